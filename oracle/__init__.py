@@ -1,0 +1,294 @@
+"""HeadQ CPU oracle -- TEST INFRASTRUCTURE ONLY.
+
+A plain, slow and obviously correct CPU restatement of HeadQ ("HeadQ:
+Model-Visible Distortion and Score-Space Correction for KV-Cache Quantization";
+the gist.science technical summary, sections 2 and 3).  Only the test-suite,
+the smoke check and the benchmark's CPU-baseline leg may import it.  It shares
+no code with the CUDA library and never imports it.
+
+The codec and the attention are in ``headq_oracle.c`` (exact fp32 codec,
+fp64 attention), compiled by :func:`build`; the query-PCA calibration is
+``numpy.linalg.eigh`` of the pooled second-moment matrix in fp64.
+
+All array arguments are numpy arrays; keys/values/queries are fp32 (bf16
+workloads pass their bf16 values converted exactly to fp32).
+"""
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "headq_oracle.c")
+_LIB = os.path.join(_HERE, "libheadq_oracle.so")
+
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+          "-fno-unsafe-math-optimizations", "-fopenmp", "-fPIC", "-shared",
+          "-fvisibility=hidden", "-Wall", "-Wno-unused-function"]
+
+
+def build(force=False):
+    """Compile the C oracle with gcc (no implicit FMA contraction, no fast-math)."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + ".tmp.%d" % os.getpid()
+    subprocess.check_call(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"])
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        L = ctypes.c_int64
+        D = ctypes.c_double
+        lib.hqo_set_threads.argtypes = [I]
+        lib.hqo_set_threads.restype = I
+        lib.hqo_base_quantize.argtypes = [P, L, I, P, P, P]
+        lib.hqo_base_dequantize.argtypes = [P, P, P, L, I, P]
+        lib.hqo_cache_write.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, P]
+        lib.hqo_side_dequantize.argtypes = [P, P, L, I, P]
+        lib.hqo_side_quantize.argtypes = [P, L, I, P, P]
+        lib.hqo_attend.argtypes = [P, I, I, I, I, I, I, P, P, P, P, P, D, D, P, P, P]
+        lib.hqo_decode.argtypes = [P, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P,
+                                   P, P, P, D, D, P, P]
+        lib.hqo_attn_kl.argtypes = [P, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P,
+                                    P, P, P, P, P, D, D, P, P, P, P]
+        for f in ("hqo_base_quantize", "hqo_base_dequantize", "hqo_cache_write",
+                  "hqo_side_dequantize", "hqo_side_quantize", "hqo_attend", "hqo_decode", "hqo_attn_kl"):
+            getattr(lib, f).restype = I
+        _lib = lib
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError("oracle %s failed with code %d" % (what, rc))
+
+
+def set_threads(n):
+    """Number of OpenMP threads the oracle uses (returns the effective count)."""
+    return _load().hqo_set_threads(int(n))
+
+
+def group_size(d):
+    return d if d < 32 else 32
+
+
+# --------------------------------------------------------------------------
+# Step 1: calibration (gist.science summary, section 3, step 1): a rank-r
+# basis U_h per KV head from the post-RoPE calibration queries.  The basis is
+# the top-r eigenvectors of the pooled uncentred second moment (1/M) Q^T Q of
+# the G query heads that read KV head h, eigenvalues descending; each column is
+# signed so that its entry of largest magnitude is positive (lowest index on a
+# tie).  center=True subtracts the pooled mean first (plain-PCA reading).
+# --------------------------------------------------------------------------
+def calibrate(q_cal, Hkv, r, center=False):
+    q_cal = np.asarray(q_cal, dtype=np.float64)
+    N, Hq, d = q_cal.shape
+    G = Hq // Hkv
+    U = np.zeros((Hkv, d, r), dtype=np.float32)
+    eig = np.zeros((Hkv, r), dtype=np.float32)
+    for kv in range(Hkv):
+        X = q_cal[:, kv * G:(kv + 1) * G, :].reshape(N * G, d)
+        if center:
+            X = X - X.mean(axis=0, keepdims=True)
+        C = (X.T @ X) / X.shape[0]
+        w, V = np.linalg.eigh(C)
+        order = np.argsort(-w, kind="stable")[:r]
+        Vr = V[:, order]
+        for i in range(r):
+            j = int(np.argmax(np.abs(Vr[:, i])))
+            if Vr[j, i] < 0:
+                Vr[:, i] = -Vr[:, i]
+        U[kv] = Vr.astype(np.float32)
+        eig[kv] = w[order].astype(np.float32)
+    return U, eig
+
+
+# --------------------------------------------------------------------------
+# Step 2: cache write.
+# --------------------------------------------------------------------------
+def base_quantize(x):
+    """B_b on the last axis: returns (codes uint8 [..., d/4], scale, min [..., ng])."""
+    x = _f32(x)
+    d = x.shape[-1]
+    lead = x.shape[:-1]
+    rows = int(np.prod(lead)) if lead else 1
+    ng = d // group_size(d)
+    codes = np.zeros(lead + (d // 4,), np.uint8)
+    sc = np.zeros(lead + (ng,), np.float32)
+    mn = np.zeros(lead + (ng,), np.float32)
+    _check(_load().hqo_base_quantize(_p(x), rows, d, _p(codes), _p(sc), _p(mn)),
+           "base_quantize")
+    return codes, sc, mn
+
+
+def base_dequantize(codes, sc, mn):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    d = codes.shape[-1] * 4
+    lead = codes.shape[:-1]
+    rows = int(np.prod(lead)) if lead else 1
+    out = np.zeros(lead + (d,), np.float32)
+    _check(_load().hqo_base_dequantize(_p(codes), _p(_f32(sc)), _p(_f32(mn)), rows,
+                                       d, _p(out)), "base_dequantize")
+    return out
+
+
+def cache_write(k, U, v=None, vmode="dense"):
+    """Encode keys k [B, Hkv, n, d] (and 2-bit values when vmode == '2bit').
+
+    Returns a dict of planes kc, ks, km, zc, zs (and vc, vs, vm) plus y, the
+    projection U_h^T e before the side quantiser.
+    """
+    k = _f32(k)
+    U = _f32(U)
+    B, Hkv, n, d = k.shape
+    r = U.shape[-1]
+    ng = d // group_size(d)
+    out = dict(
+        kc=np.zeros((B, Hkv, n, d // 4), np.uint8),
+        ks=np.zeros((B, Hkv, n, ng), np.float32),
+        km=np.zeros((B, Hkv, n, ng), np.float32),
+        zc=np.zeros((B, Hkv, n, r // 2), np.uint8),
+        zs=np.zeros((B, Hkv, n), np.float32),
+        y=np.zeros((B, Hkv, n, r), np.float32),
+    )
+    _check(_load().hqo_cache_write(_p(k), B, Hkv, n, d, r, _p(U), _p(out["kc"]),
+                                   _p(out["ks"]), _p(out["km"]), _p(out["zc"]),
+                                   _p(out["zs"]), _p(out["y"])), "cache_write")
+    if vmode == "2bit":
+        out["vc"], out["vs"], out["vm"] = base_quantize(v)
+    return out
+
+
+def side_quantize(y):
+    """Q_q on the last axis of y: returns (zc uint8 [..., r/2], zs [...])."""
+    y = _f32(y)
+    r = y.shape[-1]
+    lead = y.shape[:-1]
+    rows = int(np.prod(lead)) if lead else 1
+    zc = np.zeros(lead + (r // 2,), np.uint8)
+    zs = np.zeros(lead, np.float32)
+    _check(_load().hqo_side_quantize(_p(y), rows, r, _p(zc), _p(zs)), "side_quantize")
+    return zc, zs
+
+
+def side_dequantize(zc, zs):
+    zc = np.ascontiguousarray(zc, dtype=np.uint8)
+    r = zc.shape[-1] * 2
+    lead = zc.shape[:-1]
+    rows = int(np.prod(lead)) if lead else 1
+    out = np.zeros(lead + (r,), np.float32)
+    _check(_load().hqo_side_dequantize(_p(zc), _p(_f32(zs)), rows, r, _p(out)),
+           "side_dequantize")
+    return out
+
+
+# --------------------------------------------------------------------------
+# Step 3: cache read (decode attention).
+# --------------------------------------------------------------------------
+def attend(q, khat, v, U=None, zhat=None, sm_scale=None, sigma=1.0, seq_lens=None,
+           want_logits=False):
+    """fp64 attention with the additive logit correction.
+
+    q [B, Hq, d]; khat, v [B, Hkv, T, d]; zhat [B, Hkv, T, r] or None.
+    Returns (out [B,Hq,d], lse [B,Hq]) or also logits [B,Hq,T].
+    """
+    q = _f32(q)
+    khat = _f32(khat)
+    v = _f32(v)
+    B, Hq, d = q.shape
+    _, Hkv, T, _ = khat.shape
+    if zhat is not None:
+        zhat = np.ascontiguousarray(zhat, dtype=np.float64)
+        U = _f32(U)
+        r = U.shape[-1]
+    else:
+        r = 0
+        U = np.zeros((Hkv, d, 0), np.float32)
+    sm = 1.0 / np.sqrt(d) if sm_scale is None else float(sm_scale)
+    sl = None if seq_lens is None else np.ascontiguousarray(seq_lens, np.int32)
+    out = np.zeros((B, Hq, d), np.float64)
+    lse = np.zeros((B, Hq), np.float64)
+    lg = np.zeros((B, Hq, T), np.float64) if want_logits else None
+    _check(_load().hqo_attend(_p(q), B, Hq, Hkv, T, d, r, _p(sl), _p(khat), _p(zhat),
+                              _p(U), _p(v), sm, float(sigma), _p(out), _p(lse),
+                              _p(lg)), "attend")
+    return (out, lse, lg) if want_logits else (out, lse)
+
+
+def _vplanes(planes, vmode, v):
+    if vmode == "2bit":
+        return 1, None, planes["vc"], _f32(planes["vs"]), _f32(planes["vm"])
+    return 0, _f32(v), None, None, None
+
+
+def decode(q, planes, U, v=None, vmode="dense", sm_scale=None, sigma=1.0,
+           seq_lens=None):
+    """Cache read from stored planes ([B, Hkv, T, ...]); returns (out, lse) fp64."""
+    q = _f32(q)
+    U = _f32(U)
+    B, Hq, d = q.shape
+    _, Hkv, T, _ = planes["kc"].shape
+    r = U.shape[-1]
+    sm = 1.0 / np.sqrt(d) if sm_scale is None else float(sm_scale)
+    vm_, vd, vc, vs, vmn = _vplanes(planes, vmode, v)
+    sl = None if seq_lens is None else np.ascontiguousarray(seq_lens, np.int32)
+    out = np.zeros((B, Hq, d), np.float64)
+    lse = np.zeros((B, Hq), np.float64)
+    c = lambda a, t: np.ascontiguousarray(a, dtype=t)
+    _check(_load().hqo_decode(
+        _p(q), B, Hq, Hkv, T, d, r, _p(sl), _p(c(planes["kc"], np.uint8)),
+        _p(_f32(planes["ks"])), _p(_f32(planes["km"])), _p(c(planes["zc"], np.uint8)),
+        _p(_f32(planes["zs"])), _p(U), vm_, _p(vd), _p(vc), _p(vs), _p(vmn), sm,
+        float(sigma), _p(out), _p(lse)), "decode")
+    return out, lse
+
+
+# --------------------------------------------------------------------------
+# Step 4: diagnostics (section 2 of the summary).
+# --------------------------------------------------------------------------
+def attn_kl(q, planes, U, k_full, v_full, v=None, vmode="dense", sm_scale=None,
+            sigma=1.0, seq_lens=None):
+    """Returns (kl, fisher_var, a2_vdist, dout2), each fp64 [B, Hq]."""
+    q = _f32(q)
+    U = _f32(U)
+    B, Hq, d = q.shape
+    _, Hkv, T, _ = planes["kc"].shape
+    r = U.shape[-1]
+    sm = 1.0 / np.sqrt(d) if sm_scale is None else float(sm_scale)
+    vm_, vd, vc, vs, vmn = _vplanes(planes, vmode, v)
+    sl = None if seq_lens is None else np.ascontiguousarray(seq_lens, np.int32)
+    res = [np.zeros((B, Hq), np.float64) for _ in range(4)]
+    c = lambda a, t: np.ascontiguousarray(a, dtype=t)
+    _check(_load().hqo_attn_kl(
+        _p(q), B, Hq, Hkv, T, d, r, _p(sl), _p(c(planes["kc"], np.uint8)),
+        _p(_f32(planes["ks"])), _p(_f32(planes["km"])), _p(c(planes["zc"], np.uint8)),
+        _p(_f32(planes["zs"])), _p(U), vm_, _p(vd), _p(vc), _p(vs), _p(vmn),
+        _p(_f32(k_full)), _p(_f32(v_full)), sm, float(sigma), *[_p(a) for a in res]),
+        "attn_kl")
+    return tuple(res)
+
+
+def exact_attention(q, k, v, sm_scale=None, seq_lens=None):
+    """Full-precision attention (fp64) with no quantisation at all."""
+    return attend(q, k, v, sm_scale=sm_scale, sigma=0.0, seq_lens=seq_lens)
