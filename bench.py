@@ -1,0 +1,551 @@
+#!/usr/bin/env python
+"""HeadQ decode benchmark on B200: cached tokens/s, HBM GB/s and roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl headq|reference]
+                    [--workload NAME]
+
+One *step* is one serving decode step of one layer over a synthetic batch:
+``headq_cache_write`` of the step's new token for every (sequence, KV head)
+(base code + side code, written at position T-1), then ``headq_decode_attn``
+over the T cached tokens (query projection, streaming the packed cache,
+logits with the side-code correction, online softmax, value readout and the
+split combine).  The default workload is the long-context GQA layer (batch 1,
+32 query heads over 8 KV heads, d=128, T=131072, r=16, 2-bit keys + 4-bit side
+code + bf16 values), the bandwidth-bound case.  Calibration (one-off, offline)
+and the KL diagnostic (needs the full-precision cache) are timed beside the
+step and reported under "rows".
+
+Timing: W untimed warm-up steps, then exactly K steps replayed from a CUDA
+graph, bracketed by a barrier and a device synchronise, measured with CUDA
+events on the launching stream; the maximum over ranks is reported.  Two
+copies of the cache (2 x 348 MB > the 126 MB L2) alternate between steps, so
+every step reads its cache from HBM.  ``e2e`` is the same step through the
+public Python API with the step's inputs (query, new key/value) copied from
+pinned host memory and the output read back to the host every step.
+
+With --gpus N under torchrun every rank runs its own independent layer (weak
+scaling, no collective on the data path).  ``--impl reference`` times the CPU
+oracle on the host cores instead (rank 0 only).
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bit_decode_attention_sm_b200 import configs, synth  # noqa: E402
+
+DEFAULT_WORKLOAD = configs.WORKLOADS[3].name
+METRIC = "HeadQ decode-attn cached tokens/s and HBM GB/s (% of B200 peak), 1 GPU"
+UNIT = "cached tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["headq", "reference"], default="headq")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-rows", action="store_true", help="skip calibrate/write/kl rows")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU, NCCL; gloo in CPU tests)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def rank_seed(base_seed, rank):
+    """Each rank decodes its own independent layer (weak scaling)."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(x, device=None):
+    """Maximum of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# measurement helpers
+# ---------------------------------------------------------------------------
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(kernel_file, summary_file):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source
+    is still the one that was profiled (else None)."""
+    try:
+        src = open(os.path.join(ROOT, "bit_decode_attention_sm_b200", "csrc",
+                                kernel_file), "rb").read()
+        sha = hashlib.sha256(src).hexdigest()
+        fields = {}
+        for line in open(os.path.join(ROOT, "profiles", summary_file)):
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+        if fields.get("kernel_source_sha256") != sha:
+            return None
+        return float(fields["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def gpu_smi_id(ordinal):
+    """nvidia-smi identifier (UUID) of CUDA device `ordinal` in this process."""
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(ordinal).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        return ids[ordinal] if ordinal < len(ids) else str(ordinal)
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples while the GPU is busy."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                 power=float(parts[3]) if parts[3] not in ("", "[N/A]") else 0.0,
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        busy = [r for r in rows if r["power"] >= 0.5 * max(x["power"] for x in rows)] or rows
+        reasons = set()
+        for r in busy:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy),
+                "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(busy)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle, timed on the host cores (cpu_baseline / --impl reference)
+# ---------------------------------------------------------------------------
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_decode_rate(w, L, U, budget_s=12.0, max_T=None):
+    """Cached tokens/s of the oracle's cache read on a bounded sample of the layer:
+    the first T_s tokens of every (sequence, KV head), all query heads."""
+    import oracle
+    cores = oracle.set_threads(host_cores())
+    T_full = L.keys.shape[2]
+    max_T = T_full if max_T is None else min(max_T, T_full)
+    T_s = min(256, max_T)
+
+    def sample(Ts):
+        k = L.keys[:, :, :Ts]
+        v = L.values[:, :, :Ts]
+        planes = oracle.cache_write(k, U, v=v, vmode=w.vmode)
+        return planes, v
+
+    planes, v = sample(T_s)
+    t0 = time.perf_counter()
+    oracle.decode(L.queries, planes, U, v=v, vmode=w.vmode)
+    dt = time.perf_counter() - t0
+    # grow the sample until one call takes about a third of the budget
+    while T_s < max_T and dt < budget_s / 3:
+        T_s = min(max_T, int(T_s * max(2.0, (budget_s / 3) / max(dt, 1e-3))))
+        planes, v = sample(T_s)
+        t0 = time.perf_counter()
+        oracle.decode(L.queries, planes, U, v=v, vmode=w.vmode)
+        dt = time.perf_counter() - t0
+    reps, total = 1, dt
+    while total < budget_s * 0.66:
+        t0 = time.perf_counter()
+        oracle.decode(L.queries, planes, U, v=v, vmode=w.vmode)
+        total += time.perf_counter() - t0
+        reps += 1
+    B = L.keys.shape[0]
+    return {"value": B * T_s * reps / total, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": "oracle cache read (fp64 attention from the exact fp32 codec) of the "
+                      "first %d of %d tokens of every sequence and KV head, all %d query "
+                      "heads, %d call(s), %.1f s" % (T_s, T_full, L.queries.shape[1], reps,
+                                                      total)}
+
+
+def run_reference(args):
+    """--impl reference: the oracle on the host cores, same metric and config."""
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    w = configs.workload(args.workload)
+    L = synth.make_layer(w)
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    cores = oracle.set_threads(host_cores())
+    budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    T_s = 256
+    planes, v = None, None
+    while True:
+        planes = oracle.cache_write(L.keys[:, :, :T_s], U, v=L.values[:, :, :T_s],
+                                    vmode=w.vmode)
+        v = L.values[:, :, :T_s]
+        t0 = time.perf_counter()
+        oracle.decode(L.queries, planes, U, v=v, vmode=w.vmode)
+        dt = time.perf_counter() - t0
+        if dt >= budget / 2 or T_s >= w.T:
+            break
+        T_s = min(w.T, T_s * 2)
+    for _ in range(args.warmup):
+        oracle.decode(L.queries, planes, U, v=v, vmode=w.vmode)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.decode(L.queries, planes, U, v=v, vmode=w.vmode)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = w.B * T_s / (ms / 1e3)
+    sample = ("oracle cache read of the first %d of %d tokens of every sequence and KV head "
+              "per step" % (T_s, w.T))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, note="CPU oracle; L2 not applicable"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, note):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T,
+            "r": w.r, "keys": "2-bit group-32 base code + %d x 4-bit side code" % w.r,
+            "values": "bf16 dense" if w.vmode == "dense" else "2-bit group-32",
+            "l2": note}
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+def _events(torch):
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def run_headq(args):
+    import torch
+    import torch.distributed as dist
+    from bit_decode_attention_sm_b200 import headq as hq
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    w = configs.workload(args.workload)
+    L = synth.make_layer(w, seed=rank_seed(w.seed, rank))
+    dt = torch.bfloat16 if w.kv_dtype == "bf16" else torch.float32
+    B, Hq, Hkv, d, T = w.B, w.Hq, w.Hkv, w.d, w.T
+    stream = torch.cuda.current_stream()
+
+    # calibration on the GPU (row C1), then the full prefill write of both copies
+    q_cal = torch.from_numpy(L.q_cal).to(dev).to(dt)
+    U, _ = hq.headq_calibrate(q_cal, Hkv, w.r)
+    k_all = torch.from_numpy(L.keys).to(dev).to(dt)
+    v_all = torch.from_numpy(L.values).to(dev).to(dt)
+    caches = []
+    for _ in range(2):
+        c = hq.HeadQCache(B, Hkv, T, d, w.r, vmode=w.vmode, v_dtype=dt, device=dev)
+        hq.headq_cache_write(c, k_all, v_all, U)
+        caches.append(c)
+    q = torch.from_numpy(L.queries).to(dev).to(dt)
+    k_new = k_all[:, :, T - 1:T].contiguous()
+    v_new = v_all[:, :, T - 1:T].contiguous()
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    ws = hq.decode_workspace(caches[0], Hq, T)
+    splits, chunk, n_dec = hq.decode_plan(caches[0], Hq, T)
+    torch.cuda.synchronize()
+
+    def step(c):
+        hq.headq_cache_write(c, k_new, v_new, U, t0=T - 1)
+        hq.headq_decode_attn(c, q, U, T=T, out=out, lse=lse, ws=ws)
+
+    for i in range(max(args.warmup, 3)):
+        step(caches[i % 2])
+    torch.cuda.synchronize()
+    hq.headq_workspace_status(ws)
+
+    # capture one step per cache copy
+    graphs = []
+    use_graph = True
+    try:
+        for c in caches:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(c)
+            graphs.append(g)
+        for g in graphs:
+            g.replay()
+        torch.cuda.synchronize()
+    except Exception:
+        use_graph = False
+        graphs = []
+
+    def run_step(i):
+        if use_graph:
+            graphs[i % 2].replay()
+        else:
+            step(caches[i % 2])
+
+    sampler = ClockSampler(gpu_smi_id(local_rank))
+    sampler.start()
+    K = args.steps
+    barrier(dev)
+    torch.cuda.synchronize()
+    e0, e1 = _events(torch)
+    e0.record(stream)
+    for i in range(K):
+        run_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(dev)
+    ms_local = e0.elapsed_time(e1) / K
+    # keep the same step running for a short soak so the clock record has samples
+    t_end = time.time() + 1.5
+    i = 0
+    while time.time() < t_end:
+        run_step(i)
+        i += 1
+        if i % 200 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = max_over_ranks(ms_local, dev)
+    hq.headq_workspace_status(ws)
+
+    # decode call alone, back to back from a graph, for the roofline
+    dec_ms = None
+    try:
+        M = 20
+        gd = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gd):
+            for j in range(M):
+                hq.headq_decode_attn(caches[j % 2], q, U, T=T, out=out, lse=lse, ws=ws)
+        gd.replay()
+        torch.cuda.synchronize()
+        a, b_ = _events(torch)
+        R = max(5, min(100, 2000 // M))
+        a.record(stream)
+        for _ in range(R):
+            gd.replay()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        dec_ms = a.elapsed_time(b_) / (R * M)
+        del gd
+    except Exception:
+        a, b_ = _events(torch)
+        a.record(stream)
+        for j in range(50):
+            hq.headq_decode_attn(caches[j % 2], q, U, T=T, out=out, lse=lse, ws=ws)
+        b_.record(stream)
+        torch.cuda.synchronize()
+        dec_ms = a.elapsed_time(b_) / 50
+    dec_ms = max_over_ranks(dec_ms, dev)
+
+    # end to end through the public API: pinned host inputs in, output out, every step
+    q_h = torch.from_numpy(L.queries).to(dt).pin_memory()
+    kn_h = k_new.cpu().pin_memory()
+    vn_h = v_new.cpu().pin_memory()
+    out_h = torch.empty((B, Hq, d), dtype=torch.float32).pin_memory()
+    q_d, kn_d, vn_d = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+    Ke = max(10, min(K, 200))
+    barrier(dev)
+    torch.cuda.synchronize()
+    a, b_ = _events(torch)
+    a.record(stream)
+    for i in range(Ke):
+        c = caches[i % 2]
+        q_d.copy_(q_h, non_blocking=True)
+        kn_d.copy_(kn_h, non_blocking=True)
+        vn_d.copy_(vn_h, non_blocking=True)
+        hq.headq_cache_write(c, kn_d, vn_d, U, t0=T - 1)
+        hq.headq_decode_attn(c, q_d, U, T=T, out=out, lse=lse, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+        stream.synchronize()
+    b_.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b_) / Ke, dev)
+    h2d = q_h.numel() * q_h.element_size() + 2 * kn_h.numel() * kn_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+
+    # rows beside the step: calibration, the full prefill write, the KL diagnostic
+    rows = None
+    if not args.no_rows and rank == 0:
+        rows = measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, caches[0], dt, stream)
+
+    if world > 1:
+        barrier(dev)
+    bytes_tok = caches[0].nbytes_per_token()
+    alg_bytes = B * Hkv * T * bytes_tok
+    peak, peak_kind = measured_hbm_peak()
+    achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
+    traffic = recorded_traffic("decode_attn.cu", "decode_attn_longctx.md")
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        U_np = U.cpu().numpy()
+        cpu = oracle_decode_rate(w, L, U_np)
+    value = world * B * T / (ms * 1e-3)
+    line = {
+        "impl": "headq", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w, note="inputs larger than L2: two 348 MB cache copies "
+                                          "alternate between steps" if w.T == 131072 else
+                                          "two cache copies alternate between steps"),
+        "parallelism": "independent layer per rank" if world > 1 else "1 GPU",
+        "hbm_gbs_per_step": world * alg_bytes / (ms * 1e-3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "headq_decode_attn (split kernel + combine), %d splits of %d "
+                               "tokens" % (splits, chunk),
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "launch_ms": dec_ms, "peak_kind": peak_kind + " copy bandwidth"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * B * T / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": K * (1 + n_dec),
+        "cuda_graph": use_graph,
+        "clocks": clocks,
+        "rows": rows,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for c in caches:
+        del c
+    graphs.clear()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream):
+    """Times of the steps measured beside the decode step, with CUDA events."""
+    rows = {}
+
+    def timed(fn, reps):
+        fn()
+        torch.cuda.synchronize()
+        a, b = _events(torch)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    ms = timed(lambda: hq.headq_calibrate(q_cal, w.Hkv, w.r), 3)
+    rows["calibrate"] = {"ms": ms, "queries": int(q_cal.shape[0])}
+    B, Hkv, T = w.B, w.Hkv, w.T
+    tok = B * Hkv * T
+    ms = timed(lambda: hq.headq_cache_write(cache, k_all, v_all, U), 5)
+    in_b = tok * w.d * 2 * k_all.element_size()
+    rows["cache_write_prefill"] = {"ms": ms, "tokens": B * T,
+                                   "hbm_gbs": (in_b + tok * cache.nbytes_per_token()) / ms / 1e6}
+    ms = timed(lambda: hq.headq_attn_kl(cache, q, U, k_all, v_all), 3)
+    rows["attn_kl"] = {"ms": ms, "hbm_gbs": (in_b + tok * cache.nbytes_per_token()) / ms / 1e6}
+    return rows
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_headq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,69 @@
+"""Build libheadq.so (the CUDA C-ABI library) in-tree for sm_100a with nvcc.
+
+    python -m bit_decode_attention_sm_b200.build [--verbose]
+
+Each translation unit is compiled to an object under ``_build/`` and linked
+into ``bit_decode_attention_sm_b200/libheadq.so``.  The codec file is compiled
+with ``-fmad=false`` so no multiply and add is fused behind the intrinsics'
+back; no file uses fast-math, so division, square root and denormals keep
+IEEE semantics.
+"""
+
+import os
+import shutil
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+BUILD = os.path.join(PKG, "_build")
+LIB = os.path.join(PKG, "libheadq.so")
+
+SOURCES = ["headq_api.cu", "cache_write.cu", "decode_attn.cu", "attn_kl.cu",
+           "calibrate.cu"]
+PER_FILE_FLAGS = {"cache_write.cu": ["-fmad=false"]}
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
+          "-I" + INCLUDE, "-I" + CSRC]
+
+
+def nvcc():
+    for c in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", shutil.which("nvcc")):
+        if c and os.path.exists(c):
+            return c
+    raise RuntimeError("nvcc not found")
+
+
+def _stale(target, deps):
+    if not os.path.exists(target):
+        return True
+    t = os.path.getmtime(target)
+    return any(os.path.getmtime(d) > t for d in deps)
+
+
+def build(force=False, verbose=False):
+    os.makedirs(BUILD, exist_ok=True)
+    headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")]
+    headers.append(os.path.join(INCLUDE, "headq.h"))
+    objs = []
+    for src in SOURCES:
+        path = os.path.join(CSRC, src)
+        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
+        objs.append(obj)
+        if force or _stale(obj, [path, *headers]):
+            cmd = [nvcc(), *ARCH, *COMMON, *PER_FILE_FLAGS.get(src, [])]
+            if verbose:
+                cmd += ["-Xptxas", "-v"]
+            cmd += ["-c", path, "-o", obj]
+            subprocess.check_call(cmd)
+    if force or _stale(LIB, objs):
+        tmp = LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs])
+        os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))

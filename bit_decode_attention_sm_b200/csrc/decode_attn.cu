@@ -1,0 +1,251 @@
+// HeadQ decode attention (cache read): "HeadQ: Model-Visible Distortion and
+// Score-Space Correction for KV-Cache Quantization", gist.science summary,
+// section 3, step 3 -- the runtime query turns the stored side code into an
+// additive logit correction,
+//   s^_j = sm_scale * ( q . k^base_j + sigma * (U_h^T q) . z^_j ),
+// followed by softmax and the attention-weighted readout o = sum_j p_j v_j
+// (section 2.2).
+//
+// The base-code logit is evaluated in factored form: with group sums
+// Q_g = sum_{c in g} q_c,
+//   q . k^base_j = sum_g ( min_{j,g} Q_g + scale_{j,g} sum_{c in g} q_c code_{j,c} ),
+// which is exact algebra of the dequantisation min + code*scale, so each code is
+// used once per query head without rebuilding the key.
+//
+// Split-T flash decoding: CTA (split, kv, b) covers a contiguous chunk of tokens
+// for the G query heads of one KV head and keeps a running max m, sum l and
+// unnormalised output o (online softmax); a combine kernel merges the splits by
+// their log-sum-exp.  When there is a single split the CTA writes the result.
+#include <math.h>
+
+#include "headq_internal.cuh"
+
+namespace headq {
+namespace {
+
+constexpr int kTile = 32;      // tokens per inner step (one per lane in phase 2)
+constexpr int kThreads = 128;
+constexpr int kMaxOut = 16;    // (G * d) / kThreads outputs per thread at most
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+template <int D>
+__device__ __forceinline__ float value_at(const DecodeParams& p, size_t row, int c) {
+  if (p.c.vmode == HEADQ_V_2BIT) {
+    constexpr int NG = num_groups(D);
+    const int g = c / group_size(D);
+    const float code = static_cast<float>(code2(p.c.v_codes + row * (D / 4), c));
+    return __fadd_rn(p.c.v_min[row * NG + g], __fmul_rn(code, p.c.v_scale[row * NG + g]));
+  }
+  return load_elem(p.c.v, row * D + c, p.c.v_dtype == HEADQ_BF16);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+decode_split_kernel(const DecodeParams p) {
+  constexpr int NG = num_groups(D);
+  constexpr int GS = group_size(D);
+  const int G = p.G, r = p.c.r, Hkv = p.c.Hkv;
+  extern __shared__ float sm[];
+  float* q_s = sm;                // [G][D]
+  float* qg_s = q_s + G * D;      // [G][NG]   group sums of q
+  float* qt_s = qg_s + G * NG;    // [G][r]    sigma * U_h^T q
+  float* s_s = qt_s + G * r;      // [G][kTile] logits, then weights
+  float* m_s = s_s + G * kTile;   // [G]
+  float* l_s = m_s + G;           // [G]
+  float* a_s = l_s + G;           // [G]
+
+  const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int Tb = p.T;
+  if (p.seq_lens) Tb = max(0, min(p.seq_lens[b], p.T));
+  const int t_begin = split * p.chunk;
+  const int t_end = min(Tb, t_begin + p.chunk);
+  const size_t bk = static_cast<size_t>(b) * Hkv + kv;
+  const int h0 = kv * G;
+
+  for (int i = tid; i < G * D; i += kThreads)
+    q_s[i] = load_elem(p.q, (static_cast<size_t>(b) * p.Hq + h0) * D + i, p.q_bf16);
+  for (int h = tid; h < G; h += kThreads) {
+    m_s[h] = -INFINITY;
+    l_s[h] = 0.0f;
+  }
+  __syncthreads();
+  for (int i = tid; i < G * NG; i += kThreads) {
+    const int h = i / NG, g = i - h * NG;
+    float acc = 0.0f;
+    for (int c = 0; c < GS; ++c) acc += q_s[h * D + g * GS + c];
+    qg_s[i] = acc;
+  }
+  for (int i = tid; i < G * r; i += kThreads) {
+    const int h = i / r, ii = i - h * r;
+    const float* U = p.U + static_cast<size_t>(kv) * D * r;
+    float acc = 0.0f;
+    for (int c = 0; c < D; ++c) acc = fmaf(U[c * r + ii], q_s[h * D + c], acc);
+    qt_s[i] = p.corr_sign * acc;
+  }
+  __syncthreads();
+
+  float o[kMaxOut];
+#pragma unroll
+  for (int k = 0; k < kMaxOut; ++k) o[k] = 0.0f;
+
+  for (int t0 = t_begin; t0 < t_end; t0 += kTile) {
+    const int nt = min(kTile, t_end - t0);
+    // phase 1: logits of (head, token) pairs
+    for (int idx = tid; idx < G * kTile; idx += kThreads) {
+      const int h = idx / kTile, j = idx - h * kTile;
+      float s = -INFINITY;
+      if (j < nt) {
+        const size_t row = bk * p.c.T_cap + t0 + j;
+        const uint8_t* cr = p.c.k_codes + row * (D / 4);
+        const float* qh = q_s + h * D;
+        float acc = 0.0f;
+        for (int g = 0; g < NG; ++g) {
+          float pg = 0.0f;
+          for (int c = 0; c < GS; ++c)
+            pg = fmaf(qh[g * GS + c], static_cast<float>(code2(cr, g * GS + c)), pg);
+          acc = fmaf(p.c.k_min[row * NG + g], qg_s[h * NG + g], acc);
+          acc = fmaf(p.c.k_scale[row * NG + g], pg, acc);
+        }
+        if (r > 0) {
+          const uint8_t* zr = p.c.z_codes + row * (r / 2);
+          float cz = 0.0f;
+          for (int i = 0; i < r; ++i)
+            cz = fmaf(qt_s[h * r + i], static_cast<float>(nibble(zr, i)), cz);
+          acc = fmaf(p.c.z_scale[row], cz, acc);
+        }
+        s = acc * p.sm_scale;
+      }
+      s_s[idx] = s;
+    }
+    __syncthreads();
+    // phase 2: online softmax update, one warp per head
+    for (int h = warp; h < G; h += kThreads / 32) {
+      const float s = s_s[h * kTile + lane];
+      const float m_old = m_s[h];
+      const float m_new = fmaxf(m_old, warp_max(s));
+      const float pj = lane < nt ? expf(s - m_new) : 0.0f;
+      const float alpha = expf(m_old - m_new);
+      const float sum = warp_sum(pj);
+      s_s[h * kTile + lane] = pj;
+      __syncwarp();
+      if (lane == 0) {
+        l_s[h] = l_s[h] * alpha + sum;
+        m_s[h] = m_new;
+        a_s[h] = alpha;
+      }
+    }
+    __syncthreads();
+    // phase 3: rescale and accumulate p_j v_j
+#pragma unroll
+    for (int k = 0; k < kMaxOut; ++k) {
+      const int idx = tid + k * kThreads;
+      if (idx < G * D) {
+        const int h = idx / D, c = idx - h * D;
+        float acc = o[k] * a_s[h];
+        const float* pw = s_s + h * kTile;
+        for (int j = 0; j < nt; ++j)
+          acc = fmaf(pw[j], value_at<D>(p, bk * p.c.T_cap + t0 + j, c), acc);
+        o[k] = acc;
+      }
+    }
+    __syncthreads();
+  }
+
+  // epilogue: partial (o, m, l) or the final result
+#pragma unroll
+  for (int k = 0; k < kMaxOut; ++k) {
+    const int idx = tid + k * kThreads;
+    if (idx < G * D) {
+      const int h = idx / D, c = idx - h * D;
+      const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
+      if (p.splits == 1) {
+        const float l = l_s[h];
+        p.out[bh * D + c] = l > 0.0f ? o[k] / l : 0.0f;
+      } else {
+        float* pt = p.part + (bh * p.splits + split) * (D + 2);
+        pt[c] = o[k];
+      }
+    }
+  }
+  for (int h = tid; h < G; h += kThreads) {
+    const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
+    if (p.splits == 1) {
+      if (p.lse) p.lse[bh] = l_s[h] > 0.0f ? m_s[h] + logf(l_s[h]) : -INFINITY;
+    } else {
+      float* pt = p.part + (bh * p.splits + split) * (D + 2);
+      pt[D] = m_s[h];
+      pt[D + 1] = l_s[h];
+    }
+  }
+}
+
+// Merge the T-splits of one (b, h): exact log-sum-exp combination.
+template <int D>
+__global__ void decode_combine_kernel(const DecodeParams p) {
+  const size_t bh = blockIdx.x;
+  const int S = p.splits;
+  const float* pb = p.part + bh * S * (D + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, pb[s * (D + 2) + D]);
+  float L = 0.0f;
+  for (int s = 0; s < S; ++s) {
+    const float m = pb[s * (D + 2) + D];
+    if (m > -INFINITY) L += expf(m - M) * pb[s * (D + 2) + D + 1];
+  }
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    float acc = 0.0f;
+    for (int s = 0; s < S; ++s) {
+      const float m = pb[s * (D + 2) + D];
+      if (m > -INFINITY) acc += expf(m - M) * pb[s * (D + 2) + c];
+    }
+    p.out[bh * D + c] = L > 0.0f ? acc / L : 0.0f;
+  }
+  if (threadIdx.x == 0 && p.lse) p.lse[bh] = L > 0.0f ? M + logf(L) : -INFINITY;
+}
+
+template <int D>
+cudaError_t launch_d(const DecodeParams& p, cudaStream_t s) {
+  const int G = p.G, r = p.c.r;
+  const size_t smem = sizeof(float) * (static_cast<size_t>(G) * D + G * num_groups(D) +
+                                       G * r + G * kTile + 3 * G);
+  auto k = decode_split_kernel<D>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(p.splits, p.c.Hkv, p.c.B);
+  k<<<grid, kThreads, smem, s>>>(p);
+  if (p.splits > 1) {
+    decode_combine_kernel<D><<<p.c.B * p.Hq, D < 32 ? 32 : (D > 128 ? 128 : D), 0, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s) {
+  switch (p.c.d) {
+    case 8: return launch_d<8>(p, s);
+    case 16: return launch_d<16>(p, s);
+    case 32: return launch_d<32>(p, s);
+    case 64: return launch_d<64>(p, s);
+    case 128: return launch_d<128>(p, s);
+    case 256: return launch_d<256>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace headq

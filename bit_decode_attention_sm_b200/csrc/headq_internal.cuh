@@ -1,0 +1,108 @@
+// Internal declarations shared by the CUDA translation units of libheadq.
+// Host-side argument checking lives in headq_api.cu; each kernel file exports
+// one launcher taking a plain parameter struct.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "headq.h"
+
+namespace headq {
+
+// First bytes of every decode / attn_kl workspace: the device error word.
+constexpr size_t kWsHeaderBytes = 256;
+constexpr unsigned kDevErrWaitTimeout = 1u;
+
+__host__ __device__ constexpr int group_size(int d) { return d < 32 ? d : 32; }
+__host__ __device__ constexpr int num_groups(int d) { return d / group_size(d); }
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// element i of a tensor that is either fp32 or bf16
+__device__ __forceinline__ float load_elem(const void* p, size_t i, bool bf16) {
+  return bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(p)[i])
+              : static_cast<const float*>(p)[i];
+}
+
+// 2-bit code of channel c in a packed row
+__device__ __forceinline__ int code2(const uint8_t* row, int c) {
+  return (row[c >> 2] >> (2 * (c & 3))) & 3;
+}
+
+// signed 4-bit side code i in a packed row
+__device__ __forceinline__ int nibble(const uint8_t* row, int i) {
+  int v = (row[i >> 1] >> (4 * (i & 1))) & 0xF;
+  return v >= 8 ? v - 16 : v;
+}
+
+struct CacheWriteParams {
+  headq_cache c;
+  const void* k;
+  const void* v;
+  bool in_bf16;
+  int t0, n;
+  const float* U;
+};
+
+struct DecodeParams {
+  headq_cache c;
+  const void* q;
+  bool q_bf16;
+  int Hq, G, T;
+  const int32_t* seq_lens;
+  const float* U;
+  float sm_scale;
+  float corr_sign;
+  int splits;      // T-splits per (b, kv)
+  int chunk;       // tokens per split (multiple of 64)
+  float* part;     // [B, Hq, splits, d + 2] partial (o, m, l)
+  unsigned* err;   // device error word
+  float* out;
+  float* lse;
+};
+
+struct AttnKlParams {
+  headq_cache c;
+  const void* q;
+  bool q_bf16;
+  int Hq, G, T;
+  const int32_t* seq_lens;
+  const void* k_full;
+  const void* v_full;
+  bool kv_bf16;
+  const float* U;
+  float sm_scale;
+  float corr_sign;
+  int splits, chunk;
+  double* part;    // [B, Hq, splits, 7 + d]
+  unsigned* err;
+  float *kl, *fvar, *a2v, *dout2;
+};
+
+struct CalibrateParams {
+  const void* q;
+  bool bf16;
+  int N, Hq, Hkv, G, d, r;
+  bool center;
+  double* gram;    // [Hkv, d, d]
+  double* vt;      // [Hkv, d, d] rotation accumulator (rows = eigenvectors)
+  float* U;
+  float* eig;
+};
+
+cudaError_t launch_cache_write(const CacheWriteParams& p, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_attn_kl(const AttnKlParams& p, cudaStream_t s);
+cudaError_t launch_calibrate(const CalibrateParams& p, cudaStream_t s);
+
+// split planning shared by the workspace-size query and the launch
+struct SplitPlan {
+  int splits, chunk;
+};
+SplitPlan plan_splits(int units, int T, int min_chunk);
+
+}  // namespace headq

@@ -1,0 +1,207 @@
+/*
+ * headq.h -- C ABI of libheadq, HeadQ decode attention for NVIDIA B200 (sm_100a).
+ *
+ * HeadQ ("HeadQ: Model-Visible Distortion and Score-Space Correction for
+ * KV-Cache Quantization"; arXiv abstract and the gist.science technical summary,
+ * section 3 "Methodology: HeadQ") stores every cached key as
+ *   - a 2-bit base code  k^base_j = B_b(k_j)                    (section 3, step 2)
+ *   - a low-rank side code z_j = Q_q(U_h^T (k_j - k^base_j))     (section 3, step 2)
+ * in a rank-r basis U_h learned from post-RoPE calibration queries (step 1), and
+ * reads it with an additive logit correction                     (section 3, step 3)
+ *   s^_j = q^T k^base_j / sqrt(d) + q^T U_h z^_j / sqrt(d),
+ * followed by softmax and the attention-weighted value readout.  Section 2 of the
+ * summary defines the diagnostics (attention KL, the Fisher-weighted score-error
+ * variance, the A^2-weighted value distortion) that headq_attn_kl computes.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers, allocated and owned by the caller;
+ *     the library allocates no memory and keeps no state between calls.
+ *   - Work is enqueued asynchronously on `stream`; results are valid once the
+ *     stream has reached that point.  Argument errors are detected on the host,
+ *     before anything is launched, and returned synchronously.
+ *   - Every pointer must be 16-byte aligned.  Layouts are dense, row-major, with
+ *     the last index fastest.
+ *   - Shapes: d is 8, 16, 32, 64, 128 or 256; the base code works on groups of
+ *     32 channels (group = d when d < 32); r is even with 0 <= r <= min(d, 32);
+ *     Hq is a multiple of Hkv and query head h reads KV head h / (Hq / Hkv);
+ *     T_cap (the cache capacity in tokens) is a multiple of 16.
+ *   - Codec bit layout: channel c of a 2-bit code is bits 2*(c%4)..2*(c%4)+1 of
+ *     byte c/4; side-code entry i is a 4-bit two's-complement nibble in byte i/2
+ *     (even i in the low nibble).  Scales and minima are IEEE fp32.
+ *   - Exact codec arithmetic (bit-reproducible): for each token and group of 32
+ *     channels, mn = min x, mx = max x (a -0 extreme stored as +0),
+ *     scale = (mx - mn) / 3, code = clamp(rint((x - mn) / scale), 0, 3) with
+ *     round-half-even (all codes 0 when scale == 0); the residual is
+ *     e = x - (mn + code*scale) (product rounded first); the projection
+ *     y = U_h^T e accumulates channel by channel in order with one fused
+ *     multiply-add per term; the side scale is s = max|y| / 7 and the side code
+ *     w = clamp(rint(y / s), -7, 7) (all 0 when s == 0).  Every operation is one
+ *     IEEE fp32 operation (division correctly rounded, no flush-to-zero).
+ */
+#ifndef HEADQ_H
+#define HEADQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *headq_stream_t;
+
+typedef enum {
+    HEADQ_OK = 0,
+    HEADQ_ERR_INVALID_ARG = 1, /* null/misaligned pointer, inconsistent sizes    */
+    HEADQ_ERR_UNSUPPORTED = 2, /* valid request outside the supported shapes     */
+    HEADQ_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required     */
+    HEADQ_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed            */
+    HEADQ_ERR_DEVICE = 5       /* a kernel flagged a device-side error (timeout) */
+} headq_status;
+
+typedef enum { HEADQ_F32 = 0, HEADQ_BF16 = 1 } headq_dtype;
+
+typedef enum {
+    HEADQ_V_DENSE = 0, /* V stored as v_dtype, [B, Hkv, T_cap, d]               */
+    HEADQ_V_2BIT = 1   /* V stored with the 2-bit base code of the keys, no side */
+} headq_vmode;
+
+/*
+ * The packed HeadQ cache: structure-of-arrays planes in HBM, each indexed
+ * [b][kv][t] with t < T_cap.  Planes (NG = d / min(32, d) groups per token):
+ *   k_codes  uint8 [B, Hkv, T_cap, d/4]   2-bit base key code
+ *   k_scale  fp32  [B, Hkv, T_cap, NG]    base-code scale per group
+ *   k_min    fp32  [B, Hkv, T_cap, NG]    base-code minimum per group
+ *   z_codes  uint8 [B, Hkv, T_cap, r/2]   4-bit side code (unused when r == 0)
+ *   z_scale  fp32  [B, Hkv, T_cap]        side-code scale
+ *   v        v_dtype [B, Hkv, T_cap, d]   dense values   (vmode DENSE)
+ *   v_codes/v_scale/v_min as k_codes/k_scale/k_min        (vmode 2BIT)
+ * Pointers of planes the mode does not use may be NULL.
+ */
+typedef struct {
+    int B, Hkv, T_cap, d, r;
+    headq_vmode vmode;
+    headq_dtype v_dtype;
+    uint8_t *k_codes;
+    float *k_scale, *k_min;
+    uint8_t *z_codes;
+    float *z_scale;
+    void *v;
+    uint8_t *v_codes;
+    float *v_scale, *v_min;
+} headq_cache;
+
+/* Library version as 10000*major + 100*minor + patch. */
+int headq_version(void);
+
+/* Static, human-readable text for a status code. */
+const char *headq_status_string(headq_status s);
+
+/*
+ * headq_calibrate -- query-PCA basis U_h per KV head (summary section 3, step 1:
+ * each layer and head gets a rank-r basis from a PCA of its post-RoPE
+ * calibration queries).
+ *   q_cal   [N, Hq, d] (dtype), calibration queries after RoPE.
+ *   U_out   fp32 [Hkv, d, r]: U_out[(kv*d + c)*r + i] is entry c of basis vector i.
+ *   eig_out fp32 [Hkv, r] (nullable): the matching eigenvalues, descending.
+ * The basis is the top-r eigenvectors of the second moment (1/M) X^T X of the
+ * M = N*G calibration queries of the G query heads that share KV head kv
+ * (center != 0 subtracts their mean first), computed in fp64 by cyclic Jacobi
+ * rotations; each column is signed so that its largest-magnitude entry is
+ * positive (lowest index on a tie).
+ *   ws: device workspace of at least headq_calibrate_workspace_bytes(...) bytes.
+ * Requires 1 <= r <= d <= 128.
+ */
+headq_status headq_calibrate(const void *q_cal, headq_dtype dtype, int N, int Hq,
+                             int Hkv, int d, int r, int center, float *U_out,
+                             float *eig_out, void *ws, size_t ws_bytes,
+                             headq_stream_t stream);
+size_t headq_calibrate_workspace_bytes(int N, int Hq, int Hkv, int d);
+
+/*
+ * headq_cache_write -- encode n new tokens per (b, kv) into cache positions
+ * [t0, t0 + n) (summary section 3, step 2: base code, residual, projection onto
+ * U_h, side quantizer, store base code and side code).
+ *   k, v  [B, Hkv, n, d] of kv_dtype.  k is encoded; v is copied (DENSE, rounded
+ *         to nearest-even when the cache is bf16 and v is fp32) or encoded with
+ *         the 2-bit base code (2BIT).  v may be NULL to leave V untouched.
+ *   U     fp32 [Hkv, d, r] from headq_calibrate (ignored when r == 0).
+ * Bit-exact with the arithmetic stated at the top of this header.
+ * Requires 0 <= t0, 0 <= n, t0 + n <= T_cap.  n == 0 is a no-op.
+ */
+headq_status headq_cache_write(const headq_cache *cache, const void *k, const void *v,
+                               headq_dtype kv_dtype, int t0, int n, const float *U,
+                               headq_stream_t stream);
+
+/*
+ * headq_decode_attn -- one decode step of attention over the HeadQ cache
+ * (summary section 3, step 3: the runtime query decodes the side code into the
+ * additive logit correction; softmax and the readout o = sum_j p_j v_j of
+ * section 2.2).  For every (b, h), kv = h / (Hq/Hkv), tokens j < T_b:
+ *   s^_j = sm_scale * ( q.k^base_j + corr_sign * (U_h^T q) . z^_j )
+ *   out[b,h] = sum_j softmax(s^)_j v^_j ,  lse[b,h] = log sum_j exp(s^_j)
+ * with k^base_j = mn + code*scale per group, z^_j = w_j * s_j, and v^_j the dense
+ * value or its 2-bit dequantisation.
+ *   q         [B, Hq, d] (q_dtype)
+ *   seq_lens  int32 [B] (nullable): T_b; NULL means T_b = T for every b.
+ *             0 <= T_b <= T <= T_cap.  T_b == 0 gives out = 0, lse = -inf.
+ *   sm_scale  logit scale; pass 1/sqrt(d) for the pages' formula.
+ *   corr_sign +1 HeadQ, 0 base code only, -1 the wrong-sign control (section 4).
+ *   out       fp32 [B, Hq, d];  lse fp32 [B, Hq] (nullable).
+ *   ws        device workspace of at least headq_decode_workspace_bytes(...)
+ *             bytes whose first 256 bytes were zero before its first use (they
+ *             hold the device error word; see headq_workspace_status).
+ * Accumulation is fp32; the result matches the fp64 definition to a relative
+ * error of about 1e-5 of the row maximum.
+ */
+headq_status headq_decode_attn(const headq_cache *cache, const void *q,
+                               headq_dtype q_dtype, int Hq, const int32_t *seq_lens,
+                               int T, const float *U, float sm_scale, int corr_sign,
+                               float *out, float *lse, void *ws, size_t ws_bytes,
+                               headq_stream_t stream);
+size_t headq_decode_workspace_bytes(const headq_cache *cache, int Hq, int T);
+
+/*
+ * headq_decode_plan -- the launch plan headq_decode_attn uses for these sizes on
+ * the current device: *splits T-splits of *chunk tokens per (b, kv), and the
+ * number of kernels one call launches (returned).  0 on invalid sizes.
+ */
+int headq_decode_plan(const headq_cache *cache, int Hq, int T, int *splits, int *chunk);
+
+/*
+ * headq_attn_kl -- model-visible distortion of the cache against the
+ * full-precision keys and values (summary section 2.1: score perturbation
+ * delta_j = s^_j - s_j, attention KL and its local Fisher form; section 2.2:
+ * readout error and the A^2 weighting).  With s_j = sm_scale * q.k_j (full
+ * keys), p = softmax(s), p~ = softmax(s^) and v^ as read from the cache:
+ *   kl         = KL(p || p~)                    fp32 [B, Hq]
+ *   fisher_var = Var_p(s^ - s)                  fp32 [B, Hq]
+ *   a2_vdist   = sum_j p_j^2 |v^_j - v_j|^2     fp32 [B, Hq]
+ *   dout2      = |sum_j p_j (v^_j - v_j)|^2     fp32 [B, Hq] (nullable)
+ *   k_full, v_full [B, Hkv, T, d] of kv_dtype (the unquantised cache).
+ * Other arguments as headq_decode_attn; workspace from
+ * headq_attn_kl_workspace_bytes (first 256 bytes zero before first use).
+ * Accumulators are fp64.
+ */
+headq_status headq_attn_kl(const headq_cache *cache, const void *q, headq_dtype q_dtype,
+                           int Hq, const int32_t *seq_lens, int T, const void *k_full,
+                           const void *v_full, headq_dtype kv_dtype, const float *U,
+                           float sm_scale, int corr_sign, float *kl, float *fisher_var,
+                           float *a2_vdist, float *dout2, void *ws, size_t ws_bytes,
+                           headq_stream_t stream);
+size_t headq_attn_kl_workspace_bytes(const headq_cache *cache, int Hq, int T);
+
+/*
+ * headq_workspace_status -- waits for `stream`, reads the device error word of a
+ * decode / attn_kl workspace, clears it, and returns HEADQ_ERR_DEVICE if a
+ * kernel that used the workspace gave up a bounded wait (it then wrote no
+ * result), else HEADQ_OK.  Synchronous; call it off the hot path.
+ */
+headq_status headq_workspace_status(void *ws, headq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HEADQ_H */

@@ -1,0 +1,144 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every entry
+point include/headq.h declares, and rejects bad arguments on the host before
+anything is launched.  No call here reaches a kernel launch."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "headq.h")
+
+
+@pytest.fixture(scope="module")
+def hq():
+    from bit_decode_attention_sm_b200 import build, headq
+    build.build()
+    return headq
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(headq_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(hq):
+    names = declared_functions()
+    assert "headq_decode_attn" in names and len(names) >= 10
+    lib = hq.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(hq.EXPORTS)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", hq.LIB_PATH], text=True)
+    exported = set(re.findall(r"\bT (headq_\w+)", out))
+    assert set(names) <= exported
+
+
+def test_version_and_status_strings(hq):
+    lib = hq.lib()
+    assert lib.headq_version() == 100
+    for code in range(6):
+        assert lib.headq_status_string(code)
+    assert lib.headq_status_string(99) == b"unknown status"
+
+
+FAKE = 0x7f0000000000  # 16-byte aligned address, never dereferenced
+
+
+def make_cache(hq, d=128, r=16, T_cap=1024, B=1, Hkv=2, vmode=0, **over):
+    s = hq.CacheStruct()
+    s.B, s.Hkv, s.T_cap, s.d, s.r, s.vmode, s.v_dtype = B, Hkv, T_cap, d, r, vmode, 1
+    for i, f in enumerate(("k_codes", "k_scale", "k_min", "z_codes", "z_scale", "v",
+                           "v_codes", "v_scale", "v_min")):
+        setattr(s, f, FAKE + 0x100000 * i)
+    for k, v in over.items():
+        setattr(s, k, v)
+    return s
+
+
+def _write(hq, cs, k=FAKE, t0=0, n=1, U=FAKE):
+    return hq.lib().headq_cache_write(ctypes.byref(cs), ctypes.c_void_p(k), None, 1, t0, n,
+                                      ctypes.c_void_p(U), None)
+
+
+def test_cache_write_rejects(hq):
+    L = hq.lib()
+    assert L.headq_cache_write(None, None, None, 1, 0, 1, None, None) == 1
+    assert _write(hq, make_cache(hq, d=48)) == 2
+    assert _write(hq, make_cache(hq, r=3)) == 2
+    assert _write(hq, make_cache(hq, r=34, d=64)) == 2
+    assert _write(hq, make_cache(hq, T_cap=100)) == 2
+    assert _write(hq, make_cache(hq, k_codes=FAKE + 1)) == 1
+    assert _write(hq, make_cache(hq, z_scale=0)) == 1
+    assert _write(hq, make_cache(hq, v=0)) == 1
+    assert _write(hq, make_cache(hq, vmode=1, v_codes=0)) == 1
+    assert _write(hq, make_cache(hq), k=0) == 1
+    assert _write(hq, make_cache(hq), k=FAKE + 8) == 1
+    assert _write(hq, make_cache(hq), U=0) == 1
+    assert _write(hq, make_cache(hq), t0=1000, n=100) == 1
+    assert _write(hq, make_cache(hq), t0=-1) == 1
+    # n == 0 is a no-op that launches nothing
+    assert _write(hq, make_cache(hq), n=0) == 0
+
+
+def _decode(hq, cs, Hq=4, T=512, corr=1, ws_bytes=1 << 30, q=FAKE, out=FAKE, ws=FAKE):
+    return hq.lib().headq_decode_attn(
+        ctypes.byref(cs), ctypes.c_void_p(q), 1, Hq, None, T, ctypes.c_void_p(FAKE),
+        ctypes.c_float(0.1), corr, ctypes.c_void_p(out), None, ctypes.c_void_p(ws), ws_bytes,
+        None)
+
+
+def test_decode_rejects(hq):
+    cs = make_cache(hq)
+    assert _decode(hq, cs, Hq=3) == 1
+    assert _decode(hq, cs, corr=2) == 1
+    assert _decode(hq, cs, T=2048) == 1
+    assert _decode(hq, cs, q=0) == 1
+    assert _decode(hq, cs, out=FAKE + 4) == 1
+    assert _decode(hq, cs, ws=0) == 3
+    assert _decode(hq, cs, ws_bytes=16) == 3
+    assert _decode(hq, make_cache(hq, d=256), Hq=2 * 9) == 2      # G*d > 2048
+    assert _decode(hq, make_cache(hq, d=40)) == 2
+
+
+def test_workspace_and_plan(hq):
+    L = hq.lib()
+    cs = make_cache(hq, B=1, Hkv=8)
+    sp, ch = ctypes.c_int(), ctypes.c_int()
+    nk = L.headq_decode_plan(ctypes.byref(cs), 32, 131072 // 128, ctypes.byref(sp),
+                             ctypes.byref(ch))
+    assert nk in (1, 2) and sp.value >= 1 and ch.value % 64 == 0
+    assert sp.value * ch.value >= 1024
+    n = L.headq_decode_workspace_bytes(ctypes.byref(cs), 32, 1024)
+    assert n >= 256 + 4 * 32 * sp.value * (128 + 2)
+    assert L.headq_decode_workspace_bytes(None, 32, 1024) == 0
+    assert L.headq_attn_kl_workspace_bytes(ctypes.byref(cs), 32, 1024) >= 256
+    assert L.headq_calibrate_workspace_bytes(1024, 32, 8, 128) >= 2 * 8 * 128 * 128 * 8
+    assert L.headq_workspace_status(None, None) == 1
+
+
+def test_calibrate_rejects(hq):
+    L = hq.lib()
+    P = ctypes.c_void_p
+    big = 1 << 30
+    assert L.headq_calibrate(P(FAKE), 1, 64, 8, 2, 256, 8, 0, P(FAKE), None, P(FAKE), big,
+                             None) == 2
+    assert L.headq_calibrate(P(FAKE), 1, 64, 8, 3, 64, 8, 0, P(FAKE), None, P(FAKE), big,
+                             None) == 1
+    assert L.headq_calibrate(P(FAKE), 1, 64, 8, 2, 64, 65, 0, P(FAKE), None, P(FAKE), big,
+                             None) == 2
+    assert L.headq_calibrate(P(FAKE), 1, 64, 8, 2, 64, 8, 0, P(FAKE), None, P(FAKE), 8,
+                             None) == 3
+    assert L.headq_calibrate(None, 1, 64, 8, 2, 64, 8, 0, P(FAKE), None, P(FAKE), big,
+                             None) == 1
+
+
+def test_binding_refuses_cpu_tensors(hq):
+    import torch
+    q = torch.zeros(1, 4, 64)
+    with pytest.raises(ValueError):
+        hq.headq_calibrate(q, 1, 8)

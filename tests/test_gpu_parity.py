@@ -1,0 +1,235 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Cache write: every plane bit-exact (fp32 planes compared as bit patterns).
+Decode: max relative error per output row <= 2e-3 of the row maximum.
+Diagnostics: relative 1e-2 or absolute 1e-6, whichever is looser.
+Calibration: projector distance |U U^T - U_ref U_ref^T|_F <= 1e-3, eigenvalues
+to relative 1e-4.
+
+Reduced sizes keep each workload's distribution and head layout and still span
+several tiles, several T-splits and a ragged tail; the full-size cases run the
+exact launch configuration of the benchmark and check sampled rows the oracle
+recomputes from scratch.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from bit_decode_attention_sm_b200 import configs, synth
+from parity_helpers import (DECODE_RTOL, assert_diag_close, assert_planes_equal, gpu_cache,
+                            gpu_query, layer, oracle_side, planes_to_numpy, roundup,
+                            row_rel_err, torch_dtype)
+
+pytestmark = pytest.mark.gpu
+
+CASES = [(0, {}), (1, dict(T=300)), (2, dict(T=1000, B=2)), (3, dict(T=2500)),
+         (4, dict(T=700, B=3))]
+IDS = ["cfg%d" % c[0] for c in CASES]
+
+
+def _headq():
+    from bit_decode_attention_sm_b200 import headq
+    return headq
+
+
+@pytest.mark.parametrize("i,kw", CASES, ids=IDS)
+def test_cache_write_bit_exact(i, kw):
+    w, L = layer(i, **kw)
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    ref = oracle.cache_write(L.keys, U, v=L.values, vmode=w.vmode)
+    cache, _ = gpu_cache(w, L, U)
+    got = planes_to_numpy(cache, 0, L.keys.shape[2])
+    assert_planes_equal(got, ref, w.r, w.vmode, w.kv_dtype, values=L.values)
+
+
+def test_cache_write_chunks_and_offset():
+    """A prefill chunk followed by one-token appends at an odd offset writes the
+    same planes as the oracle on the whole sequence."""
+    import torch
+    hq = _headq()
+    w, L = layer(2, T=203, B=2)
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    ref = oracle.cache_write(L.keys, U, v=L.values)
+    dt = torch_dtype(w)
+    t0 = 5
+    cache = hq.HeadQCache(2, w.Hkv, roundup(t0 + 203, 16), w.d, w.r, v_dtype=dt)
+    Ut = torch.from_numpy(U).cuda()
+    k = torch.from_numpy(L.keys).cuda().to(dt)
+    v = torch.from_numpy(L.values).cuda().to(dt)
+    hq.headq_cache_write(cache, k[:, :, :190].contiguous(), v[:, :, :190].contiguous(), Ut,
+                         t0=t0)
+    for t in range(190, 203):
+        hq.headq_cache_write(cache, k[:, :, t:t + 1].contiguous(), v[:, :, t:t + 1].contiguous(),
+                             Ut, t0=t0 + t)
+    got = planes_to_numpy(cache, t0, 203)
+    assert_planes_equal(got, ref, w.r, w.vmode, w.kv_dtype, values=L.values)
+
+
+@pytest.mark.parametrize("sigma", [1, 0, -1])
+@pytest.mark.parametrize("i,kw", CASES, ids=IDS)
+def test_decode_matches_oracle(i, kw, sigma):
+    hq = _headq()
+    w, L = layer(i, **kw)
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    _, out_ref, lse_ref = oracle_side(w, L, U, sigma=float(sigma))
+    cache, Ut = gpu_cache(w, L, U)
+    T = L.keys.shape[2]
+    ws = hq.decode_workspace(cache, w.Hq, T)
+    out, lse = hq.headq_decode_attn(cache, gpu_query(w, L), Ut, T=T, corr_sign=sigma, ws=ws)
+    hq.headq_workspace_status(ws)
+    err = row_rel_err(out.cpu().numpy(), out_ref)
+    assert err <= DECODE_RTOL, err
+    np.testing.assert_allclose(lse.cpu().numpy(), lse_ref, rtol=1e-5, atol=1e-4)
+
+
+def test_decode_from_oracle_planes():
+    """The decode kernel alone: planes written by the oracle, uploaded as they are."""
+    import torch
+    hq = _headq()
+    w, L = layer(3, T=1500)
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    planes, out_ref, _ = oracle_side(w, L, U)
+    T = L.keys.shape[2]
+    cache = hq.HeadQCache(1, w.Hkv, roundup(T, 16), w.d, w.r, v_dtype=torch.bfloat16)
+    for name, t in cache.planes().items():
+        src = planes[name] if name != "v" else None
+        if name == "v":
+            t[:, :, :T] = torch.from_numpy(L.values).to(torch.bfloat16).cuda()
+        else:
+            t[:, :, :T] = torch.from_numpy(np.ascontiguousarray(src)).cuda()
+    out, _ = hq.headq_decode_attn(cache, gpu_query(w, L), torch.from_numpy(U).cuda(), T=T)
+    assert row_rel_err(out.cpu().numpy(), out_ref) <= DECODE_RTOL
+
+
+def test_decode_ragged_sequences():
+    """Per-sequence lengths 0, 1, 33 and T with capacity beyond T."""
+    import torch
+    hq = _headq()
+    w, L = layer(2, T=777, B=4)
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    sl = np.array([0, 1, 33, 777], np.int32)
+    _, out_ref, lse_ref = oracle_side(w, L, U, seq_lens=sl)
+    cache, Ut = gpu_cache(w, L, U, T_cap=1024)
+    out, lse = hq.headq_decode_attn(cache, gpu_query(w, L), Ut, T=777,
+                                    seq_lens=torch.from_numpy(sl).cuda())
+    o, l = out.cpu().numpy(), lse.cpu().numpy()
+    assert (o[0] == 0).all() and np.isneginf(l[0]).all()
+    assert row_rel_err(o[1:], out_ref[1:]) <= DECODE_RTOL
+    np.testing.assert_allclose(l[1:], lse_ref[1:], rtol=1e-5, atol=1e-4)
+
+
+SMALL = [  # (d, r, Hq, Hkv, T, B) beyond the five workloads: every head dim, GQA groups
+    (8, 4, 2, 1, 16, 2), (16, 2, 4, 2, 45, 1), (32, 8, 8, 1, 130, 2),
+    (64, 16, 14, 2, 129, 1), (128, 32, 8, 8, 70, 1), (256, 16, 8, 2, 300, 1),
+    (128, 0, 4, 4, 90, 1),
+]
+
+
+@pytest.mark.parametrize("d,r,Hq,Hkv,T,B", SMALL)
+@pytest.mark.parametrize("kv_dtype,vmode", [("bf16", "dense"), ("f32", "dense"),
+                                            ("bf16", "2bit")])
+def test_small_shapes(d, r, Hq, Hkv, T, B, kv_dtype, vmode):
+    hq = _headq()
+    base = configs.workload(1)
+    w = base.with_(d=d, r=r, r_s=max(2, min(8, d // 2)), Hq=Hq, Hkv=Hkv, B=B, T=T,
+                   n_cal=64, kv_dtype=kv_dtype, vmode=vmode)
+    L = synth.make_layer(w)
+    if r > 0:
+        U, _ = oracle.calibrate(L.q_cal, Hkv, r)
+    else:
+        U = np.zeros((Hkv, d, 0), np.float32)
+    planes, out_ref, lse_ref = oracle_side(w, L, U)
+    cache, Ut = gpu_cache(w, L, U)
+    got = planes_to_numpy(cache, 0, T)
+    assert_planes_equal(got, planes, r, vmode, kv_dtype, values=L.values)
+    out, lse = hq.headq_decode_attn(cache, gpu_query(w, L), Ut, T=T)
+    assert row_rel_err(out.cpu().numpy(), out_ref) <= DECODE_RTOL
+    np.testing.assert_allclose(lse.cpu().numpy(), lse_ref, rtol=1e-5, atol=1e-4)
+
+
+@pytest.mark.parametrize("sigma", [1, -1])
+@pytest.mark.parametrize("i,kw", CASES, ids=IDS)
+def test_attn_kl_matches_oracle(i, kw, sigma):
+    import torch
+    hq = _headq()
+    w, L = layer(i, **kw)
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    planes = oracle.cache_write(L.keys, U, v=L.values, vmode=w.vmode)
+    ref = oracle.attn_kl(L.queries, planes, U, L.keys, L.values, v=L.values, vmode=w.vmode,
+                         sigma=float(sigma))
+    cache, Ut = gpu_cache(w, L, U)
+    dt = torch_dtype(w)
+    kf = torch.from_numpy(L.keys).cuda().to(dt)
+    vf = torch.from_numpy(L.values).cuda().to(dt)
+    got = hq.headq_attn_kl(cache, gpu_query(w, L), Ut, kf, vf, corr_sign=sigma)
+    for g, r_, name in zip(got, ref, ("kl", "fisher_var", "a2_vdist", "dout2")):
+        assert_diag_close(g.cpu().numpy(), r_, name)
+
+
+@pytest.mark.parametrize("i", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("center", [False, True])
+def test_calibrate_matches_oracle(i, center):
+    import torch
+    hq = _headq()
+    w, L = layer(i, T=16, B=1)
+    U_ref, eig_ref = oracle.calibrate(L.q_cal, w.Hkv, w.r, center=center)
+    q = torch.from_numpy(L.q_cal).cuda().to(torch_dtype(w))
+    U, eig = hq.headq_calibrate(q, w.Hkv, w.r, center=center)
+    U, eig = U.cpu().numpy().astype(np.float64), eig.cpu().numpy()
+    for kv in range(w.Hkv):
+        P = U[kv] @ U[kv].T
+        Pr = U_ref[kv].astype(np.float64) @ U_ref[kv].T.astype(np.float64)
+        assert np.linalg.norm(P - Pr) <= 1e-3
+        np.testing.assert_allclose(eig[kv], eig_ref[kv], rtol=1e-4)
+        # same sign rule: columns agree, not just the subspace
+        assert np.abs(U[kv] - U_ref[kv]).max() <= 1e-3
+
+
+def test_wrong_sign_and_base_only_through_the_abi():
+    """Section 4 control on the GPU: sigma=-1 gives larger KL than sigma=0 and +1."""
+    import torch
+    hq = _headq()
+    w, L = layer(2, T=512, B=2)
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    cache, Ut = gpu_cache(w, L, U)
+    dt = torch_dtype(w)
+    kf = torch.from_numpy(L.keys).cuda().to(dt)
+    vf = torch.from_numpy(L.values).cuda().to(dt)
+    q = gpu_query(w, L)
+    kl = {s: hq.headq_attn_kl(cache, q, Ut, kf, vf, corr_sign=s)[0].mean().item()
+          for s in (1, 0, -1)}
+    assert kl[1] < kl[0] < kl[-1], kl
+
+
+FULL = [1, 2, 3, 4]
+
+
+@pytest.mark.parametrize("i", FULL, ids=["cfg%d-full" % i for i in FULL])
+def test_full_size_sampled_rows(i):
+    """Full workload size, the benchmark's launch configuration; the oracle
+    re-encodes two sampled (b, kv) sequences from the inputs and decodes their
+    query heads."""
+    import torch
+    hq = _headq()
+    w = configs.workload(i)
+    L = synth.make_layer(w)
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    cache, Ut = gpu_cache(w, L, U)
+    out, lse = hq.headq_decode_attn(cache, gpu_query(w, L), Ut, T=w.T)
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    rng = np.random.default_rng(100 + i)
+    picks = {(int(rng.integers(w.B)), int(rng.integers(w.Hkv))) for _ in range(2)}
+    for b, kv in sorted(picks):
+        sub = synth.LayerInputs(L.keys[b:b + 1, kv:kv + 1], L.values[b:b + 1, kv:kv + 1],
+                                L.queries[b:b + 1, kv * w.G:(kv + 1) * w.G], None, {})
+        w1 = w.with_(B=1, Hkv=1, Hq=w.G)
+        planes, out_ref, lse_ref = oracle_side(w1, sub, U[kv:kv + 1])
+        got = planes_to_numpy(cache, 0, w.T, b=b, kv=kv)
+        assert_planes_equal(got, planes, w.r, w.vmode, w.kv_dtype, values=sub.values)
+        o = out[b:b + 1, kv * w.G:(kv + 1) * w.G]
+        assert row_rel_err(o, out_ref) <= DECODE_RTOL
+        np.testing.assert_allclose(lse[b:b + 1, kv * w.G:(kv + 1) * w.G], lse_ref,
+                                   rtol=1e-5, atol=1e-4)
+    del cache
+    torch.cuda.empty_cache()
