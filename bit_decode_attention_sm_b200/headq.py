@@ -29,7 +29,8 @@ STATUS = {0: "HEADQ_OK", 1: "HEADQ_ERR_INVALID_ARG", 2: "HEADQ_ERR_UNSUPPORTED",
 EXPORTS = ("headq_version", "headq_status_string", "headq_calibrate",
            "headq_calibrate_workspace_bytes", "headq_cache_write", "headq_decode_attn",
            "headq_decode_workspace_bytes", "headq_decode_plan", "headq_attn_kl",
-           "headq_attn_kl_workspace_bytes", "headq_workspace_status")
+           "headq_attn_kl_workspace_bytes", "headq_workspace_status",
+           "headq_decode_attn_noalloc")
 
 
 class HeadQError(RuntimeError):
@@ -76,6 +77,7 @@ def lib():
             "headq_attn_kl": ([CP, P, I, I, P, I, P, P, I, P, F, I, P, P, P, P, P, Z, P], I),
             "headq_attn_kl_workspace_bytes": ([CP, I, I], Z),
             "headq_workspace_status": ([P, P], I),
+            "headq_decode_attn_noalloc": ([CP, P, I, I, P, I, P, F, I, P, P, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)

@@ -170,6 +170,32 @@ size_t headq_decode_workspace_bytes(const headq_cache *cache, int Hq, int T);
 int headq_decode_plan(const headq_cache *cache, int Hq, int T, int *splits, int *chunk);
 
 /*
+ * headq_decode_attn_noalloc -- headq_decode_attn without a caller workspace.
+ * The HeadQ pages have no counterpart to this: it exists for callers that hold
+ * only their input and output buffers and cannot allocate device memory (a
+ * plugin inside a host framework that hands it tensors but no allocator,
+ * code running where cudaMalloc is forbidden after start-up, or a caller that
+ * must not grow its memory footprint per request).
+ *   Arguments and results are those of headq_decode_attn minus ws/ws_bytes.
+ *   Scratch: a fixed 4 MiB array inside the library (per GPU, resident from
+ *   load until process exit).  A request whose workspace
+ *   (headq_decode_workspace_bytes) exceeds 4 MiB returns HEADQ_ERR_WORKSPACE
+ *   and launches nothing.
+ *   The first call on a device does a one-time, synchronous set-up on that
+ *   device (looks up the array's device address, clears its header); make that
+ *   first call before any stream capture.
+ *   Every call on a device shares the one array and leaves its contents behind:
+ *   calls whose work overlaps on the GPU (different streams, or different host
+ *   threads, without ordering between them) race on it and must be serialised
+ *   by the caller.  Allocates nothing (no cudaMalloc, no cudaFree).
+ */
+headq_status headq_decode_attn_noalloc(const headq_cache *cache, const void *q,
+                                       headq_dtype q_dtype, int Hq,
+                                       const int32_t *seq_lens, int T, const float *U,
+                                       float sm_scale, int corr_sign, float *out,
+                                       float *lse, headq_stream_t stream);
+
+/*
  * headq_attn_kl -- model-visible distortion of the cache against the
  * full-precision keys and values (summary section 2.1: score perturbation
  * delta_j = s^_j - s_j, attention KL and its local Fisher form; section 2.2:
