@@ -216,18 +216,23 @@ __global__ void decode_combine_kernel(const DecodeParams p) {
 }
 
 template <int D>
-cudaError_t launch_d(const DecodeParams& p, cudaStream_t s) {
-  const int G = p.G, r = p.c.r;
-  const size_t smem = sizeof(float) * (static_cast<size_t>(G) * D + G * num_groups(D) +
-                                       G * r + G * kTile + 3 * G);
-  auto k = decode_split_kernel<D>;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+cudaError_t launch_d(const DecodeParams& p, bool mma, cudaStream_t s) {
+  if (mma) {
+    const cudaError_t e = launch_decode_mma(p, s);
     if (e != cudaSuccess) return e;
+  } else {
+    const int G = p.G, r = p.c.r;
+    const size_t smem = sizeof(float) * (static_cast<size_t>(G) * D + G * num_groups(D) +
+                                         G * r + G * kTile + 3 * G);
+    auto k = decode_split_kernel<D>;
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+    }
+    dim3 grid(p.splits, p.c.Hkv, p.c.B);
+    k<<<grid, kThreads, smem, s>>>(p);
   }
-  dim3 grid(p.splits, p.c.Hkv, p.c.B);
-  k<<<grid, kThreads, smem, s>>>(p);
   if (p.splits > 1) {
     decode_combine_kernel<D><<<p.c.B * p.Hq, D < 32 ? 32 : (D > 128 ? 128 : D), 0, s>>>(p);
   }
@@ -236,14 +241,39 @@ cudaError_t launch_d(const DecodeParams& p, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s) {
+DecodePlan decode_plan(const headq_cache& c, int Hq, int T) {
+  DecodePlan dp{1, 64, 1, false};
+  const int G = c.Hkv > 0 ? Hq / c.Hkv : 0;
+  const int units = c.B * c.Hkv;
+  if (T <= 0 || units <= 0) return dp;
+  const int occ = mma_decode_supported(c, G) ? mma_decode_ctas_per_sm(c, G) : 0;
+  if (occ > 0) {
+    // one wave: every CTA resident, each streaming one contiguous chunk
+    int s = (occ * sm_count()) / units;
+    const int max_s = (T + 63) / 64;
+    s = s < 1 ? 1 : (s > max_s ? max_s : s);
+    int chunk = (T + s - 1) / s;
+    chunk = (chunk + 63) / 64 * 64;
+    dp.chunk = chunk;
+    dp.splits = (T + chunk - 1) / chunk;
+    dp.mma = true;
+  } else {
+    const SplitPlan sp = plan_splits(units, T, 256);
+    dp.splits = sp.splits;
+    dp.chunk = sp.chunk;
+  }
+  dp.kernels = dp.splits > 1 ? 2 : 1;
+  return dp;
+}
+
+cudaError_t launch_decode(const DecodeParams& p, bool mma, cudaStream_t s) {
   switch (p.c.d) {
-    case 8: return launch_d<8>(p, s);
-    case 16: return launch_d<16>(p, s);
-    case 32: return launch_d<32>(p, s);
-    case 64: return launch_d<64>(p, s);
-    case 128: return launch_d<128>(p, s);
-    case 256: return launch_d<256>(p, s);
+    case 8: return launch_d<8>(p, false, s);
+    case 16: return launch_d<16>(p, false, s);
+    case 32: return launch_d<32>(p, false, s);
+    case 64: return launch_d<64>(p, mma, s);
+    case 128: return launch_d<128>(p, mma, s);
+    case 256: return launch_d<256>(p, false, s);
     default: return cudaErrorInvalidValue;
   }
 }

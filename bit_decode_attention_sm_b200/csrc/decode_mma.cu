@@ -1,0 +1,662 @@
+// HeadQ decode attention, bandwidth kernel for sm_100a ("HeadQ: Model-Visible
+// Distortion and Score-Space Correction for KV-Cache Quantization", gist.science
+// summary, section 3, step 3: the runtime query turns the side code into an
+// additive logit correction; the readout is the attention-weighted sum of values).
+//
+// Same mathematics as decode_attn.cu's generic kernel; this one is built to stream
+// the packed cache at HBM speed:
+//
+//  * TMA pipeline.  One producer warp fills kStages shared-memory stages of 64
+//    tokens with 1-D bulk copies of the contiguous code / scale / side planes and
+//    a 3-D tensor copy (128-byte swizzle) of the bf16 value tile; four consumer
+//    warps each take 16 tokens of every stage.  mbarriers carry completion; every
+//    wait is bounded and flags the workspace error word on expiry.
+//  * q . code on tensor cores.  mma.m16n8k16 (fp16 in, fp32 accumulate) with the
+//    16 tokens of a warp on M and the query heads on N, each head's query split
+//    into an fp16 high and low part in adjacent columns (so 4 heads fill N = 8 and
+//    high + low add up inside one thread).  2-bit codes are exact small integers:
+//    0x6400 | (code << 2k) is the fp16 value 1024 + code*4^k, and one exact fp16
+//    FMA turns it back into the code.  Channels map to MMA k-slots so that each
+//    thread's codes are one 16-bit word per 32-channel group, and each group keeps
+//    its own accumulator, so the per-group scale and minimum are applied exactly as
+//    the dequantisation min + code*scale defines them:
+//        q.k^base_j = sum_g ( min_{j,g} Q_g + scale_{j,g} sum_{c in g} q_c code_{j,c} ).
+//    The side-code correction is one more MMA on the unpacked signed nibbles
+//    against sigma * U_h^T q (also split high / low), scaled by the side scale.
+//  * softmax in the log2 domain with a lazily refreshed running max (the output is
+//    rescaled only when the max grows by more than 2^8), per warp.
+//  * p . V on tensor cores.  mma.m16n8k16 (bf16) with the value dims on M (A = V^T
+//    fed by ldmatrix.trans from the swizzled tile) and the heads on N, p split into
+//    bf16 high and low parts in adjacent columns; the probabilities move from the
+//    logit layout to the B-operand layout with four warp shuffles.
+//  * the four warps' (max, sum, output) are merged through shared memory at the
+//    end; splits are merged by the common log-sum-exp combine kernel.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "headq_internal.cuh"
+
+namespace headq {
+namespace {
+
+constexpr int kCW = 4;                   // consumer warps
+constexpr int kTile = 16 * kCW;          // tokens per stage
+constexpr int kThreads = (kCW + 1) * 32; // + one producer warp
+constexpr int kStages = 4;
+constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at B200 clocks
+constexpr unsigned kFull = 0xffffffffu;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescale = 8.0f;         // log2 units the stale max may lag
+
+template <int D, int R>
+struct Layout {
+  static constexpr int NG = D / 32;
+  static constexpr int kVBoxes = D / 64;             // 64-dim boxes per token row
+  static constexpr int kVBox = kTile * 128;          // 64 tokens x 128 bytes
+  static constexpr int kKc = kVBoxes * kVBox;
+  static constexpr int kKs = kKc + kTile * (D / 4);
+  static constexpr int kKm = kKs + kTile * NG * 4;
+  static constexpr int kZc = kKm + kTile * NG * 4;
+  static constexpr int kZs = kZc + kTile * (R / 2);
+  static constexpr int kEnd = kZs + (R > 0 ? kTile * 4 : 0);
+  static constexpr int kStage = (kEnd + 1023) / 1024 * 1024;
+  static constexpr int kRowBytes = D / 4 + 8 * NG + (R > 0 ? R / 2 + 4 : 0);
+};
+
+template <int D, int R, int NT>
+constexpr size_t smem_bytes() {
+  using L = Layout<D, R>;
+  return 1024 + size_t(kStages) * L::kStage +
+         sizeof(float) * (4 * NT) * (D + L::NG + (R > 0 ? R : 1)) + 16 * kStages + 16;
+}
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase of the given parity to complete; false after ~2 s.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long start = clock64();
+  for (;;) {
+    for (int k = 0; k < 32; ++k)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - start > kWaitCycles) return false;
+  }
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                       uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4],
+                                        const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
+      " {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4],
+                                         const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
+      " {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// ---------------------------------------------------------------- unpacking
+// y holds one 16-bit word of eight 2-bit codes c0..c7 (code k at bits 2k) in both
+// halves.  Returns fp16 pairs (c0,c1) (c2,c3) (c4,c5) (c6,c7), exactly.
+__device__ __forceinline__ void unpack_codes(uint32_t y, uint32_t (&v)[4]) {
+  const uint32_t z = y >> 8;
+  // (1024 + c, 1024 + 4c') * (1, 1/4) - (1024, 256)
+  v[0] = hfma2((y & 0x000C0003u) | 0x64006400u, 0x34003C00u, 0xDC00E400u);
+  // (1024 + 16c, 1024 + 64c') * (1/16, 1/64) - (64, 16)
+  v[1] = hfma2((y & 0x00C00030u) | 0x64006400u, 0x24002C00u, 0xCC00D400u);
+  v[2] = hfma2((z & 0x000C0003u) | 0x64006400u, 0x34003C00u, 0xDC00E400u);
+  v[3] = hfma2((z & 0x00C00030u) | 0x64006400u, 0x24002C00u, 0xCC00D400u);
+}
+// y holds one 16-bit word of four offset nibbles (w + 8, nibble k at bits 4k) in
+// both halves.  Returns fp16 pairs (w0,w1) (w2,w3), exactly.
+__device__ __forceinline__ void unpack_side(uint32_t y, uint32_t& n01, uint32_t& n23) {
+  const uint32_t z = y >> 8;
+  // (1024 + n, 1024 + 16n') * (1, 1/16) - (1032, 72)
+  n01 = hfma2((y & 0x00F0000Fu) | 0x64006400u, 0x2C003C00u, 0xD480E408u);
+  n23 = hfma2((z & 0x00F0000Fu) | 0x64006400u, 0x2C003C00u, 0xD480E408u);
+}
+__device__ __forceinline__ uint32_t half_part_pair(float a, float b, bool lo) {
+  __half ha = __float2half_rn(a), hb = __float2half_rn(b);
+  if (lo) {
+    ha = __float2half_rn(a - __half2float(ha));
+    hb = __float2half_rn(b - __half2float(hb));
+  }
+  return static_cast<uint32_t>(__half_as_ushort(ha)) |
+         (static_cast<uint32_t>(__half_as_ushort(hb)) << 16);
+}
+__device__ __forceinline__ uint32_t bf16_part_pair(float a, float b, bool lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 f = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - f.x, b - f.y);
+  const __nv_bfloat162 r = lo ? l : h;
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// ---------------------------------------------------------------- the kernel
+template <int D, int R, int NT>
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
+decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap) {
+  using L = Layout<D, R>;
+  constexpr int NG = L::NG;
+  constexpr int KS = D / 16;   // k-steps of 16 channels
+  constexpr int MT = D / 16;   // 16-dim row blocks of the output
+  constexpr int GM = 4 * NT;   // head slots
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  float* q_s = reinterpret_cast<float*>(smem + size_t(kStages) * L::kStage);  // [GM][D]
+  float* qsum_s = q_s + GM * D;                                               // [GM][NG]
+  float* qt_s = qsum_s + GM * NG;                                             // [GM][R]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(qt_s + GM * (R > 0 ? R : 1)) + 15) & ~uintptr_t(15));
+  // bars[s] = stage full, bars[kStages + s] = stage empty
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
+  const int G = p.G, Hkv = p.c.Hkv;
+  int Tb = p.T;
+  if (p.seq_lens) Tb = max(0, min(p.seq_lens[b], p.T));
+  const int t_begin = split * p.chunk;
+  const int t_end = min(Tb, t_begin + p.chunk);
+  const int ntiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
+  const size_t bk = static_cast<size_t>(b) * Hkv + kv;
+  const int h0 = kv * G;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_addr(&bars[s]), 1);
+      mbar_init(smem_addr(&bars[kStages + s]), kCW);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // query prep: q, group sums, sigma * U_h^T q
+  for (int i = tid; i < GM * D; i += kThreads)
+    q_s[i] = i < G * D ? load_elem(p.q, (static_cast<size_t>(b) * p.Hq + h0) * D + i, p.q_bf16)
+                       : 0.0f;
+  __syncthreads();
+  for (int i = tid; i < GM * NG; i += kThreads) {
+    const int h = i / NG, g = i - h * NG;
+    float acc = 0.0f;
+    for (int c = 0; c < 32; ++c) acc += q_s[h * D + g * 32 + c];
+    qsum_s[i] = acc;
+  }
+  if constexpr (R > 0) {
+    const float* U = p.U + static_cast<size_t>(kv) * D * R;
+    for (int i = tid; i < GM * R; i += kThreads) {
+      const int h = i / R, ii = i - h * R;
+      float acc = 0.0f;
+      for (int c = 0; c < D; ++c) acc = fmaf(U[c * R + ii], q_s[h * D + c], acc);
+      qt_s[i] = p.corr_sign * acc;
+    }
+  }
+  __syncthreads();
+
+  // ------------------------------------------------------------ producer warp
+  if (warp == kCW) {
+    if (lane == 0 && ntiles > 0) {
+      bool ok = true;
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % kStages, use = i / kStages;
+        if (use > 0 && !mbar_wait(smem_addr(&bars[kStages + s]), (use - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        const int t0 = t_begin + i * kTile;
+        const int n16 = (min(kTile, t_end - t0) + 15) & ~15;
+        const uint32_t full = smem_addr(&bars[s]);
+        mbar_expect_tx(full, L::kVBoxes * L::kVBox + n16 * L::kRowBytes);
+        uint8_t* st = stages + size_t(s) * L::kStage;
+        const size_t row0 = bk * p.c.T_cap + t0;
+        bulk_g2s(smem_addr(st + L::kKc), p.c.k_codes + row0 * (D / 4), n16 * (D / 4), full);
+        bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + row0 * NG, n16 * NG * 4, full);
+        bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + row0 * NG, n16 * NG * 4, full);
+        if constexpr (R > 0) {
+          bulk_g2s(smem_addr(st + L::kZc), p.c.z_codes + row0 * (R / 2), n16 * (R / 2), full);
+          bulk_g2s(smem_addr(st + L::kZs), p.c.z_scale + row0, n16 * 4, full);
+        }
+#pragma unroll
+        for (int bx = 0; bx < L::kVBoxes; ++bx)
+          tma_3d(smem_addr(st + bx * L::kVBox), &vmap, bx * 64, t0, static_cast<int>(bk), full);
+        ++issued;
+      }
+      if (!ok && p.err) atomicOr(p.err, kDevErrWaitTimeout);
+      // never leave with copies in flight: wait (bounded) for the last use of each stage
+      for (int s = 0; s < kStages && s < issued; ++s) {
+        const int last_use = (issued - 1 - s) / kStages;
+        mbar_wait(smem_addr(&bars[s]), last_use & 1);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumer warps
+  const int g = lane >> 2, t = lane & 3;
+  const int jw = 16 * warp;
+
+  // B operands of q . code: column n = g is head (g >> 1), fp16 high (g even) or
+  // low (g odd) part; k-step ks = 2*grp + e, k-slots (2t, 2t+1) <-> channels
+  // 32*grp + 8t + 4e + {0, 1}, (2t+8, 2t+9) <-> 32*grp + 8t + 4e + {2, 3}.
+  uint32_t bq[KS][NT][2];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const int ch0 = 32 * (ks >> 1) + 8 * t + 4 * (ks & 1);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const float* qh = q_s + (4 * nt + (g >> 1)) * D + ch0;
+      bq[ks][nt][0] = half_part_pair(qh[0], qh[1], g & 1);
+      bq[ks][nt][1] = half_part_pair(qh[2], qh[3], g & 1);
+    }
+  }
+  uint32_t bz[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    bz[nt][0] = bz[nt][1] = 0;
+    if constexpr (R == 16) {
+      const float* z = qt_s + (4 * nt + (g >> 1)) * R + 4 * t;
+      bz[nt][0] = half_part_pair(z[0], z[1], g & 1);
+      bz[nt][1] = half_part_pair(z[2], z[3], g & 1);
+    } else if constexpr (R == 8) {
+      const float* z = qt_s + (4 * nt + (g >> 1)) * R + 2 * t;
+      bz[nt][0] = half_part_pair(z[0], z[1], g & 1);
+    }
+  }
+  // group sums of this thread's output head (4*nt + t)
+  float qsum[NT][NG];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int gg = 0; gg < NG; ++gg) qsum[nt][gg] = qsum_s[(4 * nt + t) * NG + gg];
+
+  const uint32_t sel = (2 * t) | ((2 * t + 1) << 4) | ((2 * t) << 8) | ((2 * t + 1) << 12);
+  const uint32_t sel8 = t | (4 << 4) | (t << 8) | (4 << 12);
+  const float scale2 = p.sm_scale * kLog2e;
+  // ldmatrix row owned by this lane: matrix (lane >> 3), row (lane & 7)
+  const int lm_tok = jw + 8 * (lane >> 4) + (lane & 7);
+  const int lm_chunk_hi = (lane >> 3) & 1;
+
+  float m2[NT], l[NT];
+  float o[MT][NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    m2[nt] = -INFINITY;
+    l[nt] = 0.0f;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+  }
+
+  bool ok = true;
+  for (int i = 0; i < ntiles; ++i) {
+    const int s = i % kStages;
+    if (!mbar_wait(smem_addr(&bars[s]), (i / kStages) & 1)) {
+      ok = false;
+      break;
+    }
+    uint8_t* st = stages + size_t(s) * L::kStage;
+    const int t0 = t_begin + i * kTile;
+    const int nvalid = min(kTile, t_end - t0);
+    const int j0 = jw + g, j1 = j0 + 8;
+    const bool val0 = j0 < nvalid, val1 = j1 < nvalid;
+
+    if (nvalid < jw + 16) {  // tail of the split: clear value rows past the end
+      for (int idx = lane; idx < 16 * 8 * L::kVBoxes; idx += 32) {
+        const int bx = idx % L::kVBoxes, rem = idx / L::kVBoxes;
+        const int row = jw + rem / 8, c16 = rem % 8;
+        if (row >= nvalid)
+          *reinterpret_cast<uint4*>(st + bx * L::kVBox + row * 128 + c16 * 16) =
+              make_uint4(0, 0, 0, 0);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+    }
+
+    // ---- q . code and the side-code correction on tensor cores
+    float acc[NG + (R > 0 ? 1 : 0)][NT][4];
+#pragma unroll
+    for (int a = 0; a < NG + (R > 0 ? 1 : 0); ++a)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) acc[a][nt][0] = acc[a][nt][1] = acc[a][nt][2] = acc[a][nt][3] = 0.f;
+
+    uint32_t cw0[D / 16], cw1[D / 16];
+#pragma unroll
+    for (int v4 = 0; v4 < D / 64; ++v4) {
+      const uint4 a = *reinterpret_cast<const uint4*>(st + L::kKc + j0 * (D / 4) + 16 * v4);
+      const uint4 c = *reinterpret_cast<const uint4*>(st + L::kKc + j1 * (D / 4) + 16 * v4);
+      cw0[4 * v4 + 0] = a.x; cw0[4 * v4 + 1] = a.y; cw0[4 * v4 + 2] = a.z; cw0[4 * v4 + 3] = a.w;
+      cw1[4 * v4 + 0] = c.x; cw1[4 * v4 + 1] = c.y; cw1[4 * v4 + 2] = c.z; cw1[4 * v4 + 3] = c.w;
+    }
+#pragma unroll
+    for (int gg = 0; gg < NG; ++gg) {
+      uint32_t u0[4], u1[4];
+      unpack_codes(__byte_perm(cw0[2 * gg], cw0[2 * gg + 1], sel), u0);
+      unpack_codes(__byte_perm(cw1[2 * gg], cw1[2 * gg + 1], sel), u1);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const uint32_t a[4] = {u0[2 * e], u1[2 * e], u0[2 * e + 1], u1[2 * e + 1]};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_f16(acc[gg][nt], a, bq[2 * gg + e][nt]);
+      }
+    }
+    float zs0 = 0.f, zs1 = 0.f;
+    if constexpr (R > 0) {
+      uint32_t a[4];
+      if constexpr (R == 16) {
+        const uint2 z0 = *reinterpret_cast<const uint2*>(st + L::kZc + j0 * 8);
+        const uint2 z1 = *reinterpret_cast<const uint2*>(st + L::kZc + j1 * 8);
+        unpack_side(__byte_perm(z0.x, z0.y, sel) ^ 0x88888888u, a[0], a[2]);
+        unpack_side(__byte_perm(z1.x, z1.y, sel) ^ 0x88888888u, a[1], a[3]);
+      } else {
+        const uint32_t z0 = *reinterpret_cast<const uint32_t*>(st + L::kZc + j0 * 4);
+        const uint32_t z1 = *reinterpret_cast<const uint32_t*>(st + L::kZc + j1 * 4);
+        uint32_t dummy;
+        unpack_side(__byte_perm(z0, 0u, sel8) ^ 0x00880088u, a[0], dummy);
+        unpack_side(__byte_perm(z1, 0u, sel8) ^ 0x00880088u, a[1], dummy);
+        a[2] = a[3] = 0u;
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_f16(acc[NG][nt], a, bz[nt]);
+      zs0 = reinterpret_cast<const float*>(st + L::kZs)[j0];
+      zs1 = reinterpret_cast<const float*>(st + L::kZs)[j1];
+    }
+    float ks0[NG], km0[NG], ks1[NG], km1[NG];
+#pragma unroll
+    for (int gg = 0; gg < NG; ++gg) {
+      ks0[gg] = reinterpret_cast<const float*>(st + L::kKs)[j0 * NG + gg];
+      km0[gg] = reinterpret_cast<const float*>(st + L::kKm)[j0 * NG + gg];
+      ks1[gg] = reinterpret_cast<const float*>(st + L::kKs)[j1 * NG + gg];
+      km1[gg] = reinterpret_cast<const float*>(st + L::kKm)[j1 * NG + gg];
+    }
+
+    // ---- logits, online softmax, p in the B-operand layout
+    uint32_t bp[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int gg = 0; gg < NG; ++gg) {
+        s0 = fmaf(ks0[gg], acc[gg][nt][0] + acc[gg][nt][1], s0);
+        s0 = fmaf(km0[gg], qsum[nt][gg], s0);
+        s1 = fmaf(ks1[gg], acc[gg][nt][2] + acc[gg][nt][3], s1);
+        s1 = fmaf(km1[gg], qsum[nt][gg], s1);
+      }
+      if constexpr (R > 0) {
+        s0 = fmaf(zs0, acc[NG][nt][0] + acc[NG][nt][1], s0);
+        s1 = fmaf(zs1, acc[NG][nt][2] + acc[NG][nt][3], s1);
+      }
+      const float x0 = val0 ? s0 * scale2 : -INFINITY;
+      const float x1 = val1 ? s1 * scale2 : -INFINITY;
+      float mx = fmaxf(x0, x1);
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+      const float mnew = fmaxf(m2[nt], mx);
+      const bool resc = mnew > m2[nt] + kRescale;
+      if (__any_sync(kFull, resc)) {
+        const float alpha = resc ? exp2f(m2[nt] - mnew) : 1.0f;
+        if (resc) m2[nt] = mnew;
+        l[nt] *= alpha;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          o[mt][nt][0] *= alpha; o[mt][nt][1] *= alpha;
+          o[mt][nt][2] *= alpha; o[mt][nt][3] *= alpha;
+        }
+      }
+      const float p0 = x0 == -INFINITY ? 0.f : exp2f(x0 - m2[nt]);
+      const float p1 = x1 == -INFINITY ? 0.f : exp2f(x1 - m2[nt]);
+      l[nt] += p0 + p1;
+      // B operand of p . V: (tokens 2t, 2t+1 | 2t+8, 2t+9) x column g
+      const int sa = 8 * t + (g >> 1), sb = sa + 4;
+      const float va = __shfl_sync(kFull, p0, sa), vb = __shfl_sync(kFull, p0, sb);
+      const float vc = __shfl_sync(kFull, p1, sa), vd = __shfl_sync(kFull, p1, sb);
+      bp[nt][0] = bf16_part_pair(va, vb, g & 1);
+      bp[nt][1] = bf16_part_pair(vc, vd, g & 1);
+    }
+
+    // ---- p . V on tensor cores (A = V^T from the swizzled tile)
+    const uint32_t vbase = smem_addr(st);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int chunk = 2 * mt + lm_chunk_hi;
+      const uint32_t addr = vbase + (chunk >> 3) * L::kVBox + lm_tok * 128 +
+                            (((chunk & 7) ^ (lm_tok & 7)) << 4);
+      uint32_t a[4];
+      ldsm_x4_trans(addr, a);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_bf16(o[mt][nt], a, bp[nt]);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&bars[kStages + s]));
+  }
+  if (!ok && lane == 0 && p.err) atomicOr(p.err, kDevErrWaitTimeout);
+
+  // ---- merge the consumer warps' partial softmax states
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    l[nt] += __shfl_xor_sync(kFull, l[nt], 4);
+    l[nt] += __shfl_xor_sync(kFull, l[nt], 8);
+    l[nt] += __shfl_xor_sync(kFull, l[nt], 16);
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+  float* mo = reinterpret_cast<float*>(stages);  // [kCW][GM][D]
+  float* mm = mo + kCW * GM * D;                 // [kCW][GM]
+  float* ml = mm + kCW * GM;                     // [kCW][GM]
+  int* bad = reinterpret_cast<int*>(ml + kCW * GM);
+  if (tid == 0) *bad = 0;
+  asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+  if (!ok) *bad = 1;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int h = 4 * nt + t;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      mo[(warp * GM + h) * D + 16 * mt + g] = o[mt][nt][0] + o[mt][nt][1];
+      mo[(warp * GM + h) * D + 16 * mt + g + 8] = o[mt][nt][2] + o[mt][nt][3];
+    }
+    if (g == 0) {
+      mm[warp * GM + h] = m2[nt];
+      ml[warp * GM + h] = l[nt];
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+  if (*bad) return;
+  for (int idx = tid; idx < G * D; idx += kCW * 32) {
+    const int h = idx / D, c = idx - h * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCW; ++w) M = fmaxf(M, mm[w * GM + h]);
+    float O = 0.f, Ls = 0.f;
+    if (M > -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kCW; ++w) {
+        const float f = exp2f(mm[w * GM + h] - M);
+        O = fmaf(f, mo[(w * GM + h) * D + c], O);
+        Ls = fmaf(f, ml[w * GM + h], Ls);
+      }
+    }
+    const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
+    if (p.splits == 1) {
+      p.out[bh * D + c] = Ls > 0.f ? O / Ls : 0.f;
+      if (c == 0 && p.lse) p.lse[bh] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
+    } else {
+      float* pt = p.part + (bh * p.splits + split) * (D + 2);
+      pt[c] = O;
+      if (c == 0) {
+        pt[D] = Ls > 0.f ? M * kLn2 : -INFINITY;
+        pt[D + 1] = Ls;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(f);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+constexpr int kMaxDev = 64;
+
+template <int D, int R, int NT>
+struct Variant {
+  static int occupancy[kMaxDev];  // CTAs per SM, 0 = not yet known
+  static std::mutex mu;
+
+  // Once per device: raise the dynamic shared memory limit and ask the
+  // occupancy calculator how many CTAs fit on one SM.
+  static int ctas_per_sm() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+      cudaGetLastError();
+      return 0;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (occupancy[dev] == 0) {
+      auto k = decode_mma_kernel<D, R, NT>;
+      const int smem = static_cast<int>(smem_bytes<D, R, NT>());
+      int n = 0;
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+              cudaSuccess ||
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kThreads, smem) != cudaSuccess) {
+        cudaGetLastError();
+        n = -1;
+      }
+      occupancy[dev] = n > 0 ? n : -1;
+    }
+    return occupancy[dev] > 0 ? occupancy[dev] : 0;
+  }
+
+  static cudaError_t launch(const DecodeParams& p, cudaStream_t s) {
+    if (ctas_per_sm() == 0) return cudaErrorInvalidConfiguration;
+    EncodeTiled enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    CUtensorMap vmap;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(p.c.T_cap),
+                                static_cast<cuuint64_t>(p.c.B) * p.c.Hkv};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                   static_cast<cuuint64_t>(p.c.T_cap) * D * 2};
+    const cuuint32_t box[3] = {64, kTile, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&vmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.c.v, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    dim3 grid(p.splits, p.c.Hkv, p.c.B);
+    decode_mma_kernel<D, R, NT><<<grid, kThreads, smem_bytes<D, R, NT>(), s>>>(p, vmap);
+    return cudaGetLastError();
+  }
+};
+template <int D, int R, int NT>
+int Variant<D, R, NT>::occupancy[kMaxDev];
+template <int D, int R, int NT>
+std::mutex Variant<D, R, NT>::mu;
+
+template <typename F>
+auto dispatch(int d, int r, int G, F&& f) -> decltype(f(Variant<128, 16, 1>{})) {
+  const int nt = G <= 4 ? 1 : 2;
+#define HEADQ_MMA_CASE(DD, RR, NN) \
+  if (d == DD && r == RR && nt == NN) return f(Variant<DD, RR, NN>{});
+  HEADQ_MMA_CASE(128, 16, 1) HEADQ_MMA_CASE(128, 16, 2)
+  HEADQ_MMA_CASE(128, 8, 1) HEADQ_MMA_CASE(128, 8, 2)
+  HEADQ_MMA_CASE(128, 0, 1) HEADQ_MMA_CASE(128, 0, 2)
+  HEADQ_MMA_CASE(64, 16, 1) HEADQ_MMA_CASE(64, 16, 2)
+  HEADQ_MMA_CASE(64, 8, 1) HEADQ_MMA_CASE(64, 8, 2)
+  HEADQ_MMA_CASE(64, 0, 1) HEADQ_MMA_CASE(64, 0, 2)
+#undef HEADQ_MMA_CASE
+  return decltype(f(Variant<128, 16, 1>{}))();
+}
+
+}  // namespace
+
+bool mma_decode_supported(const headq_cache& c, int G) {
+  return c.vmode == HEADQ_V_DENSE && c.v_dtype == HEADQ_BF16 && (c.d == 64 || c.d == 128) &&
+         (c.r == 0 || c.r == 8 || c.r == 16) && G >= 1 && G <= 8 && encode_fn() != nullptr;
+}
+
+int mma_decode_ctas_per_sm(const headq_cache& c, int G) {
+  return dispatch(c.d, c.r, G, [](auto v) { return decltype(v)::ctas_per_sm(); });
+}
+
+cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s) {
+  // 0 means no variant matched; otherwise the launch status + 1
+  const int e = dispatch(p.c.d, p.c.r, p.G, [&](auto v) {
+    return static_cast<int>(decltype(v)::launch(p, s)) + 1;
+  });
+  return e == 0 ? cudaErrorInvalidValue : static_cast<cudaError_t>(e - 1);
+}
+
+}  // namespace headq

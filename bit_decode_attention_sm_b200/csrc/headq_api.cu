@@ -17,7 +17,7 @@ static bool supported_d(int d) {
   return d == 8 || d == 16 || d == 32 || d == 64 || d == 128 || d == 256;
 }
 
-static int sm_count() {
+int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
@@ -87,9 +87,9 @@ static headq_status check_read_args(const headq_cache* c, const void* q, headq_d
 static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 static size_t decode_ws(const headq_cache* c, int Hq, int T) {
-  const SplitPlan sp = plan_splits(c->B * c->Hkv, T, 256);
+  const DecodePlan dp = decode_plan(*c, Hq, T);
   return kWsHeaderBytes +
-         round256(sizeof(float) * static_cast<size_t>(c->B) * Hq * sp.splits * (c->d + 2));
+         round256(sizeof(float) * static_cast<size_t>(c->B) * Hq * dp.splits * (c->d + 2));
 }
 
 static size_t kl_ws(const headq_cache* c, int Hq, int T) {
@@ -185,10 +185,10 @@ HEADQ_API int headq_decode_plan(const headq_cache* cache, int Hq, int T, int* sp
                                 int* chunk) {
   if (!cache || cache->B < 0 || cache->Hkv <= 0 || Hq <= 0 || T < 0 || !supported_d(cache->d))
     return 0;
-  const SplitPlan sp = plan_splits(cache->B * cache->Hkv, T, 256);
-  if (splits) *splits = sp.splits;
-  if (chunk) *chunk = sp.chunk;
-  return sp.splits > 1 ? 2 : 1;
+  const DecodePlan dp = decode_plan(*cache, Hq, T);
+  if (splits) *splits = dp.splits;
+  if (chunk) *chunk = dp.chunk;
+  return dp.kernels;
 }
 
 HEADQ_API headq_status headq_decode_attn(const headq_cache* cache, const void* q,
@@ -203,7 +203,7 @@ HEADQ_API headq_status headq_decode_attn(const headq_cache* cache, const void* q
   if (seq_lens && !aligned16(seq_lens)) return HEADQ_ERR_INVALID_ARG;
   if (!ws || !aligned16(ws) || ws_bytes < decode_ws(cache, Hq, T)) return HEADQ_ERR_WORKSPACE;
   if (cache->B == 0) return HEADQ_OK;
-  const SplitPlan sp = plan_splits(cache->B * cache->Hkv, T, 256);
+  const DecodePlan sp = decode_plan(*cache, Hq, T);
   DecodeParams p{};
   p.c = *cache;
   p.q = q;
@@ -221,7 +221,7 @@ HEADQ_API headq_status headq_decode_attn(const headq_cache* cache, const void* q
   p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeaderBytes);
   p.out = out;
   p.lse = lse;
-  return launch_decode(p, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+  return launch_decode(p, sp.mma, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? HEADQ_OK
              : HEADQ_ERR_CUDA;
 }

@@ -95,7 +95,6 @@ struct CalibrateParams {
 };
 
 cudaError_t launch_cache_write(const CacheWriteParams& p, cudaStream_t s);
-cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_attn_kl(const AttnKlParams& p, cudaStream_t s);
 cudaError_t launch_calibrate(const CalibrateParams& p, cudaStream_t s);
 
@@ -104,5 +103,19 @@ struct SplitPlan {
   int splits, chunk;
 };
 SplitPlan plan_splits(int units, int T, int min_chunk);
+int sm_count();
+
+// The decode kernel and T-split plan chosen for these sizes on the current
+// device; the workspace query, headq_decode_plan and the launch all use it.
+struct DecodePlan {
+  int splits, chunk, kernels;
+  bool mma;  // tensor-core TMA kernel (decode_mma.cu) instead of the generic one
+};
+DecodePlan decode_plan(const headq_cache& c, int Hq, int T);
+cudaError_t launch_decode(const DecodeParams& p, bool mma, cudaStream_t s);
+
+bool mma_decode_supported(const headq_cache& c, int G);
+int mma_decode_ctas_per_sm(const headq_cache& c, int G);
+cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s);
 
 }  // namespace headq
