@@ -164,6 +164,7 @@ decode_split_kernel(const DecodeParams p) {
   }
 
   // epilogue: partial (o, m, l) or the final result
+  const PartView pv = part_view(p.part, static_cast<size_t>(p.c.B) * p.Hq, p.splits, D);
 #pragma unroll
   for (int k = 0; k < kMaxOut; ++k) {
     const int idx = tid + k * kThreads;
@@ -174,8 +175,7 @@ decode_split_kernel(const DecodeParams p) {
         const float l = l_s[h];
         p.out[bh * D + c] = l > 0.0f ? o[k] / l : 0.0f;
       } else {
-        float* pt = p.part + (bh * p.splits + split) * (D + 2);
-        pt[c] = o[k];
+        pv.o[(bh * p.splits + split) * D + c] = o[k];
       }
     }
   }
@@ -184,35 +184,61 @@ decode_split_kernel(const DecodeParams p) {
     if (p.splits == 1) {
       if (p.lse) p.lse[bh] = l_s[h] > 0.0f ? m_s[h] + logf(l_s[h]) : -INFINITY;
     } else {
-      float* pt = p.part + (bh * p.splits + split) * (D + 2);
-      pt[D] = m_s[h];
-      pt[D + 1] = l_s[h];
+      pv.m[bh * p.splits + split] = m_s[h];
+      pv.l[bh * p.splits + split] = l_s[h];
     }
   }
 }
 
-// Merge the T-splits of one (b, h): exact log-sum-exp combination.
+// Merge the T-splits of one (b, h): exact log-sum-exp combination.  Warp 0
+// forms the split weights e^{m_s - M} in shared memory; every thread then
+// streams one output column over the splits with independent loads in flight.
+constexpr int kCombineThreads = 128;
+constexpr int kCombineMaxSplits = 2048;
+
 template <int D>
-__global__ void decode_combine_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kCombineThreads)
+decode_combine_kernel(const DecodeParams p) {
+  __shared__ float w_s[kCombineMaxSplits];
+  __shared__ float ML[2];
   const size_t bh = blockIdx.x;
   const int S = p.splits;
-  const float* pb = p.part + bh * S * (D + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, pb[s * (D + 2) + D]);
-  float L = 0.0f;
-  for (int s = 0; s < S; ++s) {
-    const float m = pb[s * (D + 2) + D];
-    if (m > -INFINITY) L += expf(m - M) * pb[s * (D + 2) + D + 1];
-  }
-  for (int c = threadIdx.x; c < D; c += blockDim.x) {
-    float acc = 0.0f;
-    for (int s = 0; s < S; ++s) {
-      const float m = pb[s * (D + 2) + D];
-      if (m > -INFINITY) acc += expf(m - M) * pb[s * (D + 2) + c];
+  const PartView pv = part_view(p.part, static_cast<size_t>(p.c.B) * p.Hq, S, D);
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    float M = -INFINITY;
+    for (int s = lane; s < S; s += 32) M = fmaxf(M, pv.m[bh * S + s]);
+    M = warp_max(M);
+    float L = 0.0f;
+    for (int s = lane; s < S; s += 32) {
+      const float m = pv.m[bh * S + s];
+      const float w = m > -INFINITY ? expf(m - M) : 0.0f;
+      w_s[s] = w;
+      L = fmaf(w, pv.l[bh * S + s], L);
     }
+    L = warp_sum(L);
+    if (lane == 0) {
+      ML[0] = M;
+      ML[1] = L;
+    }
+  }
+  __syncthreads();
+  const float L = ML[1];
+  for (int c = threadIdx.x; c < D; c += kCombineThreads) {
+    const float* po = pv.o + bh * S * D + c;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int s = 0;
+    for (; s + 4 <= S; s += 4) {
+      a0 = fmaf(w_s[s], po[(s + 0) * D], a0);
+      a1 = fmaf(w_s[s + 1], po[(s + 1) * D], a1);
+      a2 = fmaf(w_s[s + 2], po[(s + 2) * D], a2);
+      a3 = fmaf(w_s[s + 3], po[(s + 3) * D], a3);
+    }
+    for (; s < S; ++s) a0 = fmaf(w_s[s], po[s * D], a0);
+    const float acc = (a0 + a1) + (a2 + a3);
     p.out[bh * D + c] = L > 0.0f ? acc / L : 0.0f;
   }
-  if (threadIdx.x == 0 && p.lse) p.lse[bh] = L > 0.0f ? M + logf(L) : -INFINITY;
+  if (threadIdx.x == 0 && p.lse) p.lse[bh] = L > 0.0f ? ML[0] + logf(L) : -INFINITY;
 }
 
 template <int D>
@@ -233,8 +259,9 @@ cudaError_t launch_d(const DecodeParams& p, bool mma, cudaStream_t s) {
     dim3 grid(p.splits, p.c.Hkv, p.c.B);
     k<<<grid, kThreads, smem, s>>>(p);
   }
-  if (p.splits > 1) {
-    decode_combine_kernel<D><<<p.c.B * p.Hq, D < 32 ? 32 : (D > 128 ? 128 : D), 0, s>>>(p);
+  if (p.splits > 1 && !(mma && p.fused)) {  // unless the split kernel merged its splits
+    if (p.splits > kCombineMaxSplits) return cudaErrorInvalidConfiguration;
+    decode_combine_kernel<D><<<p.c.B * p.Hq, kCombineThreads, 0, s>>>(p);
   }
   return cudaGetLastError();
 }
@@ -242,27 +269,32 @@ cudaError_t launch_d(const DecodeParams& p, bool mma, cudaStream_t s) {
 }  // namespace
 
 DecodePlan decode_plan(const headq_cache& c, int Hq, int T) {
-  DecodePlan dp{1, 64, 1, false};
+  DecodePlan dp{1, 64, 1, false, false};
   const int G = c.Hkv > 0 ? Hq / c.Hkv : 0;
   const int units = c.B * c.Hkv;
   if (T <= 0 || units <= 0) return dp;
   const int occ = mma_decode_supported(c, G) ? mma_decode_ctas_per_sm(c, G) : 0;
   if (occ > 0) {
-    // one wave: every CTA resident, each streaming one contiguous chunk
+    // one wave: every CTA resident, each streaming one contiguous chunk of a
+    // multiple of 16 tokens (so every bulk copy stays 16-byte aligned); the last
+    // CTA of each (b, kv) merges the splits, so one kernel per call
     int s = (occ * sm_count()) / units;
     const int max_s = (T + 63) / 64;
     s = s < 1 ? 1 : (s > max_s ? max_s : s);
+    if (s > kMaxMmaSplits) s = kMaxMmaSplits;
     int chunk = (T + s - 1) / s;
-    chunk = (chunk + 63) / 64 * 64;
+    chunk = (chunk + 15) / 16 * 16;
     dp.chunk = chunk;
     dp.splits = (T + chunk - 1) / chunk;
     dp.mma = true;
+    dp.fused = units <= kMaxFusedUnits;
+    dp.kernels = (dp.splits > 1 && !dp.fused) ? 2 : 1;
   } else {
     const SplitPlan sp = plan_splits(units, T, 256);
     dp.splits = sp.splits;
     dp.chunk = sp.chunk;
+    dp.kernels = dp.splits > 1 ? 2 : 1;
   }
-  dp.kernels = dp.splits > 1 ? 2 : 1;
   return dp;
 }
 

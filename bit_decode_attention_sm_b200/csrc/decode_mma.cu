@@ -71,8 +71,10 @@ struct Layout {
 template <int D, int R, int NT>
 constexpr size_t smem_bytes() {
   using L = Layout<D, R>;
+  // stages | q [GM][D] | group sums [GM][NG] | sigma U^T q [GM][R] | U [D][R] | barriers
   return 1024 + size_t(kStages) * L::kStage +
-         sizeof(float) * (4 * NT) * (D + L::NG + (R > 0 ? R : 1)) + 16 * kStages + 16;
+         sizeof(float) * ((4 * NT) * (D + L::NG + (R > 0 ? R : 1)) + D * (R > 0 ? R : 1)) +
+         16 * kStages + 16;
 }
 
 // ---------------------------------------------------------------- PTX helpers
@@ -198,6 +200,8 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   constexpr int KS = D / 16;   // k-steps of 16 channels
   constexpr int MT = D / 16;   // 16-dim row blocks of the output
   constexpr int GM = 4 * NT;   // head slots
+  constexpr int RR = R > 0 ? R : 1;
+  constexpr int kCT = kCW * 32;  // consumer threads
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -205,9 +209,10 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   uint8_t* stages = smem;
   float* q_s = reinterpret_cast<float*>(smem + size_t(kStages) * L::kStage);  // [GM][D]
   float* qsum_s = q_s + GM * D;                                               // [GM][NG]
-  float* qt_s = qsum_s + GM * NG;                                             // [GM][R]
+  float* qt_s = qsum_s + GM * NG;                                             // [GM][RR]
+  float* u_s = qt_s + GM * RR;                                                // [D][RR]
   uint64_t* bars = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(qt_s + GM * (R > 0 ? R : 1)) + 15) & ~uintptr_t(15));
+      (reinterpret_cast<uintptr_t>(u_s + D * RR) + 15) & ~uintptr_t(15));
   // bars[s] = stage full, bars[kStages + s] = stage empty
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -228,29 +233,10 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // query prep: q, group sums, sigma * U_h^T q
-  for (int i = tid; i < GM * D; i += kThreads)
-    q_s[i] = i < G * D ? load_elem(p.q, (static_cast<size_t>(b) * p.Hq + h0) * D + i, p.q_bf16)
-                       : 0.0f;
-  __syncthreads();
-  for (int i = tid; i < GM * NG; i += kThreads) {
-    const int h = i / NG, g = i - h * NG;
-    float acc = 0.0f;
-    for (int c = 0; c < 32; ++c) acc += q_s[h * D + g * 32 + c];
-    qsum_s[i] = acc;
-  }
-  if constexpr (R > 0) {
-    const float* U = p.U + static_cast<size_t>(kv) * D * R;
-    for (int i = tid; i < GM * R; i += kThreads) {
-      const int h = i / R, ii = i - h * R;
-      float acc = 0.0f;
-      for (int c = 0; c < D; ++c) acc = fmaf(U[c * R + ii], q_s[h * D + c], acc);
-      qt_s[i] = p.corr_sign * acc;
-    }
-  }
   __syncthreads();
 
   // ------------------------------------------------------------ producer warp
+  // starts streaming at once; the consumers prepare the query meanwhile
   if (warp == kCW) {
     if (lane == 0 && ntiles > 0) {
       bool ok = true;
@@ -290,6 +276,32 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   }
 
   // ------------------------------------------------------------ consumer warps
+  // query prep: q, U_h, group sums, sigma * U_h^T q
+  for (int i = tid; i < GM * D; i += kCT)
+    q_s[i] = i < G * D ? load_elem(p.q, (static_cast<size_t>(b) * p.Hq + h0) * D + i, p.q_bf16)
+                       : 0.0f;
+  if constexpr (R > 0) {
+    const float4* U4 = reinterpret_cast<const float4*>(p.U + static_cast<size_t>(kv) * D * R);
+    for (int i = tid; i < D * R / 4; i += kCT) reinterpret_cast<float4*>(u_s)[i] = U4[i];
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
+  for (int i = tid; i < GM * NG; i += kCT) {
+    const int h = i / NG, g = i - h * NG;
+    float acc = 0.0f;
+    for (int c = 0; c < 32; ++c) acc += q_s[h * D + g * 32 + c];
+    qsum_s[i] = acc;
+  }
+  if constexpr (R > 0) {
+    for (int i = tid; i < GM * R; i += kCT) {
+      const int h = i / R, ii = i - h * R;
+      float acc = 0.0f;
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) acc = fmaf(u_s[c * R + ii], q_s[h * D + c], acc);
+      qt_s[i] = p.corr_sign * acc;
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
+
   const int g = lane >> 2, t = lane & 3;
   const int jw = 16 * warp;
 
@@ -495,14 +507,14 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     l[nt] += __shfl_xor_sync(kFull, l[nt], 8);
     l[nt] += __shfl_xor_sync(kFull, l[nt], 16);
   }
-  asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   float* mo = reinterpret_cast<float*>(stages);  // [kCW][GM][D]
   float* mm = mo + kCW * GM * D;                 // [kCW][GM]
   float* ml = mm + kCW * GM;                     // [kCW][GM]
-  int* bad = reinterpret_cast<int*>(ml + kCW * GM);
-  if (tid == 0) *bad = 0;
-  asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
-  if (!ok) *bad = 1;
+  int* flags = reinterpret_cast<int*>(ml + kCW * GM);  // [0] a warp failed, [1] last CTA
+  if (tid == 0) flags[0] = 0;
+  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
+  if (!ok) flags[0] = 1;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int h = 4 * nt + t;
@@ -516,9 +528,12 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       ml[warp * GM + h] = l[nt];
     }
   }
-  asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
-  if (*bad) return;
-  for (int idx = tid; idx < G * D; idx += kCW * 32) {
+  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
+  const bool failed = flags[0] != 0;
+  const bool single = p.splits == 1;
+  if (failed && single) return;
+  const PartView pv = part_view(p.part, static_cast<size_t>(p.c.B) * p.Hq, p.splits, D);
+  for (int idx = tid; idx < G * D; idx += kCT) {
     const int h = idx / D, c = idx - h * D;
     float M = -INFINITY;
 #pragma unroll
@@ -533,18 +548,85 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       }
     }
     const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
-    if (p.splits == 1) {
+    if (single) {
       p.out[bh * D + c] = Ls > 0.f ? O / Ls : 0.f;
       if (c == 0 && p.lse) p.lse[bh] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
-    } else {
-      float* pt = p.part + (bh * p.splits + split) * (D + 2);
-      pt[c] = O;
+    } else if (!failed) {
+      pv.o[(bh * p.splits + split) * D + c] = O;
       if (c == 0) {
-        pt[D] = Ls > 0.f ? M * kLn2 : -INFINITY;
-        pt[D + 1] = Ls;
+        pv.m[bh * p.splits + split] = Ls > 0.f ? M * kLn2 : -INFINITY;
+        pv.l[bh * p.splits + split] = Ls;
       }
     }
   }
+  if (single || !p.fused) return;  // unfused: the combine kernel merges the splits
+
+  // ---- split arrival; the last CTA of this (b, kv) merges all splits.  Every
+  // CTA arrives (also one that failed), so the counter always returns to zero.
+  __threadfence();
+  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
+  if (tid == 0) {
+    const unsigned old = atomicAdd(p.counters + bk, 1u);
+    flags[1] = old == static_cast<unsigned>(p.splits - 1);
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
+  if (!flags[1]) return;
+  __threadfence();
+  const int S = p.splits;
+  float* w_s = reinterpret_cast<float*>(flags + 4);  // [G][S] split weights, past the flags
+  float* M_s = w_s + GM * S;     // [G]
+  float* L_s = M_s + GM;         // [G]
+  for (int h = warp; h < G; h += kCW) {
+    const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
+    float mx = -INFINITY;
+    for (int s = lane; s < S; s += 32) mx = fmaxf(mx, __ldcg(pv.m + bh * S + s));
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o2));
+    float ls = 0.f;
+    for (int s = lane; s < S; s += 32) {
+      const float m = __ldcg(pv.m + bh * S + s);
+      const float w = m > -INFINITY ? expf(m - mx) : 0.f;
+      w_s[h * S + s] = w;
+      ls = fmaf(w, __ldcg(pv.l + bh * S + s), ls);
+    }
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) ls += __shfl_xor_sync(kFull, ls, o2);
+    if (lane == 0) {
+      M_s[h] = mx;
+      L_s[h] = ls;
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
+  // one thread per (head, 4 dims): independent 16-byte loads over the splits
+  for (int idx = tid; idx < G * (D / 4); idx += kCT) {
+    const int h = idx / (D / 4), c4 = idx - h * (D / 4);
+    const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
+    const float4* po = reinterpret_cast<const float4*>(pv.o + bh * S * D) + c4;
+    const float* w = w_s + h * S;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), e = a;
+    int s = 0;
+    for (; s + 2 <= S; s += 2) {
+      const float4 v0 = __ldcg(po + (s + 0) * (D / 4));
+      const float4 v1 = __ldcg(po + (s + 1) * (D / 4));
+      a.x = fmaf(w[s], v0.x, a.x); a.y = fmaf(w[s], v0.y, a.y);
+      a.z = fmaf(w[s], v0.z, a.z); a.w = fmaf(w[s], v0.w, a.w);
+      e.x = fmaf(w[s + 1], v1.x, e.x); e.y = fmaf(w[s + 1], v1.y, e.y);
+      e.z = fmaf(w[s + 1], v1.z, e.z); e.w = fmaf(w[s + 1], v1.w, e.w);
+    }
+    if (s < S) {
+      const float4 v0 = __ldcg(po + s * (D / 4));
+      a.x = fmaf(w[s], v0.x, a.x); a.y = fmaf(w[s], v0.y, a.y);
+      a.z = fmaf(w[s], v0.z, a.z); a.w = fmaf(w[s], v0.w, a.w);
+    }
+    const float Lh = L_s[h];
+    const float inv = Lh > 0.f ? 1.0f / Lh : 0.f;
+    float4 r;
+    r.x = (a.x + e.x) * inv; r.y = (a.y + e.y) * inv;
+    r.z = (a.z + e.z) * inv; r.w = (a.w + e.w) * inv;
+    reinterpret_cast<float4*>(p.out + bh * D)[c4] = r;
+    if (c4 == 0 && p.lse) p.lse[bh] = Lh > 0.f ? M_s[h] + logf(Lh) : -INFINITY;
+  }
+  if (tid == 0) p.counters[bk] = 0;  // ready for the next call
 }
 
 // ---------------------------------------------------------------- host side

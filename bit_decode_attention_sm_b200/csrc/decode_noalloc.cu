@@ -31,7 +31,8 @@ std::mutex g_setup_mu;
 void* g_scratch_addr[kMaxDevices];  // device address per device, set once
 
 // Once per device, with that device current: find the array's device address
-// and clear its header (the device error word must start at zero).  Synchronous.
+// and zero it (the device error word and the split arrival counters must start
+// at zero; every decode call leaves the counters at zero again).  Synchronous.
 cudaError_t scratch_for_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -42,7 +43,7 @@ cudaError_t scratch_for_current_device(void** out) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
     if (e != cudaSuccess) return e;
-    e = cudaMemset(ptr, 0, kWsHeaderBytes);
+    e = cudaMemset(ptr, 0, kNoAllocScratchBytes);
     if (e != cudaSuccess) return e;
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return e;

@@ -86,9 +86,10 @@ static headq_status check_read_args(const headq_cache* c, const void* q, headq_d
 
 static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
+// decode workspace: [error word header][fixed arrival-counter region][partials]
 static size_t decode_ws(const headq_cache* c, int Hq, int T) {
   const DecodePlan dp = decode_plan(*c, Hq, T);
-  return kWsHeaderBytes +
+  return kWsHeaderBytes + kWsCounterBytes +
          round256(sizeof(float) * static_cast<size_t>(c->B) * Hq * dp.splits * (c->d + 2));
 }
 
@@ -218,7 +219,9 @@ HEADQ_API headq_status headq_decode_attn(const headq_cache* cache, const void* q
   p.splits = sp.splits;
   p.chunk = sp.chunk;
   p.err = static_cast<unsigned*>(ws);
-  p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeaderBytes);
+  p.counters = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kWsHeaderBytes);
+  p.fused = sp.fused;
+  p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeaderBytes + kWsCounterBytes);
   p.out = out;
   p.lse = lse;
   return launch_decode(p, sp.mma, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess

@@ -13,6 +13,11 @@ namespace headq {
 
 // First bytes of every decode / attn_kl workspace: the device error word.
 constexpr size_t kWsHeaderBytes = 256;
+// Decode workspaces then hold a fixed region of split arrival counters (one per
+// (b, kv), left at zero by every call; never overlapped by partials, whatever
+// the shape of the call), then the partials.
+constexpr int kMaxFusedUnits = 8192;
+constexpr size_t kWsCounterBytes = sizeof(unsigned) * kMaxFusedUnits;
 constexpr unsigned kDevErrWaitTimeout = 1u;
 
 __host__ __device__ constexpr int group_size(int d) { return d < 32 ? d : 32; }
@@ -48,6 +53,18 @@ struct CacheWriteParams {
   const float* U;
 };
 
+// Decode split partials: unnormalised outputs o [B*Hq][splits][d] (rows of d
+// floats, 16-byte aligned), then the running max m and sum l [B*Hq][splits].
+struct PartView {
+  float* o;
+  float* m;
+  float* l;
+};
+__host__ __device__ inline PartView part_view(float* base, size_t bhq, int splits, int d) {
+  const size_t n = bhq * static_cast<size_t>(splits);
+  return {base, base + n * d, base + n * d + n};
+}
+
 struct DecodeParams {
   headq_cache c;
   const void* q;
@@ -61,6 +78,8 @@ struct DecodeParams {
   int chunk;       // tokens per split (multiple of 64)
   float* part;     // [B, Hq, splits, d + 2] partial (o, m, l)
   unsigned* err;   // device error word
+  unsigned* counters;  // [B * Hkv] split arrival counters, zero between calls
+  bool fused;          // the split kernel merges its own splits (last CTA)
   float* out;
   float* lse;
 };
@@ -109,11 +128,13 @@ int sm_count();
 // device; the workspace query, headq_decode_plan and the launch all use it.
 struct DecodePlan {
   int splits, chunk, kernels;
-  bool mma;  // tensor-core TMA kernel (decode_mma.cu) instead of the generic one
+  bool mma;    // tensor-core TMA kernel (decode_mma.cu) instead of the generic one
+  bool fused;  // that kernel also merges the splits (no combine launch)
 };
 DecodePlan decode_plan(const headq_cache& c, int Hq, int T);
-cudaError_t launch_decode(const DecodeParams& p, bool mma, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams& p, bool mma, cudaStream_t s);  // p.fused set
 
+constexpr int kMaxMmaSplits = 1024;  // the merging CTA keeps per-split weights in smem
 bool mma_decode_supported(const headq_cache& c, int G);
 int mma_decode_ctas_per_sm(const headq_cache& c, int G);
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s);

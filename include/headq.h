@@ -150,8 +150,10 @@ headq_status headq_cache_write(const headq_cache *cache, const void *k, const vo
  *   corr_sign +1 HeadQ, 0 base code only, -1 the wrong-sign control (section 4).
  *   out       fp32 [B, Hq, d];  lse fp32 [B, Hq] (nullable).
  *   ws        device workspace of at least headq_decode_workspace_bytes(...)
- *             bytes whose first 256 bytes were zero before its first use (they
- *             hold the device error word; see headq_workspace_status).
+ *             bytes, zero-filled before its first use: it holds the device error
+ *             word (see headq_workspace_status) and per-(b, kv) arrival counters
+ *             that every call leaves at zero again.  Calls sharing a workspace
+ *             must not overlap on the GPU.
  * Accumulation is fp32; the result matches the fp64 definition to a relative
  * error of about 1e-5 of the row maximum.
  */
@@ -182,7 +184,7 @@ int headq_decode_plan(const headq_cache *cache, int Hq, int T, int *splits, int 
  *   (headq_decode_workspace_bytes) exceeds 4 MiB returns HEADQ_ERR_WORKSPACE
  *   and launches nothing.
  *   The first call on a device does a one-time, synchronous set-up on that
- *   device (looks up the array's device address, clears its header); make that
+ *   device (looks up the array's device address, zero-fills it); make that
  *   first call before any stream capture.
  *   Every call on a device shares the one array and leaves its contents behind:
  *   calls whose work overlaps on the GPU (different streams, or different host

@@ -233,3 +233,27 @@ def test_full_size_sampled_rows(i):
                                    rtol=1e-5, atol=1e-4)
     del cache
     torch.cuda.empty_cache()
+
+
+def test_one_workspace_reused_across_shapes():
+    """A decode workspace sized for the largest call serves calls of different
+    shapes in any order: partials of one call never disturb the next."""
+    import ctypes
+    hq = _headq()
+    cases = []
+    for i, kw in ((2, dict(T=1000, B=2)), (1, dict(T=300)), (3, dict(T=2500)), (1, dict(T=700))):
+        w, L = layer(i, **kw)
+        U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+        _, out_ref, lse_ref = oracle_side(w, L, U)
+        cache, Ut = gpu_cache(w, L, U)
+        cases.append((w, L, cache, Ut, out_ref, lse_ref))
+    need = max(hq.lib().headq_decode_workspace_bytes(ctypes.byref(c[2].struct()), c[0].Hq,
+                                                     c[1].keys.shape[2]) for c in cases)
+    import torch
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for rep in range(2):
+        for w, L, cache, Ut, out_ref, lse_ref in cases:
+            out, lse = hq.headq_decode_attn(cache, gpu_query(w, L), Ut, T=L.keys.shape[2], ws=ws)
+            assert row_rel_err(out.cpu().numpy(), out_ref) <= DECODE_RTOL
+            np.testing.assert_allclose(lse.cpu().numpy(), lse_ref, rtol=1e-5, atol=1e-4)
+    hq.headq_workspace_status(ws)
