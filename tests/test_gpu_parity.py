@@ -257,3 +257,60 @@ def test_one_workspace_reused_across_shapes():
             assert row_rel_err(out.cpu().numpy(), out_ref) <= DECODE_RTOL
             np.testing.assert_allclose(lse.cpu().numpy(), lse_ref, rtol=1e-5, atol=1e-4)
     hq.headq_workspace_status(ws)
+
+
+def _edge_keys(d, T, seed):
+    """Keys built to stress the codec's rounding: exact ties (x - min)/scale =
+    k + 1/2, near-ties a few ulp away, constant, signed-zero, subnormal, tiny
+    normal and huge groups, and side-code inputs on a coarse dyadic grid."""
+    rng = np.random.default_rng(seed)
+    gs = min(32, d)
+    k = np.zeros((1, 1, T, d), np.float32)
+    for t in range(T):
+        for g in range(d // gs):
+            kind = t % 8
+            if kind == 0:     # integer levels 0..6 over span 6 -> scale 2, ties at 1, 3, 5
+                x = rng.integers(0, 7, gs).astype(np.float32)
+                x[0], x[1] = 0, 6
+            elif kind == 1:   # near-ties: tie values nudged by -4..4 ulp
+                x = rng.integers(0, 7, gs).astype(np.float32)
+                x[0], x[1] = 0, 6
+                nudge = rng.integers(-4, 5, gs)
+                for j in range(2, gs):
+                    for _ in range(abs(int(nudge[j]))):
+                        x[j] = np.nextafter(x[j], np.float32(np.inf if nudge[j] > 0 else -np.inf))
+            elif kind == 2:   # constant group: scale 0, all codes 0
+                x = np.full(gs, rng.standard_normal(), np.float32)
+            elif kind == 3:   # signed zeros and zeros
+                x = np.where(rng.random(gs) < 0.5, np.float32(-0.0), np.float32(0.0))
+            elif kind == 4:   # subnormal group
+                x = (rng.integers(0, 9, gs) * np.float32(2.0 ** -149)).astype(np.float32)
+            elif kind == 5:   # tiny normals around 1e-37
+                x = (rng.standard_normal(gs) * 1e-37).astype(np.float32)
+            elif kind == 6:   # huge values
+                x = (rng.standard_normal(gs) * 1e30).astype(np.float32)
+            else:             # dyadic grid: residuals and side codes hit exact ratios
+                x = (rng.integers(-64, 65, gs) / 16.0).astype(np.float32)
+            k[0, 0, t, g * gs:(g + 1) * gs] = x
+    return k
+
+
+@pytest.mark.parametrize("d,r", [(32, 8), (128, 16), (64, 2), (8, 4)])
+def test_cache_write_rounding_edges_bit_exact(d, r):
+    import torch
+    hq = _headq()
+    T = 96
+    k = _edge_keys(d, T, seed=d + r)
+    v = _edge_keys(d, T, seed=d + r + 1)
+    rng = np.random.default_rng(5)
+    # a dyadic basis (entries k/8): projections of dyadic residuals are exact, so
+    # side-code quotients land on ties too; plus a random orthonormal basis
+    for U in (np.stack([np.round(synth.random_orthonormal(rng, d, r) * 8) / 8]).astype(np.float32),
+              np.stack([synth.random_orthonormal(rng, d, r)])):
+        for vmode in ("dense", "2bit"):
+            ref = oracle.cache_write(k, U, v=v, vmode=vmode)
+            cache = hq.HeadQCache(1, 1, T, d, r, vmode=vmode, v_dtype=torch.float32)
+            hq.headq_cache_write(cache, torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda(),
+                                 torch.from_numpy(np.ascontiguousarray(U)).cuda())
+            got = planes_to_numpy(cache, 0, T)
+            assert_planes_equal(got, ref, r, vmode, "f32", values=v)
