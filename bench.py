@@ -5,11 +5,11 @@
                     [--workload NAME]
 
 One *step* is one serving decode step of one layer over a synthetic batch:
-``headq_cache_write`` of the step's new token for every (sequence, KV head)
-(base code + side code, written at position T-1), then ``headq_decode_attn``
-over the T cached tokens (query projection, streaming the packed cache,
-logits with the side-code correction, online softmax, value readout and the
-split combine).  The default workload is the long-context GQA layer (batch 1,
+``headq_decode_append`` writes the step's new token of every (sequence, KV
+head) into position T-1 (base code + side code, bit-exact with the cache
+write) and attends over the T cached tokens (query projection, streaming the
+packed cache, logits with the side-code correction, online softmax, value
+readout and the split merge) -- one kernel on the tensor-core path.  The default workload is the long-context GQA layer (batch 1,
 32 query heads over 8 KV heads, d=128, T=131072, r=16, 2-bit keys + 4-bit side
 code + bf16 values), the bandwidth-bound case.  Calibration (one-off, offline)
 and the KL diagnostic (needs the full-precision cache) are timed beside the
@@ -341,17 +341,17 @@ def run_headq(args):
         hq.headq_cache_write(c, k_all, v_all, U)
         caches.append(c)
     q = torch.from_numpy(L.queries).to(dev).to(dt)
-    k_new = k_all[:, :, T - 1:T].contiguous()
-    v_new = v_all[:, :, T - 1:T].contiguous()
+    k_new = k_all[:, :, T - 1].contiguous()   # [B, Hkv, d]: the step's new token
+    v_new = v_all[:, :, T - 1].contiguous()
     out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
     lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
     ws = hq.decode_workspace(caches[0], Hq, T)
-    splits, chunk, n_dec = hq.decode_plan(caches[0], Hq, T)
+    splits, chunk, n_dec, n_step = hq.decode_plan(caches[0], Hq, T)
     torch.cuda.synchronize()
 
     def step(c):
-        hq.headq_cache_write(c, k_new, v_new, U, t0=T - 1)
-        hq.headq_decode_attn(c, q, U, T=T, out=out, lse=lse, ws=ws)
+        # append the new token at position T-1 and attend over the T cached tokens
+        hq.headq_decode_append(c, k_new, v_new, q, U, T=T, out=out, lse=lse, ws=ws)
 
     for i in range(max(args.warmup, 3)):
         step(caches[i % 2])
@@ -451,8 +451,7 @@ def run_headq(args):
         q_d.copy_(q_h, non_blocking=True)
         kn_d.copy_(kn_h, non_blocking=True)
         vn_d.copy_(vn_h, non_blocking=True)
-        hq.headq_cache_write(c, kn_d, vn_d, U, t0=T - 1)
-        hq.headq_decode_attn(c, q_d, U, T=T, out=out, lse=lse, ws=ws)
+        hq.headq_decode_append(c, kn_d, vn_d, q_d, U, T=T, out=out, lse=lse, ws=ws)
         out_h.copy_(out, non_blocking=True)
         stream.synchronize()
     b_.record(stream)
@@ -490,14 +489,14 @@ def run_headq(args):
         "hbm_gbs_per_step": world * alg_bytes / (ms * 1e-3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "headq_decode_attn (split kernel + combine), %d splits of %d "
-                               "tokens" % (splits, chunk),
+                     "kernel": "headq_decode_attn, %d kernel(s), %d splits of %d tokens"
+                               % (n_dec, splits, chunk),
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "launch_ms": dec_ms, "peak_kind": peak_kind + " copy bandwidth"},
         "cpu_baseline": cpu,
         "e2e": {"value": world * B * T / (e2e_ms * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": K * (1 + n_dec),
+        "gpu_launches": K * n_step,
         "cuda_graph": use_graph,
         "clocks": clocks,
         "rows": rows,

@@ -41,6 +41,12 @@ cache_write_kernel(const CacheWriteParams p) {
   const int tid = threadIdx.x;
   const size_t bk = static_cast<size_t>(b) * p.c.Hkv + kv;
   const bool cache_v_bf16 = p.c.v_dtype == HEADQ_BF16;
+  int t0 = p.t0;
+  if (p.append) {  // one new token per sequence, at position T_b - 1
+    const int Tb = p.seq_lens ? max(0, min(p.seq_lens[b], p.T)) : p.T;
+    if (Tb == 0) return;
+    t0 = Tb - 1;
+  }
 
   // ---- phase A: base code, residual, values ---------------------------------
   for (int task = tid; task < kTT * NG; task += kThreads) {
@@ -48,7 +54,7 @@ cache_write_kernel(const CacheWriteParams p) {
     const int t = tile0 + tt;
     if (t >= p.n) continue;
     const size_t in_off = (bk * p.n + t) * D + g * GS;
-    const size_t row = bk * p.c.T_cap + p.t0 + t;
+    const size_t row = bk * p.c.T_cap + t0 + t;
     float x[GS], vv[GS];
     codec::load_row<GS>(p.k, in_off, p.in_bf16, x);
     if (p.v != nullptr) codec::load_row<GS>(p.v, in_off, p.in_bf16, vv);
@@ -119,7 +125,7 @@ cache_write_kernel(const CacheWriteParams p) {
     const float rs = __frcp_rn(s);
     const int w0 = codec::side_level(y[i], s, rs);
     const int w1 = codec::side_level(y[i + 1], s, rs);
-    const size_t row = bk * p.c.T_cap + p.t0 + tile0 + tt;
+    const size_t row = bk * p.c.T_cap + t0 + tile0 + tt;
     p.c.z_codes[row * (r / 2) + (i >> 1)] = static_cast<uint8_t>((w0 & 0xF) | ((w1 & 0xF) << 4));
     if (i == 0) p.c.z_scale[row] = s;
   }

@@ -38,6 +38,7 @@
 
 #include <mutex>
 
+#include "codec.cuh"
 #include "headq_internal.cuh"
 
 namespace headq {
@@ -71,10 +72,12 @@ struct Layout {
 template <int D, int R, int NT>
 constexpr size_t smem_bytes() {
   using L = Layout<D, R>;
-  // stages | q [GM][D] | group sums [GM][NG] | sigma U^T q [GM][R] | U [D][R] | barriers
+  // stages | q [GM][D] | group sums [GM][NG] | sigma U^T q [GM][R] | U [D][R] |
+  // appended token's residual [D] and projection [R] | barriers
   return 1024 + size_t(kStages) * L::kStage +
-         sizeof(float) * ((4 * NT) * (D + L::NG + (R > 0 ? R : 1)) + D * (R > 0 ? R : 1)) +
-         16 * kStages + 16;
+         sizeof(float) * ((4 * NT) * (D + L::NG + (R > 0 ? R : 1)) + D * (R > 0 ? R : 1) + D +
+                          (R > 0 ? R : 1)) +
+         16 * kStages + 32;
 }
 
 // ---------------------------------------------------------------- PTX helpers
@@ -211,9 +214,12 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   float* qsum_s = q_s + GM * D;                                               // [GM][NG]
   float* qt_s = qsum_s + GM * NG;                                             // [GM][RR]
   float* u_s = qt_s + GM * RR;                                                // [D][RR]
+  float* enew_s = u_s + D * RR;                                               // [D]
+  float* ynew_s = enew_s + D;                                                 // [RR]
   uint64_t* bars = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(u_s + D * RR) + 15) & ~uintptr_t(15));
-  // bars[s] = stage full, bars[kStages + s] = stage empty
+      (reinterpret_cast<uintptr_t>(ynew_s + RR) + 15) & ~uintptr_t(15));
+  // bars[s] = stage full, bars[kStages + s] = stage empty, bars[2 kStages] = the
+  // appended token is in HBM
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
@@ -225,12 +231,16 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   const int ntiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
   const size_t bk = static_cast<size_t>(b) * Hkv + kv;
   const int h0 = kv * G;
+  // the CTA whose chunk holds position T_b - 1 writes this step's new token there
+  const int pos = Tb - 1;
+  const bool owner = p.k_new != nullptr && Tb > 0 && pos >= t_begin && pos < t_begin + p.chunk;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_addr(&bars[s]), 1);
       mbar_init(smem_addr(&bars[kStages + s]), kCW);
     }
+    mbar_init(smem_addr(&bars[2 * kStages]), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -249,6 +259,13 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
         }
         const int t0 = t_begin + i * kTile;
         const int n16 = (min(kTile, t_end - t0) + 15) & ~15;
+        if (owner && pos < t0 + kTile) {  // this tile holds the appended token
+          if (!mbar_wait(smem_addr(&bars[2 * kStages]), 0)) {
+            ok = false;
+            break;
+          }
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
         const uint32_t full = smem_addr(&bars[s]);
         mbar_expect_tx(full, L::kVBoxes * L::kVBox + n16 * L::kRowBytes);
         uint8_t* st = stages + size_t(s) * L::kStage;
@@ -301,6 +318,51 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
+
+  if (owner && warp == 0) {
+    // encode the new token exactly as the cache write does: lanes 0..NG-1 take
+    // the key groups, NG..2NG-1 the value groups, lanes < R the side rows
+    const size_t row = bk * p.c.T_cap + pos;
+    const size_t in = bk * D;
+    if (lane < NG) {
+      float x[32];
+      uint32_t packed[2];
+      float sc, mn;
+      codec::load_row<32>(p.k_new, in + lane * 32, p.new_bf16, x);
+      codec::quantize_group<32, true>(x, packed, sc, mn);
+      codec::store_codes<32>(p.c.k_codes + row * (D / 4) + lane * 8, packed);
+      p.c.k_scale[row * NG + lane] = sc;
+      p.c.k_min[row * NG + lane] = mn;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) enew_s[lane * 32 + k] = x[k];
+    } else if (lane < 2 * NG && p.v_new != nullptr) {
+      const int gv = lane - NG;
+      float vv[32];
+      codec::load_row<32>(p.v_new, in + gv * 32, p.new_bf16, vv);
+      codec::store_values<32>(p.c.v, row * D + gv * 32, true, vv);
+    }
+    __syncwarp();
+    if constexpr (R > 0) {
+      float y = 0.0f;
+      if (lane < R)
+        for (int c = 0; c < D; ++c) y = __fmaf_rn(u_s[c * R + lane], enew_s[c], y);
+      float a = lane < R ? fabsf(y) : 0.0f;
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o2));
+      const float zs = codec::side_scale(a);
+      const int w = lane < R ? codec::side_level(y, zs, __frcp_rn(zs)) : 0;
+      const int w_next = __shfl_down_sync(kFull, w, 1);
+      if (lane < R && (lane & 1) == 0)
+        p.c.z_codes[row * (R / 2) + (lane >> 1)] =
+            static_cast<uint8_t>((w & 0xF) | ((w_next & 0xF) << 4));
+      if (lane == 0) p.c.z_scale[row] = zs;
+    }
+    // publish to the producer's bulk copies (async proxy) of the last tile
+    __threadfence();
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&bars[2 * kStages]));
+  }
 
   const int g = lane >> 2, t = lane & 3;
   const int jw = 16 * warp;

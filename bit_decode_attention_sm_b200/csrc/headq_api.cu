@@ -183,12 +183,13 @@ HEADQ_API size_t headq_decode_workspace_bytes(const headq_cache* cache, int Hq, 
 }
 
 HEADQ_API int headq_decode_plan(const headq_cache* cache, int Hq, int T, int* splits,
-                                int* chunk) {
+                                int* chunk, int* append_kernels) {
   if (!cache || cache->B < 0 || cache->Hkv <= 0 || Hq <= 0 || T < 0 || !supported_d(cache->d))
     return 0;
   const DecodePlan dp = decode_plan(*cache, Hq, T);
   if (splits) *splits = dp.splits;
   if (chunk) *chunk = dp.chunk;
+  if (append_kernels) *append_kernels = dp.mma ? dp.kernels : dp.kernels + 1;
   return dp.kernels;
 }
 
@@ -227,6 +228,64 @@ HEADQ_API headq_status headq_decode_attn(const headq_cache* cache, const void* q
   return launch_decode(p, sp.mma, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? HEADQ_OK
              : HEADQ_ERR_CUDA;
+}
+
+HEADQ_API headq_status headq_decode_append(const headq_cache* cache, const void* k_new,
+                                           const void* v_new, headq_dtype kv_dtype,
+                                           const void* q, headq_dtype q_dtype, int Hq,
+                                           const int32_t* seq_lens, int T, const float* U,
+                                           float sm_scale, int corr_sign, float* out,
+                                           float* lse, void* ws, size_t ws_bytes,
+                                           headq_stream_t stream) {
+  headq_status st = check_read_args(cache, q, q_dtype, Hq, T, U, corr_sign);
+  if (st != HEADQ_OK) return st;
+  if (!k_new || !aligned16(k_new) || (v_new && !aligned16(v_new))) return HEADQ_ERR_INVALID_ARG;
+  if (kv_dtype != HEADQ_F32 && kv_dtype != HEADQ_BF16) return HEADQ_ERR_INVALID_ARG;
+  if (!out || !aligned16(out) || (lse && !aligned16(lse))) return HEADQ_ERR_INVALID_ARG;
+  if (seq_lens && !aligned16(seq_lens)) return HEADQ_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws) || ws_bytes < decode_ws(cache, Hq, T)) return HEADQ_ERR_WORKSPACE;
+  if (cache->B == 0) return HEADQ_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const DecodePlan sp = decode_plan(*cache, Hq, T);
+  if (!sp.mma) {
+    // generic path: the append write, then the decode
+    CacheWriteParams w{};
+    w.c = *cache;
+    w.k = k_new;
+    w.v = v_new;
+    w.in_bf16 = kv_dtype == HEADQ_BF16;
+    w.n = 1;
+    w.U = U;
+    w.append = true;
+    w.seq_lens = seq_lens;
+    w.T = T;
+    if (launch_cache_write(w, s) != cudaSuccess) return HEADQ_ERR_CUDA;
+    return headq_decode_attn(cache, q, q_dtype, Hq, seq_lens, T, U, sm_scale, corr_sign, out,
+                             lse, ws, ws_bytes, stream);
+  }
+  DecodeParams p{};
+  p.c = *cache;
+  p.q = q;
+  p.q_bf16 = q_dtype == HEADQ_BF16;
+  p.Hq = Hq;
+  p.G = Hq / cache->Hkv;
+  p.T = T;
+  p.seq_lens = seq_lens;
+  p.U = U;
+  p.sm_scale = sm_scale;
+  p.corr_sign = static_cast<float>(corr_sign);
+  p.splits = sp.splits;
+  p.chunk = sp.chunk;
+  p.err = static_cast<unsigned*>(ws);
+  p.counters = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kWsHeaderBytes);
+  p.fused = sp.fused;
+  p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeaderBytes + kWsCounterBytes);
+  p.out = out;
+  p.lse = lse;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.new_bf16 = kv_dtype == HEADQ_BF16;
+  return launch_decode(p, true, s) == cudaSuccess ? HEADQ_OK : HEADQ_ERR_CUDA;
 }
 
 HEADQ_API size_t headq_attn_kl_workspace_bytes(const headq_cache* cache, int Hq, int T) {

@@ -51,6 +51,11 @@ struct CacheWriteParams {
   bool in_bf16;
   int t0, n;
   const float* U;
+  // append mode (n == 1): sequence b's token goes to position T_b - 1, with
+  // T_b = seq_lens[b] (or T when seq_lens is null); nothing when T_b == 0
+  bool append;
+  const int32_t* seq_lens;
+  int T;
 };
 
 // Decode split partials: unnormalised outputs o [B*Hq][splits][d] (rows of d
@@ -80,6 +85,11 @@ struct DecodeParams {
   unsigned* err;   // device error word
   unsigned* counters;  // [B * Hkv] split arrival counters, zero between calls
   bool fused;          // the split kernel merges its own splits (last CTA)
+  // fused append (tensor-core kernel): the new token [B, Hkv, d] of each sequence
+  // is encoded into position T_b - 1 before the tile holding it is read
+  const void* k_new;
+  const void* v_new;
+  bool new_bf16;
   float* out;
   float* lse;
 };

@@ -30,7 +30,7 @@ EXPORTS = ("headq_version", "headq_status_string", "headq_calibrate",
            "headq_calibrate_workspace_bytes", "headq_cache_write", "headq_decode_attn",
            "headq_decode_workspace_bytes", "headq_decode_plan", "headq_attn_kl",
            "headq_attn_kl_workspace_bytes", "headq_workspace_status",
-           "headq_decode_attn_noalloc")
+           "headq_decode_attn_noalloc", "headq_decode_append")
 
 
 class HeadQError(RuntimeError):
@@ -73,11 +73,12 @@ def lib():
             "headq_cache_write": ([CP, P, P, I, I, I, P, P], I),
             "headq_decode_attn": ([CP, P, I, I, P, I, P, F, I, P, P, P, Z, P], I),
             "headq_decode_workspace_bytes": ([CP, I, I], Z),
-            "headq_decode_plan": ([CP, I, I, P, P], I),
+            "headq_decode_plan": ([CP, I, I, P, P, P], I),
             "headq_attn_kl": ([CP, P, I, I, P, I, P, P, I, P, F, I, P, P, P, P, P, Z, P], I),
             "headq_attn_kl_workspace_bytes": ([CP, I, I], Z),
             "headq_workspace_status": ([P, P], I),
             "headq_decode_attn_noalloc": ([CP, P, I, I, P, I, P, F, I, P, P, P], I),
+            "headq_decode_append": ([CP, P, P, I, P, I, I, P, I, P, F, I, P, P, P, Z, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -227,11 +228,13 @@ def decode_workspace(cache, Hq, T):
 
 
 def decode_plan(cache, Hq, T):
-    """(splits, chunk, kernels per call) that headq_decode_attn uses for these sizes."""
+    """(splits, chunk, kernels per headq_decode_attn call, kernels per
+    headq_decode_append call) for these sizes on the current device."""
     cs = cache.struct()
-    sp, ch = ctypes.c_int(0), ctypes.c_int(0)
-    nk = lib().headq_decode_plan(ctypes.byref(cs), Hq, T, ctypes.byref(sp), ctypes.byref(ch))
-    return sp.value, ch.value, nk
+    sp, ch, ak = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    nk = lib().headq_decode_plan(ctypes.byref(cs), Hq, T, ctypes.byref(sp), ctypes.byref(ch),
+                                 ctypes.byref(ak))
+    return sp.value, ch.value, nk, ak.value
 
 
 def attn_kl_workspace(cache, Hq, T):
@@ -259,6 +262,34 @@ def headq_decode_attn(cache, q, U, T=None, seq_lens=None, sm_scale=None, corr_si
     _check("headq_decode_attn", lib().headq_decode_attn(
         ctypes.byref(cs), _ptr(q), _dtype_code(q), Hq, _ptr(seq_lens), T, _ptr(U), sm,
         int(corr_sign), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def headq_decode_append(cache, k_new, v_new, q, U, T=None, seq_lens=None, sm_scale=None,
+                        corr_sign=1, out=None, lse=None, ws=None, stream=None):
+    """One decode step: write each sequence's new token (k_new, v_new [B,Hkv,d]) at
+    position T_b - 1, then attend; returns (out fp32 [B,Hq,d], lse fp32 [B,Hq])."""
+    q = _cuda(q, "q")
+    k_new = _cuda(k_new, "k_new")
+    v_new = _cuda(v_new, "v_new")
+    if v_new is not None and v_new.dtype != k_new.dtype:
+        raise TypeError("k_new and v_new must have the same dtype")
+    B, Hq, d = q.shape
+    T = cache.T_cap if T is None else int(T)
+    sm = 1.0 / math.sqrt(d) if sm_scale is None else float(sm_scale)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = decode_workspace(cache, Hq, T)
+    seq_lens = _cuda(seq_lens, "seq_lens")
+    U = _cuda(U, "U") if cache.r > 0 else None
+    cs = cache.struct()
+    _check("headq_decode_append", lib().headq_decode_append(
+        ctypes.byref(cs), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), _ptr(q), _dtype_code(q),
+        Hq, _ptr(seq_lens), T, _ptr(U), sm, int(corr_sign), _ptr(out), _ptr(lse), _ptr(ws),
+        ws.numel(), _stream(stream)))
     return out, lse
 
 

@@ -166,10 +166,31 @@ size_t headq_decode_workspace_bytes(const headq_cache *cache, int Hq, int T);
 
 /*
  * headq_decode_plan -- the launch plan headq_decode_attn uses for these sizes on
- * the current device: *splits T-splits of *chunk tokens per (b, kv), and the
- * number of kernels one call launches (returned).  0 on invalid sizes.
+ * the current device: *splits T-splits of *chunk tokens per (b, kv), the number
+ * of kernels one headq_decode_append call launches (*append_kernels, nullable),
+ * and the number of kernels one headq_decode_attn call launches (returned).
+ * 0 on invalid sizes.
  */
-int headq_decode_plan(const headq_cache *cache, int Hq, int T, int *splits, int *chunk);
+int headq_decode_plan(const headq_cache *cache, int Hq, int T, int *splits, int *chunk,
+                      int *append_kernels);
+
+/*
+ * headq_decode_append -- one serving decode step: write each sequence's new token
+ * into the cache, then attend over the cache including it (summary section 3,
+ * steps 2 and 3 in one call).  For every b with T_b >= 1 (T_b = seq_lens[b], or
+ * T when seq_lens is NULL) the new key k_new[b, kv] and value v_new[b, kv]
+ * ([B, Hkv, d] of kv_dtype; v_new may be NULL) are encoded into position T_b - 1
+ * bit-exactly as headq_cache_write would, and out/lse are those of
+ * headq_decode_attn over tokens j < T_b.  Sequences with T_b = 0 write nothing.
+ * Same arguments, workspace and conventions as headq_decode_attn.  On the
+ * tensor-core path this is a single kernel: the CTA that owns position T_b - 1
+ * encodes the token while the others stream the cache.
+ */
+headq_status headq_decode_append(const headq_cache *cache, const void *k_new,
+                                 const void *v_new, headq_dtype kv_dtype, const void *q,
+                                 headq_dtype q_dtype, int Hq, const int32_t *seq_lens, int T,
+                                 const float *U, float sm_scale, int corr_sign, float *out,
+                                 float *lse, void *ws, size_t ws_bytes, headq_stream_t stream);
 
 /*
  * headq_decode_attn_noalloc -- headq_decode_attn without a caller workspace.

@@ -314,3 +314,72 @@ def test_cache_write_rounding_edges_bit_exact(d, r):
                                  torch.from_numpy(np.ascontiguousarray(U)).cuda())
             got = planes_to_numpy(cache, 0, T)
             assert_planes_equal(got, ref, r, vmode, "f32", values=v)
+
+
+APPEND_CASES = [
+    (3, dict(T=2500), None),
+    (2, dict(T=700, B=4), np.array([700, 1, 0, 333], np.int32)),
+    (1, dict(T=300), np.array([300, 17, 1, 64, 299, 150, 0, 65], np.int32)),
+    (4, dict(T=500, B=2), np.array([500, 250], np.int32)),    # 2-bit V: generic path
+    (0, {}, None),                                             # fp32 V: generic path
+]
+
+
+@pytest.mark.parametrize("i,kw,sl", APPEND_CASES, ids=["cfg%d" % c[0] for c in APPEND_CASES])
+def test_decode_append_matches_oracle(i, kw, sl):
+    """headq_decode_append: each sequence's new token written at T_b - 1 (planes
+    bit-exact) and the attention over tokens < T_b, in one call."""
+    import torch
+    hq = _headq()
+    w, L = layer(i, **kw)
+    B, Hkv, T, d = L.keys.shape
+    lens = np.full(B, T, np.int32) if sl is None else sl
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    planes, out_ref, lse_ref = oracle_side(w, L, U, seq_lens=sl)
+    # cache holding every token except the new ones (those positions hold other data)
+    stale = synth.LayerInputs(L.keys.copy(), L.values.copy(), L.queries, L.q_cal, {})
+    rng = np.random.default_rng(1)
+    for b in range(B):
+        if lens[b] > 0:
+            stale.keys[b, :, lens[b] - 1] = rng.standard_normal((Hkv, d)).astype(np.float32)
+            stale.values[b, :, lens[b] - 1] = rng.standard_normal((Hkv, d)).astype(np.float32)
+    if w.kv_dtype == "bf16":
+        stale.keys = synth.round_bf16(stale.keys)
+        stale.values = synth.round_bf16(stale.values)
+    cache, Ut = gpu_cache(w, stale, U)
+    dt = torch_dtype(w)
+    pos = np.maximum(lens - 1, 0)
+    k_new = torch.from_numpy(np.ascontiguousarray(L.keys[np.arange(B), :, pos])).cuda().to(dt)
+    v_new = torch.from_numpy(np.ascontiguousarray(L.values[np.arange(B), :, pos])).cuda().to(dt)
+    slt = None if sl is None else torch.from_numpy(sl).cuda()
+    ws = hq.decode_workspace(cache, w.Hq, T)
+    out, lse = hq.headq_decode_append(cache, k_new, v_new, gpu_query(w, L), Ut, T=T,
+                                      seq_lens=slt, ws=ws)
+    hq.headq_workspace_status(ws)
+    o, l_ = out.cpu().numpy(), lse.cpu().numpy()
+    assert row_rel_err(o, out_ref) <= DECODE_RTOL
+    np.testing.assert_allclose(l_, lse_ref, rtol=1e-5, atol=1e-4)
+    got = planes_to_numpy(cache, 0, T)
+    for b in range(B):
+        if lens[b] == 0:
+            continue
+        p_ = lens[b] - 1
+        one = {k: a[b:b + 1, :, p_:p_ + 1] for k, a in got.items()}
+        ref1 = {k: a[b:b + 1, :, p_:p_ + 1] for k, a in planes.items() if k != "y"}
+        assert_planes_equal(one, ref1, w.r, w.vmode, w.kv_dtype,
+                            values=L.values[b:b + 1, :, p_:p_ + 1])
+
+
+def test_decode_append_without_values_keeps_v():
+    """v_new = NULL writes the key planes only; the cached value stays."""
+    import torch
+    hq = _headq()
+    w, L = layer(2, T=300, B=2)
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    cache, Ut = gpu_cache(w, L, U)
+    before = cache.v.clone()
+    k_new = torch.from_numpy(np.ascontiguousarray(L.keys[:, :, -1])).cuda().to(torch.bfloat16)
+    out, _ = hq.headq_decode_append(cache, k_new, None, gpu_query(w, L), Ut, T=300)
+    assert torch.equal(cache.v, before)
+    _, out_ref, _ = oracle_side(w, L, U)
+    assert row_rel_err(out.cpu().numpy(), out_ref) <= DECODE_RTOL
