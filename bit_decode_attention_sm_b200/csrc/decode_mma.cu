@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -54,27 +55,36 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;         // log2 units the stale max may lag
 
-template <int D, int R>
+// Shared-memory stage of kTile tokens.  Dense bf16 values (V2 = false): the
+// swizzled value boxes come first.  2-bit values (V2 = true): their code, scale
+// and minimum planes are bulk-copied like the keys'.
+template <int D, int R, bool V2 = false>
 struct Layout {
   static constexpr int NG = D / 32;
-  static constexpr int kVBoxes = D / 64;             // 64-dim boxes per token row
+  static constexpr int kVBoxes = V2 ? 0 : D / 64;    // 64-dim boxes per token row
   static constexpr int kVBox = kTile * 128;          // 64 tokens x 128 bytes
   static constexpr int kKc = kVBoxes * kVBox;
   static constexpr int kKs = kKc + kTile * (D / 4);
   static constexpr int kKm = kKs + kTile * NG * 4;
   static constexpr int kZc = kKm + kTile * NG * 4;
   static constexpr int kZs = kZc + kTile * (R / 2);
-  static constexpr int kEnd = kZs + (R > 0 ? kTile * 4 : 0);
+  static constexpr int kVc = kZs + (R > 0 ? kTile * 4 : 0);
+  static constexpr int kVs = kVc + (V2 ? kTile * (D / 4) : 0);
+  static constexpr int kVm = kVs + (V2 ? kTile * NG * 4 : 0);
+  static constexpr int kEnd = kVm + (V2 ? kTile * NG * 4 : 0);
   static constexpr int kStage = (kEnd + 1023) / 1024 * 1024;
-  static constexpr int kRowBytes = D / 4 + 8 * NG + (R > 0 ? R / 2 + 4 : 0);
+  static constexpr int kRowBytes =
+      D / 4 + 8 * NG + (R > 0 ? R / 2 + 4 : 0) + (V2 ? D / 4 + 8 * NG : 0);
+  static constexpr int kCodeTile = V2 ? 16 * D * 2 : 0;  // per consumer warp, bf16 codes
 };
 
-template <int D, int R, int NT>
+template <int D, int R, int NT, bool V2>
 constexpr size_t smem_bytes() {
-  using L = Layout<D, R>;
-  // stages | q [GM][D] | group sums [GM][NG] | sigma U^T q [GM][R] | U [D][R] |
-  // appended token's residual [D] and projection [R] | barriers
-  return 1024 + size_t(kStages) * L::kStage +
+  using L = Layout<D, R, V2>;
+  // stages | per-warp value code tiles | q [GM][D] | group sums [GM][NG] |
+  // sigma U^T q [GM][R] | U [D][R] | appended token's residual [D] and
+  // projection [R] | barriers
+  return 1024 + size_t(kStages) * L::kStage + size_t(kCW) * L::kCodeTile +
          sizeof(float) * ((4 * NT) * (D + L::NG + (R > 0 ? R : 1)) + D * (R > 0 ? R : 1) + D +
                           (R > 0 ? R : 1)) +
          16 * kStages + 32;
@@ -177,6 +187,24 @@ __device__ __forceinline__ void unpack_side(uint32_t y, uint32_t& n01, uint32_t&
   n01 = hfma2((y & 0x00F0000Fu) | 0x64006400u, 0x2C003C00u, 0xD480E408u);
   n23 = hfma2((z & 0x00F0000Fu) | 0x64006400u, 0x2C003C00u, 0xD480E408u);
 }
+// y holds one 16-bit word of eight 2-bit codes c0..c7 in both halves.  Returns
+// bf16 pairs (c0,c1) (c2,c3) (c4,c5) (c6,c7), exactly: 0x4300 | (code << 2k) is
+// the bf16 value 128 + code*4^k (k <= 2, inside the 7-bit mantissa), and one
+// exact bf16 FMA turns it back into the code.
+__device__ __forceinline__ uint32_t hfma2_bf16(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ void unpack_codes_bf16(uint32_t y, uint32_t (&v)[4]) {
+  const uint32_t y2 = y >> 2, y8 = y >> 8, y10 = y >> 10;
+  // (128 + c, 128 + 4c') * (1, 1/4) - (128, 32)
+  v[0] = hfma2_bf16((y & 0x000C0003u) | 0x43004300u, 0x3E803F80u, 0xC200C300u);
+  // (128 + 4c, 128 + 16c') * (1/4, 1/16) - (32, 8)
+  v[1] = hfma2_bf16((y2 & 0x0030000Cu) | 0x43004300u, 0x3D803E80u, 0xC100C200u);
+  v[2] = hfma2_bf16((y8 & 0x000C0003u) | 0x43004300u, 0x3E803F80u, 0xC200C300u);
+  v[3] = hfma2_bf16((y10 & 0x0030000Cu) | 0x43004300u, 0x3D803E80u, 0xC100C200u);
+}
 __device__ __forceinline__ uint32_t half_part_pair(float a, float b, bool lo) {
   __half ha = __float2half_rn(a), hb = __float2half_rn(b);
   if (lo) {
@@ -195,10 +223,10 @@ __device__ __forceinline__ uint32_t bf16_part_pair(float a, float b, bool lo) {
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int D, int R, int NT>
+template <int D, int R, int NT, bool V2>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
 decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap) {
-  using L = Layout<D, R>;
+  using L = Layout<D, R, V2>;
   constexpr int NG = L::NG;
   constexpr int KS = D / 16;   // k-steps of 16 channels
   constexpr int MT = D / 16;   // 16-dim row blocks of the output
@@ -210,7 +238,8 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  float* q_s = reinterpret_cast<float*>(smem + size_t(kStages) * L::kStage);  // [GM][D]
+  uint8_t* ctiles = smem + size_t(kStages) * L::kStage;  // [kCW][16][D] bf16 value codes
+  float* q_s = reinterpret_cast<float*>(ctiles + size_t(kCW) * L::kCodeTile);  // [GM][D]
   float* qsum_s = q_s + GM * D;                                               // [GM][NG]
   float* qt_s = qsum_s + GM * NG;                                             // [GM][RR]
   float* u_s = qt_s + GM * RR;                                                // [D][RR]
@@ -277,9 +306,15 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
           bulk_g2s(smem_addr(st + L::kZc), p.c.z_codes + row0 * (R / 2), n16 * (R / 2), full);
           bulk_g2s(smem_addr(st + L::kZs), p.c.z_scale + row0, n16 * 4, full);
         }
+        if constexpr (V2) {
+          bulk_g2s(smem_addr(st + L::kVc), p.c.v_codes + row0 * (D / 4), n16 * (D / 4), full);
+          bulk_g2s(smem_addr(st + L::kVs), p.c.v_scale + row0 * NG, n16 * NG * 4, full);
+          bulk_g2s(smem_addr(st + L::kVm), p.c.v_min + row0 * NG, n16 * NG * 4, full);
+        } else {
 #pragma unroll
-        for (int bx = 0; bx < L::kVBoxes; ++bx)
-          tma_3d(smem_addr(st + bx * L::kVBox), &vmap, bx * 64, t0, static_cast<int>(bk), full);
+          for (int bx = 0; bx < L::kVBoxes; ++bx)
+            tma_3d(smem_addr(st + bx * L::kVBox), &vmap, bx * 64, t0, static_cast<int>(bk), full);
+        }
         ++issued;
       }
       if (!ok && p.err) atomicOr(p.err, kDevErrWaitTimeout);
@@ -339,7 +374,16 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       const int gv = lane - NG;
       float vv[32];
       codec::load_row<32>(p.v_new, in + gv * 32, p.new_bf16, vv);
-      codec::store_values<32>(p.c.v, row * D + gv * 32, true, vv);
+      if constexpr (V2) {
+        uint32_t packed[2];
+        float sc, mn;
+        codec::quantize_group<32, false>(vv, packed, sc, mn);
+        codec::store_codes<32>(p.c.v_codes + row * (D / 4) + gv * 8, packed);
+        p.c.v_scale[row * NG + gv] = sc;
+        p.c.v_min[row * NG + gv] = mn;
+      } else {
+        codec::store_values<32>(p.c.v, row * D + gv * 32, true, vv);
+      }
     }
     __syncwarp();
     if constexpr (R > 0) {
@@ -410,8 +454,12 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
 
   float m2[NT], l[NT];
   float o[MT][NT][4];
+  float vmin_acc[NT][V2 ? NG : 1];  // 2-bit values: sum_j p_j min_{j,g} per group
+  uint8_t* ctile = ctiles + size_t(warp) * L::kCodeTile;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int gg = 0; gg < (V2 ? NG : 1); ++gg) vmin_acc[nt][gg] = 0.f;
     m2[nt] = -INFINITY;
     l[nt] = 0.0f;
 #pragma unroll
@@ -431,7 +479,24 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     const int j0 = jw + g, j1 = j0 + 8;
     const bool val0 = j0 < nvalid, val1 = j1 < nvalid;
 
-    if (nvalid < jw + 16) {  // tail of the split: clear value rows past the end
+    if constexpr (V2) {
+      // this warp's 16 tokens of value codes -> bf16 code tile (chunk c of row t
+      // stored at c ^ (t & 7): conflict-free ldmatrix)
+      for (int task = lane; task < 16 * (D / 16); task += 32) {
+        const int tt = task / (D / 16), blk = task - tt * (D / 16);
+        const uint32_t wv = *reinterpret_cast<const uint32_t*>(st + L::kVc + (jw + tt) * (D / 4) +
+                                                               4 * blk);
+        uint32_t lo4[4], hi4[4];
+        unpack_codes_bf16(__byte_perm(wv, 0u, 0x1010u), lo4);
+        unpack_codes_bf16(__byte_perm(wv, 0u, 0x3232u), hi4);
+        const int c0 = 2 * blk, c1 = 2 * blk + 1;
+        *reinterpret_cast<uint4*>(ctile + tt * (D * 2) + ((c0 ^ (tt & 7)) << 4)) =
+            make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+        *reinterpret_cast<uint4*>(ctile + tt * (D * 2) + ((c1 ^ (tt & 7)) << 4)) =
+            make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+      }
+      __syncwarp();
+    } else if (nvalid < jw + 16) {  // tail of the split: clear value rows past the end
       for (int idx = lane; idx < 16 * 8 * L::kVBoxes; idx += 32) {
         const int bx = idx % L::kVBoxes, rem = idx / L::kVBoxes;
         const int row = jw + rem / 8, c16 = rem % 8;
@@ -502,6 +567,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
 
     // ---- logits, online softmax, p in the B-operand layout
     uint32_t bp[NT][2];
+    uint32_t bpv[V2 ? NG : 1][NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       float s0 = 0.f, s1 = 0.f;
@@ -528,6 +594,10 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
         const float alpha = resc ? exp2f(m2[nt] - mnew) : 1.0f;
         if (resc) m2[nt] = mnew;
         l[nt] *= alpha;
+        if constexpr (V2) {
+#pragma unroll
+          for (int gg = 0; gg < NG; ++gg) vmin_acc[nt][gg] *= alpha;
+        }
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
           o[mt][nt][0] *= alpha; o[mt][nt][1] *= alpha;
@@ -541,21 +611,53 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       const int sa = 8 * t + (g >> 1), sb = sa + 4;
       const float va = __shfl_sync(kFull, p0, sa), vb = __shfl_sync(kFull, p0, sb);
       const float vc = __shfl_sync(kFull, p1, sa), vd = __shfl_sync(kFull, p1, sb);
-      bp[nt][0] = bf16_part_pair(va, vb, g & 1);
-      bp[nt][1] = bf16_part_pair(vc, vd, g & 1);
+      if constexpr (V2) {
+        // per 32-dim group: p_j * scale_{j,g} (0 for masked tokens, whatever the
+        // stale scale), and the running sum of p_j * min_{j,g}
+        const float* vs = reinterpret_cast<const float*>(st + L::kVs);
+        const float* vm = reinterpret_cast<const float*>(st + L::kVm);
+        const int ta = jw + 2 * t, tb = ta + 1, tc = ta + 8, td = ta + 9;
+#pragma unroll
+        for (int gg = 0; gg < NG; ++gg) {
+          const float pa = va > 0.f ? va * vs[ta * NG + gg] : 0.f;
+          const float pb = vb > 0.f ? vb * vs[tb * NG + gg] : 0.f;
+          const float pc = vc > 0.f ? vc * vs[tc * NG + gg] : 0.f;
+          const float pd = vd > 0.f ? vd * vs[td * NG + gg] : 0.f;
+          bpv[gg][nt][0] = bf16_part_pair(pa, pb, g & 1);
+          bpv[gg][nt][1] = bf16_part_pair(pc, pd, g & 1);
+          if (p0 > 0.f) vmin_acc[nt][gg] = fmaf(p0, vm[j0 * NG + gg], vmin_acc[nt][gg]);
+          if (p1 > 0.f) vmin_acc[nt][gg] = fmaf(p1, vm[j1 * NG + gg], vmin_acc[nt][gg]);
+        }
+      } else {
+        bp[nt][0] = bf16_part_pair(va, vb, g & 1);
+        bp[nt][1] = bf16_part_pair(vc, vd, g & 1);
+      }
     }
 
     // ---- p . V on tensor cores (A = V^T from the swizzled tile)
-    const uint32_t vbase = smem_addr(st);
+    if constexpr (V2) {
+      const uint32_t cbase = smem_addr(ctile);
+      const int lt = lm_tok - jw;  // row within this warp's code tile
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const int chunk = 2 * mt + lm_chunk_hi;
-      const uint32_t addr = vbase + (chunk >> 3) * L::kVBox + lm_tok * 128 +
-                            (((chunk & 7) ^ (lm_tok & 7)) << 4);
-      uint32_t a[4];
-      ldsm_x4_trans(addr, a);
+      for (int mt = 0; mt < MT; ++mt) {
+        const int chunk = 2 * mt + lm_chunk_hi;
+        uint32_t a[4];
+        ldsm_x4_trans(cbase + lt * (D * 2) + ((chunk ^ (lt & 7)) << 4), a);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_bf16(o[mt][nt], a, bp[nt]);
+        for (int nt = 0; nt < NT; ++nt) mma_bf16(o[mt][nt], a, bpv[mt >> 1][nt]);
+      }
+    } else {
+      const uint32_t vbase = smem_addr(st);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const int chunk = 2 * mt + lm_chunk_hi;
+        const uint32_t addr = vbase + (chunk >> 3) * L::kVBox + lm_tok * 128 +
+                              (((chunk & 7) ^ (lm_tok & 7)) << 4);
+        uint32_t a[4];
+        ldsm_x4_trans(addr, a);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_bf16(o[mt][nt], a, bp[nt]);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&bars[kStages + s]));
@@ -568,6 +670,14 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     l[nt] += __shfl_xor_sync(kFull, l[nt], 4);
     l[nt] += __shfl_xor_sync(kFull, l[nt], 8);
     l[nt] += __shfl_xor_sync(kFull, l[nt], 16);
+    if constexpr (V2) {
+#pragma unroll
+      for (int gg = 0; gg < NG; ++gg) {
+        vmin_acc[nt][gg] += __shfl_xor_sync(kFull, vmin_acc[nt][gg], 4);
+        vmin_acc[nt][gg] += __shfl_xor_sync(kFull, vmin_acc[nt][gg], 8);
+        vmin_acc[nt][gg] += __shfl_xor_sync(kFull, vmin_acc[nt][gg], 16);
+      }
+    }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   float* mo = reinterpret_cast<float*>(stages);  // [kCW][GM][D]
@@ -582,8 +692,9 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     const int h = 4 * nt + t;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
-      mo[(warp * GM + h) * D + 16 * mt + g] = o[mt][nt][0] + o[mt][nt][1];
-      mo[(warp * GM + h) * D + 16 * mt + g + 8] = o[mt][nt][2] + o[mt][nt][3];
+      const float vmn = V2 ? vmin_acc[nt][V2 ? (mt >> 1) : 0] : 0.f;
+      mo[(warp * GM + h) * D + 16 * mt + g] = (o[mt][nt][0] + o[mt][nt][1]) + vmn;
+      mo[(warp * GM + h) * D + 16 * mt + g + 8] = (o[mt][nt][2] + o[mt][nt][3]) + vmn;
     }
     if (g == 0) {
       mm[warp * GM + h] = m2[nt];
@@ -714,7 +825,7 @@ EncodeTiled encode_fn() {
 
 constexpr int kMaxDev = 64;
 
-template <int D, int R, int NT>
+template <int D, int R, int NT, bool V2>
 struct Variant {
   static int occupancy[kMaxDev];  // CTAs per SM, 0 = not yet known
   static std::mutex mu;
@@ -729,8 +840,8 @@ struct Variant {
     }
     std::lock_guard<std::mutex> lock(mu);
     if (occupancy[dev] == 0) {
-      auto k = decode_mma_kernel<D, R, NT>;
-      const int smem = static_cast<int>(smem_bytes<D, R, NT>());
+      auto k = decode_mma_kernel<D, R, NT, V2>;
+      const int smem = static_cast<int>(smem_bytes<D, R, NT, V2>());
       int n = 0;
       if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
               cudaSuccess ||
@@ -745,9 +856,15 @@ struct Variant {
 
   static cudaError_t launch(const DecodeParams& p, cudaStream_t s) {
     if (ctas_per_sm() == 0) return cudaErrorInvalidConfiguration;
+    CUtensorMap vmap;
+    dim3 grid(p.splits, p.c.Hkv, p.c.B);
+    if (V2) {  // no value tensor map: the 2-bit value planes are bulk-copied
+      memset(&vmap, 0, sizeof(vmap));
+      decode_mma_kernel<D, R, NT, V2><<<grid, kThreads, smem_bytes<D, R, NT, V2>(), s>>>(p, vmap);
+      return cudaGetLastError();
+    }
     EncodeTiled enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    CUtensorMap vmap;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(p.c.T_cap),
                                 static_cast<cuuint64_t>(p.c.B) * p.c.Hkv};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
@@ -759,45 +876,53 @@ struct Variant {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
-    dim3 grid(p.splits, p.c.Hkv, p.c.B);
-    decode_mma_kernel<D, R, NT><<<grid, kThreads, smem_bytes<D, R, NT>(), s>>>(p, vmap);
+    decode_mma_kernel<D, R, NT, V2><<<grid, kThreads, smem_bytes<D, R, NT, V2>(), s>>>(p, vmap);
     return cudaGetLastError();
   }
 };
-template <int D, int R, int NT>
-int Variant<D, R, NT>::occupancy[kMaxDev];
-template <int D, int R, int NT>
-std::mutex Variant<D, R, NT>::mu;
+template <int D, int R, int NT, bool V2>
+int Variant<D, R, NT, V2>::occupancy[kMaxDev];
+template <int D, int R, int NT, bool V2>
+std::mutex Variant<D, R, NT, V2>::mu;
 
 template <typename F>
-auto dispatch(int d, int r, int G, F&& f) -> decltype(f(Variant<128, 16, 1>{})) {
+auto dispatch(int d, int r, int G, bool v2, F&& f) -> decltype(f(Variant<128, 16, 1, false>{})) {
   const int nt = G <= 4 ? 1 : 2;
-#define HEADQ_MMA_CASE(DD, RR, NN) \
-  if (d == DD && r == RR && nt == NN) return f(Variant<DD, RR, NN>{});
-  HEADQ_MMA_CASE(128, 16, 1) HEADQ_MMA_CASE(128, 16, 2)
-  HEADQ_MMA_CASE(128, 8, 1) HEADQ_MMA_CASE(128, 8, 2)
-  HEADQ_MMA_CASE(128, 0, 1) HEADQ_MMA_CASE(128, 0, 2)
-  HEADQ_MMA_CASE(64, 16, 1) HEADQ_MMA_CASE(64, 16, 2)
-  HEADQ_MMA_CASE(64, 8, 1) HEADQ_MMA_CASE(64, 8, 2)
-  HEADQ_MMA_CASE(64, 0, 1) HEADQ_MMA_CASE(64, 0, 2)
+#define HEADQ_MMA_CASE(DD, RR, NN, VV) \
+  if (d == DD && r == RR && nt == NN && v2 == VV) return f(Variant<DD, RR, NN, VV>{});
+  HEADQ_MMA_CASE(128, 16, 1, false) HEADQ_MMA_CASE(128, 16, 2, false)
+  HEADQ_MMA_CASE(128, 8, 1, false) HEADQ_MMA_CASE(128, 8, 2, false)
+  HEADQ_MMA_CASE(128, 0, 1, false) HEADQ_MMA_CASE(128, 0, 2, false)
+  HEADQ_MMA_CASE(64, 16, 1, false) HEADQ_MMA_CASE(64, 16, 2, false)
+  HEADQ_MMA_CASE(64, 8, 1, false) HEADQ_MMA_CASE(64, 8, 2, false)
+  HEADQ_MMA_CASE(64, 0, 1, false) HEADQ_MMA_CASE(64, 0, 2, false)
+  HEADQ_MMA_CASE(128, 16, 1, true) HEADQ_MMA_CASE(128, 16, 2, true)
+  HEADQ_MMA_CASE(128, 8, 1, true) HEADQ_MMA_CASE(128, 8, 2, true)
+  HEADQ_MMA_CASE(64, 16, 1, true) HEADQ_MMA_CASE(64, 16, 2, true)
+  HEADQ_MMA_CASE(64, 8, 1, true) HEADQ_MMA_CASE(64, 8, 2, true)
 #undef HEADQ_MMA_CASE
-  return decltype(f(Variant<128, 16, 1>{}))();
+  return decltype(f(Variant<128, 16, 1, false>{}))();
 }
+
+bool is_v2(const headq_cache& c) { return c.vmode == HEADQ_V_2BIT; }
 
 }  // namespace
 
 bool mma_decode_supported(const headq_cache& c, int G) {
-  return c.vmode == HEADQ_V_DENSE && c.v_dtype == HEADQ_BF16 && (c.d == 64 || c.d == 128) &&
-         (c.r == 0 || c.r == 8 || c.r == 16) && G >= 1 && G <= 8 && encode_fn() != nullptr;
+  if (c.d != 64 && c.d != 128) return false;
+  if (G < 1 || G > 8) return false;
+  if (c.vmode == HEADQ_V_2BIT) return c.r == 8 || c.r == 16;
+  return c.vmode == HEADQ_V_DENSE && c.v_dtype == HEADQ_BF16 &&
+         (c.r == 0 || c.r == 8 || c.r == 16) && encode_fn() != nullptr;
 }
 
 int mma_decode_ctas_per_sm(const headq_cache& c, int G) {
-  return dispatch(c.d, c.r, G, [](auto v) { return decltype(v)::ctas_per_sm(); });
+  return dispatch(c.d, c.r, G, is_v2(c), [](auto v) { return decltype(v)::ctas_per_sm(); });
 }
 
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s) {
   // 0 means no variant matched; otherwise the launch status + 1
-  const int e = dispatch(p.c.d, p.c.r, p.G, [&](auto v) {
+  const int e = dispatch(p.c.d, p.c.r, p.G, is_v2(p.c), [&](auto v) {
     return static_cast<int>(decltype(v)::launch(p, s)) + 1;
   });
   return e == 0 ? cudaErrorInvalidValue : static_cast<cudaError_t>(e - 1);
