@@ -111,18 +111,25 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def recorded_traffic(kernel_file, summary_file):
+def recorded_traffic(kernel_files, summary_file):
     """DRAM bytes per launch from a committed ncu summary, if the kernel source
-    is still the one that was profiled (else None)."""
+    (the given files, concatenated) is still the one that was profiled (else None)."""
     try:
-        src = open(os.path.join(ROOT, "bit_decode_attention_sm_b200", "csrc",
-                                kernel_file), "rb").read()
+        if isinstance(kernel_files, str):
+            kernel_files = [kernel_files]
+        src = b"".join(open(os.path.join(ROOT, "bit_decode_attention_sm_b200", "csrc", f),
+                            "rb").read() for f in kernel_files)
         sha = hashlib.sha256(src).hexdigest()
         fields = {}
         for line in open(os.path.join(ROOT, "profiles", summary_file)):
             if ":" in line and line.strip().startswith("- "):
                 k, v = line.strip()[2:].split(":", 1)
-                fields[k.strip()] = v.strip().strip("`")
+                v = v.strip()
+                if v.startswith("`"):
+                    v = v[1:].split("`", 1)[0]
+                else:
+                    v = v.split()[0] if v else v
+                fields[k.strip()] = v
         if fields.get("kernel_source_sha256") != sha:
             return None
         return float(fields["dram_bytes_per_launch"])
@@ -471,7 +478,8 @@ def run_headq(args):
     alg_bytes = B * Hkv * T * bytes_tok
     peak, peak_kind = measured_hbm_peak()
     achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
-    traffic = recorded_traffic("decode_attn.cu", "decode_attn_longctx.md")
+    traffic = (recorded_traffic(["decode_mma.cu", "codec.cuh"], "decode_mma_longctx.md")
+               if w.name == DEFAULT_WORKLOAD else None)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -511,9 +519,21 @@ def run_headq(args):
     return 0
 
 
+# fp64 FMA lanes per SM per clock on B200 (148 SMs, 1965 MHz max clock):
+# 148 x 64 x 2 x 1.965e9 = 37.2 TFLOP/s, the published fp64 figure
+FP64_FMA_PER_SM_CLK = 64
+
+
+def fp64_peak_tflops(sm_count=148, mhz=1965.0):
+    return sm_count * FP64_FMA_PER_SM_CLK * 2 * mhz * 1e6 / 1e12
+
+
 def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream):
-    """Times of the steps measured beside the decode step, with CUDA events."""
+    """The other rows of the path, timed with CUDA events, each against its roofline:
+    the prefill cache write and the KL diagnostic against HBM bandwidth (bytes they
+    must move), calibration against the fp64 ALU peak (its Gram matrix FLOPs)."""
     rows = {}
+    peak, peak_kind = measured_hbm_peak()
 
     def timed(fn, reps):
         fn()
@@ -526,16 +546,33 @@ def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / reps
 
-    ms = timed(lambda: hq.headq_calibrate(q_cal, w.Hkv, w.r), 3)
-    rows["calibrate"] = {"ms": ms, "queries": int(q_cal.shape[0])}
-    B, Hkv, T = w.B, w.Hkv, w.T
+    def hbm_row(ms, nbytes, **extra):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return dict(ms=ms, algorithmic_bytes=nbytes,
+                    roofline={"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                              "frac": gbs / peak, "peak_kind": peak_kind + " copy bandwidth"},
+                    **extra)
+
+    B, Hkv, T, d = w.B, w.Hkv, w.T, w.d
     tok = B * Hkv * T
+    kv_in = tok * d * 2 * k_all.element_size()          # the bf16 K and V read
+    planes = tok * cache.nbytes_per_token()              # the packed cache
     ms = timed(lambda: hq.headq_cache_write(cache, k_all, v_all, U), 5)
-    in_b = tok * w.d * 2 * k_all.element_size()
-    rows["cache_write_prefill"] = {"ms": ms, "tokens": B * T,
-                                   "hbm_gbs": (in_b + tok * cache.nbytes_per_token()) / ms / 1e6}
-    ms = timed(lambda: hq.headq_attn_kl(cache, q, U, k_all, v_all), 3)
-    rows["attn_kl"] = {"ms": ms, "hbm_gbs": (in_b + tok * cache.nbytes_per_token()) / ms / 1e6}
+    rows["cache_write_prefill"] = hbm_row(ms, kv_in + planes, tokens=B * T,
+                                          note="reads K,V and writes every plane")
+    ws = hq.attn_kl_workspace(cache, w.Hq, T)
+    ms = timed(lambda: hq.headq_attn_kl(cache, q, U, k_all, v_all, ws=ws), 3)
+    rows["attn_kl"] = hbm_row(ms, kv_in + planes, note="reads the packed cache and full K,V")
+    ms = timed(lambda: hq.headq_calibrate(q_cal, Hkv, w.r), 3)
+    M = q_cal.shape[0] * w.G
+    flops = 2.0 * Hkv * M * d * d
+    pk = fp64_peak_tflops(torch.cuda.get_device_properties(0).multi_processor_count)
+    tf = flops / (ms * 1e-3) / 1e12
+    rows["calibrate"] = dict(ms=ms, queries=int(q_cal.shape[0]),
+                             roofline={"bound": "alu", "achieved": tf, "peak": pk,
+                                       "unit": "TFLOP/s", "frac": tf / pk,
+                                       "peak_kind": "fp64 from unit counts and max clock",
+                                       "work": "Gram matrix, 2*Hkv*N*G*d^2 flops"})
     return rows
 
 
