@@ -277,19 +277,369 @@ __global__ void attn_kl_combine_kernel(const AttnKlParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Staged kernel (d = 64 or 128): 32-token tiles of every plane and of the full
+// K and V are copied to shared memory with double-buffered cp.async (rows past
+// the end zero-filled); the key error dk = k^ - k and the value error
+// dv = v^ - v are formed once per token and shared by the G query heads.
+constexpr int kSTT = 32;         // tokens per tile
+constexpr int kSThreads = 256;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+template <int D>
+struct KlStage {
+  static constexpr int NG = D / 32;
+  int frow;   // bytes per staged full-precision row (padded)
+  int cvrow;  // bytes per staged cache-value row (dense, padded)
+  int kf, vf, cv, kc, ks, km, zc, zs, vc, vs, vm, bytes;
+  __host__ __device__ KlStage(int esz, int cv_esz, int r, bool v2) {
+    frow = D * esz + 16;
+    cvrow = D * cv_esz + 16;
+    kf = 0;
+    vf = kf + kSTT * frow;
+    cv = vf + kSTT * frow;
+    kc = cv + (v2 ? 0 : kSTT * cvrow);
+    ks = kc + kSTT * (D / 4);
+    km = ks + kSTT * NG * 4;
+    zc = km + kSTT * NG * 4;
+    zs = zc + kSTT * (r / 2 > 0 ? r / 2 : 0);
+    vc = zs + (r > 0 ? kSTT * 4 : 0);
+    vs = vc + (v2 ? kSTT * (D / 4) : 0);
+    vm = vs + (v2 ? kSTT * NG * 4 : 0);
+    bytes = (vm + (v2 ? kSTT * NG * 4 : 0) + 127) / 128 * 128;
+  }
+};
+
+// copy `bytes_per_row` x rows (contiguous in global, rows of `rb` bytes) into
+// shared rows of stride `dst_stride`, zero-filling rows >= valid
+__device__ __forceinline__ void stage_rows(uint8_t* dst, int dst_stride, const uint8_t* src, int rb,
+                                           int valid, int tid) {
+  const int chunks = rb / 16;
+  for (int e = tid; e < kSTT * chunks; e += kSThreads) {
+    const int row = e / chunks, c = e - row * chunks;
+    const bool ok = row < valid;
+    cp_async16(dst + row * dst_stride + c * 16, ok ? src + static_cast<size_t>(row) * rb + c * 16 : src,
+               ok);
+  }
+}
+// a contiguous block (rows of rb bytes packed), valid rows only
+__device__ __forceinline__ void stage_block(uint8_t* dst, const uint8_t* src, int rb, int valid,
+                                            int tid) {
+  const int total = (kSTT * rb) / 16;
+  const int vbytes = valid * rb;
+  for (int e = tid; e < total; e += kSThreads) {
+    const bool ok = e * 16 < vbytes;
+    cp_async16(dst + e * 16, ok ? src + e * 16 : src, ok);
+  }
+}
+
+__device__ __forceinline__ float ld_smem_elem(const uint8_t* row, int c, bool bf16) {
+  return bf16 ? bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(row)[c])
+              : reinterpret_cast<const float*>(row)[c];
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSThreads)
+attn_kl_staged_kernel(const AttnKlParams p) {
+  constexpr int NG = D / 32;
+  constexpr int DS = D + 4;  // padded fp32 rows of dk / dv
+  const int G = p.G, r = p.c.r, Hkv = p.c.Hkv;
+  const bool v2 = p.c.vmode == HEADQ_V_2BIT;
+  const bool cv_bf16 = p.c.v_dtype == HEADQ_BF16;
+  const int esz = p.kv_bf16 ? 2 : 4;
+  const KlStage<D> L(esz, cv_bf16 ? 2 : 4, r, v2);
+
+  extern __shared__ __align__(128) uint8_t sm8[];
+  uint8_t* stg[2] = {sm8, sm8 + L.bytes};
+  float* dk_s = reinterpret_cast<float*>(sm8 + 2 * L.bytes);  // [kSTT][DS]
+  float* dv_s = dk_s + kSTT * DS;                              // [kSTT][DS]
+  float* q_s = dv_s + kSTT * DS;                               // [G][D]
+  float* qt_s = q_s + G * D;                                   // [G][r]
+  float* s_s = qt_s + G * (r > 0 ? r : 1);                     // [G][kSTT]
+  float* d_s = s_s + G * kSTT;                                 // [G][kSTT]
+  float* n2_s = d_s + G * kSTT;                                // [kSTT]
+  float* m_s = n2_s + kSTT;                                    // [G]
+  float* md_s = m_s + G;                                       // [G]
+  float* a_s = md_s + G;                                       // [G]
+  double* acc_s = reinterpret_cast<double*>(
+      (reinterpret_cast<uintptr_t>(a_s + G) + 7) & ~uintptr_t(7));  // [G][5]
+
+  const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int Tb = p.T;
+  if (p.seq_lens) Tb = max(0, min(p.seq_lens[b], p.T));
+  const int t_begin = split * p.chunk;
+  const int t_end = min(Tb, t_begin + p.chunk);
+  const int ntiles = t_end > t_begin ? (t_end - t_begin + kSTT - 1) / kSTT : 0;
+  const size_t bk = static_cast<size_t>(b) * Hkv + kv;
+  const int h0 = kv * G;
+
+  auto issue = [&](int i) {
+    const int t0 = t_begin + i * kSTT;
+    const int nv = min(kSTT, t_end - t0);
+    uint8_t* st = stg[i & 1];
+    const size_t frow0 = bk * p.T + t0, crow0 = bk * p.c.T_cap + t0;
+    stage_rows(st + L.kf, L.frow, static_cast<const uint8_t*>(p.k_full) + frow0 * D * esz,
+               D * esz, nv, tid);
+    stage_rows(st + L.vf, L.frow, static_cast<const uint8_t*>(p.v_full) + frow0 * D * esz,
+               D * esz, nv, tid);
+    if (!v2) {
+      const int cesz = cv_bf16 ? 2 : 4;
+      stage_rows(st + L.cv, L.cvrow, static_cast<const uint8_t*>(p.c.v) + crow0 * D * cesz,
+                 D * cesz, nv, tid);
+    } else {
+      stage_block(st + L.vc, p.c.v_codes + crow0 * (D / 4), D / 4, nv, tid);
+      stage_block(st + L.vs, reinterpret_cast<const uint8_t*>(p.c.v_scale + crow0 * NG), NG * 4, nv, tid);
+      stage_block(st + L.vm, reinterpret_cast<const uint8_t*>(p.c.v_min + crow0 * NG), NG * 4, nv, tid);
+    }
+    stage_block(st + L.kc, p.c.k_codes + crow0 * (D / 4), D / 4, nv, tid);
+    stage_block(st + L.ks, reinterpret_cast<const uint8_t*>(p.c.k_scale + crow0 * NG), NG * 4, nv, tid);
+    stage_block(st + L.km, reinterpret_cast<const uint8_t*>(p.c.k_min + crow0 * NG), NG * 4, nv, tid);
+    if (r > 0) {
+      if ((kSTT * (r / 2)) % 16 == 0)
+        stage_block(st + L.zc, p.c.z_codes + crow0 * (r / 2), r / 2, nv, tid);
+      stage_block(st + L.zs, reinterpret_cast<const uint8_t*>(p.c.z_scale + crow0), 4, nv, tid);
+    }
+    cp_async_commit();
+  };
+  if (ntiles > 0) issue(0);
+
+  for (int i = tid; i < G * D; i += kSThreads)
+    q_s[i] = load_elem(p.q, (static_cast<size_t>(b) * p.Hq + h0) * D + i, p.q_bf16);
+  for (int h = tid; h < G; h += kSThreads) {
+    m_s[h] = -INFINITY;
+    md_s[h] = -INFINITY;
+    for (int k = 0; k < 5; ++k) acc_s[h * 5 + k] = 0.0;
+  }
+  __syncthreads();
+  for (int i = tid; i < G * r; i += kSThreads) {
+    const int h = i / r, ii = i - h * r;
+    const float* U = p.U + static_cast<size_t>(kv) * D * r;
+    float acc = 0.0f;
+    for (int c = 0; c < D; ++c) acc = fmaf(U[c * r + ii], q_s[h * D + c], acc);
+    qt_s[i] = p.corr_sign * acc;
+  }
+
+  constexpr int kMaxDov = 8;  // (G * D) / kSThreads outputs per thread at most
+  double dov[kMaxDov];
+#pragma unroll
+  for (int k = 0; k < kMaxDov; ++k) dov[k] = 0.0;
+
+  for (int i = 0; i < ntiles; ++i) {
+    if (i + 1 < ntiles) {
+      issue(i + 1);
+      cp_async_wait1();
+    } else {
+      cp_async_wait0();
+    }
+    __syncthreads();
+    const uint8_t* st = stg[i & 1];
+    const int t0 = t_begin + i * kSTT;
+    const int nt = min(kSTT, t_end - t0);
+    // phase 0: key and value errors per (token, 4 channels); |dv|^2 per token
+    {
+      constexpr int CPT = D / 4;  // tasks per token
+      for (int task = tid; task < kSTT * CPT; task += kSThreads) {
+        const int tt = task / CPT, c4 = task - tt * CPT, c = 4 * c4, g = c / 32;
+        float n2 = 0.0f;
+        if (tt < nt) {
+          const uint8_t kb = st[L.kc + tt * (D / 4) + c4];
+          const float ksc = reinterpret_cast<const float*>(st + L.ks)[tt * NG + g];
+          const float kmn = reinterpret_cast<const float*>(st + L.km)[tt * NG + g];
+          const uint8_t* kfr = st + L.kf + tt * L.frow;
+          const uint8_t* vfr = st + L.vf + tt * L.frow;
+          float4 dk, dv;
+          float* dkp = &dk.x;
+          float* dvp = &dv.x;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float kh = __fadd_rn(kmn, __fmul_rn(static_cast<float>((kb >> (2 * k)) & 3), ksc));
+            dkp[k] = kh - ld_smem_elem(kfr, c + k, p.kv_bf16);
+            float vh;
+            if (v2) {
+              const uint8_t vb = st[L.vc + tt * (D / 4) + c4];
+              const float vsc = reinterpret_cast<const float*>(st + L.vs)[tt * NG + g];
+              const float vmn = reinterpret_cast<const float*>(st + L.vm)[tt * NG + g];
+              vh = __fadd_rn(vmn, __fmul_rn(static_cast<float>((vb >> (2 * k)) & 3), vsc));
+            } else {
+              vh = ld_smem_elem(st + L.cv + tt * L.cvrow, c + k, cv_bf16);
+            }
+            dvp[k] = vh - ld_smem_elem(vfr, c + k, p.kv_bf16);
+            n2 = fmaf(dvp[k], dvp[k], n2);
+          }
+          *reinterpret_cast<float4*>(dk_s + tt * DS + c) = dk;
+          *reinterpret_cast<float4*>(dv_s + tt * DS + c) = dv;
+        }
+        // the CPT tasks of a token are CPT consecutive lanes of one warp
+#pragma unroll
+        for (int o = CPT >= 32 ? 16 : CPT / 2; o > 0; o >>= 1) n2 += __shfl_xor_sync(kFull, n2, o);
+        if (c4 == 0) n2_s[tt] = tt < nt ? n2 : 0.0f;
+      }
+    }
+    __syncthreads();
+    // phase 1: logits s and score perturbations delta per (head, token)
+    for (int task = tid; task < G * kSTT; task += kSThreads) {
+      const int h = task / kSTT, tt = task - h * kSTT;
+      float sv = -INFINITY, dl = 0.0f;
+      if (tt < nt) {
+        const float* qh = q_s + h * D;
+        const uint8_t* kfr = st + L.kf + tt * L.frow;
+        const float* dkr = dk_s + tt * DS;
+        float sf = 0.0f, de = 0.0f;
+        if (p.kv_bf16) {
+#pragma unroll 4
+          for (int c = 0; c < D; c += 8) {
+            const uint4 kw = *reinterpret_cast<const uint4*>(kfr + 2 * c);
+            const uint32_t w4[4] = {kw.x, kw.y, kw.z, kw.w};
+            const float4 d0 = *reinterpret_cast<const float4*>(dkr + c);
+            const float4 d1 = *reinterpret_cast<const float4*>(dkr + c + 4);
+            const float4 q0 = *reinterpret_cast<const float4*>(qh + c);
+            const float4 q1 = *reinterpret_cast<const float4*>(qh + c + 4);
+            const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+            const float dvv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              sf = fmaf(qv[2 * k], __uint_as_float(w4[k] << 16), sf);
+              sf = fmaf(qv[2 * k + 1], __uint_as_float(w4[k] & 0xffff0000u), sf);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) de = fmaf(qv[k], dvv[k], de);
+          }
+        } else {
+          for (int c = 0; c < D; ++c) {
+            sf = fmaf(qh[c], reinterpret_cast<const float*>(kfr)[c], sf);
+            de = fmaf(qh[c], dkr[c], de);
+          }
+        }
+        if (r > 0) {
+          const uint8_t* zr = p.c.z_codes + (bk * p.c.T_cap + t0 + tt) * (r / 2);
+          if ((kSTT * (r / 2)) % 16 == 0) zr = st + L.zc + tt * (r / 2);
+          float cz = 0.0f;
+          for (int ii = 0; ii < r; ++ii)
+            cz = fmaf(qt_s[h * r + ii], static_cast<float>(nibble(zr, ii)), cz);
+          de = fmaf(reinterpret_cast<const float*>(st + L.zs)[tt], cz, de);
+        }
+        sv = sf * p.sm_scale;
+        dl = de * p.sm_scale;
+      }
+      s_s[task] = sv;
+      d_s[task] = dl;
+    }
+    __syncthreads();
+    // phase 2: running fp64 accumulators, one warp per head
+    for (int h = warp; h < G; h += kSThreads / 32) {
+      const bool valid = lane < nt;
+      const float sv = s_s[h * kSTT + lane];
+      const float dl = d_s[h * kSTT + lane];
+      const float m_old = m_s[h], md_old = md_s[h];
+      const float m_new = fmaxf(m_old, warp_maxf(sv));
+      const float md_new = fmaxf(md_old, warp_maxf(valid ? dl : -INFINITY));
+      const double w = valid ? exp(static_cast<double>(sv) - m_new) : 0.0;
+      const double x = valid ? w * exp(static_cast<double>(dl) - md_new) : 0.0;
+      const double alpha = exp(static_cast<double>(m_old) - m_new);
+      const double beta = exp(static_cast<double>(md_old) - md_new);
+      const double dd = dl;
+      const double sW = warp_sumd(w), sX = warp_sumd(x);
+      const double sM1 = warp_sumd(w * dd), sM2 = warp_sumd(w * dd * dd);
+      const double sA2 = warp_sumd(w * w * static_cast<double>(n2_s[lane]));
+      s_s[h * kSTT + lane] = static_cast<float>(w);
+      __syncwarp();
+      if (lane == 0) {
+        double* a = acc_s + h * 5;
+        a[0] = a[0] * alpha + sW;
+        a[1] = a[1] * alpha * beta + sX;
+        a[2] = a[2] * alpha + sM1;
+        a[3] = a[3] * alpha + sM2;
+        a[4] = a[4] * alpha * alpha + sA2;
+        m_s[h] = m_new;
+        md_s[h] = md_new;
+        a_s[h] = static_cast<float>(alpha);
+      }
+    }
+    __syncthreads();
+    // phase 3: readout error sum_j w_j dv_j per (head, dim)
+#pragma unroll
+    for (int k = 0; k < kMaxDov; ++k) {
+      const int idx = tid + k * kSThreads;
+      if (idx < G * D) {
+        const int h = idx / D, c = idx - h * D;
+        const float* pw = s_s + h * kSTT;
+        float part = 0.0f;
+        for (int j = 0; j < nt; ++j) part = fmaf(pw[j], dv_s[j * DS + c], part);
+        dov[k] = dov[k] * static_cast<double>(a_s[h]) + part;
+      }
+    }
+    __syncthreads();
+  }
+
+  const int PS = kPartHead + D;
+#pragma unroll
+  for (int k = 0; k < kMaxDov; ++k) {
+    const int idx = tid + k * kSThreads;
+    if (idx < G * D) {
+      const int h = idx / D, c = idx - h * D;
+      const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
+      p.part[(bh * p.splits + split) * PS + kPartHead + c] = dov[k];
+    }
+  }
+  for (int h = tid; h < G; h += kSThreads) {
+    const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
+    double* pt = p.part + (bh * p.splits + split) * PS;
+    const double* a = acc_s + h * 5;
+    pt[0] = m_s[h];
+    pt[1] = a[0];
+    pt[2] = md_s[h];
+    pt[3] = a[1];
+    pt[4] = a[2];
+    pt[5] = a[3];
+    pt[6] = a[4];
+  }
+}
+
+template <int D>
+size_t staged_smem(const AttnKlParams& p) {
+  const KlStage<D> L(p.kv_bf16 ? 2 : 4, p.c.v_dtype == HEADQ_BF16 ? 2 : 4, p.c.r,
+                     p.c.vmode == HEADQ_V_2BIT);
+  const int G = p.G, r = p.c.r;
+  return 2 * size_t(L.bytes) + sizeof(float) * (2 * kSTT * (D + 4) + G * D + G * (r > 0 ? r : 1) +
+                                                2 * G * kSTT + kSTT + 3 * G) +
+         8 + sizeof(double) * G * 5;
+}
+
 template <int D>
 cudaError_t launch_d(const AttnKlParams& p, cudaStream_t s) {
   const int G = p.G, r = p.c.r;
   const size_t smem = sizeof(double) * G * 6 +
                       sizeof(float) * (static_cast<size_t>(G) * D + G * r + 2 * G * kTile +
                                        kTile + 3 * G);
+  dim3 grid(p.splits, p.c.Hkv, p.c.B);
+  if constexpr (D == 64 || D == 128) {
+    if (p.G * D <= 8 * kSThreads) {
+      const size_t ssm = staged_smem<D>(p);
+      auto k = attn_kl_staged_kernel<D>;
+      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(ssm));
+      if (e != cudaSuccess) return e;
+      k<<<grid, kSThreads, ssm, s>>>(p);
+      attn_kl_combine_kernel<D><<<p.c.B * p.Hq, D < 32 ? 32 : (D > 128 ? 128 : D), 0, s>>>(p);
+      return cudaGetLastError();
+    }
+  }
   auto k = attn_kl_split_kernel<D>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(p.splits, p.c.Hkv, p.c.B);
   k<<<grid, kThreads, smem, s>>>(p);
   attn_kl_combine_kernel<D><<<p.c.B * p.Hq, D < 32 ? 32 : (D > 128 ? 128 : D), 0, s>>>(p);
   return cudaGetLastError();

@@ -11,8 +11,8 @@
 //   A  one thread per (token, 32-channel group): vector loads of the group's keys
 //      and values straight from HBM (all issued before any arithmetic), base code,
 //      codes/scale/min stored, residual e -> shared memory, values stored/coded
-//   B  one thread per (token, 4 side rows): y = U_h^T e in channel order, one
-//      fused multiply-add per term, two terms per packed fp32x2 FMA
+//   B  one thread per (token, 8 side rows): y = U_h^T e in channel order, one
+//      fused multiply-add per term, two rows per packed fp32x2 FMA
 //   C  one thread per (token, pair of side rows): absmax scale and the two nibbles
 #include "codec.cuh"
 
@@ -87,29 +87,37 @@ cache_write_kernel(const CacheWriteParams p) {
   __syncthreads();
 
   // ---- phase B: y = U_h^T e, channel order, one FMA per term ---------------
+  // RB side rows per thread as RB/2 packed pairs, one fp32x2 FMA per pair and
+  // channel (the pairs and U stay in 64-bit registers)
   const int blocks_per_tok = r / RB;
   for (int pr = tid; pr < kTT * blocks_per_tok; pr += kThreads) {
     const int tt = pr / blocks_per_tok;
     const int i0 = (pr - tt * blocks_per_tok) * RB;
     if (tile0 + tt >= p.n) continue;
-    float y[RB];
+    uint64_t y[RB / 2];
 #pragma unroll
-    for (int k = 0; k < RB; ++k) y[k] = 0.0f;
+    for (int k = 0; k < RB / 2; ++k) y[k] = 0ull;
     const float* er = e_s + tt * ES;
 #pragma unroll 8
     for (int c = 0; c < D; ++c) {
-      const float ec = er[c];
-      if constexpr (RB == 4) {
-        const float4 u = *reinterpret_cast<const float4*>(u_s + c * r + i0);
-        codec::fma2(y[0], y[1], u.x, u.y, ec);
-        codec::fma2(y[2], y[3], u.z, u.w, ec);
+      const uint64_t e2 = codec::dup2(er[c]);
+      const uint64_t* ur = reinterpret_cast<const uint64_t*>(u_s + c * r + i0);
+      if constexpr (RB >= 4) {
+#pragma unroll
+        for (int k = 0; k < RB / 4; ++k) {
+          const ulonglong2 u = reinterpret_cast<const ulonglong2*>(ur)[k];
+          codec::fma2_pk(y[2 * k], u.x, e2);
+          codec::fma2_pk(y[2 * k + 1], u.y, e2);
+        }
       } else {
-        const float2 u = *reinterpret_cast<const float2*>(u_s + c * r + i0);
-        codec::fma2(y[0], y[1], u.x, u.y, ec);
+        codec::fma2_pk(y[0], ur[0], e2);
       }
     }
 #pragma unroll
-    for (int k = 0; k < RB; ++k) y_s[tt * (r + 1) + i0 + k] = y[k];
+    for (int k = 0; k < RB / 2; ++k) {
+      y_s[tt * (r + 1) + i0 + 2 * k] = __uint_as_float(static_cast<uint32_t>(y[k]));
+      y_s[tt * (r + 1) + i0 + 2 * k + 1] = __uint_as_float(static_cast<uint32_t>(y[k] >> 32));
+    }
   }
   __syncthreads();
 
@@ -138,7 +146,8 @@ cudaError_t launch_d(const CacheWriteParams& p, cudaStream_t s) {
                                        static_cast<size_t>(D) * r +
                                        static_cast<size_t>(kTT) * (r + 1));
   dim3 grid((p.n + kTT - 1) / kTT, p.c.Hkv, p.c.B);
-  auto k = r % 4 == 0 ? cache_write_kernel<D, 4> : cache_write_kernel<D, 2>;
+  auto k = r % 8 == 0 ? cache_write_kernel<D, 8>
+                      : (r % 4 == 0 ? cache_write_kernel<D, 4> : cache_write_kernel<D, 2>);
   if (smem > 48 * 1024) {  // only the largest head dims need the opt-in
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

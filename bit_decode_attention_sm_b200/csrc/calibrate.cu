@@ -9,13 +9,16 @@
 // is q.e, with E[(q.e)^2] = e^T E[q q^T] e, so this eigenspace is the rank-r
 // subspace that captures the most score error.
 //
-//   gram kernel    C in fp64, one CTA per (row i, kv)
-//   jacobi kernel  one CTA per kv: cyclic two-sided Jacobi rotations in fp64
-//                  (Jacobi's method; rotation angle as in Golub & Van Loan,
-//                  "Matrix Computations", symmetric Schur decomposition), the
-//                  d/2 disjoint pairs of each step from the round-robin
-//                  ("circle") schedule applied in parallel; then the r largest
-//                  eigenvalues, descending, and a sign rule per vector.
+//   gram kernel    C in fp64, one CTA per (32x32 tile pair, kv), the query rows
+//                  staged through shared memory 32 at a time
+//   jacobi kernel  one CTA per kv: cyclic two-sided Jacobi rotations on the
+//                  fp64 matrix in shared memory (Jacobi's method; rotation angle
+//                  as in Golub & Van Loan, "Matrix Computations", symmetric Schur
+//                  decomposition), the d/2 disjoint pairs of each step from the
+//                  round-robin ("circle") schedule applied in parallel, the
+//                  rotations accumulated in fp32 rows of eigenvectors, also in
+//                  shared memory; then the r largest eigenvalues, descending, and
+//                  a sign rule per vector.
 #include <math.h>
 
 #include "headq_internal.cuh"
@@ -24,7 +27,7 @@ namespace headq {
 namespace {
 
 constexpr int kGramThreads = 128;
-constexpr int kJacThreads = 256;
+constexpr int kJacThreads = 512;
 constexpr int kMaxSweeps = 40;
 
 __global__ void mean_kernel(const CalibrateParams p, double* mean) {
@@ -41,38 +44,67 @@ __global__ void mean_kernel(const CalibrateParams p, double* mean) {
   }
 }
 
+constexpr int kGT = 32;  // Gram tile edge
+
+// C tile (i0.., j0..) of kv head: sum over the M = N*G query rows, j0 >= i0;
+// the mirrored tile is written too.
 __global__ void __launch_bounds__(kGramThreads)
 gram_kernel(const CalibrateParams p, const double* mean) {
-  const int i = blockIdx.x, kv = blockIdx.y;
-  const int d = p.d;
+  const int kv = blockIdx.y;
+  const int d = p.d, tiles = (d + kGT - 1) / kGT;
+  int ti = 0, tj = blockIdx.x;  // linear index over the upper-triangle tile pairs
+  while (tj >= tiles - ti) { tj -= tiles - ti; ++ti; }
+  tj += ti;
+  const int i0 = ti * kGT, j0 = tj * kGT;
   const long M = static_cast<long>(p.N) * p.G;
-  __shared__ double xi_s[kGramThreads];
-  double acc = 0.0;
-  const int j = threadIdx.x;
-  const double mi = p.center ? mean[kv * d + i] : 0.0;
-  const double mj = (p.center && j < d) ? mean[kv * d + j] : 0.0;
-  for (long m0 = 0; m0 < M; m0 += kGramThreads) {
-    const long mm = m0 + threadIdx.x;
-    double xi = 0.0;
-    if (mm < M) {
-      const long n = mm / p.G, g = mm - n * p.G;
-      xi = load_elem(p.q, (static_cast<size_t>(n) * p.Hq + kv * p.G + g) * d + i, p.bf16) - mi;
-    }
-    xi_s[threadIdx.x] = xi;
-    __syncthreads();
-    if (j < d) {
-      const long cnt = min(static_cast<long>(kGramThreads), M - m0);
-      for (long t = 0; t < cnt; ++t) {
-        const long m = m0 + t;
+  __shared__ double xi_s[kGT][kGT + 1];  // [row m][col i]
+  __shared__ double xj_s[kGT][kGT + 1];
+  const int tid = threadIdx.x;           // 128 threads: 8 x 16, each 4 x 2 outputs
+  const int ry = tid / 16, rx = tid % 16;
+  double acc[4][2] = {};
+  for (long m0 = 0; m0 < M; m0 += kGT) {
+    for (int e = tid; e < kGT * kGT; e += kGramThreads) {
+      const int mm = e / kGT, c = e % kGT;
+      const long m = m0 + mm;
+      double a = 0.0, bb = 0.0;
+      if (m < M) {
         const long n = m / p.G, g = m - n * p.G;
-        const double xj =
-            load_elem(p.q, (static_cast<size_t>(n) * p.Hq + kv * p.G + g) * d + j, p.bf16) - mj;
-        acc += xi_s[t] * xj;
+        const size_t row = (static_cast<size_t>(n) * p.Hq + kv * p.G + g) * d;
+        if (i0 + c < d)
+          a = load_elem(p.q, row + i0 + c, p.bf16) - (p.center ? mean[kv * d + i0 + c] : 0.0);
+        if (j0 + c < d)
+          bb = load_elem(p.q, row + j0 + c, p.bf16) - (p.center ? mean[kv * d + j0 + c] : 0.0);
       }
+      xi_s[mm][c] = a;
+      xj_s[mm][c] = bb;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int mm = 0; mm < kGT; ++mm) {
+      double xi[4], xj[2];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) xi[k] = xi_s[mm][ry * 4 + k];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) xj[k] = xj_s[mm][rx * 2 + k];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b2 = 0; b2 < 2; ++b2) acc[a][b2] = fma(xi[a], xj[b2], acc[a][b2]);
     }
     __syncthreads();
   }
-  if (j < d) p.gram[(static_cast<size_t>(kv) * d + i) * d + j] = acc / static_cast<double>(M);
+  double* C = p.gram + static_cast<size_t>(kv) * d * d;
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b2 = 0; b2 < 2; ++b2) {
+      const int i = i0 + ry * 4 + a, j = j0 + rx * 2 + b2;
+      if (i < d && j < d) {
+        const double v = acc[a][b2] / static_cast<double>(M);
+        C[static_cast<size_t>(i) * d + j] = v;
+        C[static_cast<size_t>(j) * d + i] = v;
+      }
+    }
 }
 
 // member at position pos of the round-robin schedule at step k (d players)
@@ -87,16 +119,16 @@ jacobi_kernel(const CalibrateParams p) {
   extern __shared__ double A[];                 // [d][d]
   double* cs = A + d * d;                       // [half] cosines
   double* sn = cs + half;                       // [half] sines
-  int* pp = reinterpret_cast<int*>(sn + half);  // [half]
-  int* qq = pp + half;                          // [half]
+  float* Vt = reinterpret_cast<float*>(sn + half);  // [d][d] row k = eigenvector k
+  int* pp = reinterpret_cast<int*>(Vt + d * d);     // [half]
+  int* qq = pp + half;                              // [half]
   __shared__ double red[kJacThreads / 32];
   __shared__ int stop;
-  double* Vt = p.vt + static_cast<size_t>(kv) * d * d;  // row k = eigenvector k
   const int tid = threadIdx.x;
 
   for (int i = tid; i < d * d; i += kJacThreads) {
     A[i] = p.gram[static_cast<size_t>(kv) * d * d + i];
-    Vt[i] = (i / d == i % d) ? 1.0 : 0.0;
+    Vt[i] = (i / d == i % d) ? 1.0f : 0.0f;
   }
   __syncthreads();
 
@@ -127,13 +159,19 @@ jacobi_kernel(const CalibrateParams p) {
     if (tid == 0) {
       double st = 0.0;
       for (int w = 0; w < kJacThreads / 32; ++w) st += red[w];
-      stop = (off_all <= 1e-28 * st) ? 1 : 0;
+      // off-diagonal norm below 1e-12 of the total: converged (the fp64 rounding
+      // floor of a d x d matrix lies near 1e-14 of it)
+      stop = (off_all <= 1e-24 * st) ? 1 : 0;
     }
     __syncthreads();
     if (stop) break;
 
     for (int step = 0; step < d - 1; ++step) {
       for (int i = tid; i < half; i += kJacThreads) {
+        if (step > 0) {  // the entries the previous step annihilated are exactly 0
+          A[pp[i] * d + qq[i]] = 0.0;
+          A[qq[i] * d + pp[i]] = 0.0;
+        }
         int a = rr_member(i, step, d), b = rr_member(d - 1 - i, step, d);
         if (a > b) { const int t = a; a = b; b = t; }
         pp[i] = a;
@@ -150,7 +188,8 @@ jacobi_kernel(const CalibrateParams p) {
         sn[i] = s;
       }
       __syncthreads();
-      // rows p, q  (A <- J^T A)
+      // rows p, q (A <- J^T A) and the eigenvector rows (V <- V J); the column
+      // index j runs fastest across threads, so a warp reads one contiguous row
       for (int w = tid; w < half * d; w += kJacThreads) {
         const int i = w / d, j = w - i * d;
         const int a = pp[i], b = qq[i];
@@ -158,27 +197,30 @@ jacobi_kernel(const CalibrateParams p) {
         const double ap = A[a * d + j], aq = A[b * d + j];
         A[a * d + j] = c * ap - s * aq;
         A[b * d + j] = s * ap + c * aq;
+        const float cf = static_cast<float>(c), sf = static_cast<float>(s);
+        const float vp = Vt[a * d + j], vq = Vt[b * d + j];
+        Vt[a * d + j] = cf * vp - sf * vq;
+        Vt[b * d + j] = sf * vp + cf * vq;
       }
       __syncthreads();
-      // columns p, q  (A <- A J) and the eigenvector rows (V <- V J)
+      // columns p, q (A <- A J); the pair index runs fastest across threads, so
+      // a warp touches distinct columns of one row rather than one column (a
+      // column walk strides d doubles and puts every lane on the same bank)
       for (int w = tid; w < half * d; w += kJacThreads) {
-        const int i = w / d, j = w - i * d;
+        const int j = w / half, i = w - j * half;
         const int a = pp[i], b = qq[i];
         const double c = cs[i], s = sn[i];
         const double ap = A[j * d + a], aq = A[j * d + b];
         A[j * d + a] = c * ap - s * aq;
         A[j * d + b] = s * ap + c * aq;
-        const double vp = Vt[a * d + j], vq = Vt[b * d + j];
-        Vt[a * d + j] = c * vp - s * vq;
-        Vt[b * d + j] = s * vp + c * vq;
-      }
-      __syncthreads();
-      for (int i = tid; i < half; i += kJacThreads) {
-        A[pp[i] * d + qq[i]] = 0.0;
-        A[qq[i] * d + pp[i]] = 0.0;
       }
       __syncthreads();
     }
+    for (int i = tid; i < half; i += kJacThreads) {
+      A[pp[i] * d + qq[i]] = 0.0;
+      A[qq[i] * d + pp[i]] = 0.0;
+    }
+    __syncthreads();
   }
 
   // rank of each eigenvalue (descending, lower index first on ties)
@@ -190,14 +232,14 @@ jacobi_kernel(const CalibrateParams p) {
       rank += (lj > lk) || (lj == lk && j < k);
     }
     if (rank < r) {
-      const double* v = Vt + static_cast<size_t>(k) * d;
+      const float* v = Vt + static_cast<size_t>(k) * d;
       int arg = 0;
-      double best = fabs(v[0]);
+      float best = fabsf(v[0]);
       for (int c = 1; c < d; ++c)
-        if (fabs(v[c]) > best) { best = fabs(v[c]); arg = c; }
-      const double sgn = v[arg] < 0.0 ? -1.0 : 1.0;
+        if (fabsf(v[c]) > best) { best = fabsf(v[c]); arg = c; }
+      const float sgn = v[arg] < 0.0f ? -1.0f : 1.0f;
       float* U = p.U + static_cast<size_t>(kv) * d * r;
-      for (int c = 0; c < d; ++c) U[c * r + rank] = static_cast<float>(sgn * v[c]);
+      for (int c = 0; c < d; ++c) U[c * r + rank] = sgn * v[c];
       if (p.eig) p.eig[kv * r + rank] = static_cast<float>(lk);
     }
   }
@@ -208,9 +250,10 @@ jacobi_kernel(const CalibrateParams p) {
 cudaError_t launch_calibrate(const CalibrateParams& p, cudaStream_t s) {
   double* mean = p.vt + static_cast<size_t>(p.Hkv) * p.d * p.d;
   if (p.center) mean_kernel<<<p.Hkv, 128, 0, s>>>(p, mean);
-  gram_kernel<<<dim3(p.d, p.Hkv), kGramThreads, 0, s>>>(p, mean);
+  const int tiles = (p.d + kGT - 1) / kGT;
+  gram_kernel<<<dim3(tiles * (tiles + 1) / 2, p.Hkv), kGramThreads, 0, s>>>(p, mean);
   const size_t smem = sizeof(double) * (static_cast<size_t>(p.d) * p.d + p.d) +
-                      sizeof(int) * p.d;
+                      sizeof(float) * static_cast<size_t>(p.d) * p.d + sizeof(int) * p.d;
   cudaError_t e = cudaFuncSetAttribute(jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

@@ -35,6 +35,16 @@ __device__ __forceinline__ void fma2(float& y0, float& y1, float u0, float u1, f
       : "f"(u0), "f"(u1), "f"(e));
 }
 
+// Packed fp32 FMA on 64-bit register pairs: y.lo = fma(u.lo, e.lo, y.lo),
+// y.hi = fma(u.hi, e.hi, y.hi), each correctly rounded like a scalar FMA.
+__device__ __forceinline__ void fma2_pk(uint64_t& y, uint64_t u, uint64_t e2) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(y) : "l"(u), "l"(e2));
+}
+__device__ __forceinline__ uint64_t dup2(float e) {
+  const uint64_t b = __float_as_uint(e);
+  return b | (b << 32);
+}
+
 // Base code B_b of one group of GS channels held by one thread: per-token,
 // per-group asymmetric 2-bit min/max code.  Returns the packed code bytes
 // (channel k of the group at bits 2(k%4) of byte k/4), the scale and minimum;

@@ -6,7 +6,7 @@
 // Same mathematics as decode_attn.cu's generic kernel; this one is built to stream
 // the packed cache at HBM speed:
 //
-//  * TMA pipeline.  One producer warp fills kStages shared-memory stages of 64
+//  * TMA pipeline.  One producer warp fills 3-4 shared-memory stages of 64
 //    tokens with 1-D bulk copies of the contiguous code / scale / side planes and
 //    a 3-D tensor copy (128-byte swizzle) of the bf16 value tile; four consumer
 //    warps each take 16 tokens of every stage.  mbarriers carry completion; every
@@ -48,7 +48,10 @@ namespace {
 constexpr int kCW = 4;                   // consumer warps
 constexpr int kTile = 16 * kCW;          // tokens per stage
 constexpr int kThreads = (kCW + 1) * 32; // + one producer warp
-constexpr int kStages = 4;
+// pipeline depth: 4 stages of 64 tokens, 3 for the two-N-tile variants (their
+// q fragments take the shared memory of the fourth) so that two CTAs fit per SM
+template <int NT>
+constexpr int kStagesFor = NT == 1 ? 4 : 3;
 constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at B200 clocks
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -78,16 +81,22 @@ struct Layout {
   static constexpr int kCodeTile = V2 ? 16 * D * 2 : 0;  // per consumer warp, bf16 codes
 };
 
+// the two-N-tile variants keep each thread's q B-operand fragments in shared
+// memory instead of 32 registers, so that two CTAs fit on an SM
+template <int NT>
+constexpr bool kBqInSmem = NT == 2;
+
 template <int D, int R, int NT, bool V2>
 constexpr size_t smem_bytes() {
   using L = Layout<D, R, V2>;
+  constexpr size_t bq_bytes = kBqInSmem<NT> ? size_t(kCW) * 32 * (D / 16) * NT * 8 : 0;
   // stages | per-warp value code tiles | q [GM][D] | group sums [GM][NG] |
   // sigma U^T q [GM][R] | U [D][R] | appended token's residual [D] and
   // projection [R] | barriers
-  return 1024 + size_t(kStages) * L::kStage + size_t(kCW) * L::kCodeTile +
+  return 1024 + size_t(kStagesFor<NT>) * L::kStage + size_t(kCW) * L::kCodeTile + bq_bytes +
          sizeof(float) * ((4 * NT) * (D + L::NG + (R > 0 ? R : 1)) + D * (R > 0 ? R : 1) + D +
                           (R > 0 ? R : 1)) +
-         16 * kStages + 32;
+         16 * kStagesFor<NT> + 32;
 }
 
 // ---------------------------------------------------------------- PTX helpers
@@ -224,7 +233,7 @@ __device__ __forceinline__ uint32_t bf16_part_pair(float a, float b, bool lo) {
 
 // ---------------------------------------------------------------- the kernel
 template <int D, int R, int NT, bool V2>
-__global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, 2)
 decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap) {
   using L = Layout<D, R, V2>;
   constexpr int NG = L::NG;
@@ -233,13 +242,16 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   constexpr int GM = 4 * NT;   // head slots
   constexpr int RR = R > 0 ? R : 1;
   constexpr int kCT = kCW * 32;  // consumer threads
+  constexpr int kStages = kStagesFor<NT>;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* ctiles = smem + size_t(kStages) * L::kStage;  // [kCW][16][D] bf16 value codes
-  float* q_s = reinterpret_cast<float*>(ctiles + size_t(kCW) * L::kCodeTile);  // [GM][D]
+  uint8_t* ctiles = smem + size_t(kStagesFor<NT>) * L::kStage;  // [kCW][16][D] bf16 value codes
+  uint2* bq_s = reinterpret_cast<uint2*>(ctiles + size_t(kCW) * L::kCodeTile);  // [KS][NT][128]
+  float* q_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bq_s) +
+                                        (kBqInSmem<NT> ? size_t(kCW) * 32 * KS * NT * 8 : 0));
   float* qsum_s = q_s + GM * D;                                               // [GM][NG]
   float* qt_s = qsum_s + GM * NG;                                             // [GM][RR]
   float* u_s = qt_s + GM * RR;                                                // [D][RR]
@@ -414,15 +426,21 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   // B operands of q . code: column n = g is head (g >> 1), fp16 high (g even) or
   // low (g odd) part; k-step ks = 2*grp + e, k-slots (2t, 2t+1) <-> channels
   // 32*grp + 8t + 4e + {0, 1}, (2t+8, 2t+9) <-> 32*grp + 8t + 4e + {2, 3}.
-  uint32_t bq[KS][NT][2];
+  uint32_t bq[kBqInSmem<NT> ? 1 : KS][NT][2];
 #pragma unroll
   for (int ks = 0; ks < KS; ++ks) {
     const int ch0 = 32 * (ks >> 1) + 8 * t + 4 * (ks & 1);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const float* qh = q_s + (4 * nt + (g >> 1)) * D + ch0;
-      bq[ks][nt][0] = half_part_pair(qh[0], qh[1], g & 1);
-      bq[ks][nt][1] = half_part_pair(qh[2], qh[3], g & 1);
+      const uint32_t b0 = half_part_pair(qh[0], qh[1], g & 1);
+      const uint32_t b1 = half_part_pair(qh[2], qh[3], g & 1);
+      if constexpr (kBqInSmem<NT>) {
+        bq_s[(ks * NT + nt) * kCT + tid] = make_uint2(b0, b1);
+      } else {
+        bq[ks][nt][0] = b0;
+        bq[ks][nt][1] = b1;
+      }
     }
   }
   uint32_t bz[NT][2];
@@ -532,7 +550,15 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       for (int e = 0; e < 2; ++e) {
         const uint32_t a[4] = {u0[2 * e], u1[2 * e], u0[2 * e + 1], u1[2 * e + 1]};
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_f16(acc[gg][nt], a, bq[2 * gg + e][nt]);
+        for (int nt = 0; nt < NT; ++nt) {
+          if constexpr (kBqInSmem<NT>) {
+            const uint2 bv = bq_s[((2 * gg + e) * NT + nt) * kCT + tid];
+            const uint32_t b[2] = {bv.x, bv.y};
+            mma_f16(acc[gg][nt], a, b);
+          } else {
+            mma_f16(acc[gg][nt], a, bq[2 * gg + e][nt]);
+          }
+        }
       }
     }
     float zs0 = 0.f, zs1 = 0.f;
