@@ -528,6 +528,47 @@ def fp64_peak_tflops(sm_count=148, mhz=1965.0):
     return sm_count * FP64_FMA_PER_SM_CLK * 2 * mhz * 1e6 / 1e12
 
 
+PAGE_SIZE = 256
+PLANE_ATTRS = ("k_codes", "k_scale", "k_min", "z_codes", "z_scale", "v", "v_codes", "v_scale",
+               "v_min")
+
+
+def paged_decode_row(torch, hq, w, q, U, cache, timed, hbm_row):
+    """Decode over the same cache held as PAGE_SIZE-token pages of a pool in a
+    shuffled order (block table a random permutation), timed like the
+    contiguous layout beside it."""
+    B, Hkv, T = w.B, w.Hkv, w.T
+    if cache.T_cap % PAGE_SIZE:
+        return None
+    P = cache.T_cap // PAGE_SIZE
+    gen = torch.Generator().manual_seed(0)
+    table = torch.randperm(B * P, generator=gen).to(torch.int32).view(B, P)
+    pc = hq.PagedHeadQCache(B, Hkv, w.d, w.r, PAGE_SIZE, B * P, P, vmode=cache.vmode,
+                            v_dtype=cache.v_dtype, block_table=table)
+    dst_idx = pc.block_table.reshape(-1).long()
+    for name in PLANE_ATTRS:
+        src = getattr(cache, name)
+        if src is None:
+            continue
+        tail = tuple(src.shape[3:])
+        pages = src.reshape((B, Hkv, P, PAGE_SIZE) + tail).transpose(1, 2)
+        getattr(pc, name)[dst_idx] = pages.reshape((B * P, Hkv, PAGE_SIZE) + tail)
+    ws_c = hq.decode_workspace(cache, w.Hq, T)
+    ws_p = hq.decode_workspace(pc, w.Hq, T)
+    out = torch.empty((B, w.Hq, w.d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, w.Hq), dtype=torch.float32, device=q.device)
+    ms_c = timed(lambda: hq.headq_decode_attn(cache, q, U, T=T, out=out, lse=lse, ws=ws_c), 20)
+    ms_p = timed(lambda: hq.headq_decode_attn(pc, q, U, T=T, out=out, lse=lse, ws=ws_p), 20)
+    hq.headq_workspace_status(ws_p)
+    splits, chunk, _, _ = hq.decode_plan(pc, w.Hq, T)
+    row = hbm_row(ms_p, B * Hkv * T * cache.nbytes_per_token(), page_size=PAGE_SIZE,
+                  contiguous_ms=ms_c, plan="%d splits of %d tokens" % (splits, chunk),
+                  note="headq_decode_attn over a shuffled page pool; contiguous_ms is the "
+                       "same call on the contiguous planes, timed the same way")
+    del pc
+    return row
+
+
 def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream):
     """The other rows of the path, timed with CUDA events, each against its roofline:
     the prefill cache write and the KL diagnostic against HBM bandwidth (bytes they
@@ -563,6 +604,7 @@ def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream):
     ws = hq.attn_kl_workspace(cache, w.Hq, T)
     ms = timed(lambda: hq.headq_attn_kl(cache, q, U, k_all, v_all, ws=ws), 3)
     rows["attn_kl"] = hbm_row(ms, kv_in + planes, note="reads the packed cache and full K,V")
+    rows["decode_paged"] = paged_decode_row(torch, hq, w, q, U, cache, timed, hbm_row)
     ms = timed(lambda: hq.headq_calibrate(q_cal, Hkv, w.r), 3)
     M = q_cal.shape[0] * w.G
     flops = 2.0 * Hkv * M * d * d

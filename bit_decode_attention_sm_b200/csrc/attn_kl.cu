@@ -107,11 +107,13 @@ attn_kl_split_kernel(const AttnKlParams p) {
 
   for (int t0 = t_begin; t0 < t_end; t0 += kTile) {
     const int nt = min(kTile, t_end - t0);
+    // the tile's cache rows are consecutive: chunks start at multiples of 64
+    const size_t crow0 = cache_row_read(p.c, b, kv, t0, tid == 0 ? p.err : nullptr);
     // per-token value distortion |v^_j - v_j|^2
     for (int j = tid; j < kTile; j += kThreads) {
       float n2 = 0.0f;
       if (j < nt) {
-        const size_t row = bk * p.c.T_cap + t0 + j;
+        const size_t row = crow0 + j;
         const size_t frow = bk * p.T + t0 + j;
         for (int c = 0; c < D; ++c) {
           const float dv = cached_value<D>(p, row, c) - load_elem(p.v_full, frow * D + c, p.kv_bf16);
@@ -125,7 +127,7 @@ attn_kl_split_kernel(const AttnKlParams p) {
       const int h = idx / kTile, j = idx - h * kTile;
       float s = -INFINITY, dl = 0.0f;
       if (j < nt) {
-        const size_t row = bk * p.c.T_cap + t0 + j;
+        const size_t row = crow0 + j;
         const size_t frow = bk * p.T + t0 + j;
         const float* qh = q_s + h * D;
         float sf = 0.0f, de = 0.0f;
@@ -187,7 +189,7 @@ attn_kl_split_kernel(const AttnKlParams p) {
         double acc = dov[k] * static_cast<double>(a_s[h]);
         const float* pw = s_s + h * kTile;
         for (int j = 0; j < nt; ++j) {
-          const size_t row = bk * p.c.T_cap + t0 + j;
+          const size_t row = crow0 + j;
           const size_t frow = bk * p.T + t0 + j;
           const float dv = cached_value<D>(p, row, c) - load_elem(p.v_full, frow * D + c, p.kv_bf16);
           acc += static_cast<double>(pw[j]) * dv;
@@ -387,7 +389,8 @@ attn_kl_staged_kernel(const AttnKlParams p) {
     const int t0 = t_begin + i * kSTT;
     const int nv = min(kSTT, t_end - t0);
     uint8_t* st = stg[i & 1];
-    const size_t frow0 = bk * p.T + t0, crow0 = bk * p.c.T_cap + t0;
+    const size_t frow0 = bk * p.T + t0;
+    const size_t crow0 = cache_row_read(p.c, b, kv, t0, tid == 0 ? p.err : nullptr);
     stage_rows(st + L.kf, L.frow, static_cast<const uint8_t*>(p.k_full) + frow0 * D * esz,
                D * esz, nv, tid);
     stage_rows(st + L.vf, L.frow, static_cast<const uint8_t*>(p.v_full) + frow0 * D * esz,
@@ -521,8 +524,9 @@ attn_kl_staged_kernel(const AttnKlParams p) {
           }
         }
         if (r > 0) {
-          const uint8_t* zr = p.c.z_codes + (bk * p.c.T_cap + t0 + tt) * (r / 2);
-          if ((kSTT * (r / 2)) % 16 == 0) zr = st + L.zc + tt * (r / 2);
+          const uint8_t* zr = (kSTT * (r / 2)) % 16 == 0
+                                  ? st + L.zc + tt * (r / 2)
+                                  : p.c.z_codes + (cache_row_read(p.c, b, kv, t0, nullptr) + tt) * (r / 2);
           float cz = 0.0f;
           for (int ii = 0; ii < r; ++ii)
             cz = fmaf(qt_s[h * r + ii], static_cast<float>(nibble(zr, ii)), cz);

@@ -54,7 +54,9 @@ cache_write_kernel(const CacheWriteParams p) {
     const int t = tile0 + tt;
     if (t >= p.n) continue;
     const size_t in_off = (bk * p.n + t) * D + g * GS;
-    const size_t row = bk * p.c.T_cap + t0 + t;
+    const long long row_s = cache_row(p.c, b, kv, t0 + t);
+    if (row_s < 0) continue;  // block-table entry outside the pool: not written
+    const size_t row = static_cast<size_t>(row_s);
     float x[GS], vv[GS];
     codec::load_row<GS>(p.k, in_off, p.in_bf16, x);
     if (p.v != nullptr) codec::load_row<GS>(p.v, in_off, p.in_bf16, vv);
@@ -133,7 +135,9 @@ cache_write_kernel(const CacheWriteParams p) {
     const float rs = __frcp_rn(s);
     const int w0 = codec::side_level(y[i], s, rs);
     const int w1 = codec::side_level(y[i + 1], s, rs);
-    const size_t row = bk * p.c.T_cap + t0 + tile0 + tt;
+    const long long row_s = cache_row(p.c, b, kv, t0 + tile0 + tt);
+    if (row_s < 0) continue;
+    const size_t row = static_cast<size_t>(row_s);
     p.c.z_codes[row * (r / 2) + (i >> 1)] = static_cast<uint8_t>((w0 & 0xF) | ((w1 & 0xF) << 4));
     if (i == 0) p.c.z_scale[row] = s;
   }

@@ -10,15 +10,17 @@
 // subspace that captures the most score error.
 //
 //   gram kernel    C in fp64, one CTA per (32x32 tile pair, kv), the query rows
-//                  staged through shared memory 32 at a time
+//                  staged through shared memory 32 at a time, the next 32 rows
+//                  loaded into registers during the current slab's products
 //   jacobi kernel  one CTA per kv: cyclic two-sided Jacobi rotations on the
 //                  fp64 matrix in shared memory (Jacobi's method; rotation angle
 //                  as in Golub & Van Loan, "Matrix Computations", symmetric Schur
 //                  decomposition), the d/2 disjoint pairs of each step from the
-//                  round-robin ("circle") schedule applied in parallel, the
-//                  rotations accumulated in fp32 rows of eigenvectors, also in
-//                  shared memory; then the r largest eigenvalues, descending, and
-//                  a sign rule per vector.
+//                  round-robin ("circle") schedule applied in parallel (one warp
+//                  per pair for the row pass, one lane per pair for the column
+//                  pass, two barriers per step), the rotations accumulated in
+//                  fp32 rows of eigenvectors, also in shared memory; then the r
+//                  largest eigenvalues, descending, and a sign rule per vector.
 #include <math.h>
 
 #include "headq_internal.cuh"
@@ -28,26 +30,29 @@ namespace {
 
 constexpr int kGramThreads = 128;
 constexpr int kJacThreads = 512;
+constexpr int kJacWarps = kJacThreads / 32;
+constexpr int kJacPairsPerWarp = (128 / 2 + kJacWarps - 1) / kJacWarps;  // d <= 128
 constexpr int kMaxSweeps = 40;
 
 __global__ void mean_kernel(const CalibrateParams p, double* mean) {
   const int kv = blockIdx.x;
   const int d = p.d;
-  const long M = static_cast<long>(p.N) * p.G;
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     double acc = 0.0;
-    for (long m = 0; m < M; ++m) {
-      const long n = m / p.G, g = m - n * p.G;
-      acc += load_elem(p.q, (static_cast<size_t>(n) * p.Hq + kv * p.G + g) * d + c, p.bf16);
-    }
-    mean[kv * d + c] = acc / static_cast<double>(M);
+    for (int n = 0; n < p.N; ++n)
+      for (int g = 0; g < p.G; ++g)
+        acc += load_elem(p.q, (static_cast<size_t>(n) * p.Hq + kv * p.G + g) * d + c, p.bf16);
+    mean[kv * d + c] = acc / (static_cast<double>(p.N) * p.G);
   }
 }
 
-constexpr int kGT = 32;  // Gram tile edge
+constexpr int kGT = 32;                        // Gram tile edge
+constexpr int kGPer = kGT * kGT / kGramThreads;  // tile elements each thread stages
 
 // C tile (i0.., j0..) of kv head: sum over the M = N*G query rows, j0 >= i0;
-// the mirrored tile is written too.
+// the mirrored tile is written too.  Each thread stages the same column c of
+// rows mm0 + 4k of every 32-row slab; the next slab is loaded into registers
+// while the current one is multiplied.
 __global__ void __launch_bounds__(kGramThreads)
 gram_kernel(const CalibrateParams p, const double* mean) {
   const int kv = blockIdx.y;
@@ -56,29 +61,40 @@ gram_kernel(const CalibrateParams p, const double* mean) {
   while (tj >= tiles - ti) { tj -= tiles - ti; ++ti; }
   tj += ti;
   const int i0 = ti * kGT, j0 = tj * kGT;
-  const long M = static_cast<long>(p.N) * p.G;
+  const int M = p.N * p.G;
   __shared__ double xi_s[kGT][kGT + 1];  // [row m][col i]
   __shared__ double xj_s[kGT][kGT + 1];
   const int tid = threadIdx.x;           // 128 threads: 8 x 16, each 4 x 2 outputs
   const int ry = tid / 16, rx = tid % 16;
-  double acc[4][2] = {};
-  for (long m0 = 0; m0 < M; m0 += kGT) {
-    for (int e = tid; e < kGT * kGT; e += kGramThreads) {
-      const int mm = e / kGT, c = e % kGT;
-      const long m = m0 + mm;
-      double a = 0.0, bb = 0.0;
+  const int c = tid % kGT, mm0 = tid / kGT;
+  const bool ci = i0 + c < d, cj = j0 + c < d;
+  const double mi = (p.center && ci) ? mean[kv * d + i0 + c] : 0.0;
+  const double mj = (p.center && cj) ? mean[kv * d + j0 + c] : 0.0;
+  double va[kGPer], vb[kGPer];
+  auto load = [&](int m0) {
+#pragma unroll
+    for (int k = 0; k < kGPer; ++k) {
+      const int m = m0 + mm0 + 4 * k;
+      va[k] = 0.0;
+      vb[k] = 0.0;
       if (m < M) {
-        const long n = m / p.G, g = m - n * p.G;
+        const int n = m / p.G, g = m - n * p.G;
         const size_t row = (static_cast<size_t>(n) * p.Hq + kv * p.G + g) * d;
-        if (i0 + c < d)
-          a = load_elem(p.q, row + i0 + c, p.bf16) - (p.center ? mean[kv * d + i0 + c] : 0.0);
-        if (j0 + c < d)
-          bb = load_elem(p.q, row + j0 + c, p.bf16) - (p.center ? mean[kv * d + j0 + c] : 0.0);
+        if (ci) va[k] = load_elem(p.q, row + i0 + c, p.bf16) - mi;
+        if (cj) vb[k] = load_elem(p.q, row + j0 + c, p.bf16) - mj;
       }
-      xi_s[mm][c] = a;
-      xj_s[mm][c] = bb;
+    }
+  };
+  double acc[4][2] = {};
+  load(0);
+  for (int m0 = 0; m0 < M; m0 += kGT) {
+#pragma unroll
+    for (int k = 0; k < kGPer; ++k) {
+      xi_s[mm0 + 4 * k][c] = va[k];
+      xj_s[mm0 + 4 * k][c] = vb[k];
     }
     __syncthreads();
+    if (m0 + kGT < M) load(m0 + kGT);
 #pragma unroll 4
     for (int mm = 0; mm < kGT; ++mm) {
       double xi[4], xj[2];
@@ -124,7 +140,7 @@ jacobi_kernel(const CalibrateParams p) {
   int* qq = pp + half;                              // [half]
   __shared__ double red[kJacThreads / 32];
   __shared__ int stop;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
 
   for (int i = tid; i < d * d; i += kJacThreads) {
     A[i] = p.gram[static_cast<size_t>(kv) * d * d + i];
@@ -167,60 +183,65 @@ jacobi_kernel(const CalibrateParams p) {
     if (stop) break;
 
     for (int step = 0; step < d - 1; ++step) {
-      for (int i = tid; i < half; i += kJacThreads) {
-        if (step > 0) {  // the entries the previous step annihilated are exactly 0
-          A[pp[i] * d + qq[i]] = 0.0;
-          A[qq[i] * d + pp[i]] = 0.0;
-        }
-        int a = rr_member(i, step, d), b = rr_member(d - 1 - i, step, d);
-        if (a > b) { const int t = a; a = b; b = t; }
-        pp[i] = a;
-        qq[i] = b;
-        const double apq = A[a * d + b];
-        double c = 1.0, s = 0.0;
+      // rows p, q (A <- J^T A) and the eigenvector rows (V <- V J).  The warp
+      // that owns a pair also forms its rotation: only that warp writes rows p
+      // and q in this pass, so the three entries the angle needs are still the
+      // ones the previous step left.  Pair i belongs to warp i % kJacWarps.
+      // Lane k of a warp forms the rotation of the warp's k-th pair; then the
+      // warp rotates its pairs' rows one pair at a time, the lanes along j.
+      int a_l = 0, b_l = 0;
+      double c_l = 1.0, s_l = 0.0;
+      if (lane < kJacPairsPerWarp && warp + kJacWarps * lane < half) {
+        const int i = warp + kJacWarps * lane;
+        a_l = rr_member(i, step, d);
+        b_l = rr_member(d - 1 - i, step, d);
+        if (a_l > b_l) { const int t = a_l; a_l = b_l; b_l = t; }
+        const double apq = A[a_l * d + b_l];
         if (apq != 0.0) {
-          const double tau = (A[b * d + b] - A[a * d + a]) / (2.0 * apq);
+          const double tau = (A[b_l * d + b_l] - A[a_l * d + a_l]) / (2.0 * apq);
           const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
-          c = 1.0 / sqrt(1.0 + t * t);
-          s = t * c;
+          c_l = 1.0 / sqrt(1.0 + t * t);
+          s_l = t * c_l;
         }
-        cs[i] = c;
-        sn[i] = s;
+        pp[i] = a_l;
+        qq[i] = b_l;
+        cs[i] = c_l;
+        sn[i] = s_l;
       }
-      __syncthreads();
-      // rows p, q (A <- J^T A) and the eigenvector rows (V <- V J); the column
-      // index j runs fastest across threads, so a warp reads one contiguous row
-      for (int w = tid; w < half * d; w += kJacThreads) {
-        const int i = w / d, j = w - i * d;
-        const int a = pp[i], b = qq[i];
-        const double c = cs[i], s = sn[i];
-        const double ap = A[a * d + j], aq = A[b * d + j];
-        A[a * d + j] = c * ap - s * aq;
-        A[b * d + j] = s * ap + c * aq;
+      __syncwarp();  // the pivot entries are read before any row is written
+#pragma unroll
+      for (int k = 0; k < kJacPairsPerWarp; ++k) {
+        if (warp + kJacWarps * k >= half) break;
+        const int a = __shfl_sync(0xffffffffu, a_l, k), b = __shfl_sync(0xffffffffu, b_l, k);
+        const double c = __shfl_sync(0xffffffffu, c_l, k), s = __shfl_sync(0xffffffffu, s_l, k);
         const float cf = static_cast<float>(c), sf = static_cast<float>(s);
-        const float vp = Vt[a * d + j], vq = Vt[b * d + j];
-        Vt[a * d + j] = cf * vp - sf * vq;
-        Vt[b * d + j] = sf * vp + cf * vq;
+        for (int j = lane; j < d; j += 32) {
+          const double ap = A[a * d + j], aq = A[b * d + j];
+          A[a * d + j] = c * ap - s * aq;
+          A[b * d + j] = s * ap + c * aq;
+          const float vp = Vt[a * d + j], vq = Vt[b * d + j];
+          Vt[a * d + j] = cf * vp - sf * vq;
+          Vt[b * d + j] = sf * vp + cf * vq;
+        }
       }
       __syncthreads();
-      // columns p, q (A <- A J); the pair index runs fastest across threads, so
-      // a warp touches distinct columns of one row rather than one column (a
-      // column walk strides d doubles and puts every lane on the same bank)
-      for (int w = tid; w < half * d; w += kJacThreads) {
-        const int j = w / half, i = w - j * half;
+      // columns p, q (A <- A J).  The pair index runs across lanes, so a warp
+      // touches distinct columns of one row (a column walk strides d doubles and
+      // puts every lane on one bank).  The pivot entries A[p][q] = A[q][p] are
+      // set to exactly 0, the value the rotation annihilates them to.
+      for (int i0 = 0; i0 < half; i0 += 32) {
+        const int i = i0 + lane;
+        if (i >= half) break;
         const int a = pp[i], b = qq[i];
         const double c = cs[i], s = sn[i];
-        const double ap = A[j * d + a], aq = A[j * d + b];
-        A[j * d + a] = c * ap - s * aq;
-        A[j * d + b] = s * ap + c * aq;
+        for (int j = warp; j < d; j += kJacWarps) {
+          const double ap = A[j * d + a], aq = A[j * d + b];
+          A[j * d + a] = j == b ? 0.0 : c * ap - s * aq;
+          A[j * d + b] = j == a ? 0.0 : s * ap + c * aq;
+        }
       }
       __syncthreads();
     }
-    for (int i = tid; i < half; i += kJacThreads) {
-      A[pp[i] * d + qq[i]] = 0.0;
-      A[qq[i] * d + pp[i]] = 0.0;
-    }
-    __syncthreads();
   }
 
   // rank of each eigenvalue (descending, lower index first on ties)

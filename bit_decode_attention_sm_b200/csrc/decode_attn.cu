@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(kThreads)
 decode_split_kernel(const DecodeParams p) {
   constexpr int NG = num_groups(D);
   constexpr int GS = group_size(D);
-  const int G = p.G, r = p.c.r, Hkv = p.c.Hkv;
+  const int G = p.G, r = p.c.r;
   extern __shared__ float sm[];
   float* q_s = sm;                // [G][D]
   float* qg_s = q_s + G * D;      // [G][NG]   group sums of q
@@ -71,7 +71,6 @@ decode_split_kernel(const DecodeParams p) {
   if (p.seq_lens) Tb = max(0, min(p.seq_lens[b], p.T));
   const int t_begin = split * p.chunk;
   const int t_end = min(Tb, t_begin + p.chunk);
-  const size_t bk = static_cast<size_t>(b) * Hkv + kv;
   const int h0 = kv * G;
 
   for (int i = tid; i < G * D; i += kThreads)
@@ -102,12 +101,14 @@ decode_split_kernel(const DecodeParams p) {
 
   for (int t0 = t_begin; t0 < t_end; t0 += kTile) {
     const int nt = min(kTile, t_end - t0);
+    // the tile's rows are consecutive: chunks start at multiples of 64 tokens
+    const size_t row0 = cache_row_read(p.c, b, kv, t0, tid == 0 ? p.err : nullptr);
     // phase 1: logits of (head, token) pairs
     for (int idx = tid; idx < G * kTile; idx += kThreads) {
       const int h = idx / kTile, j = idx - h * kTile;
       float s = -INFINITY;
       if (j < nt) {
-        const size_t row = bk * p.c.T_cap + t0 + j;
+        const size_t row = row0 + j;
         const uint8_t* cr = p.c.k_codes + row * (D / 4);
         const float* qh = q_s + h * D;
         float acc = 0.0f;
@@ -156,7 +157,7 @@ decode_split_kernel(const DecodeParams p) {
         float acc = o[k] * a_s[h];
         const float* pw = s_s + h * kTile;
         for (int j = 0; j < nt; ++j)
-          acc = fmaf(pw[j], value_at<D>(p, bk * p.c.T_cap + t0 + j, c), acc);
+          acc = fmaf(pw[j], value_at<D>(p, row0 + j, c), acc);
         o[k] = acc;
       }
     }
@@ -275,15 +276,17 @@ DecodePlan decode_plan(const headq_cache& c, int Hq, int T) {
   if (T <= 0 || units <= 0) return dp;
   const int occ = mma_decode_supported(c, G) ? mma_decode_ctas_per_sm(c, G) : 0;
   if (occ > 0) {
-    // one wave: every CTA resident, each streaming one contiguous chunk of a
-    // multiple of 16 tokens (so every bulk copy stays 16-byte aligned); the last
-    // CTA of each (b, kv) merges the splits, so one kernel per call
+    // one wave: every CTA resident, each streaming one contiguous chunk; the
+    // last CTA of each (b, kv) merges the splits, so one kernel per call
     int s = (occ * sm_count()) / units;
     const int max_s = (T + 63) / 64;
     s = s < 1 ? 1 : (s > max_s ? max_s : s);
     if (s > kMaxMmaSplits) s = kMaxMmaSplits;
+    // a multiple of 16 tokens (so every bulk copy stays 16-byte aligned); of
+    // 64 for a paged cache, so that no 64-token tile straddles two pages
+    const int align = c.page_size > 0 ? 64 : 16;
     int chunk = (T + s - 1) / s;
-    chunk = (chunk + 15) / 16 * 16;
+    chunk = (chunk + align - 1) / align * align;
     dp.chunk = chunk;
     dp.splits = (T + chunk - 1) / chunk;
     dp.mma = true;

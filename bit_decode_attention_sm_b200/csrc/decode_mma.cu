@@ -310,7 +310,8 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
         const uint32_t full = smem_addr(&bars[s]);
         mbar_expect_tx(full, L::kVBoxes * L::kVBox + n16 * L::kRowBytes);
         uint8_t* st = stages + size_t(s) * L::kStage;
-        const size_t row0 = bk * p.c.T_cap + t0;
+        const CacheSlab sl = cache_slab_read(p.c, b, kv, t0, p.err);
+        const size_t row0 = static_cast<size_t>(sl.slab) * slab_rows(p.c) + sl.off;
         bulk_g2s(smem_addr(st + L::kKc), p.c.k_codes + row0 * (D / 4), n16 * (D / 4), full);
         bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + row0 * NG, n16 * NG * 4, full);
         bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + row0 * NG, n16 * NG * 4, full);
@@ -325,7 +326,8 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
         } else {
 #pragma unroll
           for (int bx = 0; bx < L::kVBoxes; ++bx)
-            tma_3d(smem_addr(st + bx * L::kVBox), &vmap, bx * 64, t0, static_cast<int>(bk), full);
+            tma_3d(smem_addr(st + bx * L::kVBox), &vmap, bx * 64, sl.off, static_cast<int>(sl.slab),
+                   full);
         }
         ++issued;
       }
@@ -369,9 +371,13 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   if (owner && warp == 0) {
     // encode the new token exactly as the cache write does: lanes 0..NG-1 take
     // the key groups, NG..2NG-1 the value groups, lanes < R the side rows
-    const size_t row = bk * p.c.T_cap + pos;
+    const long long orow = cache_row(p.c, b, kv, pos);
+    if (orow < 0 && lane == 0 && p.err) atomicOr(p.err, kDevErrBadPage);
+    const size_t row = orow < 0 ? 0 : static_cast<size_t>(orow);
     const size_t in = bk * D;
-    if (lane < NG) {
+    if (orow < 0) {
+      // a block-table entry outside the pool: the token is not written
+    } else if (lane < NG) {
       float x[32];
       uint32_t packed[2];
       float sc, mn;
@@ -398,7 +404,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       }
     }
     __syncwarp();
-    if constexpr (R > 0) {
+    if (R > 0 && orow >= 0) {
       float y = 0.0f;
       if (lane < R)
         for (int c = 0; c < D; ++c) y = __fmaf_rn(u_s[c * R + lane], enew_s[c], y);
@@ -891,10 +897,12 @@ struct Variant {
     }
     EncodeTiled enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(p.c.T_cap),
-                                static_cast<cuuint64_t>(p.c.B) * p.c.Hkv};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
-                                   static_cast<cuuint64_t>(p.c.T_cap) * D * 2};
+    // [slab][row in slab][channel]: one slab per (b, kv), or per (page, kv)
+    const bool paged = p.c.page_size > 0;
+    const cuuint64_t rows = static_cast<cuuint64_t>(paged ? p.c.page_size : p.c.T_cap);
+    const cuuint64_t slabs = static_cast<cuuint64_t>(paged ? p.c.num_pages : p.c.B) * p.c.Hkv;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), rows, slabs};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, rows * D * 2};
     const cuuint32_t box[3] = {64, kTile, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     if (enc(&vmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.c.v, dims, strides, box, estr,

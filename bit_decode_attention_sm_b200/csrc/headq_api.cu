@@ -51,6 +51,14 @@ static headq_status check_cache(const headq_cache* c) {
   if (!supported_d(c->d)) return HEADQ_ERR_UNSUPPORTED;
   if (c->r % 2 != 0 || c->r > c->d || c->r > 32) return HEADQ_ERR_UNSUPPORTED;
   if (c->T_cap % 16 != 0) return HEADQ_ERR_UNSUPPORTED;
+  if (c->page_size < 0) return HEADQ_ERR_INVALID_ARG;
+  if (c->page_size > 0) {  // paged pools: whole 64-token tiles per page
+    if (c->page_size % 64 != 0) return HEADQ_ERR_UNSUPPORTED;
+    if (!c->block_table || !aligned16(c->block_table)) return HEADQ_ERR_INVALID_ARG;
+    if (c->num_pages <= 0 || c->max_pages <= 0) return HEADQ_ERR_INVALID_ARG;
+    if (static_cast<long long>(c->max_pages) * c->page_size != c->T_cap)
+      return HEADQ_ERR_INVALID_ARG;
+  }
   if (c->vmode != HEADQ_V_DENSE && c->vmode != HEADQ_V_2BIT) return HEADQ_ERR_INVALID_ARG;
   if (c->v_dtype != HEADQ_F32 && c->v_dtype != HEADQ_BF16) return HEADQ_ERR_INVALID_ARG;
   if (!c->k_codes || !c->k_scale || !c->k_min) return HEADQ_ERR_INVALID_ARG;
@@ -103,7 +111,7 @@ static size_t kl_ws(const headq_cache* c, int Hq, int T) {
 
 using namespace headq;
 
-HEADQ_API int headq_version(void) { return 100; }
+HEADQ_API int headq_version(void) { return 101; }
 
 HEADQ_API const char* headq_status_string(headq_status s) {
   switch (s) {

@@ -19,6 +19,7 @@ constexpr size_t kWsHeaderBytes = 256;
 constexpr int kMaxFusedUnits = 8192;
 constexpr size_t kWsCounterBytes = sizeof(unsigned) * kMaxFusedUnits;
 constexpr unsigned kDevErrWaitTimeout = 1u;
+constexpr unsigned kDevErrBadPage = 2u;  // a block-table entry outside the pool
 
 __host__ __device__ constexpr int group_size(int d) { return d < 32 ? d : 32; }
 __host__ __device__ constexpr int num_groups(int d) { return d / group_size(d); }
@@ -42,6 +43,53 @@ __device__ __forceinline__ int code2(const uint8_t* row, int c) {
 __device__ __forceinline__ int nibble(const uint8_t* row, int i) {
   int v = (row[i >> 1] >> (4 * (i & 1))) & 0xF;
   return v >= 8 ? v - 16 : v;
+}
+
+// Where token t of sequence b, KV head kv lives.  The planes are slabs of
+// slab_rows() consecutive rows: contiguous planes have one slab per (b, kv)
+// ([b][kv][t], slab b*Hkv + kv, offset t); a paged cache one per (page, kv)
+// ([page][kv][t % page_size], page from the block table).  slab < 0 when that
+// entry lies outside the pool.  The 64 tokens of a 64-aligned tile share one
+// page (page_size is a multiple of 64), so they occupy consecutive rows.
+struct CacheSlab {
+  long long slab;
+  int off;
+};
+
+__device__ __forceinline__ int slab_rows(const headq_cache& c) {
+  return c.page_size ? c.page_size : c.T_cap;
+}
+
+__device__ __forceinline__ CacheSlab cache_slab(const headq_cache& c, int b, int kv, int t) {
+  if (c.page_size == 0) return {static_cast<long long>(b) * c.Hkv + kv, t};
+  const int i = t / c.page_size;
+  const int pg = c.block_table[static_cast<size_t>(b) * c.max_pages + i];
+  if (pg < 0 || pg >= c.num_pages) return {-1, 0};
+  return {static_cast<long long>(pg) * c.Hkv + kv, t - i * c.page_size};
+}
+
+// plane row of the token, -1 when its block-table entry is outside the pool
+__device__ __forceinline__ long long cache_row(const headq_cache& c, int b, int kv, int t) {
+  const CacheSlab s = cache_slab(c, b, kv, t);
+  return s.slab < 0 ? -1 : s.slab * slab_rows(c) + s.off;
+}
+
+// cache_slab for a read: a bad entry reads slab 0 (always valid memory) and
+// raises kDevErrBadPage in the error word, when there is one
+__device__ __forceinline__ CacheSlab cache_slab_read(const headq_cache& c, int b, int kv, int t,
+                                                     unsigned* err) {
+  CacheSlab s = cache_slab(c, b, kv, t);
+  if (s.slab < 0) {
+    if (err) atomicOr(err, kDevErrBadPage);
+    s = {0, t % c.page_size};
+  }
+  return s;
+}
+
+__device__ __forceinline__ size_t cache_row_read(const headq_cache& c, int b, int kv, int t,
+                                                 unsigned* err) {
+  const CacheSlab s = cache_slab_read(c, b, kv, t, err);
+  return static_cast<size_t>(s.slab) * slab_rows(c) + s.off;
 }
 
 struct CacheWriteParams {

@@ -48,7 +48,9 @@ class CacheStruct(ctypes.Structure):
                 ("k_min", ctypes.c_void_p), ("z_codes", ctypes.c_void_p),
                 ("z_scale", ctypes.c_void_p), ("v", ctypes.c_void_p),
                 ("v_codes", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
-                ("v_min", ctypes.c_void_p)]
+                ("v_min", ctypes.c_void_p),
+                ("page_size", ctypes.c_int), ("num_pages", ctypes.c_int),
+                ("max_pages", ctypes.c_int), ("block_table", ctypes.c_void_p)]
 
 
 _lib = None
@@ -129,27 +131,34 @@ class HeadQCache:
     [B,Hkv,T_cap,d] (dense) or v_codes/v_scale/v_min (2-bit).
     """
 
+    page_size = num_pages = max_pages = 0
+    block_table = None
+
     def __init__(self, B, Hkv, T_cap, d, r, vmode="dense", v_dtype=torch.bfloat16,
                  device="cuda"):
         if T_cap % 16:
             raise ValueError("T_cap must be a multiple of 16")
         self.B, self.Hkv, self.T_cap, self.d, self.r = B, Hkv, T_cap, d, r
+        self._alloc((B, Hkv, T_cap), vmode, v_dtype, device)
+
+    def _alloc(self, lead, vmode, v_dtype, device):
+        d, r = self.d, self.r
         self.vmode = vmode
         self.v_dtype = v_dtype
         ng = d // min(32, d)
         u8, f32 = torch.uint8, torch.float32
-        self.k_codes = torch.zeros((B, Hkv, T_cap, d // 4), dtype=u8, device=device)
-        self.k_scale = torch.zeros((B, Hkv, T_cap, ng), dtype=f32, device=device)
-        self.k_min = torch.zeros((B, Hkv, T_cap, ng), dtype=f32, device=device)
-        self.z_codes = torch.zeros((B, Hkv, T_cap, max(r // 2, 1)), dtype=u8, device=device)
-        self.z_scale = torch.zeros((B, Hkv, T_cap), dtype=f32, device=device)
+        self.k_codes = torch.zeros(lead + (d // 4,), dtype=u8, device=device)
+        self.k_scale = torch.zeros(lead + (ng,), dtype=f32, device=device)
+        self.k_min = torch.zeros(lead + (ng,), dtype=f32, device=device)
+        self.z_codes = torch.zeros(lead + (max(r // 2, 1),), dtype=u8, device=device)
+        self.z_scale = torch.zeros(lead, dtype=f32, device=device)
         self.v = self.v_codes = self.v_scale = self.v_min = None
         if vmode == "dense":
-            self.v = torch.zeros((B, Hkv, T_cap, d), dtype=v_dtype, device=device)
+            self.v = torch.zeros(lead + (d,), dtype=v_dtype, device=device)
         elif vmode == "2bit":
-            self.v_codes = torch.zeros((B, Hkv, T_cap, d // 4), dtype=u8, device=device)
-            self.v_scale = torch.zeros((B, Hkv, T_cap, ng), dtype=f32, device=device)
-            self.v_min = torch.zeros((B, Hkv, T_cap, ng), dtype=f32, device=device)
+            self.v_codes = torch.zeros(lead + (d // 4,), dtype=u8, device=device)
+            self.v_scale = torch.zeros(lead + (ng,), dtype=f32, device=device)
+            self.v_min = torch.zeros(lead + (ng,), dtype=f32, device=device)
         else:
             raise ValueError("vmode is 'dense' or '2bit'")
 
@@ -188,7 +197,37 @@ class HeadQCache:
             s.v_codes = self.v_codes.data_ptr()
             s.v_scale = self.v_scale.data_ptr()
             s.v_min = self.v_min.data_ptr()
+        if self.page_size:
+            s.page_size, s.num_pages, s.max_pages = self.page_size, self.num_pages, self.max_pages
+            s.block_table = self.block_table.data_ptr()
         return s
+
+
+class PagedHeadQCache(HeadQCache):
+    """HeadQ cache planes held as pools of fixed-size pages (``headq_cache``
+    paged layout): every plane is [num_pages, Hkv, page_size, ...] and
+    ``block_table`` int32 [B, max_pages] names the pool page that holds tokens
+    [i*page_size, (i+1)*page_size) of sequence b.  page_size is a multiple of
+    64; a sequence holds up to T_cap = max_pages * page_size tokens.  The
+    default block table gives sequence b pages b*max_pages .. b*max_pages +
+    max_pages - 1 (it needs num_pages >= B * max_pages); any other table may be
+    assigned to ``block_table`` before a call."""
+
+    def __init__(self, B, Hkv, d, r, page_size, num_pages, max_pages, vmode="dense",
+                 v_dtype=torch.bfloat16, device="cuda", block_table=None):
+        if page_size <= 0 or page_size % 64:
+            raise ValueError("page_size must be a positive multiple of 64")
+        self.B, self.Hkv, self.d, self.r = B, Hkv, d, r
+        self.page_size, self.num_pages, self.max_pages = page_size, num_pages, max_pages
+        self.T_cap = max_pages * page_size
+        if block_table is None:
+            if num_pages < B * max_pages:
+                raise ValueError("the default block table needs B * max_pages pages")
+            block_table = torch.arange(B * max_pages, dtype=torch.int32).view(B, max_pages)
+        self.block_table = block_table.to(device=device, dtype=torch.int32).contiguous()
+        if tuple(self.block_table.shape) != (B, max_pages):
+            raise ValueError("block_table must be [B, max_pages]")
+        self._alloc((num_pages, Hkv, page_size), vmode, v_dtype, device)
 
 
 def headq_calibrate(q_cal, Hkv, r, center=False, stream=None):

@@ -69,7 +69,8 @@ typedef enum {
 
 /*
  * The packed HeadQ cache: structure-of-arrays planes in HBM, each indexed
- * [b][kv][t] with t < T_cap.  Planes (NG = d / min(32, d) groups per token):
+ * [b][kv][t] with t < T_cap (contiguous layout, page_size == 0; the paged
+ * layout is described below).  Planes (NG = d / min(32, d) groups per token):
  *   k_codes  uint8 [B, Hkv, T_cap, d/4]   2-bit base key code
  *   k_scale  fp32  [B, Hkv, T_cap, NG]    base-code scale per group
  *   k_min    fp32  [B, Hkv, T_cap, NG]    base-code minimum per group
@@ -78,6 +79,19 @@ typedef enum {
  *   v        v_dtype [B, Hkv, T_cap, d]   dense values   (vmode DENSE)
  *   v_codes/v_scale/v_min as k_codes/k_scale/k_min        (vmode 2BIT)
  * Pointers of planes the mode does not use may be NULL.
+ *
+ * Paged layout (page_size > 0), for serving loops that hand out cache memory in
+ * fixed pages.  Every plane is a pool of num_pages pages, indexed
+ * [page][kv][t % page_size] in place of [b][kv][t]:
+ *   k_codes  uint8 [num_pages, Hkv, page_size, d/4]   (and so on for each plane)
+ * block_table int32 [B, max_pages] (device) gives the pool page that holds
+ * tokens [i*page_size, (i+1)*page_size) of sequence b at block_table[b*max_pages+i];
+ * pages may be shared by no two (b, i) that are written.  page_size is a
+ * multiple of 64 and T_cap == max_pages * page_size is the capacity of one
+ * sequence.  Entries a call reaches must lie in [0, num_pages): a read of an
+ * entry outside that range is redirected to page 0 and sets the device error
+ * word (decode and diagnostic calls), a write to one is dropped.  With
+ * page_size == 0 the last four fields are ignored.
  */
 typedef struct {
     int B, Hkv, T_cap, d, r;
@@ -90,6 +104,10 @@ typedef struct {
     void *v;
     uint8_t *v_codes;
     float *v_scale, *v_min;
+    int page_size;               /* 0: contiguous planes; else tokens per page   */
+    int num_pages;               /* pages in each plane's pool (paged)           */
+    int max_pages;               /* block_table entries per sequence (paged)     */
+    const int32_t *block_table;  /* [B, max_pages] pool page of each logical page */
 } headq_cache;
 
 /* Library version as 10000*major + 100*minor + patch. */
@@ -245,7 +263,8 @@ size_t headq_attn_kl_workspace_bytes(const headq_cache *cache, int Hq, int T);
  * headq_workspace_status -- waits for `stream`, reads the device error word of a
  * decode / attn_kl workspace, clears it, and returns HEADQ_ERR_DEVICE if a
  * kernel that used the workspace gave up a bounded wait (it then wrote no
- * result), else HEADQ_OK.  Synchronous; call it off the hot path.
+ * result) or met a block-table entry outside the page pool (its result is
+ * then undefined), else HEADQ_OK.  Synchronous; call it off the hot path.
  */
 headq_status headq_workspace_status(void *ws, headq_stream_t stream);
 

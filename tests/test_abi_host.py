@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported(hq):
 
 def test_version_and_status_strings(hq):
     lib = hq.lib()
-    assert lib.headq_version() == 100
+    assert lib.headq_version() == 101
     for code in range(6):
         assert lib.headq_status_string(code)
     assert lib.headq_status_string(99) == b"unknown status"
@@ -119,6 +119,48 @@ def test_workspace_and_plan(hq):
     assert L.headq_attn_kl_workspace_bytes(ctypes.byref(cs), 32, 1024) >= 256
     assert L.headq_calibrate_workspace_bytes(1024, 32, 8, 128) >= 2 * 8 * 128 * 128 * 8
     assert L.headq_workspace_status(None, None) == 1
+
+
+def test_paged_cache_rejects(hq):
+    """Paged layout fields are checked before any launch."""
+    def paged(**over):
+        kw = dict(T_cap=1024, page_size=64, num_pages=40, max_pages=16, block_table=FAKE + 0x900000)
+        kw.update(over)
+        return make_cache(hq, **kw)
+    assert _write(hq, paged(page_size=48)) == 2
+    assert _write(hq, paged(page_size=-64)) == 1
+    assert _write(hq, paged(block_table=0)) == 1
+    assert _write(hq, paged(block_table=FAKE + 0x900004)) == 1
+    assert _write(hq, paged(num_pages=0)) == 1
+    assert _write(hq, paged(max_pages=0)) == 1
+    assert _write(hq, paged(max_pages=8)) == 1            # 8 * 64 != T_cap
+    assert _decode(hq, paged(page_size=96, max_pages=10, T_cap=960)) == 2
+    assert _write(hq, paged(), n=0) == 0                  # valid, and a no-op
+    # the tensor-core plan keeps every 64-token tile inside one page
+    cs = paged(B=1, Hkv=8, T_cap=131072, max_pages=2048, num_pages=2048)
+    sp, ch = ctypes.c_int(), ctypes.c_int()
+    hq.lib().headq_decode_plan(ctypes.byref(cs), 32, 131072, ctypes.byref(sp), ctypes.byref(ch),
+                               None)
+    assert ch.value % 64 == 0 and sp.value * ch.value >= 131072
+
+
+def test_paged_cache_struct_on_host(hq):
+    """PagedHeadQCache lays the planes out as page pools and passes its table."""
+    import torch
+    c = hq.PagedHeadQCache(2, 4, 128, 16, 128, 9, 3, device="cpu")
+    assert c.T_cap == 384 and tuple(c.k_codes.shape) == (9, 4, 128, 32)
+    assert tuple(c.z_scale.shape) == (9, 4, 128) and tuple(c.v.shape) == (9, 4, 128, 128)
+    assert c.block_table.tolist() == [[0, 1, 2], [3, 4, 5]]
+    s = c.struct()
+    assert (s.page_size, s.num_pages, s.max_pages, s.T_cap) == (128, 9, 3, 384)
+    assert s.block_table == c.block_table.data_ptr()
+    with pytest.raises(ValueError):
+        hq.PagedHeadQCache(2, 4, 128, 16, 100, 9, 3, device="cpu")
+    with pytest.raises(ValueError):
+        hq.PagedHeadQCache(4, 4, 128, 16, 128, 9, 3, device="cpu")   # pool too small
+    t = torch.tensor([[5, 0, 1], [2, 3, 4]], dtype=torch.int32)
+    c2 = hq.PagedHeadQCache(2, 4, 128, 16, 128, 9, 3, device="cpu", block_table=t)
+    assert c2.block_table.tolist() == t.tolist()
 
 
 def test_calibrate_rejects(hq):
