@@ -564,9 +564,45 @@ def paged_decode_row(torch, hq, w, q, U, cache, timed, hbm_row):
     row = hbm_row(ms_p, B * Hkv * T * cache.nbytes_per_token(), page_size=PAGE_SIZE,
                   contiguous_ms=ms_c, plan="%d splits of %d tokens" % (splits, chunk),
                   note="headq_decode_attn over a shuffled page pool; contiguous_ms is the "
-                       "same call on the contiguous planes, timed the same way")
+                       "same call on the contiguous planes, timed the same way (CUDA graph "
+                       "of 20 back-to-back calls)")
     del pc
     return row
+
+
+CP_WORLD = 8
+
+
+def cp_rank_row(torch, hq, w, q, U, cache, timed, hbm_row):
+    """One rank of a CP_WORLD-way split-T decode of this workload: the local
+    decode over its token range (the first range, as a cache holding T/CP_WORLD
+    tokens) and the merge of CP_WORLD exchanged partials.  The all-gather
+    between them crosses NVLink and is not part of this one-GPU measurement."""
+    from bit_decode_attention_sm_b200 import context_parallel as cp
+    B, Hq, d, T = w.B, w.Hq, w.d, w.T
+    t_lo, n = cp.shard_range(T, 0, CP_WORLD)
+    BH = B * Hq
+    stride = cp.part_stride(BH, d)
+    buf = torch.zeros(CP_WORLD * stride, dtype=torch.float32, device=q.device)
+    o = buf[:BH * d].view(B, Hq, d)
+    lse = buf[BH * d:BH * d + BH].view(B, Hq)
+    ws = hq.decode_workspace(cache, Hq, n)
+    hq.headq_decode_attn(cache, q, U, T=n, out=o, lse=lse, ws=ws)
+    for r in range(1, CP_WORLD):  # stand-in partials for the other ranks
+        buf[r * stride:(r + 1) * stride].copy_(buf[:stride])
+    out = torch.empty((BH, d), dtype=torch.float32, device=q.device)
+    lse_m = torch.empty(BH, dtype=torch.float32, device=q.device)
+    ms_dec = timed(lambda: hq.headq_decode_attn(cache, q, U, T=n, out=o, lse=lse, ws=ws), 20)
+    ms_merge = timed(lambda: hq.headq_merge_partials(buf, CP_WORLD, BH, d, stride, out=out,
+                                                     lse=lse_m), 20)
+    splits, chunk, _, _ = hq.decode_plan(cache, Hq, n)
+    return hbm_row(ms_dec + ms_merge, B * w.Hkv * n * cache.nbytes_per_token(), world=CP_WORLD,
+                   local_tokens=n, decode_ms=ms_dec, merge_ms=ms_merge,
+                   exchange_bytes_per_rank=4 * stride,
+                   plan="%d splits of %d tokens" % (splits, chunk),
+                   note="rank-local work of a split-T step: decode over T/world tokens, "
+                        "then headq_merge_partials, each from a CUDA graph of 20 calls; the "
+                        "all-gather is not measured on one GPU")
 
 
 def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream):
@@ -587,6 +623,27 @@ def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / reps
 
+    def gtimed(fn, reps=20, replays=10):
+        """Per-call time of fn from a CUDA graph of `reps` back-to-back calls
+        (no host launch cost between them); plain calls if capture fails."""
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(reps):
+                    fn()
+            g.replay()
+            torch.cuda.synchronize()
+            a, b = _events(torch)
+            a.record(stream)
+            for _ in range(replays):
+                g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            del g
+            return a.elapsed_time(b) / (replays * reps)
+        except Exception:
+            return timed(fn, reps)
+
     def hbm_row(ms, nbytes, **extra):
         gbs = nbytes / (ms * 1e-3) / 1e9
         return dict(ms=ms, algorithmic_bytes=nbytes,
@@ -604,7 +661,8 @@ def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream):
     ws = hq.attn_kl_workspace(cache, w.Hq, T)
     ms = timed(lambda: hq.headq_attn_kl(cache, q, U, k_all, v_all, ws=ws), 3)
     rows["attn_kl"] = hbm_row(ms, kv_in + planes, note="reads the packed cache and full K,V")
-    rows["decode_paged"] = paged_decode_row(torch, hq, w, q, U, cache, timed, hbm_row)
+    rows["decode_paged"] = paged_decode_row(torch, hq, w, q, U, cache, gtimed, hbm_row)
+    rows["context_parallel_rank"] = cp_rank_row(torch, hq, w, q, U, cache, gtimed, hbm_row)
     ms = timed(lambda: hq.headq_calibrate(q_cal, Hkv, w.r), 3)
     M = q_cal.shape[0] * w.G
     flops = 2.0 * Hkv * M * d * d

@@ -166,11 +166,11 @@ HEADQ_API headq_status headq_cache_write(const headq_cache* cache, const void* k
                                          const float* U, headq_stream_t stream) {
   headq_status st = check_cache(cache);
   if (st != HEADQ_OK) return st;
-  if (!k || !aligned16(k) || (v && !aligned16(v))) return HEADQ_ERR_INVALID_ARG;
   if (kv_dtype != HEADQ_F32 && kv_dtype != HEADQ_BF16) return HEADQ_ERR_INVALID_ARG;
   if (t0 < 0 || n < 0 || static_cast<long>(t0) + n > cache->T_cap) return HEADQ_ERR_INVALID_ARG;
+  if (n == 0 || cache->B == 0) return HEADQ_OK;  // nothing to read: k, v, U unused
+  if (!k || !aligned16(k) || (v && !aligned16(v))) return HEADQ_ERR_INVALID_ARG;
   if (cache->r > 0 && (!U || !aligned16(U))) return HEADQ_ERR_INVALID_ARG;
-  if (n == 0 || cache->B == 0) return HEADQ_OK;
   CacheWriteParams p{};
   p.c = *cache;
   p.k = k;

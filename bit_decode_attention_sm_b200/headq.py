@@ -30,7 +30,8 @@ EXPORTS = ("headq_version", "headq_status_string", "headq_calibrate",
            "headq_calibrate_workspace_bytes", "headq_cache_write", "headq_decode_attn",
            "headq_decode_workspace_bytes", "headq_decode_plan", "headq_attn_kl",
            "headq_attn_kl_workspace_bytes", "headq_workspace_status",
-           "headq_decode_attn_noalloc", "headq_decode_append")
+           "headq_decode_attn_noalloc", "headq_decode_append", "headq_shard_seq_lens",
+           "headq_merge_partials")
 
 
 class HeadQError(RuntimeError):
@@ -81,6 +82,8 @@ def lib():
             "headq_workspace_status": ([P, P], I),
             "headq_decode_attn_noalloc": ([CP, P, I, I, P, I, P, F, I, P, P, P], I),
             "headq_decode_append": ([CP, P, P, I, P, I, I, P, I, P, F, I, P, P, P, Z, P], I),
+            "headq_shard_seq_lens": ([P, I, I, I, I, P, P], I),
+            "headq_merge_partials": ([P, P, I, I, I, Z, P, P, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -352,6 +355,31 @@ def headq_attn_kl(cache, q, U, k_full, v_full, T=None, seq_lens=None, sm_scale=N
         _ptr(v_full), _dtype_code(k_full), _ptr(U), sm, int(corr_sign),
         *[_ptr(t) for t in res], _ptr(ws), ws.numel(), _stream(stream)))
     return tuple(res)
+
+
+def headq_shard_seq_lens(seq_lens, B, T, t_lo, n, out=None, device="cuda", stream=None):
+    """int32 [B] local lengths clamp(T_b - t_lo, 0, n) of a token range [t_lo, t_lo+n)."""
+    seq_lens = _cuda(seq_lens, "seq_lens")
+    dev = seq_lens.device if seq_lens is not None else device
+    out = torch.empty(B, dtype=torch.int32, device=dev) if out is None else out
+    _check("headq_shard_seq_lens", lib().headq_shard_seq_lens(
+        _ptr(seq_lens), int(B), int(T), int(t_lo), int(n), _ptr(out), _stream(stream)))
+    return out
+
+
+def headq_merge_partials(parts, S, BH, d, part_stride, out=None, lse=None, stream=None):
+    """Combine S partial decodes held in one fp32 buffer of S blocks of
+    part_stride floats, each [out (BH*d) | lse (BH) | padding]; returns
+    (out fp32 [BH, d], lse fp32 [BH])."""
+    parts = _cuda(parts, "parts")
+    if parts.dtype != torch.float32 or parts.numel() < S * part_stride:
+        raise ValueError("parts must be fp32 with S * part_stride elements")
+    out = torch.empty((BH, d), dtype=torch.float32, device=parts.device) if out is None else out
+    lse = torch.empty(BH, dtype=torch.float32, device=parts.device) if lse is None else lse
+    _check("headq_merge_partials", lib().headq_merge_partials(
+        _ptr(parts), ctypes.c_void_p(parts.data_ptr() + 4 * BH * d), int(S), int(BH), int(d),
+        int(part_stride), _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
 
 
 def headq_workspace_status(ws, stream=None):

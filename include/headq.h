@@ -146,7 +146,8 @@ size_t headq_calibrate_workspace_bytes(int N, int Hq, int Hkv, int d);
  *         the 2-bit base code (2BIT).  v may be NULL to leave V untouched.
  *   U     fp32 [Hkv, d, r] from headq_calibrate (ignored when r == 0).
  * Bit-exact with the arithmetic stated at the top of this header.
- * Requires 0 <= t0, 0 <= n, t0 + n <= T_cap.  n == 0 is a no-op.
+ * Requires 0 <= t0, 0 <= n, t0 + n <= T_cap.  n == 0 is a no-op (k, v and U
+ * are then not read and may be NULL).
  */
 headq_status headq_cache_write(const headq_cache *cache, const void *k, const void *v,
                                headq_dtype kv_dtype, int t0, int n, const float *U,
@@ -258,6 +259,39 @@ headq_status headq_attn_kl(const headq_cache *cache, const void *q, headq_dtype 
                            float *a2_vdist, float *dout2, void *ws, size_t ws_bytes,
                            headq_stream_t stream);
 size_t headq_attn_kl_workspace_bytes(const headq_cache *cache, int Hq, int T);
+
+/*
+ * Split-T across devices (context-parallel decode).  Each device holds a
+ * contiguous range [t_lo, t_lo + n) of every sequence's cached tokens, at local
+ * positions [0, n) of its own cache, and runs headq_decode_attn over it with
+ * the local lengths from headq_shard_seq_lens.  Its (out, lse) is a normalised
+ * partial; after an all-gather of the partials every device combines them with
+ * headq_merge_partials into the attention over all tokens.  This is the
+ * flash-decoding split merge across devices: HeadQ changes only the logits
+ * (summary section 3, step 3), so softmax over a union of token sets is
+ * recovered exactly from the parts' log-sum-exps.
+ *
+ * headq_shard_seq_lens -- out[b] = clamp(T_b - t_lo, 0, n), T_b = seq_lens[b]
+ * clamped to [0, T] (or T when seq_lens is NULL).  seq_lens, out: int32 [B].
+ */
+headq_status headq_shard_seq_lens(const int32_t *seq_lens, int B, int T, int t_lo, int n,
+                                  int32_t *out, headq_stream_t stream);
+
+/*
+ * headq_merge_partials -- combine S partial decode results of the same BH rows
+ * (BH = B * Hq).  Part s has its output at o_parts + s*part_stride, fp32
+ * [BH, d], and its log-sum-exp at lse_parts + s*part_stride, fp32 [BH] (one
+ * all-gathered buffer of [out | lse] blocks fits this directly); part_stride is
+ * in floats and a multiple of 4.  Per row:
+ *   M = max_s lse_s,  out = sum_s e^{lse_s - M} o_s / sum_s e^{lse_s - M},
+ *   lse = M + log sum_s e^{lse_s - M}
+ * A part with lse = -inf (no tokens) contributes nothing; a row no part covers
+ * gets out = 0, lse = -inf, as headq_decode_attn gives for T_b = 0.
+ *   out fp32 [BH, d]; lse fp32 [BH] (nullable).  Neither may alias a part.
+ */
+headq_status headq_merge_partials(const float *o_parts, const float *lse_parts, int S, int BH,
+                                  int d, size_t part_stride, float *out, float *lse,
+                                  headq_stream_t stream);
 
 /*
  * headq_workspace_status -- waits for `stream`, reads the device error word of a

@@ -264,6 +264,27 @@ def decode(q, planes, U, v=None, vmode="dense", sm_scale=None, sigma=1.0,
     return out, lse
 
 
+def merge_partials(outs, lses):
+    """Attention over the union of S disjoint token sets from the S partial
+    results: o_s is the softmax-weighted readout over set s and lse_s the
+    log-sum-exp of its logits, so the softmax over the union weighs part s by
+    exp(lse_s) (written relative to the largest lse).  A part with no tokens has
+    lse_s = -inf and weight 0; a row no part covers gets out = 0, lse = -inf.
+    outs [S, ..., d], lses [S, ...]; returns (out, lse) fp64."""
+    outs = np.asarray(outs, np.float64)
+    lses = np.asarray(lses, np.float64)
+    M = lses.max(axis=0)
+    covered = np.isfinite(M)
+    M0 = np.where(covered, M, 0.0)
+    w = np.where(np.isfinite(lses), np.exp(lses - M0), 0.0)
+    L = w.sum(axis=0)
+    L1 = np.where(L > 0, L, 1.0)
+    out = (w[..., None] * outs).sum(axis=0) / L1[..., None]
+    out = np.where(covered[..., None], out, 0.0)
+    lse = np.where(covered, M0 + np.log(L1), -np.inf)
+    return out, lse
+
+
 # --------------------------------------------------------------------------
 # Step 4: diagnostics (section 2 of the summary).
 # --------------------------------------------------------------------------

@@ -81,8 +81,9 @@ def test_cache_write_rejects(hq):
     assert _write(hq, make_cache(hq), U=0) == 1
     assert _write(hq, make_cache(hq), t0=1000, n=100) == 1
     assert _write(hq, make_cache(hq), t0=-1) == 1
-    # n == 0 is a no-op that launches nothing
+    # n == 0 is a no-op that launches nothing and reads no input pointer
     assert _write(hq, make_cache(hq), n=0) == 0
+    assert _write(hq, make_cache(hq), k=0, U=0, n=0) == 0
 
 
 def _decode(hq, cs, Hq=4, T=512, corr=1, ws_bytes=1 << 30, q=FAKE, out=FAKE, ws=FAKE):

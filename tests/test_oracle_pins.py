@@ -340,6 +340,43 @@ def test_empty_and_single_token_sequences():
     np.testing.assert_array_equal(out[1], np.repeat(v[1, :, 0], 2, axis=0).astype(np.float64))
 
 
+def test_merge_of_token_shards_equals_whole():
+    """Split-T: decoding disjoint token ranges separately and merging the
+    partials by their log-sum-exps equals one decode over all tokens (softmax
+    over a union of token sets); ranges a sequence never reaches contribute
+    nothing, and a sequence of length 0 stays out = 0, lse = -inf."""
+    k, v, q, U = _tiny_layer(d=32, T=100, Hkv=2, G=2, B=3, r=8, seed=21)
+    planes = oracle.cache_write(k, U)
+    seq_lens = np.array([100, 30, 0], np.int32)
+    whole, whole_lse = oracle.decode(q, planes, U, v=v, seq_lens=seq_lens)
+    bounds = [0, 17, 64, 100]
+    outs, lses = [], []
+    for lo, hi in zip(bounds[:-1], bounds[1:]):
+        sub = {n: a[:, :, lo:hi] for n, a in planes.items()}
+        loc = np.clip(seq_lens - lo, 0, hi - lo).astype(np.int32)
+        o, l_ = oracle.decode(q, sub, U, v=v[:, :, lo:hi], seq_lens=loc)
+        outs.append(o)
+        lses.append(l_)
+    assert np.isneginf(lses[2][1]).all() and all(np.isneginf(l_[2]).all() for l_ in lses)
+    out, lse = oracle.merge_partials(outs, lses)
+    np.testing.assert_allclose(out, whole, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse[:2], whole_lse[:2], rtol=1e-13)
+    assert (out[2] == 0).all() and np.isneginf(lse[2]).all()
+    # the order of the parts does not matter; one part is returned unchanged
+    out_r, lse_r = oracle.merge_partials(outs[::-1], lses[::-1])
+    np.testing.assert_allclose(out_r, out, rtol=1e-13, atol=1e-15)
+    o1, l1 = oracle.merge_partials(outs[:1], lses[:1])
+    np.testing.assert_allclose(o1, outs[0], rtol=1e-15, atol=0)
+    # library check: per-range SDPA merged equals SDPA over all tokens
+    khat = oracle.base_dequantize(planes["kc"], planes["ks"], planes["km"])
+    ref, ref_lse = _sdpa(q, khat, v, 1 / np.sqrt(32))
+    po, pl = zip(*[_sdpa(q, khat[:, :, lo:hi], v[:, :, lo:hi], 1 / np.sqrt(32))
+                   for lo, hi in zip(bounds[:-1], bounds[1:])])
+    mo, ml = oracle.merge_partials(np.stack(po), np.stack(pl))
+    np.testing.assert_allclose(mo, ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(ml, ref_lse, rtol=1e-12)
+
+
 def test_output_inside_value_bounding_box():
     k, v, q, U = _tiny_layer(d=64, T=100, Hkv=2, G=3, B=2, r=8, seed=13)
     planes = oracle.cache_write(k, U)
