@@ -470,7 +470,7 @@ def run_headq(args):
     # rows beside the step: calibration, the full prefill write, the KL diagnostic
     rows = None
     if not args.no_rows and rank == 0:
-        rows = measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, caches[0], dt, stream)
+        rows = measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, caches[0], dt, stream, L)
 
     if world > 1:
         barrier(dev)
@@ -605,7 +605,54 @@ def cp_rank_row(torch, hq, w, q, U, cache, timed, hbm_row):
                         "all-gather is not measured on one GPU")
 
 
-def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream):
+A2_OBS = 16        # observation queries per sequence
+A2_KEEP = 0.05     # fraction of each sequence's tokens whose values stay exact
+# fp32 FMA lanes per SM per clock (CUDA cores) on B200
+FP32_FMA_PER_SM_CLK = 128
+
+
+def a2_policy_row(torch, hq, w, q, U, cache, k_all, v_all, dt, L, timed, gtimed, hbm_row):
+    """The A^2 value policy on this workload: scores from A2_OBS observation
+    queries per sequence (two logit passes on CUDA cores, against the fp32 ALU
+    peak), the top-K selection with the copy of the kept values, and the decode
+    followed by the value fixup (against HBM, the cache plus the kept values)."""
+    B, Hq, Hkv, d, T = w.B, w.Hq, w.Hkv, w.d, w.T
+    qo = torch.from_numpy(synth.make_observation_queries(w, L, A2_OBS)).to(q.device).to(dt)
+    K = max(1, int(A2_KEEP * T))
+    ws = hq.a2_workspace(cache, A2_OBS, Hq, T)
+    scores = torch.empty((B, Hkv, T), dtype=torch.float32, device=q.device)
+    keep_idx = torch.empty((B, Hkv, K), dtype=torch.int32, device=q.device)
+    keep_v = torch.empty((B, Hkv, K, d), dtype=dt, device=q.device)
+    ms_sc = timed(lambda: hq.headq_a2_scores(cache, qo, k_all, v_all, ws=ws, out=scores), 3)
+    ms_sel = timed(lambda: hq.headq_a2_select(scores, K, v_all, keep_idx=keep_idx, keep_v=keep_v), 5)
+    hq.headq_workspace_status(ws)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    dws = hq.decode_workspace(cache, Hq, T)
+
+    def dec_fix():
+        hq.headq_decode_attn(cache, q, U, T=T, out=out, lse=lse, ws=dws)
+        hq.headq_a2_value_fixup(cache, q, U, keep_idx, keep_v, out, lse, T=T)
+
+    ms_dec = gtimed(lambda: hq.headq_decode_attn(cache, q, U, T=T, out=out, lse=lse, ws=dws))
+    ms_df = gtimed(dec_fix)
+    flops = 2 * 2.0 * B * Hq * A2_OBS * T * d   # two passes of the observation logits
+    sm_count = torch.cuda.get_device_properties(0).multi_processor_count
+    pk = sm_count * FP32_FMA_PER_SM_CLK * 2 * 1965e6 / 1e12
+    tf = flops / (ms_sc * 1e-3) / 1e12
+    keep_bytes = B * Hkv * K * (4 + d * keep_v.element_size())
+    row = hbm_row(ms_df, B * Hkv * T * cache.nbytes_per_token() + keep_bytes, kept_per_seq=K,
+                  observation_queries=A2_OBS, decode_ms=ms_dec, fixup_ms=ms_df - ms_dec,
+                  select_ms=ms_sel, note="ms = decode + value fixup (CUDA graph of 20); "
+                  "scores_roofline: the two observation-logit passes on CUDA cores")
+    row["scores_ms"] = ms_sc
+    row["scores_roofline"] = {"bound": "alu", "achieved": tf, "peak": pk, "unit": "TFLOP/s",
+                              "frac": tf / pk, "peak_kind": "fp32 CUDA cores from unit counts "
+                              "and max clock", "work": "2 passes x 2*B*Hq*n_obs*T*d flops"}
+    return row
+
+
+def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream, L):
     """The other rows of the path, timed with CUDA events, each against its roofline:
     the prefill cache write and the KL diagnostic against HBM bandwidth (bytes they
     must move), calibration against the fp64 ALU peak (its Gram matrix FLOPs)."""
@@ -663,6 +710,9 @@ def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream):
     rows["attn_kl"] = hbm_row(ms, kv_in + planes, note="reads the packed cache and full K,V")
     rows["decode_paged"] = paged_decode_row(torch, hq, w, q, U, cache, gtimed, hbm_row)
     rows["context_parallel_rank"] = cp_rank_row(torch, hq, w, q, U, cache, gtimed, hbm_row)
+    if w.vmode == "2bit":  # the policy chooses which 2-bit values to keep exact
+        rows["a2_policy"] = a2_policy_row(torch, hq, w, q, U, cache, k_all, v_all, dt, L, timed,
+                                          gtimed, hbm_row)
     ms = timed(lambda: hq.headq_calibrate(q_cal, Hkv, w.r), 3)
     M = q_cal.shape[0] * w.G
     flops = 2.0 * Hkv * M * d * d

@@ -1,0 +1,603 @@
+// A^2 value policy for the full-KV composition ("HeadQ: Model-Visible
+// Distortion and Score-Space Correction for KV-Cache Quantization"; abstract,
+// and the gist.science summary, section 2: under fixed attention the readout
+// error of value distortions dv_j has the A^2-weighted diagonal surrogate
+// D_V = sum_j p_j^2 |dv_j|^2, and value compression should put its precision
+// where that weight is large; section 5 composes HeadQ keys with 2-bit values
+// under an A^2 value policy, which the pages do not spell out).
+//
+// Policy as built here: with a budget of K tokens per (b, kv) whose values stay
+// exact (the input precision) and 2-bit codes for the rest, D_V (summed over a
+// set of observation queries and the G query heads of the KV head) loses the
+// term of every kept token, so the K tokens with the largest
+//   a_j = |v^_j - v_j|^2 * sum_{obs o, head h} p_{o,h,j}^2
+// minimise it exactly (top-K, ties to the lower position).  p is the attention
+// of the observation queries over the exact keys.
+//
+//   a2 pass kernel (x2)  pass 0: per 64-token tile, each observation query's
+//                        logit max and exp-sum (two halves per tile); lse
+//                        kernel merges them.  Pass 1: a_j per token.
+//   a2 select kernel     per (b, kv): radix select of the K-th largest a_j over
+//                        the 32-bit patterns (a_j >= 0, so the bit order is the
+//                        value order), ordered compaction of the kept positions
+//                        (ascending), and a copy of their exact values.
+//   a2 fixup kernel      after a decode: out += sum_{kept j < T_b}
+//                        exp(s^_j - lse) (v_j - v^_j), which turns the decode's
+//                        readout over v^_j into the readout over the mixed values
+//                        (same softmax weights; exact algebra).
+#include <math.h>
+
+#include "headq_internal.cuh"
+
+#define HEADQ_API extern "C" __attribute__((visibility("default")))
+
+namespace headq {
+namespace {
+
+constexpr int kAT = 64;          // tokens per score tile
+constexpr int kAThreads = 256;   // 64 tokens x 4 query lanes
+constexpr int kAQC = 16;         // observation queries staged per chunk
+constexpr int kSelThreads = 1024;
+constexpr int kFixThreads = 256;
+constexpr int kFixTok = 32;      // kept tokens per fixup step
+constexpr int kFixMaxOut = 2048 / kFixThreads;
+
+struct A2Params {
+  headq_cache c;
+  const void* q_obs;
+  bool q_bf16;
+  int n_obs, Hq, G, T;
+  const int32_t* seq_lens;
+  const void* k_full;
+  const void* v_full;
+  bool kv_bf16;
+  float sm_scale;
+  int ntiles;
+  float2* part;   // [B*Hkv, ntiles, 2, NQ] (max, exp-sum) per tile half
+  float* lse;     // [B*Hkv, NQ], query index o*G + g
+  float* scores;  // [B*Hkv, T]
+  unsigned* err;
+};
+
+__device__ __forceinline__ int seq_len(const int32_t* seq_lens, int b, int T) {
+  return seq_lens ? max(0, min(seq_lens[b], T)) : T;
+}
+
+// the cached (dequantised) value of channel c at plane row `row`
+__device__ __forceinline__ float value_hat(const headq_cache& c, size_t row, int ch, int d) {
+  if (c.vmode == HEADQ_V_2BIT) {
+    const int GS = d < 32 ? d : 32, NG = d / GS;
+    const int g = ch / GS;
+    const float mn = c.v_min[row * NG + g], sc = c.v_scale[row * NG + g];
+    return __fadd_rn(mn, __fmul_rn(static_cast<float>(code2(c.v_codes + row * (d / 4), ch)), sc));
+  }
+  return load_elem(c.v, row * d + ch, c.v_dtype == HEADQ_BF16);
+}
+
+// Pass 0 (SCORE false): tile partials of the softmax normaliser of each
+// observation query.  Pass 1 (SCORE true): a_j of each token of the tile.
+template <int D, bool SCORE>
+__global__ void __launch_bounds__(kAThreads) a2_pass_kernel(const A2Params p) {
+  extern __shared__ float sm[];
+  constexpr int KS = D + 4;             // key row stride: 16-byte rows, 8 rows per bank sweep
+  float* k_s = sm;                      // [kAT][KS]
+  float* q_s = k_s + kAT * KS;          // [kAQC][D]
+  float* red_s = q_s + kAQC * D;        // [kAThreads]
+  float* dv2_s = red_s + kAThreads;     // [kAT]
+
+  const int tile = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, j = tid % kAT, lane4 = tid / kAT;  // 4 query lanes
+  const int Tb = seq_len(p.seq_lens, b, p.T);
+  const int t0 = tile * kAT;
+  const int G = p.G, NQ = p.n_obs * G;
+  const size_t bk = static_cast<size_t>(b) * p.c.Hkv + kv;
+  const bool valid = t0 + j < Tb;
+
+  for (int e = tid; e < kAT * D; e += kAThreads) {
+    const int jj = e / D, ch = e - jj * D;
+    float x = 0.0f;
+    if (t0 + jj < Tb) x = load_elem(p.k_full, (bk * p.T + t0 + jj) * D + ch, p.kv_bf16);
+    k_s[jj * KS + ch] = x;
+  }
+  if constexpr (SCORE) {  // |v^_j - v_j|^2, channels split over the 4 lanes
+    float a = 0.0f;
+    if (valid) {
+      const size_t row = cache_row_read(p.c, b, kv, t0 + j, lane4 == 0 ? p.err : nullptr);
+      for (int ch = lane4 * (D / 4); ch < (lane4 + 1) * (D / 4); ++ch) {
+        const float dv = value_hat(p.c, row, ch, D) -
+                         load_elem(p.v_full, (bk * p.T + t0 + j) * D + ch, p.kv_bf16);
+        a = fmaf(dv, dv, a);
+      }
+    }
+    red_s[tid] = a;
+    __syncthreads();
+    if (tid < kAT) dv2_s[tid] = (red_s[tid] + red_s[tid + kAT]) + (red_s[tid + 2 * kAT] + red_s[tid + 3 * kAT]);
+  }
+
+  float acc2 = 0.0f;  // SCORE: sum of p^2 of token j over this lane's queries
+  for (int q0 = 0; q0 < NQ; q0 += kAQC) {
+    const int nq = min(kAQC, NQ - q0);
+    __syncthreads();
+    for (int e = tid; e < kAQC * D; e += kAThreads) {
+      const int qq = e / D, ch = e - qq * D;
+      float x = 0.0f;
+      if (qq < nq) {
+        const int qi = q0 + qq, o = qi / G, g = qi - o * G;
+        x = load_elem(p.q_obs, ((static_cast<size_t>(b) * p.n_obs + o) * p.Hq + kv * G + g) * D + ch,
+                      p.q_bf16);
+      }
+      q_s[e] = x;
+    }
+    __syncthreads();
+    // lane4 takes queries lane4, lane4 + 4, lane4 + 8, lane4 + 12 of the chunk
+    float s[kAQC / 4];
+#pragma unroll
+    for (int u = 0; u < kAQC / 4; ++u) s[u] = 0.0f;
+    // 128-bit loads: the 4 queries of a lane are the same for the whole warp
+    // (broadcast), the key rows differ by token (no bank conflict at stride KS)
+    const float4* kr = reinterpret_cast<const float4*>(k_s + j * KS);
+#pragma unroll 4
+    for (int c4 = 0; c4 < D / 4; ++c4) {
+      const float4 kc = kr[c4];
+#pragma unroll
+      for (int u = 0; u < kAQC / 4; ++u) {
+        const float4 qv = reinterpret_cast<const float4*>(q_s + (lane4 + 4 * u) * D)[c4];
+        s[u] = fmaf(qv.x, kc.x, s[u]);
+        s[u] = fmaf(qv.y, kc.y, s[u]);
+        s[u] = fmaf(qv.z, kc.z, s[u]);
+        s[u] = fmaf(qv.w, kc.w, s[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kAQC / 4; ++u) {
+      const int qq = lane4 + 4 * u;
+      if (qq >= nq) break;  // uniform across the warp (lane4 is per warp)
+      const float sv = valid ? s[u] * p.sm_scale : -INFINITY;
+      if constexpr (!SCORE) {
+        float m = sv;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o2));
+        float l = valid ? expf(sv - m) : 0.0f;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o2);
+        if ((tid & 31) == 0) {
+          const int half = (j >> 5);
+          p.part[((bk * p.ntiles + tile) * 2 + half) * NQ + q0 + qq] = make_float2(m, l);
+        }
+      } else {
+        const float pj = valid ? expf(sv - p.lse[bk * NQ + q0 + qq]) : 0.0f;
+        acc2 = fmaf(pj, pj, acc2);
+      }
+    }
+  }
+  if constexpr (SCORE) {
+    __syncthreads();
+    red_s[tid] = acc2;
+    __syncthreads();
+    if (tid < kAT && t0 + tid < p.T) {
+      const float w = (red_s[tid] + red_s[tid + kAT]) + (red_s[tid + 2 * kAT] + red_s[tid + 3 * kAT]);
+      p.scores[bk * p.T + t0 + tid] = t0 + tid < Tb ? w * dv2_s[tid] : 0.0f;
+    }
+  }
+}
+
+// lse of every observation query from the tile partials; one CTA per (b, kv)
+__global__ void a2_lse_kernel(const A2Params p) {
+  const size_t bk = blockIdx.x;
+  const int NQ = p.n_obs * p.G;
+  for (int qi = threadIdx.x; qi < NQ; qi += blockDim.x) {
+    float M = -INFINITY;
+    for (int e = 0; e < 2 * p.ntiles; ++e) M = fmaxf(M, p.part[(bk * p.ntiles * 2 + e) * NQ + qi].x);
+    float L = 0.0f;
+    if (M != -INFINITY)
+      for (int e = 0; e < 2 * p.ntiles; ++e) {
+        const float2 ml = p.part[(bk * p.ntiles * 2 + e) * NQ + qi];
+        if (ml.x != -INFINITY) L += ml.y * expf(ml.x - M);
+      }
+    p.lse[bk * NQ + qi] = M == -INFINITY ? -INFINITY : M + logf(L);
+  }
+}
+
+// exclusive prefix count of `flag` over the CTA (threads in order); returns it
+// and the CTA total through *total.  Uses wsum (kSelThreads / 32 entries).
+__device__ __forceinline__ int block_excl_count(bool flag, int* wsum, int* total) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, flag);
+  const int in_warp = __popc(bal & ((1u << lane) - 1u));
+  __syncthreads();
+  if (lane == 0) wsum[warp] = __popc(bal);
+  __syncthreads();
+  if (warp == 0) {
+    const int v = lane < kSelThreads / 32 ? wsum[lane] : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane < kSelThreads / 32) wsum[lane] = x - v;  // exclusive
+    if (lane == 31) wsum[kSelThreads / 32] = x;       // total
+  }
+  __syncthreads();
+  *total = wsum[kSelThreads / 32];
+  return wsum[warp] + in_warp;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+a2_select_kernel(const float* scores, int Hkv, const int32_t* seq_lens, int T, int K,
+                 const void* v_full, int esz, int d, int32_t* keep_idx, void* keep_v) {
+  __shared__ unsigned hist[256];
+  __shared__ unsigned s_pre;
+  __shared__ int s_rem;
+  __shared__ int wsum[kSelThreads / 32 + 1];
+  const size_t bk = blockIdx.x;
+  const int b = static_cast<int>(bk / Hkv);
+  const int tid = threadIdx.x;
+  const int Tb = seq_len(seq_lens, b, T);
+  const int Keff = min(K, Tb);
+  const unsigned* key = reinterpret_cast<const unsigned*>(scores + bk * T);
+  int32_t* out_idx = keep_idx + bk * K;
+
+  // radix select, 8 bits at a time from the top: s_pre ends as the bit pattern
+  // of the Keff-th largest score, s_rem as how many of the kept tokens equal it
+  if (tid == 0) {
+    s_pre = 0u;
+    s_rem = Keff;
+  }
+  unsigned mask = 0u;
+  for (int shift = 24; shift >= 0 && Keff > 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0u;
+    __syncthreads();
+    const unsigned pre = s_pre;
+    for (int t = tid; t < Tb; t += kSelThreads) {
+      const unsigned u = key[t];
+      if ((u & mask) == pre) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int rem = s_rem, bin = 255;
+      for (; bin > 0; --bin) {
+        const int h = static_cast<int>(hist[bin]);
+        if (h >= rem) break;
+        rem -= h;
+      }
+      s_rem = rem;
+      s_pre = pre | (static_cast<unsigned>(bin) << shift);
+    }
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  const unsigned tau = s_pre;
+  const int need_eq = s_rem;
+
+  // ordered compaction: every token above tau, and the first need_eq equal to it
+  int base = 0, eq_base = 0;
+  for (int t0 = 0; t0 < Tb && Keff > 0; t0 += kSelThreads) {
+    const int t = t0 + tid;
+    const unsigned u = t < Tb ? key[t] : 0u;
+    const bool eq = t < Tb && u == tau;
+    int eq_total = 0;
+    const int eq_rank = block_excl_count(eq, wsum, &eq_total);
+    const bool take = t < Tb && (u > tau || (eq && eq_base + eq_rank < need_eq));
+    int take_total = 0;
+    const int pos = block_excl_count(take, wsum, &take_total);
+    if (take && base + pos < Keff) out_idx[base + pos] = t;
+    base += take_total;
+    eq_base += eq_total;
+  }
+  for (int k = Keff + tid; k < K; k += kSelThreads) out_idx[k] = -1;
+  __syncthreads();
+
+  // exact values of the kept tokens (raw elements of v_full), zero for the pad
+  const int row_bytes = d * esz;
+  const uint8_t* vsrc = static_cast<const uint8_t*>(v_full);
+  uint8_t* vdst = static_cast<uint8_t*>(keep_v) + bk * K * row_bytes;
+  for (int e = tid; e < K * (row_bytes / 4); e += kSelThreads) {
+    const int k = e / (row_bytes / 4), w = e - k * (row_bytes / 4);
+    uint32_t x = 0u;
+    if (k < Keff) {
+      const int t = out_idx[k];
+      x = reinterpret_cast<const uint32_t*>(vsrc + (bk * T + t) * row_bytes)[w];
+    }
+    reinterpret_cast<uint32_t*>(vdst + static_cast<size_t>(k) * row_bytes)[w] = x;
+  }
+}
+
+struct FixParams {
+  headq_cache c;
+  const void* q;
+  bool q_bf16;
+  int Hq, G, T;
+  const int32_t* seq_lens;
+  const float* U;
+  float sm_scale, corr_sign;
+  const int32_t* keep_idx;
+  const void* keep_v;
+  bool keep_bf16;
+  int K;
+  float* out;
+  const float* lse;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p) {
+  constexpr int GS = group_size(D), NG = num_groups(D);
+  extern __shared__ float sm[];
+  const int G = p.G, r = p.c.r;
+  float* q_s = sm;                    // [G][D]
+  float* qg_s = q_s + G * D;          // [G][NG]
+  float* qt_s = qg_s + G * NG;        // [G][r]
+  float* lse_s = qt_s + G * r;        // [G]
+  float* p_s = lse_s + G;             // [kFixTok][G]
+  float* dv_s = p_s + kFixTok * G;    // [kFixTok][D]
+  int* idx_s = reinterpret_cast<int*>(dv_s + kFixTok * D);  // [kFixTok]
+
+  const int kv = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int h0 = kv * G;
+  const int Tb = seq_len(p.seq_lens, b, p.T);
+  if (Tb == 0) return;  // out = 0, lse = -inf: nothing to correct
+  const size_t bk = static_cast<size_t>(b) * p.c.Hkv + kv;
+
+  for (int i = tid; i < G * D; i += kFixThreads)
+    q_s[i] = load_elem(p.q, (static_cast<size_t>(b) * p.Hq + h0) * D + i, p.q_bf16);
+  for (int h = tid; h < G; h += kFixThreads) lse_s[h] = p.lse[static_cast<size_t>(b) * p.Hq + h0 + h];
+  __syncthreads();
+  for (int i = tid; i < G * NG; i += kFixThreads) {
+    const int h = i / NG, g = i - h * NG;
+    float acc = 0.0f;
+    for (int c = 0; c < GS; ++c) acc += q_s[h * D + g * GS + c];
+    qg_s[i] = acc;
+  }
+  for (int i = tid; i < G * r; i += kFixThreads) {
+    const int h = i / r, ii = i - h * r;
+    const float* U = p.U + static_cast<size_t>(kv) * D * r;
+    float acc = 0.0f;
+    for (int c = 0; c < D; ++c) acc = fmaf(U[c * r + ii], q_s[h * D + c], acc);
+    qt_s[i] = p.corr_sign * acc;
+  }
+
+  float acc[kFixMaxOut];
+#pragma unroll
+  for (int k = 0; k < kFixMaxOut; ++k) acc[k] = 0.0f;
+
+  for (int k0 = 0; k0 < p.K; k0 += kFixTok) {
+    __syncthreads();
+    if (tid < kFixTok) {
+      const int t = k0 + tid < p.K ? p.keep_idx[bk * p.K + k0 + tid] : -1;
+      idx_s[tid] = (t >= 0 && t < Tb) ? t : -1;
+    }
+    __syncthreads();
+    // weights exp(s^_j - lse) of the kept tokens, per head
+    for (int pr = tid; pr < kFixTok * G; pr += kFixThreads) {
+      const int tt = pr / G, h = pr - tt * G;
+      const int t = idx_s[tt];
+      float w = 0.0f;
+      if (t >= 0) {
+        const size_t row = cache_row_read(p.c, b, kv, t, nullptr);
+        const uint8_t* cr = p.c.k_codes + row * (D / 4);
+        const float* qh = q_s + h * D;
+        float s = 0.0f;
+        for (int g = 0; g < NG; ++g) {
+          float pg = 0.0f;
+          for (int c = 0; c < GS; ++c)
+            pg = fmaf(qh[g * GS + c], static_cast<float>(code2(cr, g * GS + c)), pg);
+          s = fmaf(p.c.k_min[row * NG + g], qg_s[h * NG + g], s);
+          s = fmaf(p.c.k_scale[row * NG + g], pg, s);
+        }
+        if (r > 0) {
+          const uint8_t* zr = p.c.z_codes + row * (r / 2);
+          float cz = 0.0f;
+          for (int i = 0; i < r; ++i) cz = fmaf(qt_s[h * r + i], static_cast<float>(nibble(zr, i)), cz);
+          s = fmaf(p.c.z_scale[row], cz, s);
+        }
+        w = expf(s * p.sm_scale - lse_s[h]);
+      }
+      p_s[tt * G + h] = w;
+    }
+    // exact value minus cached value of the kept tokens
+    for (int e = tid; e < kFixTok * D; e += kFixThreads) {
+      const int tt = e / D, c = e - tt * D;
+      const int t = idx_s[tt];
+      float dv = 0.0f;
+      if (t >= 0) {
+        const size_t row = cache_row_read(p.c, b, kv, t, nullptr);
+        const float v = load_elem(p.keep_v, (bk * p.K + k0 + tt) * D + c, p.keep_bf16);
+        dv = v - value_hat(p.c, row, c, D);
+      }
+      dv_s[e] = dv;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kFixMaxOut; ++k) {
+      const int idx = tid + k * kFixThreads;
+      if (idx < G * D) {
+        const int h = idx / D, c = idx - h * D;
+        float a = acc[k];
+#pragma unroll
+        for (int tt = 0; tt < kFixTok; ++tt) a = fmaf(p_s[tt * G + h], dv_s[tt * D + c], a);
+        acc[k] = a;
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kFixMaxOut; ++k) {
+    const int idx = tid + k * kFixThreads;
+    if (idx < G * D) {
+      const int h = idx / D, c = idx - h * D;
+      p.out[(static_cast<size_t>(b) * p.Hq + h0 + h) * D + c] += acc[k];
+    }
+  }
+}
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+int score_tiles(int T) { return (T + kAT - 1) / kAT; }
+
+size_t a2_ws_bytes(const headq_cache* c, int n_obs, int Hq, int T) {
+  const size_t NQ = static_cast<size_t>(n_obs) * (Hq / c->Hkv);
+  const size_t units = static_cast<size_t>(c->B) * c->Hkv;
+  return kWsHeaderBytes + round256(sizeof(float2) * units * score_tiles(T) * 2 * NQ) +
+         round256(sizeof(float) * units * NQ);
+}
+
+template <int D>
+cudaError_t launch_scores(const A2Params& p, cudaStream_t s) {
+  const size_t smem = sizeof(float) * (kAT * (D + 4) + kAQC * D + kAThreads + kAT);
+  auto k0 = a2_pass_kernel<D, false>;
+  auto k1 = a2_pass_kernel<D, true>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k0, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(p.ntiles, p.c.Hkv, p.c.B);
+  k0<<<grid, kAThreads, smem, s>>>(p);
+  const int NQ = p.n_obs * p.G;
+  a2_lse_kernel<<<p.c.B * p.c.Hkv, NQ < 1024 ? (NQ + 31) / 32 * 32 : 1024, 0, s>>>(p);
+  k1<<<grid, kAThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_fixup(const FixParams& p, cudaStream_t s) {
+  const int G = p.G;
+  const size_t smem = sizeof(float) * (static_cast<size_t>(G) * D + G * num_groups(D) +
+                                       G * p.c.r + G + kFixTok * G + kFixTok * D) +
+                      sizeof(int) * kFixTok;
+  auto k = a2_fixup_kernel<D>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  k<<<dim3(p.c.Hkv, p.c.B), kFixThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace headq
+
+using namespace headq;
+
+HEADQ_API size_t headq_a2_workspace_bytes(const headq_cache* cache, int n_obs, int Hq, int T) {
+  if (!cache || cache->Hkv <= 0 || n_obs <= 0 || Hq <= 0 || T < 0) return 0;
+  return a2_ws_bytes(cache, n_obs, Hq, T);
+}
+
+HEADQ_API headq_status headq_a2_scores(const headq_cache* cache, const void* q_obs,
+                                       headq_dtype q_dtype, int n_obs, int Hq,
+                                       const int32_t* seq_lens, int T, const void* k_full,
+                                       const void* v_full, headq_dtype kv_dtype, float sm_scale,
+                                       float* scores, void* ws, size_t ws_bytes,
+                                       headq_stream_t stream) {
+  headq_status st = check_cache(cache);
+  if (st != HEADQ_OK) return st;
+  if (!q_obs || !aligned16(q_obs)) return HEADQ_ERR_INVALID_ARG;
+  if (q_dtype != HEADQ_F32 && q_dtype != HEADQ_BF16) return HEADQ_ERR_INVALID_ARG;
+  if (Hq <= 0 || Hq % cache->Hkv != 0 || T < 0 || T > cache->T_cap || n_obs <= 0)
+    return HEADQ_ERR_INVALID_ARG;
+  if (kv_dtype != HEADQ_F32 && kv_dtype != HEADQ_BF16) return HEADQ_ERR_INVALID_ARG;
+  if (!k_full || !v_full || !scores || !aligned16(k_full) || !aligned16(v_full) ||
+      !aligned16(scores) || (seq_lens && !aligned16(seq_lens)))
+    return HEADQ_ERR_INVALID_ARG;
+  if (cache->d < 8 || cache->d > 256) return HEADQ_ERR_UNSUPPORTED;
+  if (!ws || !aligned16(ws) || ws_bytes < a2_ws_bytes(cache, n_obs, Hq, T))
+    return HEADQ_ERR_WORKSPACE;
+  if (cache->B == 0 || T == 0) return HEADQ_OK;
+  A2Params p{};
+  p.c = *cache;
+  p.q_obs = q_obs;
+  p.q_bf16 = q_dtype == HEADQ_BF16;
+  p.n_obs = n_obs;
+  p.Hq = Hq;
+  p.G = Hq / cache->Hkv;
+  p.T = T;
+  p.seq_lens = seq_lens;
+  p.k_full = k_full;
+  p.v_full = v_full;
+  p.kv_bf16 = kv_dtype == HEADQ_BF16;
+  p.sm_scale = sm_scale;
+  p.ntiles = score_tiles(T);
+  p.err = static_cast<unsigned*>(ws);
+  const size_t units = static_cast<size_t>(cache->B) * cache->Hkv;
+  const size_t NQ = static_cast<size_t>(n_obs) * p.G;
+  p.part = reinterpret_cast<float2*>(static_cast<char*>(ws) + kWsHeaderBytes);
+  p.lse = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeaderBytes +
+                                   round256(sizeof(float2) * units * p.ntiles * 2 * NQ));
+  p.scores = scores;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  switch (cache->d) {
+    case 8: e = launch_scores<8>(p, s); break;
+    case 16: e = launch_scores<16>(p, s); break;
+    case 32: e = launch_scores<32>(p, s); break;
+    case 64: e = launch_scores<64>(p, s); break;
+    case 128: e = launch_scores<128>(p, s); break;
+    case 256: e = launch_scores<256>(p, s); break;
+    default: return HEADQ_ERR_UNSUPPORTED;
+  }
+  return e == cudaSuccess ? HEADQ_OK : HEADQ_ERR_CUDA;
+}
+
+HEADQ_API headq_status headq_a2_select(const float* scores, int B, int Hkv,
+                                       const int32_t* seq_lens, int T, int K, const void* v_full,
+                                       headq_dtype kv_dtype, int d, int32_t* keep_idx,
+                                       void* keep_v, headq_stream_t stream) {
+  if (B < 0 || Hkv <= 0 || T < 0 || K < 0 || d <= 0 || d % 8 != 0) return HEADQ_ERR_INVALID_ARG;
+  if (kv_dtype != HEADQ_F32 && kv_dtype != HEADQ_BF16) return HEADQ_ERR_INVALID_ARG;
+  if (B == 0 || K == 0) return HEADQ_OK;
+  if (!scores || !v_full || !keep_idx || !keep_v || !aligned16(scores) || !aligned16(v_full) ||
+      !aligned16(keep_idx) || !aligned16(keep_v) || (seq_lens && !aligned16(seq_lens)))
+    return HEADQ_ERR_INVALID_ARG;
+  a2_select_kernel<<<B * Hkv, kSelThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      scores, Hkv, seq_lens, T, K, v_full, kv_dtype == HEADQ_BF16 ? 2 : 4, d, keep_idx, keep_v);
+  return cudaGetLastError() == cudaSuccess ? HEADQ_OK : HEADQ_ERR_CUDA;
+}
+
+HEADQ_API headq_status headq_a2_value_fixup(const headq_cache* cache, const void* q,
+                                            headq_dtype q_dtype, int Hq, const int32_t* seq_lens,
+                                            int T, const float* U, float sm_scale, int corr_sign,
+                                            const int32_t* keep_idx, const void* keep_v,
+                                            headq_dtype keep_dtype, int K, float* out,
+                                            const float* lse, headq_stream_t stream) {
+  headq_status st = check_read_args(cache, q, q_dtype, Hq, T, U, corr_sign);
+  if (st != HEADQ_OK) return st;
+  if (K < 0 || (keep_dtype != HEADQ_F32 && keep_dtype != HEADQ_BF16)) return HEADQ_ERR_INVALID_ARG;
+  if (!out || !lse || !aligned16(out) || !aligned16(lse) || (seq_lens && !aligned16(seq_lens)))
+    return HEADQ_ERR_INVALID_ARG;
+  if (cache->B == 0 || K == 0) return HEADQ_OK;
+  if (!keep_idx || !keep_v || !aligned16(keep_idx) || !aligned16(keep_v))
+    return HEADQ_ERR_INVALID_ARG;
+  FixParams p{};
+  p.c = *cache;
+  p.q = q;
+  p.q_bf16 = q_dtype == HEADQ_BF16;
+  p.Hq = Hq;
+  p.G = Hq / cache->Hkv;
+  p.T = T;
+  p.seq_lens = seq_lens;
+  p.U = U;
+  p.sm_scale = sm_scale;
+  p.corr_sign = static_cast<float>(corr_sign);
+  p.keep_idx = keep_idx;
+  p.keep_v = keep_v;
+  p.keep_bf16 = keep_dtype == HEADQ_BF16;
+  p.K = K;
+  p.out = out;
+  p.lse = lse;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  switch (cache->d) {
+    case 8: e = launch_fixup<8>(p, s); break;
+    case 16: e = launch_fixup<16>(p, s); break;
+    case 32: e = launch_fixup<32>(p, s); break;
+    case 64: e = launch_fixup<64>(p, s); break;
+    case 128: e = launch_fixup<128>(p, s); break;
+    case 256: e = launch_fixup<256>(p, s); break;
+    default: return HEADQ_ERR_UNSUPPORTED;
+  }
+  return e == cudaSuccess ? HEADQ_OK : HEADQ_ERR_CUDA;
+}

@@ -230,6 +230,20 @@ __device__ __forceinline__ uint32_t bf16_part_pair(float a, float b, bool lo) {
   const __nv_bfloat162 r = lo ? l : h;
   return *reinterpret_cast<const uint32_t*>(&r);
 }
+// x rounded to the nearest bf16 (ties to even), as an fp32 value; finite x
+__device__ __forceinline__ float bf16_round(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return __uint_as_float((u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u);
+}
+// bf16_part_pair with one conversion: the lanes that want the low part first
+// subtract the high part (lo_f = 1) and convert the residual, which is then
+// exactly the low part; the others convert the value itself (lo_f = 0)
+__device__ __forceinline__ uint32_t bf16_part_pair1(float a, float b, float lo_f) {
+  const float a2 = fmaf(-lo_f, bf16_round(a), a);
+  const float b2 = fmaf(-lo_f, bf16_round(b), b);
+  const __nv_bfloat162 r = __floats2bfloat162_rn(a2, b2);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
 
 // ---------------------------------------------------------------- the kernel
 template <int D, int R, int NT, bool V2>
@@ -643,9 +657,35 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       const int sa = 8 * t + (g >> 1), sb = sa + 4;
       const float va = __shfl_sync(kFull, p0, sa), vb = __shfl_sync(kFull, p0, sb);
       const float vc = __shfl_sync(kFull, p1, sa), vd = __shfl_sync(kFull, p1, sb);
-      if constexpr (V2) {
+      if constexpr (V2 && NG == 4) {
         // per 32-dim group: p_j * scale_{j,g} (0 for masked tokens, whatever the
-        // stale scale), and the running sum of p_j * min_{j,g}
+        // stale scale), and the running sum of p_j * min_{j,g}; the scales of
+        // the four tokens of this lane's B operand and the minima of its two
+        // logit tokens come in one vector load each
+        const float4* vs4 = reinterpret_cast<const float4*>(st + L::kVs);
+        const float4* vm4 = reinterpret_cast<const float4*>(st + L::kVm);
+        const int ta = jw + 2 * t;
+        const float4 vsc[4] = {vs4[ta], vs4[ta + 1], vs4[ta + 8], vs4[ta + 9]};
+        const float4 vmn[2] = {vm4[j0], vm4[j1]};
+        const float lo_f = (g & 1) ? 1.0f : 0.0f;
+        const float sa4[4][4] = {{vsc[0].x, vsc[0].y, vsc[0].z, vsc[0].w},
+                                 {vsc[1].x, vsc[1].y, vsc[1].z, vsc[1].w},
+                                 {vsc[2].x, vsc[2].y, vsc[2].z, vsc[2].w},
+                                 {vsc[3].x, vsc[3].y, vsc[3].z, vsc[3].w}};
+        const float m4[2][4] = {{vmn[0].x, vmn[0].y, vmn[0].z, vmn[0].w},
+                                {vmn[1].x, vmn[1].y, vmn[1].z, vmn[1].w}};
+#pragma unroll
+        for (int gg = 0; gg < NG; ++gg) {
+          const float pa = va > 0.f ? va * sa4[0][gg] : 0.f;
+          const float pb = vb > 0.f ? vb * sa4[1][gg] : 0.f;
+          const float pc = vc > 0.f ? vc * sa4[2][gg] : 0.f;
+          const float pd = vd > 0.f ? vd * sa4[3][gg] : 0.f;
+          bpv[gg][nt][0] = bf16_part_pair1(pa, pb, lo_f);
+          bpv[gg][nt][1] = bf16_part_pair1(pc, pd, lo_f);
+          if (p0 > 0.f) vmin_acc[nt][gg] = fmaf(p0, m4[0][gg], vmin_acc[nt][gg]);
+          if (p1 > 0.f) vmin_acc[nt][gg] = fmaf(p1, m4[1][gg], vmin_acc[nt][gg]);
+        }
+      } else if constexpr (V2) {
         const float* vs = reinterpret_cast<const float*>(st + L::kVs);
         const float* vm = reinterpret_cast<const float*>(st + L::kVm);
         const int ta = jw + 2 * t, tb = ta + 1, tc = ta + 8, td = ta + 9;

@@ -9,7 +9,7 @@
 
 namespace headq {
 
-static bool aligned16(const void* p) {
+bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
 
@@ -45,7 +45,7 @@ SplitPlan plan_splits(int units, int T, int min_chunk) {
   return sp;
 }
 
-static headq_status check_cache(const headq_cache* c) {
+headq_status check_cache(const headq_cache* c) {
   if (!c) return HEADQ_ERR_INVALID_ARG;
   if (c->B < 0 || c->Hkv <= 0 || c->T_cap < 0 || c->r < 0) return HEADQ_ERR_INVALID_ARG;
   if (!supported_d(c->d)) return HEADQ_ERR_UNSUPPORTED;
@@ -78,8 +78,8 @@ static headq_status check_cache(const headq_cache* c) {
   return HEADQ_OK;
 }
 
-static headq_status check_read_args(const headq_cache* c, const void* q, headq_dtype qd,
-                                    int Hq, int T, const float* U, int corr_sign) {
+headq_status check_read_args(const headq_cache* c, const void* q, headq_dtype qd, int Hq, int T,
+                             const float* U, int corr_sign) {
   headq_status st = check_cache(c);
   if (st != HEADQ_OK) return st;
   if (!q || !aligned16(q)) return HEADQ_ERR_INVALID_ARG;

@@ -171,6 +171,12 @@ struct CalibrateParams {
   float* eig;
 };
 
+// host-side argument checks shared by the entry points (headq_api.cu)
+bool aligned16(const void* p);
+headq_status check_cache(const headq_cache* c);
+headq_status check_read_args(const headq_cache* c, const void* q, headq_dtype qd, int Hq, int T,
+                             const float* U, int corr_sign);
+
 cudaError_t launch_cache_write(const CacheWriteParams& p, cudaStream_t s);
 cudaError_t launch_attn_kl(const AttnKlParams& p, cudaStream_t s);
 cudaError_t launch_calibrate(const CalibrateParams& p, cudaStream_t s);

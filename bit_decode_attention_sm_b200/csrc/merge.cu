@@ -55,8 +55,6 @@ __global__ void shard_seq_lens_kernel(const int32_t* seq_lens, int B, int T, int
   out[b] = loc < 0 ? 0 : (loc > n ? n : loc);
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 }  // namespace headq
 

@@ -31,7 +31,8 @@ EXPORTS = ("headq_version", "headq_status_string", "headq_calibrate",
            "headq_decode_workspace_bytes", "headq_decode_plan", "headq_attn_kl",
            "headq_attn_kl_workspace_bytes", "headq_workspace_status",
            "headq_decode_attn_noalloc", "headq_decode_append", "headq_shard_seq_lens",
-           "headq_merge_partials")
+           "headq_merge_partials", "headq_a2_workspace_bytes", "headq_a2_scores",
+           "headq_a2_select", "headq_a2_value_fixup")
 
 
 class HeadQError(RuntimeError):
@@ -84,6 +85,10 @@ def lib():
             "headq_decode_append": ([CP, P, P, I, P, I, I, P, I, P, F, I, P, P, P, Z, P], I),
             "headq_shard_seq_lens": ([P, I, I, I, I, P, P], I),
             "headq_merge_partials": ([P, P, I, I, I, Z, P, P, P], I),
+            "headq_a2_workspace_bytes": ([CP, I, I, I], Z),
+            "headq_a2_scores": ([CP, P, I, I, I, P, I, P, P, I, F, P, P, Z, P], I),
+            "headq_a2_select": ([P, I, I, P, I, I, P, I, I, P, P, P], I),
+            "headq_a2_value_fixup": ([CP, P, I, I, P, I, P, F, I, P, P, I, I, P, P, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -380,6 +385,72 @@ def headq_merge_partials(parts, S, BH, d, part_stride, out=None, lse=None, strea
         _ptr(parts), ctypes.c_void_p(parts.data_ptr() + 4 * BH * d), int(S), int(BH), int(d),
         int(part_stride), _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
+
+
+def a2_workspace(cache, n_obs, Hq, T):
+    cs = cache.struct()
+    n = lib().headq_a2_workspace_bytes(ctypes.byref(cs), n_obs, Hq, T)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=cache.k_codes.device)
+
+
+def headq_a2_scores(cache, q_obs, k_full, v_full, T=None, seq_lens=None, sm_scale=None,
+                    ws=None, out=None, stream=None):
+    """A^2 policy scores a_j fp32 [B, Hkv, T] from observation queries
+    q_obs [B, n_obs, Hq, d] and the exact keys/values [B, Hkv, T, d]."""
+    q_obs = _cuda(q_obs, "q_obs")
+    k_full = _cuda(k_full, "k_full")
+    v_full = _cuda(v_full, "v_full")
+    seq_lens = _cuda(seq_lens, "seq_lens")
+    B, n_obs, Hq, d = q_obs.shape
+    T = k_full.shape[2] if T is None else int(T)
+    sm = 1.0 / math.sqrt(d) if sm_scale is None else float(sm_scale)
+    ws = a2_workspace(cache, n_obs, Hq, T) if ws is None else ws
+    out = torch.empty((cache.B, cache.Hkv, T), dtype=torch.float32,
+                      device=q_obs.device) if out is None else out
+    cs = cache.struct()
+    _check("headq_a2_scores", lib().headq_a2_scores(
+        ctypes.byref(cs), _ptr(q_obs), _dtype_code(q_obs), n_obs, Hq, _ptr(seq_lens), T,
+        _ptr(k_full), _ptr(v_full), _dtype_code(k_full), ctypes.c_float(sm), _ptr(out),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def headq_a2_select(scores, K, v_full, seq_lens=None, keep_idx=None, keep_v=None, stream=None):
+    """Top-K kept positions (int32 [B, Hkv, K], ascending, -1 padded) and their
+    exact values [B, Hkv, K, d] (v_full's dtype)."""
+    scores = _cuda(scores, "scores")
+    v_full = _cuda(v_full, "v_full")
+    seq_lens = _cuda(seq_lens, "seq_lens")
+    B, Hkv, T = scores.shape
+    d = v_full.shape[-1]
+    keep_idx = torch.empty((B, Hkv, K), dtype=torch.int32,
+                           device=scores.device) if keep_idx is None else keep_idx
+    keep_v = torch.empty((B, Hkv, K, d), dtype=v_full.dtype,
+                         device=scores.device) if keep_v is None else keep_v
+    _check("headq_a2_select", lib().headq_a2_select(
+        _ptr(scores), B, Hkv, _ptr(seq_lens), T, int(K), _ptr(v_full), _dtype_code(v_full), d,
+        _ptr(keep_idx), _ptr(keep_v), _stream(stream)))
+    return keep_idx, keep_v
+
+
+def headq_a2_value_fixup(cache, q, U, keep_idx, keep_v, out, lse, T=None, seq_lens=None,
+                         sm_scale=None, corr_sign=1, stream=None):
+    """out += the kept tokens' exact-minus-cached value readout (after a decode
+    that wrote out and lse with the same arguments)."""
+    q = _cuda(q, "q")
+    keep_idx = _cuda(keep_idx, "keep_idx")
+    keep_v = _cuda(keep_v, "keep_v")
+    seq_lens = _cuda(seq_lens, "seq_lens")
+    B, Hq, d = q.shape
+    T = cache.T_cap if T is None else int(T)
+    sm = 1.0 / math.sqrt(d) if sm_scale is None else float(sm_scale)
+    U = _cuda(U, "U") if cache.r > 0 else None
+    cs = cache.struct()
+    _check("headq_a2_value_fixup", lib().headq_a2_value_fixup(
+        ctypes.byref(cs), _ptr(q), _dtype_code(q), Hq, _ptr(seq_lens), T, _ptr(U),
+        ctypes.c_float(sm), int(corr_sign), _ptr(keep_idx), _ptr(keep_v), _dtype_code(keep_v),
+        keep_idx.shape[-1], _ptr(out), _ptr(lse), _stream(stream)))
+    return out
 
 
 def headq_workspace_status(ws, stream=None):

@@ -21,7 +21,9 @@ bf16 values are rounded to nearest-even from fp32.
 
 import numpy as np
 
-_STREAMS = ("key_stats", "keys", "values", "query_basis", "queries", "cal")
+# a name appended here leaves every earlier stream unchanged (children of a
+# SeedSequence depend only on their own index)
+_STREAMS = ("key_stats", "keys", "values", "query_basis", "queries", "cal", "observe")
 
 
 def _streams(seed):
@@ -144,6 +146,17 @@ def make_layer(w, T=None, B=None, seed=None, n_cal=None):
     return LayerInputs(keys, values, queries, q_cal,
                        dict(workload=w.name, B=B, T=T, seed=seed, n_cal=n_cal,
                             query_basis=A))
+
+
+def make_observation_queries(w, L, n_obs, seed=None):
+    """[B, n_obs, Hq, d] observation queries of each sequence (the queries an
+    A^2 value policy measures attention with), drawn like the decode queries
+    from the layer's query basis; bf16-representable for bf16 workloads."""
+    st = _streams(L.meta["seed"] if seed is None else seed)
+    B = L.queries.shape[0]
+    q = make_queries(st["observe"], L.meta["query_basis"], B * n_obs, w.Hq)
+    q = q.reshape(B, n_obs, w.Hq, w.d)
+    return round_bf16(q) if w.kv_dtype == "bf16" else q
 
 
 def random_orthonormal(rng, d, r):

@@ -261,6 +261,64 @@ headq_status headq_attn_kl(const headq_cache *cache, const void *q, headq_dtype 
 size_t headq_attn_kl_workspace_bytes(const headq_cache *cache, int Hq, int T);
 
 /*
+ * A^2 value policy for the full-KV composition (2-bit values).  The pages give
+ * the value-side distortion as an A^2-weighted surrogate (abstract; summary
+ * section 2: under fixed attention p the readout error of value distortions
+ * dv_j is summarised by D_V = sum_j p_j^2 |dv_j|^2) and compose HeadQ keys with
+ * 2-bit values under an "A^2 value policy" they do not define (section 5).
+ * This library's reading: a budget of K tokens per (b, kv) keeps its values
+ * exact (the input precision) and the rest use the 2-bit code; D_V, summed over
+ * a set of n_obs observation queries per sequence and the G query heads of the
+ * KV head, loses exactly the terms of the kept tokens, so keeping the K tokens
+ * with the largest
+ *   a_j = |v^_j - v_j|^2 * sum_{o < n_obs} sum_{h in kv's group} p_{o,h,j}^2
+ * minimises it (top-K; ties to the lower position).  p_{o,h,.} is the softmax
+ * of sm_scale * q_{o,h} . k_j over the exact keys j < T_b.
+ *
+ * headq_a2_scores -- a_j for every cached token.
+ *   q_obs   [B, n_obs, Hq, d] (q_dtype): observation queries of each sequence.
+ *   k_full, v_full  [B, Hkv, T, d] (kv_dtype): the exact keys and values.
+ *   scores  fp32 [B, Hkv, T]; 0 for j >= T_b.  v^_j is read from the cache.
+ *   ws      headq_a2_workspace_bytes(...) bytes (its first word is the device
+ *           error word, as for decode).
+ * Two passes of the logits (normaliser, then p^2), fp32 accumulation.
+ */
+size_t headq_a2_workspace_bytes(const headq_cache *cache, int n_obs, int Hq, int T);
+headq_status headq_a2_scores(const headq_cache *cache, const void *q_obs, headq_dtype q_dtype,
+                             int n_obs, int Hq, const int32_t *seq_lens, int T,
+                             const void *k_full, const void *v_full, headq_dtype kv_dtype,
+                             float sm_scale, float *scores, void *ws, size_t ws_bytes,
+                             headq_stream_t stream);
+
+/*
+ * headq_a2_select -- the kept set of each (b, kv): the min(K, T_b) positions
+ * j < T_b with the largest scores (scores >= 0, as headq_a2_scores returns;
+ * equal scores: lower position first), written to keep_idx int32 [B, Hkv, K]
+ * in ascending order and padded with -1, and their exact values copied from
+ * v_full [B, Hkv, T, d] (kv_dtype) into keep_v [B, Hkv, K, d] (same dtype,
+ * zero rows for the padding).  d is a multiple of 8.
+ */
+headq_status headq_a2_select(const float *scores, int B, int Hkv, const int32_t *seq_lens,
+                             int T, int K, const void *v_full, headq_dtype kv_dtype, int d,
+                             int32_t *keep_idx, void *keep_v, headq_stream_t stream);
+
+/*
+ * headq_a2_value_fixup -- after headq_decode_attn (or headq_decode_append) with
+ * the same cache, q, seq_lens, T, U, sm_scale and corr_sign has written out and
+ * lse, turn its readout over the cached values v^_j into the readout over the
+ * policy's mixed values (the exact value for every kept j < T_b, v^_j for the
+ * rest):  out[b,h] += sum_{kept j} exp(s^_j - lse[b,h]) (v_j - v^_j), where s^_j
+ * is the HeadQ logit.  The softmax weights are unchanged, so the result is the
+ * mixed-value attention itself.  keep_idx/keep_v as headq_a2_select writes them
+ * (entries < 0 or >= T_b are skipped); lse is read, not written.
+ */
+headq_status headq_a2_value_fixup(const headq_cache *cache, const void *q, headq_dtype q_dtype,
+                                  int Hq, const int32_t *seq_lens, int T, const float *U,
+                                  float sm_scale, int corr_sign, const int32_t *keep_idx,
+                                  const void *keep_v, headq_dtype keep_dtype, int K, float *out,
+                                  const float *lse, headq_stream_t stream);
+
+/*
  * Split-T across devices (context-parallel decode).  Each device holds a
  * contiguous range [t_lo, t_lo + n) of every sequence's cached tokens, at local
  * positions [0, n) of its own cache, and runs headq_decode_attn over it with

@@ -286,6 +286,76 @@ def merge_partials(outs, lses):
 
 
 # --------------------------------------------------------------------------
+# A^2 value policy (abstract; summary sections 2 and 5).  The pages name the
+# policy without defining it; the reading restated here: a budget of K tokens
+# per (b, kv) keeps exact values, the rest keep the 2-bit code, and the kept
+# set minimises the A^2 surrogate sum_j p_j^2 |v^_j - v_j|^2 summed over the
+# observation queries and the heads of the KV head.
+# --------------------------------------------------------------------------
+def cached_values(planes, vmode, v=None):
+    """v^ [B, Hkv, T, d] fp32: the 2-bit dequantised values, or the dense cache."""
+    if vmode == "2bit":
+        return base_dequantize(planes["vc"], planes["vs"], planes["vm"])
+    return _f32(v)
+
+
+def a2_scores(q_obs, k_full, v_full, v_hat, sm_scale=None, seq_lens=None):
+    """a_j = |v^_j - v_j|^2 * sum_{o, h in group(kv)} p_{o,h,j}^2, fp64 [B, Hkv, T],
+    with p_{o,h,.} = softmax_j(sm_scale * q_obs[b, o, h] . k_j) over j < T_b (exact
+    keys), and 0 for j >= T_b.  q_obs [B, n_obs, Hq, d]; k_full, v_full, v_hat
+    [B, Hkv, T, d]."""
+    q = np.asarray(q_obs, np.float64)
+    k = np.asarray(k_full, np.float64)
+    v = np.asarray(v_full, np.float64)
+    vh = np.asarray(v_hat, np.float64)
+    B, n_obs, Hq, d = q.shape
+    Hkv, T = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    sm = 1.0 / np.sqrt(d) if sm_scale is None else float(sm_scale)
+    out = np.zeros((B, Hkv, T), np.float64)
+    for b in range(B):
+        Tb = T if seq_lens is None else int(min(max(seq_lens[b], 0), T))
+        if Tb == 0:
+            continue
+        for kv in range(Hkv):
+            qs = q[b, :, kv * G:(kv + 1) * G].reshape(-1, d)          # [n_obs*G, d]
+            s = sm * (qs @ k[b, kv, :Tb].T)                             # [n_obs*G, Tb]
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p /= p.sum(axis=1, keepdims=True)
+            dv2 = ((vh[b, kv, :Tb] - v[b, kv, :Tb]) ** 2).sum(axis=1)
+            out[b, kv, :Tb] = (p * p).sum(axis=0) * dv2
+    return out
+
+
+def a2_select(scores, K, seq_lens=None):
+    """Kept positions int32 [B, Hkv, K]: the min(K, T_b) largest scores among
+    j < T_b (equal scores: lower position first), ascending, padded with -1."""
+    scores = np.asarray(scores)
+    B, Hkv, T = scores.shape
+    out = np.full((B, Hkv, K), -1, np.int32)
+    for b in range(B):
+        Tb = T if seq_lens is None else int(min(max(seq_lens[b], 0), T))
+        for kv in range(Hkv):
+            order = sorted(range(Tb), key=lambda j: (-scores[b, kv, j], j))
+            kept = sorted(order[:min(K, Tb)])
+            out[b, kv, :len(kept)] = kept
+    return out
+
+
+def a2_mixed_values(v_hat, v_full, keep_idx):
+    """The policy's values: v_j for every kept j, v^_j for the rest."""
+    mixed = np.array(v_hat, np.float32, copy=True)
+    B, Hkv, K = keep_idx.shape
+    for b in range(B):
+        for kv in range(Hkv):
+            for j in keep_idx[b, kv]:
+                if j >= 0:
+                    mixed[b, kv, j] = v_full[b, kv, j]
+    return mixed
+
+
+# --------------------------------------------------------------------------
 # Step 4: diagnostics (section 2 of the summary).
 # --------------------------------------------------------------------------
 def attn_kl(q, planes, U, k_full, v_full, v=None, vmode="dense", sm_scale=None,

@@ -377,6 +377,68 @@ def test_merge_of_token_shards_equals_whole():
     np.testing.assert_allclose(ml, ref_lse, rtol=1e-12)
 
 
+def test_a2_scores_sum_to_the_a2_diagnostic():
+    """With the decode query as the only observation query, the A^2 policy
+    scores of a KV head sum to the A^2 value distortion the diagnostic reports
+    for its G heads (an independent implementation in the C oracle)."""
+    k, v, q, U = _tiny_layer(d=32, T=60, Hkv=2, G=3, B=2, r=8, seed=17)
+    planes = oracle.cache_write(k, U, v=v, vmode="2bit")
+    vh = oracle.cached_values(planes, "2bit")
+    seq_lens = np.array([60, 23], np.int32)
+    sc = oracle.a2_scores(q[:, None], k, v, vh, seq_lens=seq_lens)
+    _, _, a2v, _ = oracle.attn_kl(q, planes, U, k, v, vmode="2bit", seq_lens=seq_lens)
+    np.testing.assert_allclose(sc.sum(axis=2), a2v.reshape(2, 2, 3).sum(axis=2), rtol=1e-10)
+    assert (sc[1, :, 23:] == 0).all() and (sc >= 0).all()
+
+
+def test_a2_scores_uniform_attention_closed_form():
+    """Zero observation queries attend uniformly: a_j = n_obs G |dv_j|^2 / T_b^2."""
+    k, v, q, U = _tiny_layer(d=16, T=40, Hkv=1, G=2, B=1, r=4, seed=18)
+    planes = oracle.cache_write(k, U, v=v, vmode="2bit")
+    vh = oracle.cached_values(planes, "2bit")
+    sc = oracle.a2_scores(np.zeros((1, 3, 2, 16), np.float32), k, v, vh)
+    dv2 = ((vh.astype(np.float64) - v) ** 2).sum(-1)
+    np.testing.assert_allclose(sc, 3 * 2 * dv2 / 40 ** 2, rtol=1e-12)
+
+
+def test_a2_selection_minimises_the_surrogate_brute_force():
+    """For every budget K the kept set leaves the smallest surrogate sum over
+    the dropped tokens of all subsets of that size (exhaustive search), and
+    among equally good sets it takes the lower positions."""
+    import itertools
+    rng = _rng(19)
+    T = 9
+    scores = rng.integers(0, 4, size=(2, 1, T)).astype(np.float64)  # many ties
+    seq_lens = np.array([9, 6], np.int32)
+    for K in range(0, T + 2):
+        kept = oracle.a2_select(scores, K, seq_lens=seq_lens)
+        for b in range(2):
+            Tb = int(seq_lens[b])
+            m = min(K, Tb)
+            got = tuple(int(j) for j in kept[b, 0] if j >= 0)
+            assert len(got) == m and list(got) == sorted(got)
+            assert (kept[b, 0, m:] == -1).all()
+            best = min((sum(scores[b, 0, j] for j in range(Tb) if j not in S), S)
+                       for S in itertools.combinations(range(Tb), m))
+            assert best[1] == got
+
+
+def test_a2_mixed_values_limits():
+    """K = 0 is plain 2-bit value attention; keeping every token is attention
+    over the exact values (same HeadQ logits in both)."""
+    k, v, q, U = _tiny_layer(d=32, T=50, Hkv=2, G=2, B=2, r=8, seed=20)
+    planes = oracle.cache_write(k, U, v=v, vmode="2bit")
+    vh = oracle.cached_values(planes, "2bit")
+    none = oracle.a2_select(np.ones((2, 2, 50)), 0)
+    every = oracle.a2_select(np.ones((2, 2, 50)), 50)
+    o2, _ = oracle.decode(q, planes, U, vmode="2bit")
+    o0, _ = oracle.decode(q, planes, U, v=oracle.a2_mixed_values(vh, v, none))
+    np.testing.assert_array_equal(o0, o2)
+    oe, _ = oracle.decode(q, planes, U, v=v)
+    om, _ = oracle.decode(q, planes, U, v=oracle.a2_mixed_values(vh, v, every))
+    np.testing.assert_array_equal(om, oe)
+
+
 def test_output_inside_value_bounding_box():
     k, v, q, U = _tiny_layer(d=64, T=100, Hkv=2, G=3, B=2, r=8, seed=13)
     planes = oracle.cache_write(k, U)
