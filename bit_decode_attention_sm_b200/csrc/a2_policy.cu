@@ -38,8 +38,8 @@ constexpr int kAT = 64;          // tokens per score tile
 constexpr int kAThreads = 256;   // 64 tokens x 4 query lanes
 constexpr int kAQC = 16;         // observation queries staged per chunk
 constexpr int kSelThreads = 1024;
-constexpr int kFixThreads = 256;
-constexpr int kFixTok = 32;      // kept tokens per fixup step
+constexpr int kFixThreads = 512;
+constexpr int kFixTok = 64;      // kept tokens per fixup step
 constexpr int kFixMaxOut = 2048 / kFixThreads;
 
 struct A2Params {
@@ -72,6 +72,40 @@ __device__ __forceinline__ float value_hat(const headq_cache& c, size_t row, int
     return __fadd_rn(mn, __fmul_rn(static_cast<float>(code2(c.v_codes + row * (d / 4), ch)), sc));
   }
   return load_elem(c.v, row * d + ch, c.v_dtype == HEADQ_BF16);
+}
+
+// 8 consecutive elements (offset a multiple of 8) of an fp32 or bf16 tensor
+__device__ __forceinline__ void load8(const void* base, size_t off, bool bf16, float (&x)[8]) {
+  if (bf16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + off);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      x[2 * k] = __uint_as_float(w[k] << 16);
+      x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+  } else {
+    const float4* f = reinterpret_cast<const float4*>(static_cast<const float*>(base) + off);
+    const float4 a = f[0], b = f[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+}
+
+// value_hat of channels c0 .. c0+7 (c0 a multiple of 8, inside one group)
+__device__ __forceinline__ void value_hat8(const headq_cache& c, size_t row, int c0, int d,
+                                           float (&x)[8]) {
+  if (c.vmode == HEADQ_V_2BIT) {
+    const int GS = d < 32 ? d : 32, NG = d / GS;
+    const int g = c0 / GS;
+    const float mn = c.v_min[row * NG + g], sc = c.v_scale[row * NG + g];
+    const uint32_t w = *reinterpret_cast<const uint16_t*>(c.v_codes + row * (d / 4) + c0 / 4);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      x[k] = __fadd_rn(mn, __fmul_rn(static_cast<float>((w >> (2 * k)) & 3u), sc));
+  } else {
+    load8(c.v, row * d + c0, c.v_dtype == HEADQ_BF16, x);
+  }
 }
 
 // Pass 0 (SCORE false): tile partials of the softmax normaliser of each
@@ -319,18 +353,38 @@ struct FixParams {
   const float* lse;
 };
 
+// shared-memory layout of one fixup chunk: the kept tokens' key planes
+template <int D>
+struct FixStage {
+  static constexpr int NG = num_groups(D);
+  static constexpr int kKcWords = (D + 15) / 16;  // 2-bit codes, 16 per word (d = 8: half)
+  static constexpr int kZcBytes = 16;      // side codes, r <= 32
+  static constexpr size_t bytes() {
+    return sizeof(uint32_t) * kFixTok * kKcWords + sizeof(float) * kFixTok * (2 * NG + 1) +
+           kFixTok * kZcBytes;
+  }
+};
+
 template <int D>
 __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p) {
   constexpr int GS = group_size(D), NG = num_groups(D);
+  using FS = FixStage<D>;
   extern __shared__ float sm[];
   const int G = p.G, r = p.c.r;
-  float* q_s = sm;                    // [G][D]
+  float* dv_s = sm;                   // [kFixTok][D]  (first: 16-byte aligned rows)
+  float* q_s = dv_s + kFixTok * D;    // [G][D]
   float* qg_s = q_s + G * D;          // [G][NG]
   float* qt_s = qg_s + G * NG;        // [G][r]
   float* lse_s = qt_s + G * r;        // [G]
   float* p_s = lse_s + G;             // [kFixTok][G]
-  float* dv_s = p_s + kFixTok * G;    // [kFixTok][D]
-  int* idx_s = reinterpret_cast<int*>(dv_s + kFixTok * D);  // [kFixTok]
+  int* idx_s = reinterpret_cast<int*>(p_s + kFixTok * G);            // [kFixTok]
+  size_t* row_s = reinterpret_cast<size_t*>(                          // [kFixTok], 8-aligned
+      (reinterpret_cast<uintptr_t>(idx_s + kFixTok) + 7) & ~uintptr_t(7));
+  uint32_t* kc_s = reinterpret_cast<uint32_t*>(row_s + kFixTok);     // [kFixTok][D/16]
+  float* ks_s = reinterpret_cast<float*>(kc_s + kFixTok * FS::kKcWords);  // [kFixTok][NG]
+  float* km_s = ks_s + kFixTok * NG;                                  // [kFixTok][NG]
+  float* zs_s = km_s + kFixTok * NG;                                  // [kFixTok]
+  uint8_t* zc_s = reinterpret_cast<uint8_t*>(zs_s + kFixTok);         // [kFixTok][16]
 
   const int kv = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int h0 = kv * G;
@@ -348,11 +402,14 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
     for (int c = 0; c < GS; ++c) acc += q_s[h * D + g * GS + c];
     qg_s[i] = acc;
   }
+  // sigma U_h^T q, with U_h staged in the (not yet used) value-difference buffer
+  float* u_s = dv_s;
+  for (int i = tid; i < D * r; i += kFixThreads) u_s[i] = p.U[static_cast<size_t>(kv) * D * r + i];
+  __syncthreads();
   for (int i = tid; i < G * r; i += kFixThreads) {
     const int h = i / r, ii = i - h * r;
-    const float* U = p.U + static_cast<size_t>(kv) * D * r;
     float acc = 0.0f;
-    for (int c = 0; c < D; ++c) acc = fmaf(U[c * r + ii], q_s[h * D + c], acc);
+    for (int c = 0; c < D; ++c) acc = fmaf(u_s[c * r + ii], q_s[h * D + c], acc);
     qt_s[i] = p.corr_sign * acc;
   }
 
@@ -364,47 +421,87 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
     __syncthreads();
     if (tid < kFixTok) {
       const int t = k0 + tid < p.K ? p.keep_idx[bk * p.K + k0 + tid] : -1;
-      idx_s[tid] = (t >= 0 && t < Tb) ? t : -1;
+      const bool ok = t >= 0 && t < Tb;
+      idx_s[tid] = ok ? t : -1;
+      row_s[tid] = ok ? cache_row_read(p.c, b, kv, t, nullptr) : 0;
     }
     __syncthreads();
-    // weights exp(s^_j - lse) of the kept tokens, per head
+    // stage the kept tokens' key planes (word-wide, all threads)
+    if constexpr (D >= 16) {
+      for (int e = tid; e < kFixTok * FS::kKcWords; e += kFixThreads) {
+        const int tt = e / FS::kKcWords, w = e - tt * FS::kKcWords;
+        kc_s[e] = idx_s[tt] >= 0
+                      ? reinterpret_cast<const uint32_t*>(p.c.k_codes + row_s[tt] * (D / 4))[w]
+                      : 0u;
+      }
+    } else {  // d = 8: a 2-byte code row, staged byte by byte into the low half
+      for (int tt = tid; tt < kFixTok; tt += kFixThreads) {
+        uint32_t x = 0u;
+        if (idx_s[tt] >= 0)
+          for (int by = 0; by < D / 4; ++by)
+            x |= static_cast<uint32_t>(p.c.k_codes[row_s[tt] * (D / 4) + by]) << (8 * by);
+        kc_s[tt] = x;
+      }
+    }
+    for (int e = tid; e < kFixTok * NG; e += kFixThreads) {
+      const int tt = e / NG, g = e - tt * NG;
+      const bool ok = idx_s[tt] >= 0;
+      ks_s[e] = ok ? p.c.k_scale[row_s[tt] * NG + g] : 0.0f;
+      km_s[e] = ok ? p.c.k_min[row_s[tt] * NG + g] : 0.0f;
+    }
+    if (r > 0) {
+      for (int e = tid; e < kFixTok * (r / 2); e += kFixThreads) {
+        const int tt = e / (r / 2), w = e - tt * (r / 2);
+        zc_s[tt * FS::kZcBytes + w] = idx_s[tt] >= 0 ? p.c.z_codes[row_s[tt] * (r / 2) + w] : 0;
+      }
+      for (int tt = tid; tt < kFixTok; tt += kFixThreads)
+        zs_s[tt] = idx_s[tt] >= 0 ? p.c.z_scale[row_s[tt]] : 0.0f;
+    }
+    // exact value minus cached value, 8 channels per task (wide loads)
+    for (int e = tid; e < kFixTok * (D / 8); e += kFixThreads) {
+      const int tt = e / (D / 8), c0 = (e - tt * (D / 8)) * 8;
+      float dv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (idx_s[tt] >= 0) {
+        float v[8], vh[8];
+        load8(p.keep_v, (bk * p.K + k0 + tt) * D + c0, p.keep_bf16, v);
+        value_hat8(p.c, row_s[tt], c0, D, vh);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) dv[k] = v[k] - vh[k];
+      }
+      float4* dst = reinterpret_cast<float4*>(dv_s + tt * D + c0);
+      dst[0] = make_float4(dv[0], dv[1], dv[2], dv[3]);
+      dst[1] = make_float4(dv[4], dv[5], dv[6], dv[7]);
+    }
+    __syncthreads();
+    // weights exp(s^_j - lse) of the kept tokens, per head, from shared memory
     for (int pr = tid; pr < kFixTok * G; pr += kFixThreads) {
       const int tt = pr / G, h = pr - tt * G;
-      const int t = idx_s[tt];
       float w = 0.0f;
-      if (t >= 0) {
-        const size_t row = cache_row_read(p.c, b, kv, t, nullptr);
-        const uint8_t* cr = p.c.k_codes + row * (D / 4);
+      if (idx_s[tt] >= 0) {
+        const uint32_t* cw = kc_s + tt * FS::kKcWords;
         const float* qh = q_s + h * D;
         float s = 0.0f;
+#pragma unroll
         for (int g = 0; g < NG; ++g) {
           float pg = 0.0f;
-          for (int c = 0; c < GS; ++c)
-            pg = fmaf(qh[g * GS + c], static_cast<float>(code2(cr, g * GS + c)), pg);
-          s = fmaf(p.c.k_min[row * NG + g], qg_s[h * NG + g], s);
-          s = fmaf(p.c.k_scale[row * NG + g], pg, s);
+#pragma unroll
+          for (int c = 0; c < GS; ++c) {
+            const int ch = g * GS + c;
+            const uint32_t code = (cw[ch >> 4] >> (2 * (ch & 15))) & 3u;
+            pg = fmaf(qh[ch], static_cast<float>(code), pg);
+          }
+          s = fmaf(km_s[tt * NG + g], qg_s[h * NG + g], s);
+          s = fmaf(ks_s[tt * NG + g], pg, s);
         }
         if (r > 0) {
-          const uint8_t* zr = p.c.z_codes + row * (r / 2);
+          const uint8_t* zr = zc_s + tt * FS::kZcBytes;
           float cz = 0.0f;
           for (int i = 0; i < r; ++i) cz = fmaf(qt_s[h * r + i], static_cast<float>(nibble(zr, i)), cz);
-          s = fmaf(p.c.z_scale[row], cz, s);
+          s = fmaf(zs_s[tt], cz, s);
         }
         w = expf(s * p.sm_scale - lse_s[h]);
       }
       p_s[tt * G + h] = w;
-    }
-    // exact value minus cached value of the kept tokens
-    for (int e = tid; e < kFixTok * D; e += kFixThreads) {
-      const int tt = e / D, c = e - tt * D;
-      const int t = idx_s[tt];
-      float dv = 0.0f;
-      if (t >= 0) {
-        const size_t row = cache_row_read(p.c, b, kv, t, nullptr);
-        const float v = load_elem(p.keep_v, (bk * p.K + k0 + tt) * D + c, p.keep_bf16);
-        dv = v - value_hat(p.c, row, c, D);
-      }
-      dv_s[e] = dv;
     }
     __syncthreads();
 #pragma unroll
@@ -466,7 +563,7 @@ cudaError_t launch_fixup(const FixParams& p, cudaStream_t s) {
   const int G = p.G;
   const size_t smem = sizeof(float) * (static_cast<size_t>(G) * D + G * num_groups(D) +
                                        G * p.c.r + G + kFixTok * G + kFixTok * D) +
-                      sizeof(int) * kFixTok;
+                      sizeof(int) * 2 * kFixTok + sizeof(size_t) * kFixTok + FixStage<D>::bytes();
   auto k = a2_fixup_kernel<D>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -565,6 +662,7 @@ HEADQ_API headq_status headq_a2_value_fixup(const headq_cache* cache, const void
                                             const float* lse, headq_stream_t stream) {
   headq_status st = check_read_args(cache, q, q_dtype, Hq, T, U, corr_sign);
   if (st != HEADQ_OK) return st;
+  if (cache->kmode != HEADQ_K_TOKEN) return HEADQ_ERR_UNSUPPORTED;
   if (K < 0 || (keep_dtype != HEADQ_F32 && keep_dtype != HEADQ_BF16)) return HEADQ_ERR_INVALID_ARG;
   if (!out || !lse || !aligned16(out) || !aligned16(lse) || (seq_lens && !aligned16(seq_lens)))
     return HEADQ_ERR_INVALID_ARG;

@@ -54,9 +54,13 @@ __device__ __forceinline__ float cached_value(const AttnKlParams& p, size_t row,
 
 template <int D>
 __device__ __forceinline__ float base_key(const AttnKlParams& p, size_t row, int c) {
+  const float code = static_cast<float>(code2(p.c.k_codes + row * (D / 4), c));
+  if (p.c.kmode == HEADQ_K_CHANNEL) {  // per channel, per 64-token block (row / 64)
+    const size_t bi = (row >> 6) * D + c;
+    return __fadd_rn(p.c.k_min[bi], __fmul_rn(code, p.c.k_scale[bi]));
+  }
   constexpr int NG = num_groups(D);
   const int g = c / group_size(D);
-  const float code = static_cast<float>(code2(p.c.k_codes + row * (D / 4), c));
   return __fadd_rn(p.c.k_min[row * NG + g], __fmul_rn(code, p.c.k_scale[row * NG + g]));
 }
 
@@ -627,7 +631,7 @@ cudaError_t launch_d(const AttnKlParams& p, cudaStream_t s) {
                                        kTile + 3 * G);
   dim3 grid(p.splits, p.c.Hkv, p.c.B);
   if constexpr (D == 64 || D == 128) {
-    if (p.G * D <= 8 * kSThreads) {
+    if (p.G * D <= 8 * kSThreads && p.c.kmode == HEADQ_K_TOKEN) {
       const size_t ssm = staged_smem<D>(p);
       auto k = attn_kl_staged_kernel<D>;
       cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -112,12 +112,21 @@ decode_split_kernel(const DecodeParams p) {
         const uint8_t* cr = p.c.k_codes + row * (D / 4);
         const float* qh = q_s + h * D;
         float acc = 0.0f;
-        for (int g = 0; g < NG; ++g) {
-          float pg = 0.0f;
-          for (int c = 0; c < GS; ++c)
-            pg = fmaf(qh[g * GS + c], static_cast<float>(code2(cr, g * GS + c)), pg);
-          acc = fmaf(p.c.k_min[row * NG + g], qg_s[h * NG + g], acc);
-          acc = fmaf(p.c.k_scale[row * NG + g], pg, acc);
+        if (p.c.kmode == HEADQ_K_CHANNEL) {  // per-channel minimum and scale of the block
+          const float* mn = p.c.k_min + (row >> 6) * D;
+          const float* sc = p.c.k_scale + (row >> 6) * D;
+          for (int c = 0; c < D; ++c) {
+            const float kh = __fadd_rn(mn[c], __fmul_rn(static_cast<float>(code2(cr, c)), sc[c]));
+            acc = fmaf(qh[c], kh, acc);
+          }
+        } else {
+          for (int g = 0; g < NG; ++g) {
+            float pg = 0.0f;
+            for (int c = 0; c < GS; ++c)
+              pg = fmaf(qh[g * GS + c], static_cast<float>(code2(cr, g * GS + c)), pg);
+            acc = fmaf(p.c.k_min[row * NG + g], qg_s[h * NG + g], acc);
+            acc = fmaf(p.c.k_scale[row * NG + g], pg, acc);
+          }
         }
         if (r > 0) {
           const uint8_t* zr = p.c.z_codes + row * (r / 2);
@@ -274,7 +283,10 @@ DecodePlan decode_plan(const headq_cache& c, int Hq, int T) {
   const int G = c.Hkv > 0 ? Hq / c.Hkv : 0;
   const int units = c.B * c.Hkv;
   if (T <= 0 || units <= 0) return dp;
-  const int occ = mma_decode_supported(c, G) ? mma_decode_ctas_per_sm(c, G) : 0;
+  // the tensor-core kernel reads the per-token base code; the per-channel code
+  // goes to the generic kernel
+  const bool mma = c.kmode == HEADQ_K_TOKEN && mma_decode_supported(c, G);
+  const int occ = mma ? mma_decode_ctas_per_sm(c, G) : 0;
   if (occ > 0) {
     // one wave: every CTA resident, each streaming one contiguous chunk; the
     // last CTA of each (b, kv) merges the splits, so one kernel per call

@@ -51,6 +51,8 @@ headq_status check_cache(const headq_cache* c) {
   if (!supported_d(c->d)) return HEADQ_ERR_UNSUPPORTED;
   if (c->r % 2 != 0 || c->r > c->d || c->r > 32) return HEADQ_ERR_UNSUPPORTED;
   if (c->T_cap % 16 != 0) return HEADQ_ERR_UNSUPPORTED;
+  if (c->kmode != HEADQ_K_TOKEN && c->kmode != HEADQ_K_CHANNEL) return HEADQ_ERR_INVALID_ARG;
+  if (c->kmode == HEADQ_K_CHANNEL && c->T_cap % 64 != 0) return HEADQ_ERR_UNSUPPORTED;
   if (c->page_size < 0) return HEADQ_ERR_INVALID_ARG;
   if (c->page_size > 0) {  // paged pools: whole 64-token tiles per page
     if (c->page_size % 64 != 0) return HEADQ_ERR_UNSUPPORTED;
@@ -168,6 +170,7 @@ HEADQ_API headq_status headq_cache_write(const headq_cache* cache, const void* k
   if (st != HEADQ_OK) return st;
   if (kv_dtype != HEADQ_F32 && kv_dtype != HEADQ_BF16) return HEADQ_ERR_INVALID_ARG;
   if (t0 < 0 || n < 0 || static_cast<long>(t0) + n > cache->T_cap) return HEADQ_ERR_INVALID_ARG;
+  if (cache->kmode == HEADQ_K_CHANNEL && t0 % 64 != 0) return HEADQ_ERR_UNSUPPORTED;
   if (n == 0 || cache->B == 0) return HEADQ_OK;  // nothing to read: k, v, U unused
   if (!k || !aligned16(k) || (v && !aligned16(v))) return HEADQ_ERR_INVALID_ARG;
   if (cache->r > 0 && (!U || !aligned16(U))) return HEADQ_ERR_INVALID_ARG;
@@ -247,6 +250,7 @@ HEADQ_API headq_status headq_decode_append(const headq_cache* cache, const void*
                                            headq_stream_t stream) {
   headq_status st = check_read_args(cache, q, q_dtype, Hq, T, U, corr_sign);
   if (st != HEADQ_OK) return st;
+  if (cache->kmode != HEADQ_K_TOKEN) return HEADQ_ERR_UNSUPPORTED;  // sealed key blocks
   if (!k_new || !aligned16(k_new) || (v_new && !aligned16(v_new))) return HEADQ_ERR_INVALID_ARG;
   if (kv_dtype != HEADQ_F32 && kv_dtype != HEADQ_BF16) return HEADQ_ERR_INVALID_ARG;
   if (!out || !aligned16(out) || (lse && !aligned16(lse))) return HEADQ_ERR_INVALID_ARG;

@@ -35,6 +35,9 @@ EXPORTS = ("headq_version", "headq_status_string", "headq_calibrate",
            "headq_a2_select", "headq_a2_value_fixup")
 
 
+KMODES = {"token": 0, "channel": 1}  # headq_kmode
+
+
 class HeadQError(RuntimeError):
     def __init__(self, fn, status):
         self.status = status
@@ -52,7 +55,8 @@ class CacheStruct(ctypes.Structure):
                 ("v_codes", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
                 ("v_min", ctypes.c_void_p),
                 ("page_size", ctypes.c_int), ("num_pages", ctypes.c_int),
-                ("max_pages", ctypes.c_int), ("block_table", ctypes.c_void_p)]
+                ("max_pages", ctypes.c_int), ("block_table", ctypes.c_void_p),
+                ("kmode", ctypes.c_int)]
 
 
 _lib = None
@@ -141,23 +145,29 @@ class HeadQCache:
 
     page_size = num_pages = max_pages = 0
     block_table = None
+    kmode = "token"
 
     def __init__(self, B, Hkv, T_cap, d, r, vmode="dense", v_dtype=torch.bfloat16,
-                 device="cuda"):
-        if T_cap % 16:
-            raise ValueError("T_cap must be a multiple of 16")
+                 device="cuda", kmode="token"):
+        if T_cap % (64 if kmode == "channel" else 16):
+            raise ValueError("T_cap must be a multiple of 16 (64 for per-channel keys)")
         self.B, self.Hkv, self.T_cap, self.d, self.r = B, Hkv, T_cap, d, r
-        self._alloc((B, Hkv, T_cap), vmode, v_dtype, device)
+        self._alloc((B, Hkv, T_cap), vmode, v_dtype, device, kmode)
 
-    def _alloc(self, lead, vmode, v_dtype, device):
+    def _alloc(self, lead, vmode, v_dtype, device, kmode="token"):
         d, r = self.d, self.r
+        if kmode not in KMODES:
+            raise ValueError("kmode is 'token' or 'channel'")
         self.vmode = vmode
         self.v_dtype = v_dtype
+        self.kmode = kmode
         ng = d // min(32, d)
         u8, f32 = torch.uint8, torch.float32
         self.k_codes = torch.zeros(lead + (d // 4,), dtype=u8, device=device)
-        self.k_scale = torch.zeros(lead + (ng,), dtype=f32, device=device)
-        self.k_min = torch.zeros(lead + (ng,), dtype=f32, device=device)
+        # per-token groups, or (per-channel code) one row of d per 64-token block
+        sshape = lead + (ng,) if kmode == "token" else lead[:-1] + (lead[-1] // 64, d)
+        self.k_scale = torch.zeros(sshape, dtype=f32, device=device)
+        self.k_min = torch.zeros(sshape, dtype=f32, device=device)
         self.z_codes = torch.zeros(lead + (max(r // 2, 1),), dtype=u8, device=device)
         self.z_scale = torch.zeros(lead, dtype=f32, device=device)
         self.v = self.v_codes = self.v_scale = self.v_min = None
@@ -182,7 +192,7 @@ class HeadQCache:
     def nbytes_per_token(self):
         """Bytes one cached token of one KV head occupies in HBM."""
         ng = self.d // min(32, self.d)
-        b = self.d // 4 + 8 * ng + self.r // 2 + 4
+        b = self.d // 4 + (8 * ng if self.kmode == "token" else self.d // 8) + self.r // 2 + 4
         if self.vmode == "2bit":
             b += self.d // 4 + 8 * ng
         else:
@@ -208,6 +218,7 @@ class HeadQCache:
         if self.page_size:
             s.page_size, s.num_pages, s.max_pages = self.page_size, self.num_pages, self.max_pages
             s.block_table = self.block_table.data_ptr()
+        s.kmode = KMODES[self.kmode]
         return s
 
 
@@ -222,7 +233,7 @@ class PagedHeadQCache(HeadQCache):
     assigned to ``block_table`` before a call."""
 
     def __init__(self, B, Hkv, d, r, page_size, num_pages, max_pages, vmode="dense",
-                 v_dtype=torch.bfloat16, device="cuda", block_table=None):
+                 v_dtype=torch.bfloat16, device="cuda", block_table=None, kmode="token"):
         if page_size <= 0 or page_size % 64:
             raise ValueError("page_size must be a positive multiple of 64")
         self.B, self.Hkv, self.d, self.r = B, Hkv, d, r
@@ -235,7 +246,7 @@ class PagedHeadQCache(HeadQCache):
         self.block_table = block_table.to(device=device, dtype=torch.int32).contiguous()
         if tuple(self.block_table.shape) != (B, max_pages):
             raise ValueError("block_table must be [B, max_pages]")
-        self._alloc((num_pages, Hkv, page_size), vmode, v_dtype, device)
+        self._alloc((num_pages, Hkv, page_size), vmode, v_dtype, device, kmode)
 
 
 def headq_calibrate(q_cal, Hkv, r, center=False, stream=None):

@@ -62,6 +62,12 @@ typedef enum {
 
 typedef enum { HEADQ_F32 = 0, HEADQ_BF16 = 1 } headq_dtype;
 
+/* The base code of the keys (B_b of summary section 3, step 2). */
+typedef enum {
+    HEADQ_K_TOKEN = 0,   /* per token, per group of 32 channels (the pages' reading) */
+    HEADQ_K_CHANNEL = 1  /* per channel, per block of 64 tokens (KIVI-style keys)   */
+} headq_kmode;
+
 typedef enum {
     HEADQ_V_DENSE = 0, /* V stored as v_dtype, [B, Hkv, T_cap, d]               */
     HEADQ_V_2BIT = 1   /* V stored with the 2-bit base code of the keys, no side */
@@ -91,7 +97,19 @@ typedef enum {
  * sequence.  Entries a call reaches must lie in [0, num_pages): a read of an
  * entry outside that range is redirected to page 0 and sets the device error
  * word (decode and diagnostic calls), a write to one is dropped.  With
- * page_size == 0 the last four fields are ignored.
+ * page_size == 0 the page fields are ignored.
+ *
+ * Key base code (kmode).  HEADQ_K_TOKEN is the layout above.  HEADQ_K_CHANNEL
+ * (an alternative base quantizer under the same side-code correction): each
+ * channel of each block of 64 consecutive tokens has its own minimum and scale
+ * (same arithmetic as the per-token code, taken along the block's tokens), so
+ * k_scale and k_min hold one row of d floats per block: plane row p of a token
+ * (b*Hkv + kv)*T_cap + t, or its paged row) has its block row at p / 64, i.e.
+ *   k_scale, k_min  fp32 [B, Hkv, T_cap/64, d]  (paged: [num_pages, Hkv, page_size/64, d])
+ * T_cap is a multiple of 64, writes start on a block boundary (t0 % 64 == 0)
+ * and a block's codes are fixed once written (headq_decode_append and the A^2
+ * fixup are unsupported in this mode); the tensor-core decode serves only the
+ * per-token code, the channel code is decoded by the generic kernel.
  */
 typedef struct {
     int B, Hkv, T_cap, d, r;
@@ -108,6 +126,7 @@ typedef struct {
     int num_pages;               /* pages in each plane's pool (paged)           */
     int max_pages;               /* block_table entries per sequence (paged)     */
     const int32_t *block_table;  /* [B, max_pages] pool page of each logical page */
+    headq_kmode kmode;           /* key base code, HEADQ_K_TOKEN by default       */
 } headq_cache;
 
 /* Library version as 10000*major + 100*minor + patch. */

@@ -56,15 +56,17 @@ def _load():
         lib.hqo_set_threads.restype = I
         lib.hqo_base_quantize.argtypes = [P, L, I, P, P, P]
         lib.hqo_base_dequantize.argtypes = [P, P, P, L, I, P]
-        lib.hqo_cache_write.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, P]
+        lib.hqo_cache_write.argtypes = [P, I, I, I, I, I, P, P, P, P, P, P, P, I, I]
+        lib.hqo_base_dequantize_channel.argtypes = [P, P, P, L, I, I, I, P]
         lib.hqo_side_dequantize.argtypes = [P, P, L, I, P]
         lib.hqo_side_quantize.argtypes = [P, L, I, P, P]
         lib.hqo_attend.argtypes = [P, I, I, I, I, I, I, P, P, P, P, P, D, D, P, P, P]
         lib.hqo_decode.argtypes = [P, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P,
-                                   P, P, P, D, D, P, P]
+                                   P, P, P, D, D, P, P, I, I]
         lib.hqo_attn_kl.argtypes = [P, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P,
-                                    P, P, P, P, P, D, D, P, P, P, P]
+                                    P, P, P, P, P, D, D, P, P, P, P, I, I]
         for f in ("hqo_base_quantize", "hqo_base_dequantize", "hqo_cache_write",
+                  "hqo_base_dequantize_channel",
                   "hqo_side_dequantize", "hqo_side_quantize", "hqo_attend", "hqo_decode", "hqo_attn_kl"):
             getattr(lib, f).restype = I
         _lib = lib
@@ -87,6 +89,10 @@ def _check(rc, what):
 def set_threads(n):
     """Number of OpenMP threads the oracle uses (returns the effective count)."""
     return _load().hqo_set_threads(int(n))
+
+
+KMODES = {"token": 0, "channel": 1}
+KBLOCK = 64  # tokens per block of the per-channel base code
 
 
 def group_size(d):
@@ -142,6 +148,18 @@ def base_quantize(x):
     return codes, sc, mn
 
 
+def base_dequantize_channel(codes, sc, mn, block=KBLOCK):
+    """Per-channel base code: codes [S..., T, d/4], sc/mn [S..., ceil(T/block), d]
+    -> k^ [S..., T, d] fp32, k^ = min_c + code * scale_c of the token's block."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    lead, T, d = codes.shape[:-2], codes.shape[-2], codes.shape[-1] * 4
+    seqs = int(np.prod(lead)) if lead else 1
+    out = np.zeros(lead + (T, d), np.float32)
+    _check(_load().hqo_base_dequantize_channel(_p(codes), _p(_f32(sc)), _p(_f32(mn)), seqs, T,
+                                               d, block, _p(out)), "base_dequantize_channel")
+    return out
+
+
 def base_dequantize(codes, sc, mn):
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     d = codes.shape[-1] * 4
@@ -153,9 +171,12 @@ def base_dequantize(codes, sc, mn):
     return out
 
 
-def cache_write(k, U, v=None, vmode="dense"):
+def cache_write(k, U, v=None, vmode="dense", kmode="token"):
     """Encode keys k [B, Hkv, n, d] (and 2-bit values when vmode == '2bit').
 
+    kmode 'token': the per-token group-32 base code (ks, km [B, Hkv, n, ng]);
+    kmode 'channel': the per-channel base code over blocks of KBLOCK tokens
+    counted from the first token written (ks, km [B, Hkv, ceil(n/KBLOCK), d]).
     Returns a dict of planes kc, ks, km, zc, zs (and vc, vs, vm) plus y, the
     projection U_h^T e before the side quantiser.
     """
@@ -164,17 +185,19 @@ def cache_write(k, U, v=None, vmode="dense"):
     B, Hkv, n, d = k.shape
     r = U.shape[-1]
     ng = d // group_size(d)
+    sshape = (B, Hkv, n, ng) if kmode == "token" else (B, Hkv, -(-n // KBLOCK), d)
     out = dict(
         kc=np.zeros((B, Hkv, n, d // 4), np.uint8),
-        ks=np.zeros((B, Hkv, n, ng), np.float32),
-        km=np.zeros((B, Hkv, n, ng), np.float32),
+        ks=np.zeros(sshape, np.float32),
+        km=np.zeros(sshape, np.float32),
         zc=np.zeros((B, Hkv, n, r // 2), np.uint8),
         zs=np.zeros((B, Hkv, n), np.float32),
         y=np.zeros((B, Hkv, n, r), np.float32),
     )
     _check(_load().hqo_cache_write(_p(k), B, Hkv, n, d, r, _p(U), _p(out["kc"]),
                                    _p(out["ks"]), _p(out["km"]), _p(out["zc"]),
-                                   _p(out["zs"]), _p(out["y"])), "cache_write")
+                                   _p(out["zs"]), _p(out["y"]), KMODES[kmode], KBLOCK),
+           "cache_write")
     if vmode == "2bit":
         out["vc"], out["vs"], out["vm"] = base_quantize(v)
     return out
@@ -243,7 +266,7 @@ def _vplanes(planes, vmode, v):
 
 
 def decode(q, planes, U, v=None, vmode="dense", sm_scale=None, sigma=1.0,
-           seq_lens=None):
+           seq_lens=None, kmode="token"):
     """Cache read from stored planes ([B, Hkv, T, ...]); returns (out, lse) fp64."""
     q = _f32(q)
     U = _f32(U)
@@ -260,7 +283,7 @@ def decode(q, planes, U, v=None, vmode="dense", sm_scale=None, sigma=1.0,
         _p(q), B, Hq, Hkv, T, d, r, _p(sl), _p(c(planes["kc"], np.uint8)),
         _p(_f32(planes["ks"])), _p(_f32(planes["km"])), _p(c(planes["zc"], np.uint8)),
         _p(_f32(planes["zs"])), _p(U), vm_, _p(vd), _p(vc), _p(vs), _p(vmn), sm,
-        float(sigma), _p(out), _p(lse)), "decode")
+        float(sigma), _p(out), _p(lse), KMODES[kmode], KBLOCK), "decode")
     return out, lse
 
 
@@ -359,7 +382,7 @@ def a2_mixed_values(v_hat, v_full, keep_idx):
 # Step 4: diagnostics (section 2 of the summary).
 # --------------------------------------------------------------------------
 def attn_kl(q, planes, U, k_full, v_full, v=None, vmode="dense", sm_scale=None,
-            sigma=1.0, seq_lens=None):
+            sigma=1.0, seq_lens=None, kmode="token"):
     """Returns (kl, fisher_var, a2_vdist, dout2), each fp64 [B, Hq]."""
     q = _f32(q)
     U = _f32(U)
@@ -375,8 +398,8 @@ def attn_kl(q, planes, U, k_full, v_full, v=None, vmode="dense", sm_scale=None,
         _p(q), B, Hq, Hkv, T, d, r, _p(sl), _p(c(planes["kc"], np.uint8)),
         _p(_f32(planes["ks"])), _p(_f32(planes["km"])), _p(c(planes["zc"], np.uint8)),
         _p(_f32(planes["zs"])), _p(U), vm_, _p(vd), _p(vc), _p(vs), _p(vmn),
-        _p(_f32(k_full)), _p(_f32(v_full)), sm, float(sigma), *[_p(a) for a in res]),
-        "attn_kl")
+        _p(_f32(k_full)), _p(_f32(v_full)), sm, float(sigma), *[_p(a) for a in res],
+        KMODES[kmode], KBLOCK), "attn_kl")
     return tuple(res)
 
 

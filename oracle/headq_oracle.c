@@ -120,6 +120,73 @@ static void base_dequantize_token(const uint8_t *packed, const float *scale,
     }
 }
 
+/* The alternative base code (KIVI-style per-channel keys): for one block of  */
+/* nt consecutive tokens x [nt, d] of one (b, kv), every channel c gets its  */
+/* own minimum and scale over the block's tokens, with the same arithmetic as */
+/* the per-token code (min/max, scale = (max - min)/3, rint half-even, clamp);*/
+/* codes are packed per token exactly as in the per-token layout.            */
+static void base_quantize_channel_block(const float *x, int nt, int d,
+                                        uint8_t *packed, float *scale,
+                                        float *minimum)
+{
+    memset(packed, 0, (size_t)nt * d / 4);
+    for (int c = 0; c < d; ++c) {
+        float lo = x[c], hi = x[c];
+        for (int t = 1; t < nt; ++t) {
+            const float v = x[(size_t)t * d + c];
+            if (v < lo) lo = v;
+            if (v > hi) hi = v;
+        }
+        lo = lo + 0.0f;
+        hi = hi + 0.0f;
+        const float s = (hi - lo) / 3.0f;
+        scale[c] = s;
+        minimum[c] = lo;
+        for (int t = 0; t < nt; ++t) {
+            int code = 0;
+            if (s != 0.0f) {
+                const float tq = nearbyintf((x[(size_t)t * d + c] - lo) / s);
+                code = tq < 0.0f ? 0 : (tq > 3.0f ? 3 : (int)tq);
+            }
+            packed[(size_t)t * (d / 4) + (c >> 2)] |= (uint8_t)(code << (2 * (c & 3)));
+        }
+    }
+}
+
+/* codes [seqs, T, d/4], scale/min [seqs, ceil(T/block), d] -> xhat [seqs, T, d] */
+HQO_API int hqo_base_dequantize_channel(const uint8_t *codes, const float *scale,
+                                        const float *minimum, int64_t seqs, int T,
+                                        int d, int block, float *xhat)
+{
+    if (!shape_ok(d, 0) || seqs < 0 || T < 0 || block <= 0) return HQO_BAD_ARG;
+    const int nblk = (T + block - 1) / block;
+#pragma omp parallel for schedule(static)
+    for (int64_t sq = 0; sq < seqs; ++sq)
+        for (int t = 0; t < T; ++t) {
+            const float *sc = scale + (sq * nblk + t / block) * d;
+            const float *mn = minimum + (sq * nblk + t / block) * d;
+            const uint8_t *pk = codes + (sq * T + t) * (d / 4);
+            for (int c = 0; c < d; ++c) {
+                const float prod = (float)code2_at(pk, c) * sc[c];
+                xhat[(sq * T + t) * d + c] = mn[c] + prod;
+            }
+        }
+    return HQO_OK;
+}
+
+HQO_API int hqo_base_dequantize(const uint8_t *codes, const float *scale,
+                                const float *minimum, int64_t rows, int d,
+                                float *xhat);
+
+static void dequantize_keys(int kmode, int block, const uint8_t *kc, const float *ks,
+                            const float *km, int64_t seqs, int T, int d, float *khat)
+{
+    if (kmode == 1)
+        hqo_base_dequantize_channel(kc, ks, km, seqs, T, d, block, khat);
+    else
+        hqo_base_dequantize(kc, ks, km, seqs * T, d, khat);
+}
+
 /* x: [rows, d] -> codes [rows, d/4], scale/min [rows, ng] */
 HQO_API int hqo_base_quantize(const float *x, int64_t rows, int d,
                               uint8_t *codes, float *scale, float *minimum)
@@ -192,11 +259,24 @@ static int nibble_at(const uint8_t *zc, int i)
  */
 HQO_API int hqo_cache_write(const float *k, int B, int Hkv, int n, int d, int r,
                             const float *U, uint8_t *kc, float *ks, float *km,
-                            uint8_t *zc, float *zs, float *y_out)
+                            uint8_t *zc, float *zs, float *y_out, int kmode, int block)
 {
     if (!shape_ok(d, r) || B < 0 || Hkv <= 0 || n < 0) return HQO_BAD_ARG;
+    if (kmode != 0 && (kmode != 1 || block <= 0)) return HQO_BAD_ARG;
     const int ng = d / group_size(d);
     const int64_t rows = (int64_t)B * Hkv * n;
+    if (kmode == 1) { /* per-channel base code over blocks of `block` tokens */
+        const int nblk = (n + block - 1) / block;
+#pragma omp parallel for schedule(static)
+        for (int64_t sb = 0; sb < (int64_t)B * Hkv * nblk; ++sb) {
+            const int64_t sq = sb / nblk;
+            const int t0 = (int)(sb % nblk) * block;
+            const int nt = n - t0 < block ? n - t0 : block;
+            base_quantize_channel_block(k + (sq * n + t0) * d, nt, d,
+                                        kc + (sq * n + t0) * (d / 4), ks + sb * d,
+                                        km + sb * d);
+        }
+    }
     int bad = 0;
 #pragma omp parallel
     {
@@ -212,9 +292,20 @@ HQO_API int hqo_cache_write(const float *k, int B, int Hkv, int n, int d, int r,
                 const int kv = (int)((row / n) % Hkv);
                 const float *x = k + row * d;
                 uint8_t *codes = kc + row * (d / 4);
-                float *sc = ks + row * ng, *mn = km + row * ng;
-                base_quantize_token(x, d, codes, sc, mn);
-                base_dequantize_token(codes, sc, mn, d, khat);
+                if (kmode == 1) {
+                    const int64_t sq = row / n;
+                    const int t = (int)(row % n), nblk = (n + block - 1) / block;
+                    const float *sc = ks + (sq * nblk + t / block) * d;
+                    const float *mn = km + (sq * nblk + t / block) * d;
+                    for (int c = 0; c < d; ++c) {
+                        const float prod = (float)code2_at(codes, c) * sc[c];
+                        khat[c] = mn[c] + prod;
+                    }
+                } else {
+                    float *sc = ks + row * ng, *mn = km + row * ng;
+                    base_quantize_token(x, d, codes, sc, mn);
+                    base_dequantize_token(codes, sc, mn, d, khat);
+                }
                 for (int c = 0; c < d; ++c) e[c] = x[c] - khat[c];
                 if (r > 0) {
                     side_project(e, U + (size_t)kv * d * r, d, r, y);
@@ -387,7 +478,8 @@ HQO_API int hqo_decode(const float *q, int B, int Hq, int Hkv, int T, int d, int
                        const float *km, const uint8_t *zc, const float *zs,
                        const float *U, int vmode, const float *v_dense,
                        const uint8_t *vc, const float *vs, const float *vm,
-                       double sm_scale, double sigma, double *out, double *lse)
+                       double sm_scale, double sigma, double *out, double *lse,
+                       int kmode, int block)
 {
     if (!shape_ok(d, r)) return HQO_BAD_ARG;
     const int64_t rows = (int64_t)B * Hkv * T;
@@ -397,7 +489,7 @@ HQO_API int hqo_decode(const float *q, int B, int Hq, int Hkv, int T, int d, int
     float *vv = NULL;
     int owned = 0, rc = HQO_NO_MEM;
     if (khat && zf && zhat) {
-        hqo_base_dequantize(kc, ks, km, rows, d, khat);
+        dequantize_keys(kmode, block, kc, ks, km, (int64_t)B * Hkv, T, d, khat);
         hqo_side_dequantize(zc, zs, rows, r, zf);
         for (int64_t i = 0; i < rows * r; ++i) zhat[i] = (double)zf[i];
         rc = values_as_read(vmode, v_dense, vc, vs, vm, rows, d, &vv, &owned);
@@ -432,7 +524,7 @@ HQO_API int hqo_attn_kl(const float *q, int B, int Hq, int Hkv, int T, int d, in
                         const uint8_t *vc, const float *vs, const float *vm,
                         const float *k_full, const float *v_full, double sm_scale,
                         double sigma, double *kl, double *fvar, double *a2v,
-                        double *dout2)
+                        double *dout2, int kmode, int block)
 {
     if (!shape_ok(d, r) || Hkv <= 0 || Hq % Hkv) return HQO_BAD_ARG;
     const int G = Hq / Hkv;
@@ -443,7 +535,7 @@ HQO_API int hqo_attn_kl(const float *q, int B, int Hq, int Hkv, int T, int d, in
     float *vv = NULL;
     int owned = 0, rc = HQO_NO_MEM;
     if (!khat || !zf || !zhat) goto done;
-    hqo_base_dequantize(kc, ks, km, rows, d, khat);
+    dequantize_keys(kmode, block, kc, ks, km, (int64_t)B * Hkv, T, d, khat);
     hqo_side_dequantize(zc, zs, rows, r, zf);
     for (int64_t i = 0; i < rows * r; ++i) zhat[i] = (double)zf[i];
     rc = values_as_read(vmode, v_dense, vc, vs, vm, rows, d, &vv, &owned);

@@ -164,6 +164,34 @@ def test_paged_cache_struct_on_host(hq):
     assert c2.block_table.tolist() == t.tolist()
 
 
+def test_channel_keys_rejects(hq):
+    """Per-channel keys: capacity and write offsets on 64-token blocks, no
+    single-token append, no A^2 fixup; an unknown key mode is an argument error."""
+    L = hq.lib()
+    assert _write(hq, make_cache(hq, kmode=7)) == 1
+    assert _write(hq, make_cache(hq, kmode=1, T_cap=1040)) == 2      # not a multiple of 64
+    assert _write(hq, make_cache(hq, kmode=1), t0=16, n=1) == 2       # not a block start
+    assert _write(hq, make_cache(hq, kmode=1), t0=64, n=0) == 0       # valid no-op
+    cs = make_cache(hq, kmode=1)
+    P = ctypes.c_void_p
+    assert L.headq_decode_append(ctypes.byref(cs), P(FAKE), None, 1, P(FAKE), 1, 4, None, 512,
+                                 P(FAKE), ctypes.c_float(0.1), 1, P(FAKE), None, P(FAKE),
+                                 1 << 30, None) == 2
+    assert L.headq_a2_value_fixup(ctypes.byref(cs), P(FAKE), 1, 4, None, 512, P(FAKE),
+                                  ctypes.c_float(0.1), 1, P(FAKE), P(FAKE), 1, 8, P(FAKE),
+                                  P(FAKE), None) == 2
+
+
+def test_channel_cache_struct_on_host(hq):
+    c = hq.HeadQCache(2, 4, 256, 128, 16, kmode="channel", device="cpu")
+    assert tuple(c.k_scale.shape) == (2, 4, 4, 128) and tuple(c.k_codes.shape) == (2, 4, 256, 32)
+    assert c.struct().kmode == 1 and c.nbytes_per_token() == 32 + 16 + 8 + 4 + 256
+    pc = hq.PagedHeadQCache(2, 4, 64, 8, 128, 5, 2, kmode="channel", device="cpu")
+    assert tuple(pc.k_min.shape) == (5, 4, 2, 64)
+    with pytest.raises(ValueError):
+        hq.HeadQCache(1, 1, 80, 64, 8, kmode="channel", device="cpu")
+
+
 def test_calibrate_rejects(hq):
     L = hq.lib()
     P = ctypes.c_void_p

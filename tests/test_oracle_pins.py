@@ -135,6 +135,124 @@ def test_base_code_is_nearest_level(d):
                 assert c[t, g * gs + k] == want
 
 
+# ---------------------------------------------------------------------------
+# The alternative base code: per-channel keys over 64-token blocks.
+# ---------------------------------------------------------------------------
+
+def test_channel_code_hand_example():
+    # d = 8, three tokens.  Channel 0 holds 1, 4, 2.5 -> min 1, scale 1, codes
+    # 0, 3, 2 (1.5 ties to even); channel 1 is constant -> scale 0, codes 0;
+    # every other channel holds 0, 3, 1.5 -> codes 0, 3, 2.
+    # Token 0 byte0 = 0|0<<2|0<<4|0<<6 = 0x00; token 1: 3|0<<2|3<<4|3<<6 = 0xF3;
+    # token 2: 2|0<<2|2<<4|2<<6 = 0xA2 (bytes 1 repeat channels 4..7: 0x00, 0xFF, 0xAA).
+    x = np.zeros((1, 1, 3, 8), np.float32)
+    x[0, 0, :, 0] = [1.0, 4.0, 2.5]
+    x[0, 0, :, 1] = 7.0
+    for c in range(2, 8):
+        x[0, 0, :, c] = [0.0, 3.0, 1.5]
+    U = np.zeros((1, 8, 2), np.float32)
+    pl = oracle.cache_write(x, U, kmode="channel")
+    assert pl["ks"].shape == (1, 1, 1, 8)
+    np.testing.assert_array_equal(pl["km"][0, 0, 0], [1, 7, 0, 0, 0, 0, 0, 0])
+    np.testing.assert_array_equal(pl["ks"][0, 0, 0], [1, 0, 1, 1, 1, 1, 1, 1])
+    np.testing.assert_array_equal(pl["kc"][0, 0], [[0x00, 0x00], [0xF3, 0xFF], [0xA2, 0xAA]])
+    khat = oracle.base_dequantize_channel(pl["kc"], pl["ks"], pl["km"])
+    np.testing.assert_array_equal(khat[0, 0, :, 0], [1.0, 4.0, 3.0])
+
+
+def test_channel_code_is_the_token_code_of_the_transpose():
+    """A block of 32 tokens quantised per channel is, arithmetic for arithmetic,
+    the per-token group-32 code of the transposed block (pinned above by hand
+    and by exhaustive search); with n = 70 the blocks are 64 + 6 tokens."""
+    rng = _rng(31)
+    for n in (32, 70):
+        x = synth.round_bf16((rng.standard_normal((2, 1, n, 64)) * 3 + 1).astype(np.float32))
+        pl = oracle.cache_write(x, np.zeros((1, 64, 2), np.float32), kmode="channel")
+        assert pl["ks"].shape == (2, 1, -(-n // 64), 64)
+        for b in range(2):
+            for blk, (t0, t1) in enumerate([(0, min(n, 64)), (64, n)][:-(-n // 64)]):
+                xt = np.ascontiguousarray(x[b, 0, t0:t1].T)          # [64 channels, nt]
+                if xt.shape[1] not in (32,):
+                    # not a group size: check min / scale and nearest levels directly
+                    mn = xt.min(axis=1) + np.float32(0)
+                    sc = (xt.max(axis=1) - xt.min(axis=1)) / np.float32(3)
+                    np.testing.assert_array_equal(pl["km"][b, 0, blk], mn)
+                    np.testing.assert_array_equal(pl["ks"][b, 0, blk], sc)
+                    c = _codes2(pl["kc"][b, 0, t0:t1], 64)           # [nt, 64]
+                    for ch in range(64):
+                        for t in range(t1 - t0):
+                            u = float(np.float32(xt[ch, t] - mn[ch]) / sc[ch])
+                            dist = [abs(u - lvl) for lvl in range(4)]
+                            best = [lvl for lvl in range(4) if dist[lvl] == min(dist)]
+                            want = best[0] if len(best) == 1 else [v for v in best if v % 2 == 0][0]
+                            assert c[t, ch] == want
+                    continue
+                codes_t, sc_t, mn_t = oracle.base_quantize(xt)           # per channel row
+                np.testing.assert_array_equal(pl["km"][b, 0, blk], mn_t[:, 0])
+                np.testing.assert_array_equal(pl["ks"][b, 0, blk], sc_t[:, 0])
+                np.testing.assert_array_equal(_codes2(pl["kc"][b, 0, t0:t1], 64).T,
+                                              _codes2(codes_t, t1 - t0))
+
+
+def test_channel_code_is_equivariant_to_a_shared_translation():
+    """Adding the same vector mu to every key (a softmax-null component, summary
+    section 2.1) leaves the per-channel codes, scales and residuals unchanged
+    and shifts the minima by mu, so the HeadQ attention is unchanged; the
+    per-token group code is not equivariant and its attention moves.  Values on
+    a dyadic grid keep every sum exact."""
+    rng = _rng(33)
+    B, Hkv, T, d, r = 1, 2, 128, 32, 8
+    # every channel of every 64-token block spans exactly 0.75 (scale 0.25):
+    # x = m + 0.25 j + delta, with the block's first two tokens at the ends
+    m = (rng.integers(-64, 64, size=(B, Hkv, 2, 1, d)) / 16).astype(np.float32)
+    j = rng.integers(0, 4, size=(B, Hkv, 2, 64, d))
+    delta = rng.integers(-3, 4, size=(B, Hkv, 2, 64, d)) / 64
+    delta = np.where(j == 0, np.abs(delta), np.where(j == 3, -np.abs(delta), delta))
+    j[..., 0, :], j[..., 1, :] = 0, 3
+    delta[..., 0:2, :] = 0
+    k = (m + 0.25 * j + delta).astype(np.float32).reshape(B, Hkv, T, d)
+    mu = (rng.integers(-256, 256, size=d) / 8).astype(np.float32)
+    v = rng.standard_normal((B, Hkv, T, d)).astype(np.float32)
+    q = rng.standard_normal((B, 4, d)).astype(np.float32)
+    U = np.stack([synth.random_orthonormal(rng, d, r) for _ in range(Hkv)])
+    outs = {}
+    for mode in ("channel", "token"):
+        p0 = oracle.cache_write(k, U, kmode=mode)
+        p1 = oracle.cache_write(k + mu, U, kmode=mode)
+        o0, _ = oracle.decode(q, p0, U, v=v, kmode=mode)
+        o1, _ = oracle.decode(q, p1, U, v=v, kmode=mode)
+        outs[mode] = (p0, p1, o0, o1)
+    p0, p1, o0, o1 = outs["channel"]
+    for name in ("kc", "ks", "zc", "zs", "y"):
+        np.testing.assert_array_equal(p1[name], p0[name])
+    np.testing.assert_array_equal(p1["km"], p0["km"] + mu)
+    np.testing.assert_allclose(o1, o0, rtol=1e-11, atol=1e-12)
+    p0, p1, o0, o1 = outs["token"]
+    assert not np.array_equal(p1["kc"], p0["kc"])
+    assert np.abs(o1 - o0).max() > 1e-3
+
+
+def test_null_space_intervention_hurts_only_the_non_equivariant_code():
+    """Summary section 4 (null-space interventions): restoring a softmax-null
+    mean component raises the Fisher damage sharply for a non-equivariant code
+    and leaves an equivariant one alone.  Synthetic keys of the 28q/4kv layer
+    (reduced), with and without a shared mean of scale 4 added after RoPE."""
+    w = configs.workload(2).with_(B=2, T=512, n_cal=256)
+    L = synth.make_layer(w)
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    mu = (16.0 * _rng(35).standard_normal(w.d)).astype(np.float32)
+    for sigma in (0.0, 1.0):       # the base code alone, and with the HeadQ correction
+        fv = {}
+        for mode in ("token", "channel"):
+            for tag, k in (("plain", L.keys), ("mean", L.keys + mu)):
+                pl = oracle.cache_write(k, U, kmode=mode)
+                _, f, _, _ = oracle.attn_kl(L.queries, pl, U, k, L.values, v=L.values,
+                                            kmode=mode, sigma=sigma)
+                fv[mode, tag] = float(np.mean(f))
+        assert fv["token", "mean"] > 2.5 * fv["token", "plain"]
+        assert abs(fv["channel", "mean"] / fv["channel", "plain"] - 1) < 0.05
+
+
 def test_projection_exact_rational_sequential_fma():
     """y_i = fl(... fl(fl(U_0i e_0) + U_1i e_1) ...) in channel order (d=8, r=4)."""
     rng = _rng(3)
