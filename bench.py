@@ -607,10 +607,6 @@ def cp_rank_row(torch, hq, w, q, U, cache, timed, hbm_row):
 
 A2_OBS = 16        # observation queries per sequence
 A2_KEEP = 0.05     # fraction of each sequence's tokens whose values stay exact
-# fp32 FMA lanes per SM per clock (CUDA cores) on B200
-FP32_FMA_PER_SM_CLK = 128
-
-
 def a2_policy_row(torch, hq, w, q, U, cache, k_all, v_all, dt, L, timed, gtimed, hbm_row):
     """The A^2 value policy on this workload: scores from A2_OBS observation
     queries per sequence (two logit passes on CUDA cores, against the fp32 ALU
@@ -636,19 +632,47 @@ def a2_policy_row(torch, hq, w, q, U, cache, k_all, v_all, dt, L, timed, gtimed,
 
     ms_dec = gtimed(lambda: hq.headq_decode_attn(cache, q, U, T=T, out=out, lse=lse, ws=dws))
     ms_df = gtimed(dec_fix)
-    flops = 2 * 2.0 * B * Hq * A2_OBS * T * d   # two passes of the observation logits
-    sm_count = torch.cuda.get_device_properties(0).multi_processor_count
-    pk = sm_count * FP32_FMA_PER_SM_CLK * 2 * 1965e6 / 1e12
-    tf = flops / (ms_sc * 1e-3) / 1e12
+    # the scores must read the exact keys and values, the cached 2-bit value
+    # planes, and write one score per token (the second pass's re-read of the
+    # keys is not algorithmic)
+    esz = k_all.element_size()
+    sc_bytes = B * Hkv * T * (2 * d * esz + (d // 4 + 8 * (d // min(32, d))) + 4)
+    sc_gbs = sc_bytes / (ms_sc * 1e-3) / 1e9
     keep_bytes = B * Hkv * K * (4 + d * keep_v.element_size())
     row = hbm_row(ms_df, B * Hkv * T * cache.nbytes_per_token() + keep_bytes, kept_per_seq=K,
                   observation_queries=A2_OBS, decode_ms=ms_dec, fixup_ms=ms_df - ms_dec,
                   select_ms=ms_sel, note="ms = decode + value fixup (CUDA graph of 20); "
-                  "scores_roofline: the two observation-logit passes on CUDA cores")
+                  "scores_roofline: the observation-logit passes (tensor cores for bf16)")
     row["scores_ms"] = ms_sc
-    row["scores_roofline"] = {"bound": "alu", "achieved": tf, "peak": pk, "unit": "TFLOP/s",
-                              "frac": tf / pk, "peak_kind": "fp32 CUDA cores from unit counts "
-                              "and max clock", "work": "2 passes x 2*B*Hq*n_obs*T*d flops"}
+    row["scores_roofline"] = dict(row["roofline"], achieved=sc_gbs,
+                                  frac=sc_gbs / row["roofline"]["peak"], traffic=None,
+                                  work="exact K and V, cached 2-bit value planes, scores")
+    row["scores_algorithmic_bytes"] = sc_bytes
+    return row
+
+
+def channel_keys_row(torch, hq, w, q, U, k_all, v_all, dt, timed, gtimed, hbm_row):
+    """The alternative base code (per-channel keys over 64-token blocks) on this
+    workload: the prefill write and the decode (generic kernel), each against HBM."""
+    B, Hkv, T, d = w.B, w.Hkv, w.T, w.d
+    if T % 64:
+        return None
+    c = hq.HeadQCache(B, Hkv, T, d, w.r, vmode=w.vmode, v_dtype=dt, device=q.device,
+                      kmode="channel")
+    ms_w = timed(lambda: hq.headq_cache_write(c, k_all, v_all, U), 3)
+    ws = hq.decode_workspace(c, w.Hq, T)
+    out = torch.empty((B, w.Hq, d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, w.Hq), dtype=torch.float32, device=q.device)
+    ms_d = gtimed(lambda: hq.headq_decode_attn(c, q, U, T=T, out=out, lse=lse, ws=ws), reps=5,
+                  replays=3)
+    tok = B * Hkv * T
+    planes = tok * c.nbytes_per_token()
+    row = hbm_row(ms_d, planes, write_ms=ms_w, bytes_per_token=c.nbytes_per_token(),
+                  note="ms: headq_decode_attn (generic kernel) on the per-channel code; "
+                       "write_roofline: the prefill write")
+    gbs = (tok * d * 2 * k_all.element_size() + planes) / (ms_w * 1e-3) / 1e9
+    row["write_roofline"] = dict(row["roofline"], achieved=gbs, frac=gbs / row["roofline"]["peak"])
+    del c
     return row
 
 
@@ -710,6 +734,8 @@ def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream, L):
     rows["attn_kl"] = hbm_row(ms, kv_in + planes, note="reads the packed cache and full K,V")
     rows["decode_paged"] = paged_decode_row(torch, hq, w, q, U, cache, gtimed, hbm_row)
     rows["context_parallel_rank"] = cp_rank_row(torch, hq, w, q, U, cache, gtimed, hbm_row)
+    rows["channel_keys"] = channel_keys_row(torch, hq, w, q, U, k_all, v_all, dt, timed, gtimed,
+                                            hbm_row)
     if w.vmode == "2bit":  # the policy chooses which 2-bit values to keep exact
         rows["a2_policy"] = a2_policy_row(torch, hq, w, q, U, cache, k_all, v_all, dt, L, timed,
                                           gtimed, hbm_row)

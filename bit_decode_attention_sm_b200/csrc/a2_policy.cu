@@ -53,7 +53,8 @@ struct A2Params {
   bool kv_bf16;
   float sm_scale;
   int ntiles;
-  float2* part;   // [B*Hkv, ntiles, 2, NQ] (max, exp-sum) per tile half
+  int ppt;        // partials per tile: 2 (CUDA-core pass) or 4 (tensor-core pass)
+  float2* part;   // [B*Hkv, ntiles, ppt, NQ] (max, exp-sum) per tile part
   float* lse;     // [B*Hkv, NQ], query index o*G + g
   float* scores;  // [B*Hkv, T]
   unsigned* err;
@@ -196,7 +197,7 @@ __global__ void __launch_bounds__(kAThreads) a2_pass_kernel(const A2Params p) {
         for (int o2 = 16; o2 > 0; o2 >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o2);
         if ((tid & 31) == 0) {
           const int half = (j >> 5);
-          p.part[((bk * p.ntiles + tile) * 2 + half) * NQ + q0 + qq] = make_float2(m, l);
+          p.part[((bk * p.ntiles + tile) * p.ppt + half) * NQ + q0 + qq] = make_float2(m, l);
         }
       } else {
         const float pj = valid ? expf(sv - p.lse[bk * NQ + q0 + qq]) : 0.0f;
@@ -215,17 +216,177 @@ __global__ void __launch_bounds__(kAThreads) a2_pass_kernel(const A2Params p) {
   }
 }
 
+// ---- the same two passes on tensor cores, for bf16 keys and queries ---------
+// A 64-token tile, 4 warps of 16 tokens; observation queries in chunks of 64.
+// Logits = K_tile (A, row-major, tokens x channels) times Q^T (B: each query's
+// channels are a column), mma.sync m16n8k16 bf16 -> fp32: products of bf16
+// values are exact, so this differs from the CUDA-core pass only in the order
+// of the fp32 sums.  Both operands come from padded shared-memory rows with
+// 32-bit loads (row stride D + 8: lanes of a fragment hit distinct banks).
+constexpr int kMT = 128;   // threads: 4 warps x 16 tokens
+constexpr int kMQ = 64;    // queries per chunk: 8 n8 tiles
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
+      " {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int D, bool SCORE>
+__global__ void __launch_bounds__(kMT) a2_pass_mma_kernel(const A2Params p) {
+  constexpr int RS = D + 8;  // bf16 elements per shared row
+  constexpr int KSTEPS = D / 16;
+  extern __shared__ __align__(16) unsigned char a2m_smem[];
+  uint16_t* k_s = reinterpret_cast<uint16_t*>(a2m_smem);          // [kAT][RS]
+  uint16_t* q_s = k_s + kAT * RS;                                   // [kMQ][RS]
+  float* dv2_s = reinterpret_cast<float*>(q_s + kMQ * RS);         // [kAT]
+
+  const int tile = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int Tb = seq_len(p.seq_lens, b, p.T);
+  const int t0 = tile * kAT;
+  const int G = p.G, NQ = p.n_obs * G;
+  const size_t bk = static_cast<size_t>(b) * p.c.Hkv + kv;
+  const uint16_t* kf = static_cast<const uint16_t*>(p.k_full);
+  const uint16_t* qo = static_cast<const uint16_t*>(p.q_obs);
+
+  for (int e = tid; e < kAT * (D / 8); e += kMT) {
+    const int row = e / (D / 8), c8 = e - row * (D / 8);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (t0 + row < Tb) v = *reinterpret_cast<const uint4*>(kf + (bk * p.T + t0 + row) * D + c8 * 8);
+    *reinterpret_cast<uint4*>(k_s + row * RS + c8 * 8) = v;
+  }
+  if constexpr (SCORE) {  // |v^_j - v_j|^2: two threads per token, half the channels each
+    const int j = tid >> 1, half = tid & 1;
+    float a = 0.0f;
+    if (t0 + j < Tb) {
+      const size_t row = cache_row_read(p.c, b, kv, t0 + j, half == 0 ? p.err : nullptr);
+      for (int c0 = half * (D / 2); c0 < (half + 1) * (D / 2); c0 += 8) {
+        float v[8], vh[8];
+        load8(p.v_full, (bk * p.T + t0 + j) * D + c0, true, v);
+        value_hat8(p.c, row, c0, D, vh);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float dv = vh[k] - v[k];
+          a = fmaf(dv, dv, a);
+        }
+      }
+    }
+    a += __shfl_xor_sync(0xffffffffu, a, 1);
+    if (half == 0) dv2_s[j] = a;
+  }
+  __syncthreads();
+
+  // this warp's 16 tokens as A fragments, all k-steps
+  uint32_t af[KSTEPS][4];
+  {
+    const uint16_t* r0 = k_s + (16 * warp + g) * RS + 2 * t;
+    const uint16_t* r1 = r0 + 8 * RS;
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+      af[ks][0] = *reinterpret_cast<const uint32_t*>(r0 + 16 * ks);
+      af[ks][1] = *reinterpret_cast<const uint32_t*>(r1 + 16 * ks);
+      af[ks][2] = *reinterpret_cast<const uint32_t*>(r0 + 16 * ks + 8);
+      af[ks][3] = *reinterpret_cast<const uint32_t*>(r1 + 16 * ks + 8);
+    }
+  }
+  const int tok0 = t0 + 16 * warp + g, tok1 = tok0 + 8;
+  const bool v0 = tok0 < Tb, v1 = tok1 < Tb;
+  float acc0 = 0.0f, acc1 = 0.0f;  // SCORE: sum of p^2 for tokens tok0, tok1
+
+  for (int q0 = 0; q0 < NQ; q0 += kMQ) {
+    const int nq = min(kMQ, NQ - q0);
+    __syncthreads();  // every warp is done with the previous chunk
+    for (int e = tid; e < kMQ * (D / 8); e += kMT) {
+      const int qq = e / (D / 8), c8 = e - qq * (D / 8);
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (qq < nq) {
+        const int qi = q0 + qq, o = qi / G, gq = qi - o * G;
+        v = *reinterpret_cast<const uint4*>(
+            qo + ((static_cast<size_t>(b) * p.n_obs + o) * p.Hq + kv * G + gq) * D + c8 * 8);
+      }
+      *reinterpret_cast<uint4*>(q_s + qq * RS + c8 * 8) = v;
+    }
+    __syncthreads();
+    float c[kMQ / 8][4];
+#pragma unroll
+    for (int nt = 0; nt < kMQ / 8; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.0f;
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+#pragma unroll
+      for (int nt = 0; nt < kMQ / 8; ++nt) {
+        if (8 * nt >= nq) break;  // uniform across the CTA
+        const uint16_t* qr = q_s + (8 * nt + g) * RS + 16 * ks + 2 * t;
+        mma_bf16_16816(c[nt], af[ks], *reinterpret_cast<const uint32_t*>(qr),
+                       *reinterpret_cast<const uint32_t*>(qr + 8));
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < kMQ / 8; ++nt) {
+      if (8 * nt >= nq) break;
+      const int n0 = 8 * nt + 2 * t;  // this lane's two query columns n0, n0 + 1
+      const float s00 = v0 ? c[nt][0] * p.sm_scale : -INFINITY;
+      const float s01 = v0 ? c[nt][1] * p.sm_scale : -INFINITY;
+      const float s10 = v1 ? c[nt][2] * p.sm_scale : -INFINITY;
+      const float s11 = v1 ? c[nt][3] * p.sm_scale : -INFINITY;
+      if constexpr (!SCORE) {
+        float m0 = fmaxf(s00, s10), m1 = fmaxf(s01, s11);
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) {
+          m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o2));
+          m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o2));
+        }
+        float l0 = (v0 ? expf(s00 - m0) : 0.0f) + (v1 ? expf(s10 - m0) : 0.0f);
+        float l1 = (v0 ? expf(s01 - m1) : 0.0f) + (v1 ? expf(s11 - m1) : 0.0f);
+#pragma unroll
+        for (int o2 = 4; o2 < 32; o2 <<= 1) {
+          l0 += __shfl_xor_sync(0xffffffffu, l0, o2);
+          l1 += __shfl_xor_sync(0xffffffffu, l1, o2);
+        }
+        if (g == 0) {
+          float2* dst = p.part + ((bk * p.ntiles + tile) * p.ppt + warp) * NQ + q0;
+          if (n0 < nq) dst[n0] = make_float2(m0, l0);
+          if (n0 + 1 < nq) dst[n0 + 1] = make_float2(m1, l1);
+        }
+      } else {
+        const float* lse = p.lse + bk * NQ + q0;
+        const float l0 = n0 < nq ? lse[n0] : 0.0f, l1 = n0 + 1 < nq ? lse[n0 + 1] : 0.0f;
+        const float p00 = (v0 && n0 < nq) ? expf(s00 - l0) : 0.0f;
+        const float p01 = (v0 && n0 + 1 < nq) ? expf(s01 - l1) : 0.0f;
+        const float p10 = (v1 && n0 < nq) ? expf(s10 - l0) : 0.0f;
+        const float p11 = (v1 && n0 + 1 < nq) ? expf(s11 - l1) : 0.0f;
+        acc0 = fmaf(p00, p00, fmaf(p01, p01, acc0));
+        acc1 = fmaf(p10, p10, fmaf(p11, p11, acc1));
+      }
+    }
+  }
+  if constexpr (SCORE) {
+    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
+    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
+    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
+    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
+    if (t == 0) {
+      if (tok0 < p.T) p.scores[bk * p.T + tok0] = v0 ? acc0 * dv2_s[16 * warp + g] : 0.0f;
+      if (tok1 < p.T) p.scores[bk * p.T + tok1] = v1 ? acc1 * dv2_s[16 * warp + g + 8] : 0.0f;
+    }
+  }
+}
+
 // lse of every observation query from the tile partials; one CTA per (b, kv)
 __global__ void a2_lse_kernel(const A2Params p) {
   const size_t bk = blockIdx.x;
   const int NQ = p.n_obs * p.G;
   for (int qi = threadIdx.x; qi < NQ; qi += blockDim.x) {
+    const int ne = p.ppt * p.ntiles;
     float M = -INFINITY;
-    for (int e = 0; e < 2 * p.ntiles; ++e) M = fmaxf(M, p.part[(bk * p.ntiles * 2 + e) * NQ + qi].x);
+    for (int e = 0; e < ne; ++e) M = fmaxf(M, p.part[(bk * ne + e) * NQ + qi].x);
     float L = 0.0f;
     if (M != -INFINITY)
-      for (int e = 0; e < 2 * p.ntiles; ++e) {
-        const float2 ml = p.part[(bk * p.ntiles * 2 + e) * NQ + qi];
+      for (int e = 0; e < ne; ++e) {
+        const float2 ml = p.part[(bk * ne + e) * NQ + qi];
         if (ml.x != -INFINITY) L += ml.y * expf(ml.x - M);
       }
     p.lse[bk * NQ + qi] = M == -INFINITY ? -INFINITY : M + logf(L);
@@ -533,12 +694,25 @@ int score_tiles(int T) { return (T + kAT - 1) / kAT; }
 size_t a2_ws_bytes(const headq_cache* c, int n_obs, int Hq, int T) {
   const size_t NQ = static_cast<size_t>(n_obs) * (Hq / c->Hkv);
   const size_t units = static_cast<size_t>(c->B) * c->Hkv;
-  return kWsHeaderBytes + round256(sizeof(float2) * units * score_tiles(T) * 2 * NQ) +
+  return kWsHeaderBytes + round256(sizeof(float2) * units * score_tiles(T) * 4 * NQ) +
          round256(sizeof(float) * units * NQ);
 }
 
 template <int D>
-cudaError_t launch_scores(const A2Params& p, cudaStream_t s) {
+cudaError_t launch_scores(A2Params p, cudaStream_t s) {
+  dim3 grid(p.ntiles, p.c.Hkv, p.c.B);
+  const int NQ = p.n_obs * p.G;
+  if constexpr (D == 64 || D == 128) {
+    if (p.kv_bf16 && p.q_bf16) {  // tensor cores
+      p.ppt = 4;
+      const size_t smem = sizeof(uint16_t) * (kAT + kMQ) * (D + 8) + sizeof(float) * kAT;
+      a2_pass_mma_kernel<D, false><<<grid, kMT, smem, s>>>(p);
+      a2_lse_kernel<<<p.c.B * p.c.Hkv, NQ < 1024 ? (NQ + 31) / 32 * 32 : 1024, 0, s>>>(p);
+      a2_pass_mma_kernel<D, true><<<grid, kMT, smem, s>>>(p);
+      return cudaGetLastError();
+    }
+  }
+  p.ppt = 2;
   const size_t smem = sizeof(float) * (kAT * (D + 4) + kAQC * D + kAThreads + kAT);
   auto k0 = a2_pass_kernel<D, false>;
   auto k1 = a2_pass_kernel<D, true>;
@@ -550,9 +724,7 @@ cudaError_t launch_scores(const A2Params& p, cudaStream_t s) {
                                static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(p.ntiles, p.c.Hkv, p.c.B);
   k0<<<grid, kAThreads, smem, s>>>(p);
-  const int NQ = p.n_obs * p.G;
   a2_lse_kernel<<<p.c.B * p.c.Hkv, NQ < 1024 ? (NQ + 31) / 32 * 32 : 1024, 0, s>>>(p);
   k1<<<grid, kAThreads, smem, s>>>(p);
   return cudaGetLastError();
@@ -623,7 +795,7 @@ HEADQ_API headq_status headq_a2_scores(const headq_cache* cache, const void* q_o
   const size_t NQ = static_cast<size_t>(n_obs) * p.G;
   p.part = reinterpret_cast<float2*>(static_cast<char*>(ws) + kWsHeaderBytes);
   p.lse = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeaderBytes +
-                                   round256(sizeof(float2) * units * p.ntiles * 2 * NQ));
+                                   round256(sizeof(float2) * units * p.ntiles * 4 * NQ));
   p.scores = scores;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;

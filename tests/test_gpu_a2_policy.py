@@ -42,14 +42,20 @@ def _to(w, a):
 
 
 CASES = [(4, dict(T=700, B=3), [700, 300, 64]), (4, dict(T=333, B=2), None),
-         (2, dict(T=500, B=2), [500, 1])]
+         (2, dict(T=500, B=2), [500, 1]), (0, {}, [300])]
 
 
-@pytest.mark.parametrize("i,kw,sl", CASES, ids=["cfg4-ragged", "cfg4", "cfg2-dense"])
+@pytest.mark.parametrize("i,kw,sl", CASES,
+                         ids=["cfg4-ragged", "cfg4", "cfg2-dense", "cfg0-fp32-2bit"])
 def test_a2_scores_match_oracle(i, kw, sl):
+    """bf16 workloads take the tensor-core passes, fp32 the CUDA-core ones."""
     import torch
     hq = _headq()
     w, L, U, planes, vh, qo = _setup(i, **kw)
+    if w.kv_dtype == "f32":  # give the fp32 workload 2-bit values, so a_j is not 0
+        w = w.with_(vmode="2bit")
+        planes = oracle.cache_write(L.keys, U, v=L.values, vmode="2bit")
+        vh = oracle.cached_values(planes, "2bit")
     sl = None if sl is None else np.array(sl, np.int32)
     ref = oracle.a2_scores(qo, L.keys, L.values, vh, seq_lens=sl)
     cache, Ut = gpu_cache(w, L, U)
