@@ -93,10 +93,11 @@ constexpr size_t smem_bytes() {
   // stages | per-warp value code tiles | q [GM][D] | group sums [GM][NG] |
   // sigma U^T q [GM][R] | U [D][R] | appended token's residual [D] and
   // projection [R] | barriers
+  // ... | the query as bulk-copied (raw bf16 or fp32) [GM][D] | barriers
   return 1024 + size_t(kStagesFor<NT>) * L::kStage + size_t(kCW) * L::kCodeTile + bq_bytes +
          sizeof(float) * ((4 * NT) * (D + L::NG + (R > 0 ? R : 1)) + D * (R > 0 ? R : 1) + D +
-                          (R > 0 ? R : 1)) +
-         16 * kStagesFor<NT> + 32;
+                          (R > 0 ? R : 1) + (4 * NT) * D) +
+         16 * kStagesFor<NT> + 64;  // barriers (2 kStages + 2) and two 16-byte alignments
 }
 
 // ---------------------------------------------------------------- PTX helpers
@@ -271,10 +272,15 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   float* u_s = qt_s + GM * RR;                                                // [D][RR]
   float* enew_s = u_s + D * RR;                                               // [D]
   float* ynew_s = enew_s + D;                                                 // [RR]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(
+  // [GM][D] floats of room, 16-byte aligned (a bulk-copy destination): the query
+  // as copied (bf16 or fp32)
+  float* qraw_s = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(ynew_s + RR) + 15) & ~uintptr_t(15));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(qraw_s + GM * D) + 15) & ~uintptr_t(15));
   // bars[s] = stage full, bars[kStages + s] = stage empty, bars[2 kStages] = the
-  // appended token is in HBM
+  // appended token is in HBM, bars[2 kStages + 1] = the query and U_h are in
+  // shared memory
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
@@ -296,6 +302,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       mbar_init(smem_addr(&bars[kStages + s]), kCW);
     }
     mbar_init(smem_addr(&bars[2 * kStages]), 1);
+    mbar_init(smem_addr(&bars[2 * kStages + 1]), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -303,6 +310,19 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   // ------------------------------------------------------------ producer warp
   // starts streaming at once; the consumers prepare the query meanwhile
   if (warp == kCW) {
+    if (lane == 0) {
+      // the query and U_h first: they head the copy queue, so the consumers'
+      // preparation does not wait behind the cache stream
+      const uint32_t qbar = smem_addr(&bars[2 * kStages + 1]);
+      const uint32_t qbytes = static_cast<uint32_t>(G * D * (p.q_bf16 ? 2 : 4));
+      mbar_expect_tx(qbar, qbytes + (R > 0 ? D * R * 4 : 0));
+      bulk_g2s(smem_addr(qraw_s),
+               static_cast<const uint8_t*>(p.q) +
+                   (static_cast<size_t>(b) * p.Hq + h0) * D * (p.q_bf16 ? 2 : 4),
+               qbytes, qbar);
+      if constexpr (R > 0)
+        bulk_g2s(smem_addr(u_s), p.U + static_cast<size_t>(kv) * D * R, D * R * 4, qbar);
+    }
     if (lane == 0 && ntiles > 0) {
       bool ok = true;
       int issued = 0;
@@ -356,14 +376,11 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   }
 
   // ------------------------------------------------------------ consumer warps
-  // query prep: q, U_h, group sums, sigma * U_h^T q
+  // query prep: q and U_h (bulk-copied by the producer), group sums, sigma U_h^T q
+  if (!mbar_wait(smem_addr(&bars[2 * kStages + 1]), 0) && tid == 0 && p.err)
+    atomicOr(p.err, kDevErrWaitTimeout);
   for (int i = tid; i < GM * D; i += kCT)
-    q_s[i] = i < G * D ? load_elem(p.q, (static_cast<size_t>(b) * p.Hq + h0) * D + i, p.q_bf16)
-                       : 0.0f;
-  if constexpr (R > 0) {
-    const float4* U4 = reinterpret_cast<const float4*>(p.U + static_cast<size_t>(kv) * D * R);
-    for (int i = tid; i < D * R / 4; i += kCT) reinterpret_cast<float4*>(u_s)[i] = U4[i];
-  }
+    q_s[i] = i < G * D ? load_elem(qraw_s, i, p.q_bf16) : 0.0f;
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   for (int i = tid; i < GM * NG; i += kCT) {
     const int h = i / NG, g = i - h * NG;
