@@ -97,7 +97,8 @@ constexpr size_t smem_bytes() {
   return 1024 + size_t(kStagesFor<NT>) * L::kStage + size_t(kCW) * L::kCodeTile + bq_bytes +
          sizeof(float) * ((4 * NT) * (D + L::NG + (R > 0 ? R : 1)) + D * (R > 0 ? R : 1) + D +
                           (R > 0 ? R : 1) + (4 * NT) * D) +
-         16 * kStagesFor<NT> + 64;  // barriers (2 kStages + 2) and two 16-byte alignments
+         32 * kStagesFor<NT> + 64;  // barriers (2 kStages + 2), stage tile starts,
+                                    // two 16-byte alignments
 }
 
 // ---------------------------------------------------------------- PTX helpers
@@ -246,6 +247,65 @@ __device__ __forceinline__ uint32_t bf16_part_pair1(float a, float b, float lo_f
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
+// The new token of sequence b, KV head kv, encoded into cache position pos
+// exactly as the cache write does (bit-exact codec): lanes 0..NG-1 take the key
+// groups, NG..2NG-1 the value groups, lanes < R the side rows.  Warp-wide; U_h
+// is in shared memory, enew_s is [D] scratch.
+template <int D, int R, bool V2>
+__device__ __forceinline__ void encode_new_token(const DecodeParams& p, int b, int kv, int pos,
+                                                 const float* u_s, float* enew_s, int lane) {
+  constexpr int NG = D / 32;
+  const size_t bk = static_cast<size_t>(b) * p.c.Hkv + kv;
+  const long long orow = cache_row(p.c, b, kv, pos);
+  if (orow < 0 && lane == 0 && p.err) atomicOr(p.err, kDevErrBadPage);
+  const size_t row = orow < 0 ? 0 : static_cast<size_t>(orow);
+  const size_t in = bk * D;
+  if (orow < 0) {
+    // a block-table entry outside the pool: the token is not written
+  } else if (lane < NG) {
+    float x[32];
+    uint32_t packed[2];
+    float sc, mn;
+    codec::load_row<32>(p.k_new, in + lane * 32, p.new_bf16, x);
+    codec::quantize_group<32, true>(x, packed, sc, mn);
+    codec::store_codes<32>(p.c.k_codes + row * (D / 4) + lane * 8, packed);
+    p.c.k_scale[row * NG + lane] = sc;
+    p.c.k_min[row * NG + lane] = mn;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) enew_s[lane * 32 + k] = x[k];
+  } else if (lane < 2 * NG && p.v_new != nullptr) {
+    const int gv = lane - NG;
+    float vv[32];
+    codec::load_row<32>(p.v_new, in + gv * 32, p.new_bf16, vv);
+    if constexpr (V2) {
+      uint32_t packed[2];
+      float sc, mn;
+      codec::quantize_group<32, false>(vv, packed, sc, mn);
+      codec::store_codes<32>(p.c.v_codes + row * (D / 4) + gv * 8, packed);
+      p.c.v_scale[row * NG + gv] = sc;
+      p.c.v_min[row * NG + gv] = mn;
+    } else {
+      codec::store_values<32>(p.c.v, row * D + gv * 32, true, vv);
+    }
+  }
+  __syncwarp();
+  if (R > 0 && orow >= 0) {
+    float y = 0.0f;
+    if (lane < R)
+      for (int c = 0; c < D; ++c) y = __fmaf_rn(u_s[c * R + lane], enew_s[c], y);
+    float a = lane < R ? fabsf(y) : 0.0f;
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o2));
+    const float zs = codec::side_scale(a);
+    const int w = lane < R ? codec::side_level(y, zs, __frcp_rn(zs)) : 0;
+    const int w_next = __shfl_down_sync(kFull, w, 1);
+    if (lane < R && (lane & 1) == 0)
+      p.c.z_codes[row * (R / 2) + (lane >> 1)] =
+          static_cast<uint8_t>((w & 0xF) | ((w_next & 0xF) << 4));
+    if (lane == 0) p.c.z_scale[row] = zs;
+  }
+}
+
 // ---------------------------------------------------------------- the kernel
 template <int D, int R, int NT, bool V2>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -278,9 +338,9 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       (reinterpret_cast<uintptr_t>(ynew_s + RR) + 15) & ~uintptr_t(15));
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(qraw_s + GM * D) + 15) & ~uintptr_t(15));
-  // bars[s] = stage full, bars[kStages + s] = stage empty, bars[2 kStages] = the
-  // appended token is in HBM, bars[2 kStages + 1] = the query and U_h are in
-  // shared memory
+  // bars[s] = stage full, bars[kStages + s] = stage empty, bars[2 kStages + 1] =
+  // the query and U_h are in shared memory (bars[2 kStages] unused)
+  int* stile_s = reinterpret_cast<int*>(bars + 2 * kStages + 2);  // [kStages] tile start, -1: end
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
@@ -292,9 +352,9 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   const int ntiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
   const size_t bk = static_cast<size_t>(b) * Hkv + kv;
   const int h0 = kv * G;
-  // the CTA whose chunk holds position T_b - 1 writes this step's new token there
-  const int pos = Tb - 1;
-  const bool owner = p.k_new != nullptr && Tb > 0 && pos >= t_begin && pos < t_begin + p.chunk;
+  // position of this step's new token (fused append), -1 when none
+  const int pos = (p.k_new != nullptr && Tb > 0) ? Tb - 1 : -1;
+  const int tile_end = t_end;  // a tile's tokens stop at the chunk end
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -323,48 +383,68 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       if constexpr (R > 0)
         bulk_g2s(smem_addr(u_s), p.U + static_cast<size_t>(kv) * D * R, D * R * 4, qbar);
     }
-    if (lane == 0 && ntiles > 0) {
-      bool ok = true;
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kStages, use = i / kStages;
-        if (use > 0 && !mbar_wait(smem_addr(&bars[kStages + s]), (use - 1) & 1)) {
-          ok = false;
-          break;
-        }
-        const int t0 = t_begin + i * kTile;
-        const int n16 = (min(kTile, t_end - t0) + 15) & ~15;
-        if (owner && pos < t0 + kTile) {  // this tile holds the appended token
-          if (!mbar_wait(smem_addr(&bars[2 * kStages]), 0)) {
-            ok = false;
-            break;
-          }
-          asm volatile("fence.proxy.async.global;" ::: "memory");
-        }
+    // The tiles of this CTA's chunk in order, one per stage, then an end marker.
+    // Appending: before issuing the tile that holds the new token (the chunk's
+    // last) this warp encodes the token, while the consumers drain the stages
+    // already in flight.
+    bool ok = true;
+    int issued = 0;
+    for (int i = 0;; ++i) {
+      const int s = i % kStages, use = i / kStages;
+      int t0 = -1;
+      if (lane == 0) {
+        if (use > 0 && !mbar_wait(smem_addr(&bars[kStages + s]), (use - 1) & 1)) ok = false;
+        if (ok && i < ntiles) t0 = t_begin + i * kTile;
+      }
+      ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+      t0 = __shfl_sync(kFull, t0, 0);
+      if (!ok) break;
+      if (t0 >= 0 && pos >= t0 && pos < t0 + kTile) {
+        // this tile holds the new token: encode it (U_h must be in shared
+        // memory), then publish it to the bulk copies (async proxy)
+        if (!mbar_wait(smem_addr(&bars[2 * kStages + 1]), 0) && lane == 0 && p.err)
+          atomicOr(p.err, kDevErrWaitTimeout);
+        encode_new_token<D, R, V2>(p, b, kv, pos, u_s, enew_s, lane);
+        __threadfence();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+        // the issuing lane orders every lane's writes before its bulk copies
+        if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
+      if (lane == 0) {
+        stile_s[s] = t0;
         const uint32_t full = smem_addr(&bars[s]);
-        mbar_expect_tx(full, L::kVBoxes * L::kVBox + n16 * L::kRowBytes);
-        uint8_t* st = stages + size_t(s) * L::kStage;
-        const CacheSlab sl = cache_slab_read(p.c, b, kv, t0, p.err);
-        const size_t row0 = static_cast<size_t>(sl.slab) * slab_rows(p.c) + sl.off;
-        bulk_g2s(smem_addr(st + L::kKc), p.c.k_codes + row0 * (D / 4), n16 * (D / 4), full);
-        bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + row0 * NG, n16 * NG * 4, full);
-        bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + row0 * NG, n16 * NG * 4, full);
-        if constexpr (R > 0) {
-          bulk_g2s(smem_addr(st + L::kZc), p.c.z_codes + row0 * (R / 2), n16 * (R / 2), full);
-          bulk_g2s(smem_addr(st + L::kZs), p.c.z_scale + row0, n16 * 4, full);
-        }
-        if constexpr (V2) {
-          bulk_g2s(smem_addr(st + L::kVc), p.c.v_codes + row0 * (D / 4), n16 * (D / 4), full);
-          bulk_g2s(smem_addr(st + L::kVs), p.c.v_scale + row0 * NG, n16 * NG * 4, full);
-          bulk_g2s(smem_addr(st + L::kVm), p.c.v_min + row0 * NG, n16 * NG * 4, full);
+        if (t0 < 0) {
+          mbar_arrive(full);  // no more tiles: the consumers stop at this stage
         } else {
+          const int n16 = (min(kTile, tile_end - t0) + 15) & ~15;
+          mbar_expect_tx(full, L::kVBoxes * L::kVBox + n16 * L::kRowBytes);
+          uint8_t* st = stages + size_t(s) * L::kStage;
+          const CacheSlab sl = cache_slab_read(p.c, b, kv, t0, p.err);
+          const size_t row0 = static_cast<size_t>(sl.slab) * slab_rows(p.c) + sl.off;
+          bulk_g2s(smem_addr(st + L::kKc), p.c.k_codes + row0 * (D / 4), n16 * (D / 4), full);
+          bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + row0 * NG, n16 * NG * 4, full);
+          bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + row0 * NG, n16 * NG * 4, full);
+          if constexpr (R > 0) {
+            bulk_g2s(smem_addr(st + L::kZc), p.c.z_codes + row0 * (R / 2), n16 * (R / 2), full);
+            bulk_g2s(smem_addr(st + L::kZs), p.c.z_scale + row0, n16 * 4, full);
+          }
+          if constexpr (V2) {
+            bulk_g2s(smem_addr(st + L::kVc), p.c.v_codes + row0 * (D / 4), n16 * (D / 4), full);
+            bulk_g2s(smem_addr(st + L::kVs), p.c.v_scale + row0 * NG, n16 * NG * 4, full);
+            bulk_g2s(smem_addr(st + L::kVm), p.c.v_min + row0 * NG, n16 * NG * 4, full);
+          } else {
 #pragma unroll
-          for (int bx = 0; bx < L::kVBoxes; ++bx)
-            tma_3d(smem_addr(st + bx * L::kVBox), &vmap, bx * 64, sl.off, static_cast<int>(sl.slab),
-                   full);
+            for (int bx = 0; bx < L::kVBoxes; ++bx)
+              tma_3d(smem_addr(st + bx * L::kVBox), &vmap, bx * 64, sl.off, static_cast<int>(sl.slab),
+                     full);
+          }
         }
         ++issued;
       }
+      if (t0 < 0) break;
+    }
+    if (lane == 0) {
       if (!ok && p.err) atomicOr(p.err, kDevErrWaitTimeout);
       // never leave with copies in flight: wait (bounded) for the last use of each stage
       for (int s = 0; s < kStages && s < issued; ++s) {
@@ -398,64 +478,6 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
-
-  if (owner && warp == 0) {
-    // encode the new token exactly as the cache write does: lanes 0..NG-1 take
-    // the key groups, NG..2NG-1 the value groups, lanes < R the side rows
-    const long long orow = cache_row(p.c, b, kv, pos);
-    if (orow < 0 && lane == 0 && p.err) atomicOr(p.err, kDevErrBadPage);
-    const size_t row = orow < 0 ? 0 : static_cast<size_t>(orow);
-    const size_t in = bk * D;
-    if (orow < 0) {
-      // a block-table entry outside the pool: the token is not written
-    } else if (lane < NG) {
-      float x[32];
-      uint32_t packed[2];
-      float sc, mn;
-      codec::load_row<32>(p.k_new, in + lane * 32, p.new_bf16, x);
-      codec::quantize_group<32, true>(x, packed, sc, mn);
-      codec::store_codes<32>(p.c.k_codes + row * (D / 4) + lane * 8, packed);
-      p.c.k_scale[row * NG + lane] = sc;
-      p.c.k_min[row * NG + lane] = mn;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) enew_s[lane * 32 + k] = x[k];
-    } else if (lane < 2 * NG && p.v_new != nullptr) {
-      const int gv = lane - NG;
-      float vv[32];
-      codec::load_row<32>(p.v_new, in + gv * 32, p.new_bf16, vv);
-      if constexpr (V2) {
-        uint32_t packed[2];
-        float sc, mn;
-        codec::quantize_group<32, false>(vv, packed, sc, mn);
-        codec::store_codes<32>(p.c.v_codes + row * (D / 4) + gv * 8, packed);
-        p.c.v_scale[row * NG + gv] = sc;
-        p.c.v_min[row * NG + gv] = mn;
-      } else {
-        codec::store_values<32>(p.c.v, row * D + gv * 32, true, vv);
-      }
-    }
-    __syncwarp();
-    if (R > 0 && orow >= 0) {
-      float y = 0.0f;
-      if (lane < R)
-        for (int c = 0; c < D; ++c) y = __fmaf_rn(u_s[c * R + lane], enew_s[c], y);
-      float a = lane < R ? fabsf(y) : 0.0f;
-#pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o2));
-      const float zs = codec::side_scale(a);
-      const int w = lane < R ? codec::side_level(y, zs, __frcp_rn(zs)) : 0;
-      const int w_next = __shfl_down_sync(kFull, w, 1);
-      if (lane < R && (lane & 1) == 0)
-        p.c.z_codes[row * (R / 2) + (lane >> 1)] =
-            static_cast<uint8_t>((w & 0xF) | ((w_next & 0xF) << 4));
-      if (lane == 0) p.c.z_scale[row] = zs;
-    }
-    // publish to the producer's bulk copies (async proxy) of the last tile
-    __threadfence();
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_addr(&bars[2 * kStages]));
-  }
 
   const int g = lane >> 2, t = lane & 3;
   const int jw = 16 * warp;
@@ -522,15 +544,16 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   }
 
   bool ok = true;
-  for (int i = 0; i < ntiles; ++i) {
+  for (int i = 0;; ++i) {
     const int s = i % kStages;
     if (!mbar_wait(smem_addr(&bars[s]), (i / kStages) & 1)) {
       ok = false;
       break;
     }
+    const int t0 = stile_s[s];  // the producer's tile for this stage, -1: no more
+    if (t0 < 0) break;
     uint8_t* st = stages + size_t(s) * L::kStage;
-    const int t0 = t_begin + i * kTile;
-    const int nvalid = min(kTile, t_end - t0);
+    const int nvalid = min(kTile, tile_end - t0);
     const int j0 = jw + g, j1 = j0 + 8;
     const bool val0 = j0 < nvalid, val1 = j1 < nvalid;
 
@@ -836,58 +859,86 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   __threadfence();
   const int S = p.splits;
   float* w_s = reinterpret_cast<float*>(flags + 4);  // [G][S] split weights, past the flags
-  float* M_s = w_s + GM * S;     // [G]
-  float* L_s = M_s + GM;         // [G]
+  // One warp per head, no CTA barrier, few round trips to L2: the first issues
+  // the (m, l) of the splits (lane-strided) together with the partial outputs
+  // of the first kMR splits (lane = 4 output dims); while those are in flight
+  // the warp reduces the maximum and writes the split weights w_s to shared
+  // memory; further rounds load the remaining splits' outputs.
+  constexpr int kSPL = 4;   // splits per lane held in registers (S <= 128)
+  constexpr int kMR = 16;   // splits per round of output loads
   for (int h = warp; h < G; h += kCW) {
     const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
+    const bool has_c4 = lane < D / 4;
+    const float4* po = reinterpret_cast<const float4*>(pv.o + bh * S * D) + lane;
+    float4 v[kMR];
+#pragma unroll
+    for (int u = 0; u < kMR; ++u)
+      v[u] = (has_c4 && u < S) ? __ldcg(po + u * (D / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float mv[kSPL], lv[kSPL];
     float mx = -INFINITY;
-    for (int s = lane; s < S; s += 32) mx = fmaxf(mx, __ldcg(pv.m + bh * S + s));
+#pragma unroll
+    for (int k = 0; k < kSPL; ++k) {
+      const int sI = lane + 32 * k;
+      mv[k] = -INFINITY;
+      lv[k] = 0.f;
+      if (sI < S) {
+        mv[k] = __ldcg(pv.m + bh * S + sI);
+        lv[k] = __ldcg(pv.l + bh * S + sI);
+      }
+      mx = fmaxf(mx, mv[k]);
+    }
+    for (int sI = lane + 32 * kSPL; sI < S; sI += 32) mx = fmaxf(mx, __ldcg(pv.m + bh * S + sI));
 #pragma unroll
     for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o2));
     float ls = 0.f;
-    for (int s = lane; s < S; s += 32) {
-      const float m = __ldcg(pv.m + bh * S + s);
-      const float w = m > -INFINITY ? expf(m - mx) : 0.f;
-      w_s[h * S + s] = w;
-      ls = fmaf(w, __ldcg(pv.l + bh * S + s), ls);
-    }
+    float* w = w_s + h * S;
 #pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) ls += __shfl_xor_sync(kFull, ls, o2);
-    if (lane == 0) {
-      M_s[h] = mx;
-      L_s[h] = ls;
+    for (int k = 0; k < kSPL; ++k) {
+      const int sI = lane + 32 * k;
+      if (sI < S) {
+        const float wk = mv[k] > -INFINITY ? expf(mv[k] - mx) : 0.f;
+        w[sI] = wk;
+        ls = fmaf(wk, lv[k], ls);
+      }
     }
+    for (int sI = lane + 32 * kSPL; sI < S; sI += 32) {
+      const float m = __ldcg(pv.m + bh * S + sI);
+      const float wk = m > -INFINITY ? expf(m - mx) : 0.f;
+      w[sI] = wk;
+      ls = fmaf(wk, __ldcg(pv.l + bh * S + sI), ls);
+    }
+    for (int o2 = 16; o2 > 0; o2 >>= 1) ls += __shfl_xor_sync(kFull, ls, o2);
+    __syncwarp();
+    float4 acc[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0;;) {
+#pragma unroll
+      for (int u = 0; u < kMR; ++u) {
+        const float wu = s0 + u < S ? w[s0 + u] : 0.f;
+        float4& a4 = acc[u & 3];
+        a4.x = fmaf(wu, v[u].x, a4.x); a4.y = fmaf(wu, v[u].y, a4.y);
+        a4.z = fmaf(wu, v[u].z, a4.z); a4.w = fmaf(wu, v[u].w, a4.w);
+      }
+      s0 += kMR;
+      if (s0 >= S) break;
+#pragma unroll
+      for (int u = 0; u < kMR; ++u)
+        v[u] = (has_c4 && s0 + u < S) ? __ldcg(po + (s0 + u) * (D / 4))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const float inv = ls > 0.f ? 1.0f / ls : 0.f;
+    if (has_c4) {
+      float4 r;
+      r.x = ((acc[0].x + acc[1].x) + (acc[2].x + acc[3].x)) * inv;
+      r.y = ((acc[0].y + acc[1].y) + (acc[2].y + acc[3].y)) * inv;
+      r.z = ((acc[0].z + acc[1].z) + (acc[2].z + acc[3].z)) * inv;
+      r.w = ((acc[0].w + acc[1].w) + (acc[2].w + acc[3].w)) * inv;
+      reinterpret_cast<float4*>(p.out + bh * D)[lane] = r;
+    }
+    if (lane == 0 && p.lse) p.lse[bh] = ls > 0.f ? mx + logf(ls) : -INFINITY;
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
-  // one thread per (head, 4 dims): independent 16-byte loads over the splits
-  for (int idx = tid; idx < G * (D / 4); idx += kCT) {
-    const int h = idx / (D / 4), c4 = idx - h * (D / 4);
-    const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
-    const float4* po = reinterpret_cast<const float4*>(pv.o + bh * S * D) + c4;
-    const float* w = w_s + h * S;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), e = a;
-    int s = 0;
-    for (; s + 2 <= S; s += 2) {
-      const float4 v0 = __ldcg(po + (s + 0) * (D / 4));
-      const float4 v1 = __ldcg(po + (s + 1) * (D / 4));
-      a.x = fmaf(w[s], v0.x, a.x); a.y = fmaf(w[s], v0.y, a.y);
-      a.z = fmaf(w[s], v0.z, a.z); a.w = fmaf(w[s], v0.w, a.w);
-      e.x = fmaf(w[s + 1], v1.x, e.x); e.y = fmaf(w[s + 1], v1.y, e.y);
-      e.z = fmaf(w[s + 1], v1.z, e.z); e.w = fmaf(w[s + 1], v1.w, e.w);
-    }
-    if (s < S) {
-      const float4 v0 = __ldcg(po + s * (D / 4));
-      a.x = fmaf(w[s], v0.x, a.x); a.y = fmaf(w[s], v0.y, a.y);
-      a.z = fmaf(w[s], v0.z, a.z); a.w = fmaf(w[s], v0.w, a.w);
-    }
-    const float Lh = L_s[h];
-    const float inv = Lh > 0.f ? 1.0f / Lh : 0.f;
-    float4 r;
-    r.x = (a.x + e.x) * inv; r.y = (a.y + e.y) * inv;
-    r.z = (a.z + e.z) * inv; r.w = (a.w + e.w) * inv;
-    reinterpret_cast<float4*>(p.out + bh * D)[c4] = r;
-    if (c4 == 0 && p.lse) p.lse[bh] = Lh > 0.f ? M_s[h] + logf(Lh) : -INFINITY;
-  }
   if (tid == 0) p.counters[bk] = 0;  // ready for the next call
 }
 

@@ -104,7 +104,7 @@ def test_merge_partials_edge_rows():
 def test_context_parallel_decode_nccl_world1():
     """ContextParallelDecode over a real NCCL group of one rank: the exchange is
     a copy and the merge of one part returns it unchanged, so the result equals
-    headq_decode_attn bit for bit."""
+    headq_decode_attn bit for bit (the decode is deterministic)."""
     import os
     import socket
     from datetime import timedelta
