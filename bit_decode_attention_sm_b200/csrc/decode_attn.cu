@@ -64,6 +64,9 @@ decode_split_kernel(const DecodeParams p) {
   float* m_s = s_s + G * kTile;   // [G]
   float* l_s = m_s + G;           // [G]
   float* a_s = l_s + G;           // [G]
+  float* v_s = a_s + G;           // [kTile][D] the tile's values, dequantised
+  float* kmn_s = v_s + kTile * D; // [D] per-channel key minima of the tile's block
+  float* ksc_s = kmn_s + D;       // [D] and scales (per-channel base code)
 
   const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -103,6 +106,18 @@ decode_split_kernel(const DecodeParams p) {
     const int nt = min(kTile, t_end - t0);
     // the tile's rows are consecutive: chunks start at multiples of 64 tokens
     const size_t row0 = cache_row_read(p.c, b, kv, t0, tid == 0 ? p.err : nullptr);
+    // the tile's values (and, per-channel code, its block's minima and scales)
+    // staged once with coalesced loads, so the readout below reads shared memory
+    for (int e = tid; e < nt * D; e += kThreads) {
+      const int j = e / D, c = e - j * D;
+      v_s[e] = value_at<D>(p, row0 + j, c);
+    }
+    if (p.c.kmode == HEADQ_K_CHANNEL)
+      for (int c = tid; c < D; c += kThreads) {
+        kmn_s[c] = p.c.k_min[(row0 >> 6) * D + c];
+        ksc_s[c] = p.c.k_scale[(row0 >> 6) * D + c];
+      }
+    __syncthreads();
     // phase 1: logits of (head, token) pairs
     for (int idx = tid; idx < G * kTile; idx += kThreads) {
       const int h = idx / kTile, j = idx - h * kTile;
@@ -113,10 +128,9 @@ decode_split_kernel(const DecodeParams p) {
         const float* qh = q_s + h * D;
         float acc = 0.0f;
         if (p.c.kmode == HEADQ_K_CHANNEL) {  // per-channel minimum and scale of the block
-          const float* mn = p.c.k_min + (row >> 6) * D;
-          const float* sc = p.c.k_scale + (row >> 6) * D;
           for (int c = 0; c < D; ++c) {
-            const float kh = __fadd_rn(mn[c], __fmul_rn(static_cast<float>(code2(cr, c)), sc[c]));
+            const float kh =
+                __fadd_rn(kmn_s[c], __fmul_rn(static_cast<float>(code2(cr, c)), ksc_s[c]));
             acc = fmaf(qh[c], kh, acc);
           }
         } else {
@@ -165,8 +179,7 @@ decode_split_kernel(const DecodeParams p) {
         const int h = idx / D, c = idx - h * D;
         float acc = o[k] * a_s[h];
         const float* pw = s_s + h * kTile;
-        for (int j = 0; j < nt; ++j)
-          acc = fmaf(pw[j], value_at<D>(p, row0 + j, c), acc);
+        for (int j = 0; j < nt; ++j) acc = fmaf(pw[j], v_s[j * D + c], acc);
         o[k] = acc;
       }
     }
@@ -259,7 +272,7 @@ cudaError_t launch_d(const DecodeParams& p, bool mma, cudaStream_t s) {
   } else {
     const int G = p.G, r = p.c.r;
     const size_t smem = sizeof(float) * (static_cast<size_t>(G) * D + G * num_groups(D) +
-                                         G * r + G * kTile + 3 * G);
+                                         G * r + G * kTile + 3 * G + kTile * D + 2 * D);
     auto k = decode_split_kernel<D>;
     if (smem > 48 * 1024) {
       cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -305,7 +318,9 @@ DecodePlan decode_plan(const headq_cache& c, int Hq, int T) {
     dp.fused = units <= kMaxFusedUnits;
     dp.kernels = (dp.splits > 1 && !dp.fused) ? 2 : 1;
   } else {
-    const SplitPlan sp = plan_splits(units, T, 256);
+    // the generic kernel is latency-bound per warp (4 warps per CTA): fill
+    // the SMs with about 4 CTAs each, chunks down to 64 tokens
+    const SplitPlan sp = plan_splits(units, T, 64, 4);
     dp.splits = sp.splits;
     dp.chunk = sp.chunk;
     dp.kernels = dp.splits > 1 ? 2 : 1;

@@ -27,13 +27,13 @@ int sm_count() {
   return n;
 }
 
-// Split each (b, kv) sequence into chunks so that the grid covers about two
-// waves of CTAs on this GPU, with chunks of at least `min_chunk` tokens and a
-// multiple of 64 tokens.
-SplitPlan plan_splits(int units, int T, int min_chunk) {
+// Split each (b, kv) sequence into chunks so that the grid covers about
+// `ctas_per_sm` CTAs per SM of this GPU, with chunks of at least `min_chunk`
+// tokens and a multiple of 64 tokens.
+SplitPlan plan_splits(int units, int T, int min_chunk, int ctas_per_sm) {
   SplitPlan sp{1, 64};
   if (T <= 0 || units <= 0) return sp;
-  const int target = 2 * sm_count();
+  const int target = ctas_per_sm * sm_count();
   int s = (target + units - 1) / units;
   const int max_s = (T + min_chunk - 1) / min_chunk;
   if (s > max_s) s = max_s;

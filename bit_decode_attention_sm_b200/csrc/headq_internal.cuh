@@ -185,7 +185,7 @@ cudaError_t launch_calibrate(const CalibrateParams& p, cudaStream_t s);
 struct SplitPlan {
   int splits, chunk;
 };
-SplitPlan plan_splits(int units, int T, int min_chunk);
+SplitPlan plan_splits(int units, int T, int min_chunk, int ctas_per_sm = 2);
 int sm_count();
 
 // The decode kernel and T-split plan chosen for these sizes on the current
