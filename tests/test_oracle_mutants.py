@@ -1,10 +1,11 @@
 """The oracle's pins catch plausible mistakes.
 
 Each case copies the oracle to a temporary directory, plants one slip in the
-C source by a textual substitution (a wrong sign, a transposed U, a wrong bit
-position, a dropped term, another rounding), builds it, and runs the pins of
-test_oracle_pins.py against that copy: at least one pin must fail.  The real
-oracle is never modified.  Everything runs on the CPU.
+C source or in its Python layer by a textual substitution (a wrong sign, a
+transposed U, a wrong bit position, a dropped term, another rounding, another
+tie rule), builds it, and runs the pins of test_oracle_pins.py against that
+copy: at least one pin must fail.  The real oracle is never modified.
+Everything runs on the CPU.
 """
 
 import importlib.util
@@ -51,6 +52,25 @@ MUTANTS = [
      "code = (int)t;"),
     ("group-of-16", "static int group_size(int d) { return d < 32 ? d : 32; }",
      "static int group_size(int d) { return d < 16 ? d : 16; }"),
+    # the per-channel base code
+    ("channel-minimum-is-maximum", "            if (v < lo) lo = v;", "            if (v > lo) lo = v;"),
+    ("channel-dequant-drops-minimum", "                xhat[(sq * T + t) * d + c] = mn[c] + prod;",
+     "                xhat[(sq * T + t) * d + c] = prod;"),
+]
+
+# slips in the Python layer of the oracle (oracle/__init__.py)
+MUTANTS_PY = [
+    ("merge-equal-weights", "w = np.where(np.isfinite(lses), np.exp(lses - M0), 0.0)",
+     "w = np.where(np.isfinite(lses), 1.0, 0.0)"),
+    ("merge-lse-without-log", "lse = np.where(covered, M0 + np.log(L1), -np.inf)",
+     "lse = np.where(covered, M0 + L1, -np.inf)"),
+    ("a2-p-not-squared", "out[b, kv, :Tb] = (p * p).sum(axis=0) * dv2",
+     "out[b, kv, :Tb] = p.sum(axis=0) * dv2"),
+    ("a2-ties-to-higher-position", "order = sorted(range(Tb), key=lambda j: (-scores[b, kv, j], j))",
+     "order = sorted(range(Tb), key=lambda j: (-scores[b, kv, j], -j))"),
+    ("a2-kept-unsorted", "kept = sorted(order[:min(K, Tb)])", "kept = order[:min(K, Tb)]"),
+    ("channel-block-of-32", "KBLOCK = 64  # tokens per block of the per-channel base code",
+     "KBLOCK = 32  # tokens per block of the per-channel base code"),
 ]
 
 PINS = [
@@ -67,16 +87,26 @@ PINS = [
     ("test_kl_direction_two_tokens", {}),
     ("test_lossless_limit_and_one_hot_value_distortion", {}),
     ("test_uniform_attention_value_distortion", {}),
+    ("test_channel_code_hand_example", {}),
+    ("test_channel_code_is_the_token_code_of_the_transpose", {}),
+    ("test_channel_code_is_equivariant_to_a_shared_translation", {}),
+    ("test_merge_of_token_shards_equals_whole", {}),
+    ("test_a2_scores_sum_to_the_a2_diagnostic", {}),
+    ("test_a2_scores_uniform_attention_closed_form", {}),
+    ("test_a2_selection_minimises_the_surrogate_brute_force", {}),
+    ("test_a2_mixed_values_limits", {}),
 ]
 
 
-def _load_mutant(tmp_path, name, old, new):
-    src = open(os.path.join(SRC_DIR, "headq_oracle.c")).read()
-    assert src.count(old) == 1, "mutation site not found exactly once: " + name
+def _load_mutant(tmp_path, name, old, new, target="headq_oracle.c"):
     d = tmp_path / ("oracle_" + name.replace("-", "_"))
     d.mkdir()
-    shutil.copy(os.path.join(SRC_DIR, "__init__.py"), d / "__init__.py")
-    (d / "headq_oracle.c").write_text(src.replace(old, new))
+    for f in ("__init__.py", "headq_oracle.c"):
+        src = open(os.path.join(SRC_DIR, f)).read()
+        if f == target:
+            assert src.count(old) == 1, "mutation site not found exactly once: " + name
+            src = src.replace(old, new)
+        (d / f).write_text(src)
     modname = "oracle_mutant_" + uuid.uuid4().hex
     spec = importlib.util.spec_from_file_location(modname, str(d / "__init__.py"))
     mod = importlib.util.module_from_spec(spec)
@@ -86,9 +116,12 @@ def _load_mutant(tmp_path, name, old, new):
     return mod
 
 
-@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_pins_catch_mutant(tmp_path, monkeypatch, name, old, new):
-    mod = _load_mutant(tmp_path, name, old, new)
+ALL = [m + ("headq_oracle.c",) for m in MUTANTS] + [m + ("__init__.py",) for m in MUTANTS_PY]
+
+
+@pytest.mark.parametrize("name,old,new,target", ALL, ids=[m[0] for m in ALL])
+def test_pins_catch_mutant(tmp_path, monkeypatch, name, old, new, target):
+    mod = _load_mutant(tmp_path, name, old, new, target)
     monkeypatch.setattr(pins, "oracle", mod)
     caught = []
     for fn, kw in PINS:
