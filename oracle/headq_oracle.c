@@ -3,7 +3,7 @@
  *
  * A plain, slow, obviously-correct CPU restatement of what HeadQ computes, used
  * only by the test-suite, the smoke check and the benchmark's CPU-baseline leg to
- * judge the CUDA library.  Nothing in the product links or calls this file, and it
+ * check the CUDA library.  Nothing in the product links or calls this file, and it
  * shares no code, header or table with the CUDA sources.
  *
  * Source: "HeadQ: Model-Visible Distortion and Score-Space Correction for KV-Cache
