@@ -78,7 +78,7 @@ struct Layout {
   static constexpr int kStage = (kEnd + 1023) / 1024 * 1024;
   static constexpr int kRowBytes =
       D / 4 + 8 * NG + (R > 0 ? R / 2 + 4 : 0) + (V2 ? D / 4 + 8 * NG : 0);
-  static constexpr int kCodeTile = V2 ? 16 * D * 2 : 0;  // per consumer warp, bf16 codes
+  static constexpr int kCodeTile = V2 ? 16 * D * 2 : 0;  // per consumer warp, fp16 codes
 };
 
 // the two-N-tile variants keep each thread's q B-operand fragments in shared
@@ -198,24 +198,6 @@ __device__ __forceinline__ void unpack_side(uint32_t y, uint32_t& n01, uint32_t&
   n01 = hfma2((y & 0x00F0000Fu) | 0x64006400u, 0x2C003C00u, 0xD480E408u);
   n23 = hfma2((z & 0x00F0000Fu) | 0x64006400u, 0x2C003C00u, 0xD480E408u);
 }
-// y holds one 16-bit word of eight 2-bit codes c0..c7 in both halves.  Returns
-// bf16 pairs (c0,c1) (c2,c3) (c4,c5) (c6,c7), exactly: 0x4300 | (code << 2k) is
-// the bf16 value 128 + code*4^k (k <= 2, inside the 7-bit mantissa), and one
-// exact bf16 FMA turns it back into the code.
-__device__ __forceinline__ uint32_t hfma2_bf16(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ void unpack_codes_bf16(uint32_t y, uint32_t (&v)[4]) {
-  const uint32_t y2 = y >> 2, y8 = y >> 8, y10 = y >> 10;
-  // (128 + c, 128 + 4c') * (1, 1/4) - (128, 32)
-  v[0] = hfma2_bf16((y & 0x000C0003u) | 0x43004300u, 0x3E803F80u, 0xC200C300u);
-  // (128 + 4c, 128 + 16c') * (1/4, 1/16) - (32, 8)
-  v[1] = hfma2_bf16((y2 & 0x0030000Cu) | 0x43004300u, 0x3D803E80u, 0xC100C200u);
-  v[2] = hfma2_bf16((y8 & 0x000C0003u) | 0x43004300u, 0x3E803F80u, 0xC200C300u);
-  v[3] = hfma2_bf16((y10 & 0x0030000Cu) | 0x43004300u, 0x3D803E80u, 0xC100C200u);
-}
 __device__ __forceinline__ uint32_t half_part_pair(float a, float b, bool lo) {
   __half ha = __float2half_rn(a), hb = __float2half_rn(b);
   if (lo) {
@@ -232,21 +214,6 @@ __device__ __forceinline__ uint32_t bf16_part_pair(float a, float b, bool lo) {
   const __nv_bfloat162 r = lo ? l : h;
   return *reinterpret_cast<const uint32_t*>(&r);
 }
-// x rounded to the nearest bf16 (ties to even), as an fp32 value; finite x
-__device__ __forceinline__ float bf16_round(float x) {
-  const uint32_t u = __float_as_uint(x);
-  return __uint_as_float((u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u);
-}
-// bf16_part_pair with one conversion: the lanes that want the low part first
-// subtract the high part (lo_f = 1) and convert the residual, which is then
-// exactly the low part; the others convert the value itself (lo_f = 0)
-__device__ __forceinline__ uint32_t bf16_part_pair1(float a, float b, float lo_f) {
-  const float a2 = fmaf(-lo_f, bf16_round(a), a);
-  const float b2 = fmaf(-lo_f, bf16_round(b), b);
-  const __nv_bfloat162 r = __floats2bfloat162_rn(a2, b2);
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
-
 // The new token of sequence b, KV head kv, encoded into cache position pos
 // exactly as the cache write does (bit-exact codec): lanes 0..NG-1 take the key
 // groups, NG..2NG-1 the value groups, lanes < R the side rows.  Warp-wide; U_h
@@ -323,7 +290,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* ctiles = smem + size_t(kStagesFor<NT>) * L::kStage;  // [kCW][16][D] bf16 value codes
+  uint8_t* ctiles = smem + size_t(kStagesFor<NT>) * L::kStage;  // [kCW][16][D] fp16 value codes
   uint2* bq_s = reinterpret_cast<uint2*>(ctiles + size_t(kCW) * L::kCodeTile);  // [KS][NT][128]
   float* q_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bq_s) +
                                         (kBqInSmem<NT> ? size_t(kCW) * 32 * KS * NT * 8 : 0));
@@ -530,7 +497,8 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   const int lm_chunk_hi = (lane >> 3) & 1;
 
   float m2[NT], l[NT];
-  float o[MT][NT][4];
+  float o[V2 ? 1 : MT][NT][4];      // dense values: columns (head, high/low part)
+  float ov[V2 ? MT : 1][4];         // 2-bit values: columns = the 8 head slots (fp16 p.V)
   float vmin_acc[NT][V2 ? NG : 1];  // 2-bit values: sum_j p_j min_{j,g} per group
   uint8_t* ctile = ctiles + size_t(warp) * L::kCodeTile;
 #pragma unroll
@@ -540,8 +508,10 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     m2[nt] = -INFINITY;
     l[nt] = 0.0f;
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+    for (int mt = 0; mt < (V2 ? 1 : MT); ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
   }
+#pragma unroll
+  for (int mt = 0; mt < (V2 ? MT : 1); ++mt) ov[mt][0] = ov[mt][1] = ov[mt][2] = ov[mt][3] = 0.f;
 
   bool ok = true;
   for (int i = 0;; ++i) {
@@ -558,15 +528,15 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     const bool val0 = j0 < nvalid, val1 = j1 < nvalid;
 
     if constexpr (V2) {
-      // this warp's 16 tokens of value codes -> bf16 code tile (chunk c of row t
+      // this warp's 16 tokens of value codes -> fp16 code tile (chunk c of row t
       // stored at c ^ (t & 7): conflict-free ldmatrix)
       for (int task = lane; task < 16 * (D / 16); task += 32) {
         const int tt = task / (D / 16), blk = task - tt * (D / 16);
         const uint32_t wv = *reinterpret_cast<const uint32_t*>(st + L::kVc + (jw + tt) * (D / 4) +
                                                                4 * blk);
         uint32_t lo4[4], hi4[4];
-        unpack_codes_bf16(__byte_perm(wv, 0u, 0x1010u), lo4);
-        unpack_codes_bf16(__byte_perm(wv, 0u, 0x3232u), hi4);
+        unpack_codes(__byte_perm(wv, 0u, 0x1010u), lo4);
+        unpack_codes(__byte_perm(wv, 0u, 0x3232u), hi4);
         const int c0 = 2 * blk, c1 = 2 * blk + 1;
         *reinterpret_cast<uint4*>(ctile + tt * (D * 2) + ((c0 ^ (tt & 7)) << 4)) =
             make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
@@ -653,7 +623,8 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
 
     // ---- logits, online softmax, p in the B-operand layout
     uint32_t bp[NT][2];
-    uint32_t bpv[V2 ? NG : 1][NT][2];
+    float pv0[NT], pv1[NT], al[NT];  // 2-bit values: p of tokens j0, j1 and the rescale
+    bool any_resc = false;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       float s0 = 0.f, s1 = 0.f;
@@ -676,6 +647,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
       const float mnew = fmaxf(m2[nt], mx);
       const bool resc = mnew > m2[nt] + kRescale;
+      al[nt] = 1.0f;
       if (__any_sync(kFull, resc)) {
         const float alpha = resc ? exp2f(m2[nt] - mnew) : 1.0f;
         if (resc) m2[nt] = mnew;
@@ -683,66 +655,87 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
         if constexpr (V2) {
 #pragma unroll
           for (int gg = 0; gg < NG; ++gg) vmin_acc[nt][gg] *= alpha;
-        }
+          al[nt] = alpha;
+          any_resc = true;
+        } else {
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          o[mt][nt][0] *= alpha; o[mt][nt][1] *= alpha;
-          o[mt][nt][2] *= alpha; o[mt][nt][3] *= alpha;
+          for (int mt = 0; mt < MT; ++mt) {
+            o[mt][nt][0] *= alpha; o[mt][nt][1] *= alpha;
+            o[mt][nt][2] *= alpha; o[mt][nt][3] *= alpha;
+          }
         }
       }
       const float p0 = x0 == -INFINITY ? 0.f : exp2f(x0 - m2[nt]);
       const float p1 = x1 == -INFINITY ? 0.f : exp2f(x1 - m2[nt]);
       l[nt] += p0 + p1;
-      // B operand of p . V: (tokens 2t, 2t+1 | 2t+8, 2t+9) x column g
-      const int sa = 8 * t + (g >> 1), sb = sa + 4;
-      const float va = __shfl_sync(kFull, p0, sa), vb = __shfl_sync(kFull, p0, sb);
-      const float vc = __shfl_sync(kFull, p1, sa), vd = __shfl_sync(kFull, p1, sb);
-      if constexpr (V2 && NG == 4) {
-        // per 32-dim group: p_j * scale_{j,g} (0 for masked tokens, whatever the
-        // stale scale), and the running sum of p_j * min_{j,g}; the scales of
-        // the four tokens of this lane's B operand and the minima of its two
-        // logit tokens come in one vector load each
-        const float4* vs4 = reinterpret_cast<const float4*>(st + L::kVs);
-        const float4* vm4 = reinterpret_cast<const float4*>(st + L::kVm);
-        const int ta = jw + 2 * t;
-        const float4 vsc[4] = {vs4[ta], vs4[ta + 1], vs4[ta + 8], vs4[ta + 9]};
-        const float4 vmn[2] = {vm4[j0], vm4[j1]};
-        const float lo_f = (g & 1) ? 1.0f : 0.0f;
-        const float sa4[4][4] = {{vsc[0].x, vsc[0].y, vsc[0].z, vsc[0].w},
-                                 {vsc[1].x, vsc[1].y, vsc[1].z, vsc[1].w},
-                                 {vsc[2].x, vsc[2].y, vsc[2].z, vsc[2].w},
-                                 {vsc[3].x, vsc[3].y, vsc[3].z, vsc[3].w}};
-        const float m4[2][4] = {{vmn[0].x, vmn[0].y, vmn[0].z, vmn[0].w},
-                                {vmn[1].x, vmn[1].y, vmn[1].z, vmn[1].w}};
-#pragma unroll
-        for (int gg = 0; gg < NG; ++gg) {
-          const float pa = va > 0.f ? va * sa4[0][gg] : 0.f;
-          const float pb = vb > 0.f ? vb * sa4[1][gg] : 0.f;
-          const float pc = vc > 0.f ? vc * sa4[2][gg] : 0.f;
-          const float pd = vd > 0.f ? vd * sa4[3][gg] : 0.f;
-          bpv[gg][nt][0] = bf16_part_pair1(pa, pb, lo_f);
-          bpv[gg][nt][1] = bf16_part_pair1(pc, pd, lo_f);
-          if (p0 > 0.f) vmin_acc[nt][gg] = fmaf(p0, m4[0][gg], vmin_acc[nt][gg]);
-          if (p1 > 0.f) vmin_acc[nt][gg] = fmaf(p1, m4[1][gg], vmin_acc[nt][gg]);
-        }
-      } else if constexpr (V2) {
-        const float* vs = reinterpret_cast<const float*>(st + L::kVs);
+      if constexpr (V2) {
+        pv0[nt] = p0;
+        pv1[nt] = p1;
+        // the running sum of p_j * min_{j,g} (masked tokens add nothing)
         const float* vm = reinterpret_cast<const float*>(st + L::kVm);
-        const int ta = jw + 2 * t, tb = ta + 1, tc = ta + 8, td = ta + 9;
 #pragma unroll
         for (int gg = 0; gg < NG; ++gg) {
-          const float pa = va > 0.f ? va * vs[ta * NG + gg] : 0.f;
-          const float pb = vb > 0.f ? vb * vs[tb * NG + gg] : 0.f;
-          const float pc = vc > 0.f ? vc * vs[tc * NG + gg] : 0.f;
-          const float pd = vd > 0.f ? vd * vs[td * NG + gg] : 0.f;
-          bpv[gg][nt][0] = bf16_part_pair(pa, pb, g & 1);
-          bpv[gg][nt][1] = bf16_part_pair(pc, pd, g & 1);
           if (p0 > 0.f) vmin_acc[nt][gg] = fmaf(p0, vm[j0 * NG + gg], vmin_acc[nt][gg]);
           if (p1 > 0.f) vmin_acc[nt][gg] = fmaf(p1, vm[j1 * NG + gg], vmin_acc[nt][gg]);
         }
       } else {
+        // B operand of p . V: (tokens 2t, 2t+1 | 2t+8, 2t+9) x column g
+        const int sa = 8 * t + (g >> 1), sb = sa + 4;
+        const float va = __shfl_sync(kFull, p0, sa), vb = __shfl_sync(kFull, p0, sb);
+        const float vc = __shfl_sync(kFull, p1, sa), vd = __shfl_sync(kFull, p1, sb);
         bp[nt][0] = bf16_part_pair(va, vb, g & 1);
         bp[nt][1] = bf16_part_pair(vc, vd, g & 1);
+      }
+    }
+
+    // 2-bit values: one fp16 B operand per 32-dim group over the 8 head slots.
+    // Column g is head slot g; its p for tokens 2t, 2t+1 (2t+8, 2t+9) is p0 (p1)
+    // of the lanes 4*(2t) + (g & 3) and 4*(2t+1) + (g & 3) in query tile g >> 2.
+    // p * scale_{j,g} lies in [0, a few]: one fp16 part (11-bit mantissa) is
+    // well inside the output tolerance; the codes are exact in fp16.
+    uint32_t bpf[V2 ? NG : 1][2];
+    if constexpr (V2) {
+      const int src_a = 8 * t + (g & 3), src_b = src_a + 4;
+      float pa = 0.f, pb = 0.f, pc = 0.f, pd = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float a_ = __shfl_sync(kFull, pv0[nt], src_a);
+        const float b_ = __shfl_sync(kFull, pv0[nt], src_b);
+        const float c_ = __shfl_sync(kFull, pv1[nt], src_a);
+        const float d_ = __shfl_sync(kFull, pv1[nt], src_b);
+        if ((g >> 2) == nt) {
+          pa = a_; pb = b_; pc = c_; pd = d_;
+        }
+      }
+      const float* vs = reinterpret_cast<const float*>(st + L::kVs);
+      const int ta = jw + 2 * t;
+#pragma unroll
+      for (int gg = 0; gg < NG; ++gg) {
+        const float qa = pa > 0.f ? pa * vs[ta * NG + gg] : 0.f;
+        const float qb = pb > 0.f ? pb * vs[(ta + 1) * NG + gg] : 0.f;
+        const float qc = pc > 0.f ? pc * vs[(ta + 8) * NG + gg] : 0.f;
+        const float qd = pd > 0.f ? pd * vs[(ta + 9) * NG + gg] : 0.f;
+        const __half2 h0 = __floats2half2_rn(qa, qb), h1 = __floats2half2_rn(qc, qd);
+        bpf[gg][0] = *reinterpret_cast<const uint32_t*>(&h0);
+        bpf[gg][1] = *reinterpret_cast<const uint32_t*>(&h1);
+      }
+      if (__any_sync(kFull, any_resc)) {
+        // rescale the output columns (head slots 2t, 2t+1) by their heads' factors
+        float f0 = 1.0f, f1 = 1.0f;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const float x0 = __shfl_sync(kFull, al[nt], (2 * t) & 3);
+          const float x1 = __shfl_sync(kFull, al[nt], (2 * t + 1) & 3);
+          if (((2 * t) >> 2) == nt) {
+            f0 = x0;
+            f1 = x1;
+          }
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          ov[mt][0] *= f0; ov[mt][1] *= f1;
+          ov[mt][2] *= f0; ov[mt][3] *= f1;
+        }
       }
     }
 
@@ -755,8 +748,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
         const int chunk = 2 * mt + lm_chunk_hi;
         uint32_t a[4];
         ldsm_x4_trans(cbase + lt * (D * 2) + ((chunk ^ (lt & 7)) << 4), a);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16(o[mt][nt], a, bpv[mt >> 1][nt]);
+        mma_f16(ov[mt], a, bpf[mt >> 1]);
       }
     } else {
       const uint32_t vbase = smem_addr(st);
@@ -795,22 +787,43 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   float* mo = reinterpret_cast<float*>(stages);  // [kCW][GM][D]
   float* mm = mo + kCW * GM * D;                 // [kCW][GM]
   float* ml = mm + kCW * GM;                     // [kCW][GM]
-  int* flags = reinterpret_cast<int*>(ml + kCW * GM);  // [0] a warp failed, [1] last CTA
+  float* vms = ml + kCW * GM;                    // [kCW][GM][NG] (2-bit values) sum p min
+  int* flags = reinterpret_cast<int*>(vms + (V2 ? kCW * GM * NG : 0));  // [0] a warp failed, [1] last CTA
   if (tid == 0) flags[0] = 0;
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   if (!ok) flags[0] = 1;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int h = 4 * nt + t;
+    if constexpr (!V2) {
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const float vmn = V2 ? vmin_acc[nt][V2 ? (mt >> 1) : 0] : 0.f;
-      mo[(warp * GM + h) * D + 16 * mt + g] = (o[mt][nt][0] + o[mt][nt][1]) + vmn;
-      mo[(warp * GM + h) * D + 16 * mt + g + 8] = (o[mt][nt][2] + o[mt][nt][3]) + vmn;
+      for (int mt = 0; mt < MT; ++mt) {
+        mo[(warp * GM + h) * D + 16 * mt + g] = o[mt][nt][0] + o[mt][nt][1];
+        mo[(warp * GM + h) * D + 16 * mt + g + 8] = o[mt][nt][2] + o[mt][nt][3];
+      }
     }
     if (g == 0) {
       mm[warp * GM + h] = m2[nt];
       ml[warp * GM + h] = l[nt];
+      if constexpr (V2) {
+#pragma unroll
+        for (int gg = 0; gg < NG; ++gg) vms[(warp * GM + h) * NG + gg] = vmin_acc[nt][gg];
+      }
+    }
+  }
+  if constexpr (V2) {  // columns = head slots 2t, 2t+1; add the minima sum of the group
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * t + e;
+      if (h < GM) {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const float vmn = vms[(warp * GM + h) * NG + (mt >> 1)];
+          mo[(warp * GM + h) * D + 16 * mt + g] = ov[mt][e] + vmn;
+          mo[(warp * GM + h) * D + 16 * mt + g + 8] = ov[mt][2 + e] + vmn;
+        }
+      }
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
