@@ -7,13 +7,15 @@
 // Bit-exact: every codec operation is one IEEE fp32 operation (codec.cuh; this
 // file is also compiled with -fmad=false).
 //
-// One CTA per (64-token tile, kv, b), three phases:
-//   A  one thread per (token, 32-channel group): vector loads of the group's keys
-//      and values straight from HBM (all issued before any arithmetic), base code,
-//      codes/scale/min stored, residual e -> shared memory, values stored/coded
-//   B  one thread per (token, 8 side rows): y = U_h^T e in channel order, one
-//      fused multiply-add per term, two rows per packed fp32x2 FMA
-//   C  one thread per (token, pair of side rows): absmax scale and the two nibbles
+// One CTA per (64-token tile, kv, b), two phases:
+//   A  one thread per (token, 32-channel group): the group's keys and values
+//      loaded straight from HBM together, base code (a short path per channel,
+//      the exact codec near a rounding tie), codes/scale/min stored, the
+//      residual written to shared memory, values copied or coded
+//   B  one thread per (token, RB side rows), RB = 16 for r = 16: y = U_h^T e in
+//      channel order, one fused multiply-add per term, two rows per packed
+//      fp32x2 FMA, U_h read as warp-wide broadcasts; then max|y| (shared by warp
+//      shuffles when a token has several threads) and the 4-bit side code
 #include "codec.cuh"
 
 namespace headq {
@@ -21,77 +23,331 @@ namespace {
 
 constexpr int kTT = 64;        // tokens per CTA
 constexpr int kThreads = 256;
+constexpr unsigned kFull = 0xffffffffu;
 
-// The value of token tt, group g of the tile: dense copy or 2-bit code.
+// The residual tile in shared memory, one fp32 per channel.  Group g of a
+// token starts at 16-byte chunk g*GC (GC = 2 mod 8: two chunks of padding per
+// 32-channel group) and a token row spans RC chunks (RC odd): the (token, group)
+// writes of phase A and the one-token-per-lane reads of phase B then fall in
+// distinct banks.
 template <int D>
+struct ResTile {
+  static constexpr int GS = group_size(D);
+  static constexpr int NG = num_groups(D);
+  static constexpr int GC = GS / 4 + 2;
+  static constexpr int RC = NG * GC + 1;
+  static constexpr int kFloats = kTT * RC * 4;
+  // float offset of channel c within a token row
+  __device__ static int off(int c) { return 4 * ((c / GS) * GC + (c % GS) / 4) + (c & 3); }
+};
+
+// U_h in shared memory as [r / RB][D][RB]: the RB rows a phase-B thread owns are
+// contiguous for every channel; blocks are padded apart by 16 bytes (8 for RB 2)
+// so the threads of a token (when it has several) read distinct banks.
+template <int D, int RB>
+struct BasisTile {
+  static constexpr int kPad = RB >= 4 ? 4 : 2;
+  static constexpr int kBlock = D * RB + kPad;
+  __host__ __device__ static int floats(int r) { return (r / RB) * kBlock; }
+};
+
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// GS values of one group as loaded: GS/8 16-byte words of bf16, or GS/4 of fp32.
+template <int GS, bool BF16>
+struct RawGroup {
+  static constexpr int kWords = BF16 ? GS / 8 : GS / 4;
+  uint4 w[kWords];
+};
+
+template <int GS, bool BF16>
+__device__ __forceinline__ void load_raw(const void* base, size_t off, RawGroup<GS, BF16>& g) {
+  if constexpr (BF16) {
+    const uint4* s = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + off);
+#pragma unroll
+    for (int k = 0; k < GS / 8; ++k) g.w[k] = s[k];
+  } else {
+    const uint4* s = reinterpret_cast<const uint4*>(static_cast<const float*>(base) + off);
+#pragma unroll
+    for (int k = 0; k < GS / 4; ++k) g.w[k] = s[k];
+  }
+}
+
+template <int GS, bool BF16>
+__device__ __forceinline__ void unpack_raw(const RawGroup<GS, BF16>& g, float (&x)[GS]) {
+  if constexpr (BF16) {
+#pragma unroll
+    for (int k = 0; k < GS / 8; ++k) {
+      const uint32_t w[4] = {g.w[k].x, g.w[k].y, g.w[k].z, g.w[k].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        x[8 * k + 2 * j] = __uint_as_float(w[j] << 16);
+        x[8 * k + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < GS / 4; ++k) {
+      x[4 * k] = __uint_as_float(g.w[k].x);
+      x[4 * k + 1] = __uint_as_float(g.w[k].y);
+      x[4 * k + 2] = __uint_as_float(g.w[k].z);
+      x[4 * k + 3] = __uint_as_float(g.w[k].w);
+    }
+  }
+}
+
+// The per-token base code of one group: the codes, scale, minimum and residuals
+// of codec::quantize_group, with fewer operations per channel.  With the scale
+// a normal number of at most 2^126, every quotient (x - min)/scale lies in
+// [0, 3 + 2^-21], and q = RN((x - min) * RN(1/scale)) rounds to the same integer
+// as RN((x - min)/scale) whenever q is more than 2^-16 away from a half-integer
+// (the error argument of codec::rint_quot), so no clamp is needed there; a
+// channel whose q lies that close to a half-integer (exact ties are common with
+// bf16 inputs) takes the exact quotient, as codec::rint_quot does.  Returns false,
+// with x partly overwritten, when the scale is outside that range: the caller
+// then runs the exact codec on the group.
+template <int GS, bool RESIDUAL>
+__device__ __forceinline__ bool quantize_group_fast(float (&x)[GS],
+                                                    uint32_t (&packed)[GS / 16 > 0 ? GS / 16 : 1],
+                                                    float& scale_out, float& min_out) {
+  float lo = x[0], hi = x[0];
+#pragma unroll
+  for (int k = 1; k + 1 < GS; k += 2) {
+    lo = fmin3(lo, x[k], x[k + 1]);
+    hi = fmax3(hi, x[k], x[k + 1]);
+  }
+  lo = fminf(lo, x[GS - 1]);
+  hi = fmaxf(hi, x[GS - 1]);
+  lo = __fadd_rn(lo, 0.0f);  // a -0 extreme is stored as +0
+  hi = __fadd_rn(hi, 0.0f);
+  const float scale = __fdiv_rn(__fsub_rn(hi, lo), 3.0f);
+  scale_out = scale;
+  min_out = lo;
+#pragma unroll
+  for (int w = 0; w < (GS / 16 > 0 ? GS / 16 : 1); ++w) packed[w] = 0u;
+  if (scale == 0.0f) {  // all codes 0; the residual is x - (min + 0) = x - min
+    if constexpr (RESIDUAL) {
+#pragma unroll
+      for (int k = 0; k < GS; ++k) x[k] = __fsub_rn(x[k], lo);
+    }
+    return true;
+  }
+  if (!(scale >= 0x1p-126f && scale <= 0x1p126f)) return false;
+  const float rs = __frcp_rn(scale);
+  float acc[GS / 8];  // eight codes per float, c * 4^j summed exactly
+#pragma unroll
+  for (int i = 0; i < GS / 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+  for (int k = 0; k < GS; ++k) {
+    const float a = __fsub_rn(x[k], lo);
+    const float q = __fmul_rn(a, rs);
+    float c = rintf(q);
+    if (!(fabsf(__fsub_rn(q, c)) < 0.5f - 0x1p-16f)) {  // near a half-integer (or NaN)
+      const float t = rintf(__fdiv_rn(a, scale));
+      c = static_cast<float>(t < 0.0f ? 0 : (t > 3.0f ? 3 : static_cast<int>(t)));
+    }
+    acc[k / 8] = __fmaf_rn(c, static_cast<float>(1u << (2 * (k % 8))), acc[k / 8]);
+    if constexpr (RESIDUAL) x[k] = __fsub_rn(x[k], __fadd_rn(lo, __fmul_rn(c, scale)));
+  }
+  if constexpr (GS >= 16) {
+#pragma unroll
+    for (int w = 0; w < GS / 16; ++w)
+      packed[w] = static_cast<uint32_t>(acc[2 * w]) | (static_cast<uint32_t>(acc[2 * w + 1]) << 16);
+  } else {
+    packed[0] = static_cast<uint32_t>(acc[0]);
+  }
+  return true;
+}
+
+// Base code of a group loaded as raw words from base + off: the short path, or,
+// for a scale outside its range, the group loaded again through the exact codec.
+template <int GS, bool RESIDUAL, bool BF16>
+__device__ __forceinline__ void quantize_raw(const void* base, size_t off, RawGroup<GS, BF16>& raw,
+                                             float (&x)[GS],
+                                             uint32_t (&packed)[GS / 16 > 0 ? GS / 16 : 1],
+                                             float& sc, float& mn) {
+  unpack_raw<GS, BF16>(raw, x);
+  if (!quantize_group_fast<GS, RESIDUAL>(x, packed, sc, mn)) {
+    load_raw<GS, BF16>(base, off, raw);
+    unpack_raw<GS, BF16>(raw, x);
+    codec::quantize_group<GS, RESIDUAL>(x, packed, sc, mn);
+  }
+}
+
+// Plane rows of a tile's tokens: when its first and last token share a slab, the
+// tile occupies consecutive rows from row0 (the common case: contiguous planes,
+// or a tile inside one page); otherwise each token is looked up.
+struct TileRows {
+  long long row0;
+  bool consecutive;
+};
+
+__device__ __forceinline__ TileRows tile_rows(const headq_cache& c, int b, int kv, int t_first,
+                                              int nt) {
+  const CacheSlab a = cache_slab(c, b, kv, t_first);
+  const CacheSlab z = cache_slab(c, b, kv, t_first + nt - 1);
+  if (a.slab >= 0 && a.slab == z.slab) return {a.slab * slab_rows(c) + a.off, true};
+  return {-1, false};
+}
+
+__device__ __forceinline__ long long tile_row(const headq_cache& c, const TileRows& tr, int b,
+                                              int kv, int t_first, int tt) {
+  return tr.consecutive ? tr.row0 + tt : cache_row(c, b, kv, t_first + tt);
+}
+
+// Dense values whose cache dtype is the input dtype are copied as 16-byte chunks
+// with consecutive lanes on consecutive chunks (whole rows of the tile), in
+// batches of kBatch chunks per thread.
+template <int D, bool BF16>
+struct ValueCopy {
+  static constexpr int kCPR = D * (BF16 ? 2 : 4) / 16;  // chunks per row
+  static constexpr int kBatch = 4;
+};
+
+// The value of one (token, group): a plain copy when the cache holds the input
+// dtype, else converted; or the 2-bit code of the full-KV composition.
+template <int D, bool BF16>
 __device__ __forceinline__ void store_value_group(const CacheWriteParams& p, size_t in_off,
+                                                  RawGroup<group_size(D), BF16>& raw,
                                                   size_t row, int g) {
   constexpr int GS = group_size(D);
   constexpr int NG = num_groups(D);
   constexpr int NW = GS / 16 > 0 ? GS / 16 : 1;
   float vv[GS];
-  codec::load_row<GS>(p.v, in_off, p.in_bf16, vv);
   if (p.c.vmode == HEADQ_V_2BIT) {
     uint32_t packed[NW];
     float sc, mn;
-    codec::quantize_group<GS, false>(vv, packed, sc, mn);
+    quantize_raw<GS, false, BF16>(p.v, in_off, raw, vv, packed, sc, mn);
     codec::store_codes<GS>(p.c.v_codes + row * (D / 4) + g * (GS / 4), packed);
     p.c.v_scale[row * NG + g] = sc;
     p.c.v_min[row * NG + g] = mn;
-  } else {
-    codec::store_values<GS>(p.c.v, row * D + g * GS, p.c.v_dtype == HEADQ_BF16, vv);
+    return;
+  }
+  const bool cache_bf16 = p.c.v_dtype == HEADQ_BF16;
+  if (cache_bf16 == BF16) {  // same dtype: the input bits are the cached bits
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.c.v) +
+                                          (row * D + g * GS) * (BF16 ? 2 : 4));
+#pragma unroll
+    for (int k = 0; k < RawGroup<GS, BF16>::kWords; ++k) dst[k] = raw.w[k];
+    return;
+  }
+  unpack_raw<GS, BF16>(raw, vv);
+  codec::store_values<GS>(p.c.v, row * D + g * GS, cache_bf16, vv);
+}
+
+// U_h of this KV head into the [r / RB][D][RB] tile, by 16-byte vectors (8-byte
+// for RB 2): a vector's rows fall in one block.
+template <int D, int RB>
+__device__ __forceinline__ void load_basis(const CacheWriteParams& p, int kv, float* u_s) {
+  using BT = BasisTile<D, RB>;
+  constexpr int V = RB >= 4 ? 4 : 2;  // floats per vector
+  const int r = p.c.r, rv = r / V;
+  const float* U = p.U + static_cast<size_t>(kv) * D * r;
+  for (int i = threadIdx.x; i < D * rv; i += kThreads) {
+    const int c = i / rv, row = (i - c * rv) * V;
+    float* dst = u_s + (row / RB) * BT::kBlock + c * RB + (row % RB);
+    if constexpr (V == 4)
+      *reinterpret_cast<float4*>(dst) = reinterpret_cast<const float4*>(U)[i];
+    else
+      *reinterpret_cast<float2*>(dst) = reinterpret_cast<const float2*>(U)[i];
   }
 }
 
-// Phases B and C, shared by both base codes: from the residuals e_s of the
-// tile's tokens, y = U_h^T e and the 4-bit side code of every token.
-template <int D, int RB>
-__device__ __forceinline__ void side_code_tile(const CacheWriteParams& p, float* e_s, float* u_s,
-                                               float* y_s, int b, int kv, int tile0, int t0) {
-  constexpr int ES = D + 4;
-  const int r = p.c.r, tid = threadIdx.x;
-  {
-    const float4* U4 = reinterpret_cast<const float4*>(p.U + static_cast<size_t>(kv) * D * r);
-    for (int i = tid; i < D * r / 4; i += kThreads) reinterpret_cast<float4*>(u_s)[i] = U4[i];
+// y (RB rows, as packed pairs) += U[c][rows] * e, for one channel c.
+template <int RB>
+__device__ __forceinline__ void fma_rows(uint64_t (&y)[RB / 2], const float* u, uint64_t e2) {
+  if constexpr (RB == 2) {
+    codec::fma2_pk(y[0], *reinterpret_cast<const uint64_t*>(u), e2);
+  } else {
+#pragma unroll
+    for (int k = 0; k < RB / 4; ++k) {
+      const ulonglong2 uu = reinterpret_cast<const ulonglong2*>(u)[k];
+      codec::fma2_pk(y[2 * k], uu.x, e2);
+      codec::fma2_pk(y[2 * k + 1], uu.y, e2);
+    }
   }
-  __syncthreads();
+}
 
-  // ---- phase B: y = U_h^T e, channel order, one FMA per term ---------------
-  // RB side rows per thread as RB/2 packed pairs, one fp32x2 FMA per pair and
-  // channel (the pairs and U stay in 64-bit registers)
-  const int blocks_per_tok = r / RB;
-  for (int pr = tid; pr < kTT * blocks_per_tok; pr += kThreads) {
-    const int tt = pr / blocks_per_tok;
-    const int i0 = (pr - tt * blocks_per_tok) * RB;
-    if (tile0 + tt >= p.n) continue;
+__device__ __forceinline__ float lo32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+
+// Phase B: from the tile's residuals, y = U_h^T e and the 4-bit side code of
+// every token.  When the threads of a token are a power of two (aligned lanes
+// of one warp) max|y| goes round by shuffles and each thread codes its own
+// rows; otherwise y passes through shared memory first.
+template <int D, int RB>
+__device__ __forceinline__ void side_code_tile(const CacheWriteParams& p, const float* e_s,
+                                               const float* u_s, float* y_s, int b, int kv,
+                                               int tile0, int t0, const TileRows& tr) {
+  using L = ResTile<D>;
+  using BT = BasisTile<D, RB>;
+  const int r = p.c.r, tid = threadIdx.x;
+  const int bpt = r / RB;                      // threads per token
+  const bool fused = (bpt & (bpt - 1)) == 0;   // kTT * bpt is a multiple of 32 either way
+  for (int pr = tid; pr < kTT * bpt; pr += kThreads) {
+    const int tt = pr / bpt, blk = pr - tt * bpt, i0 = blk * RB;
     uint64_t y[RB / 2];
 #pragma unroll
     for (int k = 0; k < RB / 2; ++k) y[k] = 0ull;
-    const float* er = e_s + tt * ES;
-#pragma unroll 8
-    for (int c = 0; c < D; ++c) {
-      const uint64_t e2 = codec::dup2(er[c]);
-      const uint64_t* ur = reinterpret_cast<const uint64_t*>(u_s + c * r + i0);
-      if constexpr (RB >= 4) {
+    const float4* er = reinterpret_cast<const float4*>(e_s) + tt * L::RC;
+    const float* ub = u_s + blk * BT::kBlock;
+#pragma unroll 1
+    for (int g = 0; g < L::NG; ++g) {  // rolled: keeps the loop in the instruction cache
 #pragma unroll
-        for (int k = 0; k < RB / 4; ++k) {
-          const ulonglong2 u = reinterpret_cast<const ulonglong2*>(ur)[k];
-          codec::fma2_pk(y[2 * k], u.x, e2);
-          codec::fma2_pk(y[2 * k + 1], u.y, e2);
-        }
-      } else {
-        codec::fma2_pk(y[0], ur[0], e2);
+      for (int j = 0; j < L::GS / 4; ++j) {
+        const int c = g * L::GS + 4 * j;
+        const float4 ev = er[g * L::GC + j];  // e_c .. e_c+3
+        fma_rows<RB>(y, ub + c * RB, codec::dup2(ev.x));
+        fma_rows<RB>(y, ub + (c + 1) * RB, codec::dup2(ev.y));
+        fma_rows<RB>(y, ub + (c + 2) * RB, codec::dup2(ev.z));
+        fma_rows<RB>(y, ub + (c + 3) * RB, codec::dup2(ev.w));
       }
     }
+    const bool live = tile0 + tt < p.n;
+    if (fused) {
+      float a = 0.0f;
 #pragma unroll
-    for (int k = 0; k < RB / 2; ++k) {
-      y_s[tt * (r + 1) + i0 + 2 * k] = __uint_as_float(static_cast<uint32_t>(y[k]));
-      y_s[tt * (r + 1) + i0 + 2 * k + 1] = __uint_as_float(static_cast<uint32_t>(y[k] >> 32));
+      for (int k = 0; k < RB / 2; ++k) a = fmax3(a, fabsf(lo32(y[k])), fabsf(hi32(y[k])));
+      for (int m = 1; m < bpt; m <<= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, m));
+      if (!live) continue;
+      const long long row_s = tile_row(p.c, tr, b, kv, t0 + tile0, tt);
+      if (row_s < 0) continue;
+      const size_t row = static_cast<size_t>(row_s);
+      const float s = codec::side_scale(a);
+      const float rs = __frcp_rn(s);
+      uint64_t bits = 0u;
+#pragma unroll
+      for (int k = 0; k < RB / 2; ++k) {
+        const int w0 = codec::side_level(lo32(y[k]), s, rs);
+        const int w1 = codec::side_level(hi32(y[k]), s, rs);
+        bits |= static_cast<uint64_t>((w0 & 0xF) | ((w1 & 0xF) << 4)) << (8 * k);
+      }
+      uint8_t* dst = p.c.z_codes + row * (r / 2) + i0 / 2;
+      if constexpr (RB == 2) *dst = static_cast<uint8_t>(bits);
+      else if constexpr (RB == 4) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(bits);
+      else if constexpr (RB == 8) *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(bits);
+      else *reinterpret_cast<uint64_t*>(dst) = bits;
+      if (blk == 0) p.c.z_scale[row] = s;
+    } else if (live) {
+#pragma unroll
+      for (int k = 0; k < RB / 2; ++k) {
+        y_s[tt * (r + 1) + i0 + 2 * k] = lo32(y[k]);
+        y_s[tt * (r + 1) + i0 + 2 * k + 1] = hi32(y[k]);
+      }
     }
   }
+  if (fused) return;
   __syncthreads();
-
-  // ---- phase C: side code, one byte (two rows) per thread --------------------
+  // one byte (two rows) per thread
   const int pairs = r / 2;
   for (int pr = tid; pr < kTT * pairs; pr += kThreads) {
     const int tt = pr / pairs, i = 2 * (pr - tt * pairs);
@@ -103,7 +359,7 @@ __device__ __forceinline__ void side_code_tile(const CacheWriteParams& p, float*
     const float rs = __frcp_rn(s);
     const int w0 = codec::side_level(y[i], s, rs);
     const int w1 = codec::side_level(y[i + 1], s, rs);
-    const long long row_s = cache_row(p.c, b, kv, t0 + tile0 + tt);
+    const long long row_s = tile_row(p.c, tr, b, kv, t0 + tile0, tt);
     if (row_s < 0) continue;
     const size_t row = static_cast<size_t>(row_s);
     p.c.z_codes[row * (r / 2) + (i >> 1)] = static_cast<uint8_t>((w0 & 0xF) | ((w1 & 0xF) << 4));
@@ -111,19 +367,28 @@ __device__ __forceinline__ void side_code_tile(const CacheWriteParams& p, float*
   }
 }
 
+// Shared-memory carve-up of both kernels: residual tile, basis tile, y rows
+// (side code through shared memory) and, for the per-channel code, the block's
+// per-channel minimum and scale.
 template <int D, int RB>
-__global__ void __launch_bounds__(kThreads, 3)
+__host__ __device__ inline size_t cache_write_smem_floats(int r, bool channel) {
+  return static_cast<size_t>(ResTile<D>::kFloats) + BasisTile<D, RB>::floats(r) +
+         static_cast<size_t>(kTT) * (r + 1) + (channel ? 2 * D : 0);
+}
+
+template <int D, int RB, bool BF16>
+__global__ void __launch_bounds__(kThreads, BF16 ? 3 : 2)
 cache_write_kernel(const CacheWriteParams p) {
   constexpr int GS = group_size(D);
   constexpr int NG = num_groups(D);
   constexpr int NW = GS / 16 > 0 ? GS / 16 : 1;
-  constexpr int ES = D + 4;  // residual row stride (floats): 16-byte rows, spread banks
+  using L = ResTile<D>;
 
-  extern __shared__ float smem[];
+  extern __shared__ float4 smem4[];
   const int r = p.c.r;
-  float* e_s = smem;                 // [kTT][ES]
-  float* u_s = e_s + kTT * ES;       // [D][r]
-  float* y_s = u_s + D * r;          // [kTT][r + 1]
+  float* e_s = reinterpret_cast<float*>(smem4);      // [kTT][RC chunks]
+  float* u_s = e_s + L::kFloats;                     // [r/RB][D][RB] (+ pad)
+  float* y_s = u_s + BasisTile<D, RB>::floats(r);    // [kTT][r + 1]
 
   const int b = blockIdx.z, kv = blockIdx.y;
   const int tile0 = blockIdx.x * kTT;
@@ -135,52 +400,123 @@ cache_write_kernel(const CacheWriteParams p) {
     if (Tb == 0) return;
     t0 = Tb - 1;
   }
+  if (r > 0) load_basis<D, RB>(p, kv, u_s);
+  const int nt = min(kTT, p.n - tile0);
+  const TileRows tr = tile_rows(p.c, b, kv, t0 + tile0, nt);
 
+  // dense values in the input dtype: one contiguous copy of the tile's rows
+  using VC = ValueCopy<D, BF16>;
+  const bool v_copy = p.v != nullptr && p.c.vmode != HEADQ_V_2BIT &&
+                      ((p.c.v_dtype == HEADQ_BF16) == BF16);
+  const int v_chunks = nt * VC::kCPR;
+  const uint4* v_src = v_copy ? reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.v) +
+                                                               (bk * p.n + tile0) * D * (BF16 ? 2 : 4))
+                              : nullptr;
+  uint4* v_dst = reinterpret_cast<uint4*>(p.c.v);
+  uint4 vb[VC::kBatch];
+  auto v_load = [&](int base) {
+#pragma unroll
+    for (int j = 0; j < VC::kBatch; ++j) {
+      const int i = base + j * kThreads + tid;
+      if (i < v_chunks) vb[j] = v_src[i];
+    }
+  };
+  auto v_store = [&](int base) {
+    if (tr.consecutive) {  // the tile's rows are one contiguous run of the plane
+      uint4* dst = v_dst + static_cast<size_t>(tr.row0) * VC::kCPR;
+#pragma unroll
+      for (int j = 0; j < VC::kBatch; ++j) {
+        const int i = base + j * kThreads + tid;
+        if (i < v_chunks) dst[i] = vb[j];
+      }
+      return;
+    }
+#pragma unroll
+    for (int j = 0; j < VC::kBatch; ++j) {
+      const int i = base + j * kThreads + tid;
+      if (i >= v_chunks) continue;
+      const int tt = i / VC::kCPR;
+      const long long row_s = cache_row(p.c, b, kv, t0 + tile0 + tt);
+      if (row_s >= 0) v_dst[static_cast<size_t>(row_s) * VC::kCPR + (i - tt * VC::kCPR)] = vb[j];
+    }
+  };
   // ---- phase A: base code, residual, values ---------------------------------
-  for (int task = tid; task < kTT * NG; task += kThreads) {
-    const int tt = task / NG, g = task - tt * NG;
-    const int t = tile0 + tt;
-    if (t >= p.n) continue;
-    const size_t in_off = (bk * p.n + t) * D + g * GS;
-    const long long row_s = cache_row(p.c, b, kv, t0 + t);
-    if (row_s < 0) continue;  // block-table entry outside the pool: not written
-    const size_t row = static_cast<size_t>(row_s);
+  // one (token, group) task: the keys' code and residual from kraw
+  auto key_group = [&](int tt, int g, size_t in_off, size_t row, RawGroup<GS, BF16>& kraw) {
     float x[GS];
-    codec::load_row<GS>(p.k, in_off, p.in_bf16, x);
     uint32_t packed[NW];
     float sc, mn;
-    codec::quantize_group<GS, true>(x, packed, sc, mn);  // x becomes the residual e
+    quantize_raw<GS, true, BF16>(p.k, in_off, kraw, x, packed, sc, mn);  // x: the residual e
     codec::store_codes<GS>(p.c.k_codes + row * (D / 4) + g * (GS / 4), packed);
     p.c.k_scale[row * NG + g] = sc;
     p.c.k_min[row * NG + g] = mn;
+    float4* er = reinterpret_cast<float4*>(e_s) + tt * L::RC + g * L::GC;
 #pragma unroll
-    for (int k = 0; k < GS; k += 4)
-      *reinterpret_cast<float4*>(e_s + tt * ES + g * GS + k) =
-          make_float4(x[k], x[k + 1], x[k + 2], x[k + 3]);
-    if (p.v != nullptr) store_value_group<D>(p, in_off, row, g);
+    for (int j = 0; j < GS / 4; ++j) er[j] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+  };
+  if (v_copy) {
+    v_load(0);
+    bool stored = false;
+    for (int task = tid; task < kTT * NG; task += kThreads) {
+      const int tt = task / NG, g = task - tt * NG;
+      if (tt >= nt) continue;
+      const size_t in_off = (bk * p.n + tile0 + tt) * D + g * GS;
+      RawGroup<GS, BF16> kraw;
+      load_raw<GS, BF16>(p.k, in_off, kraw);
+      if (!stored) {  // the copy's first batch, while the keys load
+        v_store(0);
+        stored = true;
+      }
+      const long long row_s = tile_row(p.c, tr, b, kv, t0 + tile0, tt);
+      if (row_s < 0) continue;  // block-table entry outside the pool: not written
+      key_group(tt, g, in_off, static_cast<size_t>(row_s), kraw);
+    }
+    if (!stored) v_store(0);
+    for (int base = VC::kBatch * kThreads; base < v_chunks; base += VC::kBatch * kThreads) {
+      v_load(base);
+      v_store(base);
+    }
+  } else {
+    for (int task = tid; task < kTT * NG; task += kThreads) {
+      const int tt = task / NG, g = task - tt * NG;
+      if (tt >= nt) continue;
+      const size_t in_off = (bk * p.n + tile0 + tt) * D + g * GS;
+      RawGroup<GS, BF16> kraw, vraw;
+      load_raw<GS, BF16>(p.k, in_off, kraw);
+      if (p.v != nullptr) load_raw<GS, BF16>(p.v, in_off, vraw);
+      const long long row_s = tile_row(p.c, tr, b, kv, t0 + tile0, tt);
+      if (row_s < 0) continue;
+      const size_t row = static_cast<size_t>(row_s);
+      key_group(tt, g, in_off, row, kraw);
+      if (p.v != nullptr) store_value_group<D, BF16>(p, in_off, vraw, row, g);
+    }
   }
   if (r == 0) return;  // no side code
-  side_code_tile<D, RB>(p, e_s, u_s, y_s, b, kv, tile0, t0);
+  __syncthreads();
+  side_code_tile<D, RB>(p, e_s, u_s, y_s, b, kv, tile0, t0, tr);
 }
 
 // The alternative base code, per channel over a block of 64 tokens: the CTA's
 // tile is one block (writes start on a block boundary).  Phase A1 stages the
-// keys; A2, one thread per channel: minimum, maximum and scale over the block's
-// tokens; A3, one thread per (token, 4 channels): codes, packed byte, residual.
-// Every step is the same IEEE fp32 operation as in the per-token code.
-template <int D, int RB>
-__global__ void __launch_bounds__(kThreads, 3)
+// keys (in the residual tile's layout) and stores the values; A2, one thread per
+// channel: minimum, maximum and scale over the block's tokens; A3, one thread
+// per (token, 4 channels): codes, packed byte, residual in place.  Every step is
+// the same IEEE fp32 operation as in the per-token code.
+template <int D, int RB, bool BF16>
+__global__ void __launch_bounds__(kThreads, BF16 ? 3 : 2)
 cache_write_channel_kernel(const CacheWriteParams p) {
   constexpr int GS = group_size(D);
   constexpr int NG = num_groups(D);
-  constexpr int ES = D + 4;
+  using L = ResTile<D>;
   static_assert(D <= kThreads, "one thread per channel");
 
-  extern __shared__ float smem[];
+  extern __shared__ float4 smem4[];
   const int r = p.c.r;
-  float* e_s = smem;                 // [kTT][ES]   keys, then residuals
-  float* u_s = e_s + kTT * ES;       // [D][r]      (phase A2 borrows it: [2][D])
-  float* y_s = u_s + D * (r > 2 ? r : 2);
+  float* e_s = reinterpret_cast<float*>(smem4);      // [kTT][RC chunks]: keys, then residuals
+  float* u_s = e_s + L::kFloats;
+  float* y_s = u_s + BasisTile<D, RB>::floats(r);
+  float* mn_s = y_s + kTT * (r + 1);                 // [D]
+  float* sc_s = mn_s + D;                            // [D]
 
   const int b = blockIdx.z, kv = blockIdx.y;
   const int tile0 = blockIdx.x * kTT;
@@ -188,33 +524,36 @@ cache_write_channel_kernel(const CacheWriteParams p) {
   const size_t bk = static_cast<size_t>(b) * p.c.Hkv + kv;
   const int t0 = p.t0;
   const int nt = min(kTT, p.n - tile0);
+  const TileRows tr = tile_rows(p.c, b, kv, t0 + tile0, nt);
+  if (r > 0) load_basis<D, RB>(p, kv, u_s);
 
   // A1: the block's keys, and the values (as for the per-token code)
   for (int task = tid; task < kTT * NG; task += kThreads) {
     const int tt = task / NG, g = task - tt * NG;
     if (tt >= nt) continue;
     const size_t in_off = (bk * p.n + tile0 + tt) * D + g * GS;
+    RawGroup<GS, BF16> kraw, vraw;
+    load_raw<GS, BF16>(p.k, in_off, kraw);
+    if (p.v != nullptr) load_raw<GS, BF16>(p.v, in_off, vraw);
     float x[GS];
-    codec::load_row<GS>(p.k, in_off, p.in_bf16, x);
+    unpack_raw<GS, BF16>(kraw, x);
+    float4* er = reinterpret_cast<float4*>(e_s) + tt * L::RC + g * L::GC;
 #pragma unroll
-    for (int k = 0; k < GS; k += 4)
-      *reinterpret_cast<float4*>(e_s + tt * ES + g * GS + k) =
-          make_float4(x[k], x[k + 1], x[k + 2], x[k + 3]);
+    for (int j = 0; j < GS / 4; ++j) er[j] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
     if (p.v != nullptr) {
-      const long long row_s = cache_row(p.c, b, kv, t0 + tile0 + tt);
-      if (row_s >= 0) store_value_group<D>(p, in_off, static_cast<size_t>(row_s), g);
+      const long long row_s = tile_row(p.c, tr, b, kv, t0 + tile0, tt);
+      if (row_s >= 0) store_value_group<D, BF16>(p, in_off, vraw, static_cast<size_t>(row_s), g);
     }
   }
   __syncthreads();
   const long long brow_s = cache_row(p.c, b, kv, t0 + tile0);  // the block's first row
-  float* mn_s = u_s;
-  float* sc_s = u_s + D;
   // A2: per channel, over the block's tokens
   if (tid < D) {
-    float lo = e_s[tid], hi = e_s[tid];
+    const int o = L::off(tid);
+    float lo = e_s[o], hi = e_s[o];
     for (int tt = 1; tt < nt; ++tt) {
-      lo = fminf(lo, e_s[tt * ES + tid]);
-      hi = fmaxf(hi, e_s[tt * ES + tid]);
+      lo = fminf(lo, e_s[tt * 4 * L::RC + o]);
+      hi = fmaxf(hi, e_s[tt * 4 * L::RC + o]);
     }
     lo = __fadd_rn(lo, 0.0f);  // a -0 extreme is stored as +0
     hi = __fadd_rn(hi, 0.0f);
@@ -232,48 +571,59 @@ cache_write_channel_kernel(const CacheWriteParams p) {
   for (int task = tid; task < kTT * (D / 4); task += kThreads) {
     const int tt = task / (D / 4), c4 = (task - tt * (D / 4)) * 4;
     if (tt >= nt) continue;
+    float4* ch = reinterpret_cast<float4*>(e_s + tt * 4 * L::RC + L::off(c4));
+    const float4 h = *ch;
+    const float xs[4] = {h.x, h.y, h.z, h.w};
+    float res[4];
     uint32_t byte = 0u;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int c = c4 + k;
-      const float x = e_s[tt * ES + c], lo = mn_s[c], scale = sc_s[c];
+      const float x = xs[k], lo = mn_s[c], scale = sc_s[c];
       int code = 0;
       if (scale != 0.0f) {
         const float tq = codec::rint_quot(__fsub_rn(x, lo), scale, __frcp_rn(scale));
         code = tq < 0.0f ? 0 : (tq > 3.0f ? 3 : static_cast<int>(tq));
       }
       byte |= static_cast<uint32_t>(code) << (2 * k);
-      e_s[tt * ES + c] = __fsub_rn(x, __fadd_rn(lo, __fmul_rn(static_cast<float>(code), scale)));
+      res[k] = __fsub_rn(x, __fadd_rn(lo, __fmul_rn(static_cast<float>(code), scale)));
     }
-    const long long row_s = cache_row(p.c, b, kv, t0 + tile0 + tt);
+    *ch = make_float4(res[0], res[1], res[2], res[3]);
+    const long long row_s = tile_row(p.c, tr, b, kv, t0 + tile0, tt);
     if (row_s >= 0) p.c.k_codes[static_cast<size_t>(row_s) * (D / 4) + c4 / 4] = static_cast<uint8_t>(byte);
   }
   if (r == 0) return;
-  __syncthreads();  // residuals complete; u_s is reloaded with U below
-  side_code_tile<D, RB>(p, e_s, u_s, y_s, b, kv, tile0, t0);
+  __syncthreads();  // residuals complete
+  side_code_tile<D, RB>(p, e_s, u_s, y_s, b, kv, tile0, t0, tr);
 }
 
-template <int D>
-cudaError_t launch_d(const CacheWriteParams& p, cudaStream_t s) {
-  const int r = p.c.r;
+template <int D, int RB>
+cudaError_t launch_rb(const CacheWriteParams& p, cudaStream_t s) {
   const bool channel = p.c.kmode == HEADQ_K_CHANNEL;
   if (channel && D > kThreads) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(float) * (static_cast<size_t>(kTT) * (D + 4) +
-                                       static_cast<size_t>(D) * (r > 2 ? r : 2) +
-                                       static_cast<size_t>(kTT) * (r + 1));
+  const size_t smem = sizeof(float) * cache_write_smem_floats<D, RB>(p.c.r, channel);
   dim3 grid((p.n + kTT - 1) / kTT, p.c.Hkv, p.c.B);
-  auto k = channel ? (r % 8 == 0 ? cache_write_channel_kernel<D, 8>
-                                 : (r % 4 == 0 ? cache_write_channel_kernel<D, 4>
-                                               : cache_write_channel_kernel<D, 2>))
-                   : (r % 8 == 0 ? cache_write_kernel<D, 8>
-                                 : (r % 4 == 0 ? cache_write_kernel<D, 4> : cache_write_kernel<D, 2>));
-  if (smem > 48 * 1024) {  // only the largest head dims need the opt-in
+  auto k = channel ? (p.in_bf16 ? cache_write_channel_kernel<D, RB, true>
+                               : cache_write_channel_kernel<D, RB, false>)
+                   : (p.in_bf16 ? cache_write_kernel<D, RB, true> : cache_write_kernel<D, RB, false>);
+  if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
   k<<<grid, kThreads, smem, s>>>(p);
   return cudaGetLastError();
+}
+
+// RB side rows per phase-B thread: the largest of 16, 8, 4, 2 that divides r.
+template <int D>
+cudaError_t launch_d(const CacheWriteParams& p, cudaStream_t s) {
+  const int r = p.c.r;
+  if constexpr (D >= 16)
+    if (r % 16 == 0) return launch_rb<D, 16>(p, s);
+  if (r % 8 == 0) return launch_rb<D, 8>(p, s);
+  if (r % 4 == 0) return launch_rb<D, 4>(p, s);
+  return launch_rb<D, 2>(p, s);
 }
 
 }  // namespace
