@@ -12,10 +12,10 @@
 //      loaded straight from HBM together, base code (a short path per channel,
 //      the exact codec near a rounding tie), codes/scale/min stored, the
 //      residual written to shared memory, values copied or coded
-//   B  one thread per (token, RB side rows), RB = 16 for r = 16: y = U_h^T e in
-//      channel order, one fused multiply-add per term, two rows per packed
-//      fp32x2 FMA, U_h read as warp-wide broadcasts; then max|y| (shared by warp
-//      shuffles when a token has several threads) and the 4-bit side code
+//   B  one thread per (token, RB side rows), two threads per token for r = 16:
+//      y = U_h^T e in channel order, one fused multiply-add per term, two rows per
+//      packed fp32x2 FMA, U_h read as (nearly) warp-wide broadcasts; then max|y|
+//      shared by a warp shuffle and the 4-bit side code of each thread's rows
 #include "codec.cuh"
 
 namespace headq {
@@ -28,8 +28,8 @@ constexpr unsigned kFull = 0xffffffffu;
 // The residual tile in shared memory, one fp32 per channel.  Group g of a
 // token starts at 16-byte chunk g*GC (GC = 2 mod 8: two chunks of padding per
 // 32-channel group) and a token row spans RC chunks (RC odd): the (token, group)
-// writes of phase A and the one-token-per-lane reads of phase B then fall in
-// distinct banks.
+// writes of phase A and the per-token reads of phase B then fall in distinct
+// banks.
 template <int D>
 struct ResTile {
   static constexpr int GS = group_size(D);
@@ -615,12 +615,17 @@ cudaError_t launch_rb(const CacheWriteParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// RB side rows per phase-B thread: the largest of 16, 8, 4, 2 that divides r.
+// RB side rows per phase-B thread: half the rank when that is 16, 8, 4 or 2 (two
+// threads per token: four warps of the CTA share the projection, and U_h reads
+// stay two addresses per warp instruction); else the largest of 8, 4, 2 dividing r.
 template <int D>
 cudaError_t launch_d(const CacheWriteParams& p, cudaStream_t s) {
   const int r = p.c.r;
-  if constexpr (D >= 16)
-    if (r % 16 == 0) return launch_rb<D, 16>(p, s);
+  if constexpr (D >= 32)
+    if (r == 32) return launch_rb<D, 16>(p, s);
+  if (r == 16) return launch_rb<D, 8>(p, s);
+  if (r == 8) return launch_rb<D, 4>(p, s);
+  if (r == 4) return launch_rb<D, 2>(p, s);
   if (r % 8 == 0) return launch_rb<D, 8>(p, s);
   if (r % 4 == 0) return launch_rb<D, 4>(p, s);
   return launch_rb<D, 2>(p, s);
