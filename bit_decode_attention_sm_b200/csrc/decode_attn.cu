@@ -39,34 +39,53 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// A staged tile row of 2-bit key codes: d/16 32-bit words (for d = 8, the row's
+// two bytes in one word); rows padded by one word so that the 32 tokens a warp
+// reads at once fall in distinct banks.
 template <int D>
-__device__ __forceinline__ float value_at(const DecodeParams& p, size_t row, int c) {
-  if (p.c.vmode == HEADQ_V_2BIT) {
-    constexpr int NG = num_groups(D);
-    const int g = c / group_size(D);
-    const float code = static_cast<float>(code2(p.c.v_codes + row * (D / 4), c));
-    return __fadd_rn(p.c.v_min[row * NG + g], __fmul_rn(code, p.c.v_scale[row * NG + g]));
-  }
-  return load_elem(p.c.v, row * D + c, p.c.v_dtype == HEADQ_BF16);
+struct CodeRow {
+  static constexpr int kWords = D >= 16 ? D / 16 : 1;
+  static constexpr int kCodes = D >= 16 ? 16 : D;  // codes per word
+  static constexpr int kStride = kWords + 1;
+};
+
+// Code k of w as an exact float: the bits of 2^23 + code, less 2^23 (an FMA-pipe
+// add instead of an integer conversion).
+__device__ __forceinline__ float code_f(uint32_t w, int k) {
+  return __int_as_float(0x4B000000u | ((w >> (2 * k)) & 3u)) - 8388608.0f;
 }
 
+// Generic split kernel, every shape the tensor-core kernel does not take.  Per
+// 32-token tile: the tile's codes, scales, side codes and values are staged in
+// shared memory with vector loads; one thread per (head, token) forms the logit
+// from the staged code words; one warp per head updates the online softmax; one
+// thread per (channel, head set) accumulates p_j v_j.
 template <int D>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
 decode_split_kernel(const DecodeParams p) {
   constexpr int NG = num_groups(D);
   constexpr int GS = group_size(D);
+  using CR = CodeRow<D>;
+  constexpr int KS = NG + 1;  // padded row of per-token group scales / minima
   const int G = p.G, r = p.c.r;
-  extern __shared__ float sm[];
-  float* q_s = sm;                // [G][D]
-  float* qg_s = q_s + G * D;      // [G][NG]   group sums of q
-  float* qt_s = qg_s + G * NG;    // [G][r]    sigma * U_h^T q
-  float* s_s = qt_s + G * r;      // [G][kTile] logits, then weights
-  float* m_s = s_s + G * kTile;   // [G]
-  float* l_s = m_s + G;           // [G]
-  float* a_s = l_s + G;           // [G]
-  float* v_s = a_s + G;           // [kTile][D] the tile's values, dequantised
-  float* kmn_s = v_s + kTile * D; // [D] per-channel key minima of the tile's block
-  float* ksc_s = kmn_s + D;       // [D] and scales (per-channel base code)
+  const bool channel = p.c.kmode == HEADQ_K_CHANNEL;
+  const int ZB = r > 0 ? ((r / 2 + 3) / 4 + 1) * 4 : 0;  // padded side-code row, bytes
+  extern __shared__ float4 sm4[];
+  float* v_s = reinterpret_cast<float*>(sm4);  // [kTile][D] the tile's values (float4 stores)
+  float* q_s = v_s + kTile * D;      // [G][D]
+  float* qs_s = q_s + G * D;         // [G][D]    per-channel code: q * scale of the block
+  float* qg_s = qs_s + (channel ? G * D : 0);  // [G][NG] group sums of q
+  float* qt_s = qg_s + G * NG;       // [G][r]    sigma * U_h^T q
+  float* s_s = qt_s + G * r;         // [G][kTile] logits, then weights
+  float* m_s = s_s + G * kTile;      // [G]
+  float* l_s = m_s + G;              // [G]
+  float* a_s = l_s + G;              // [G]
+  float* qm_s = a_s + G;             // [G]       per-channel code: q . minimum of the block
+  float* ks_s = qm_s + G;            // [kTile][KS] per-token code: group scales
+  float* km_s = ks_s + kTile * KS;   // [kTile][KS] and minima
+  float* zs_s = km_s + kTile * KS;   // [kTile] side scales
+  uint32_t* kc_s = reinterpret_cast<uint32_t*>(zs_s + kTile);  // [kTile][CR::kStride]
+  uint8_t* zb_s = reinterpret_cast<uint8_t*>(kc_s + kTile * CR::kStride);  // [kTile][ZB]
 
   const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -96,7 +115,6 @@ decode_split_kernel(const DecodeParams p) {
     for (int c = 0; c < D; ++c) acc = fmaf(U[c * r + ii], q_s[h * D + c], acc);
     qt_s[i] = p.corr_sign * acc;
   }
-  __syncthreads();
 
   float o[kMaxOut];
 #pragma unroll
@@ -106,55 +124,127 @@ decode_split_kernel(const DecodeParams p) {
     const int nt = min(kTile, t_end - t0);
     // the tile's rows are consecutive: chunks start at multiples of 64 tokens
     const size_t row0 = cache_row_read(p.c, b, kv, t0, tid == 0 ? p.err : nullptr);
-    // the tile's values (and, per-channel code, its block's minima and scales)
-    // staged once with coalesced loads, so the readout below reads shared memory
-    for (int e = tid; e < nt * D; e += kThreads) {
-      const int j = e / D, c = e - j * D;
-      v_s[e] = value_at<D>(p, row0 + j, c);
-    }
-    if (p.c.kmode == HEADQ_K_CHANNEL)
-      for (int c = tid; c < D; c += kThreads) {
-        kmn_s[c] = p.c.k_min[(row0 >> 6) * D + c];
-        ksc_s[c] = p.c.k_scale[(row0 >> 6) * D + c];
+    // ---- staging ------------------------------------------------------------
+    if constexpr (D >= 16) {
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(p.c.k_codes + row0 * (D / 4));
+      for (int e = tid; e < nt * CR::kWords; e += kThreads) {
+        const int j = e / CR::kWords, w = e - j * CR::kWords;
+        kc_s[j * CR::kStride + w] = src[e];
       }
+    } else {
+      const uint16_t* src = reinterpret_cast<const uint16_t*>(p.c.k_codes + row0 * (D / 4));
+      for (int j = tid; j < nt; j += kThreads) kc_s[j * CR::kStride] = src[j];
+    }
+    if (!channel) {
+      for (int e = tid; e < nt * NG; e += kThreads) {
+        const int j = e / NG, g = e - j * NG;
+        ks_s[j * KS + g] = p.c.k_scale[row0 * NG + e];
+        km_s[j * KS + g] = p.c.k_min[row0 * NG + e];
+      }
+    } else if (((t0 - t_begin) & 63) == 0) {  // a new 64-token block: fold its scale into q
+      const size_t bi = (row0 >> 6) * D;
+      for (int i = tid; i < G * D; i += kThreads) qs_s[i] = q_s[i] * p.c.k_scale[bi + (i % D)];
+      for (int h = warp; h < G; h += kThreads / 32) {
+        float acc = 0.0f;
+        for (int c = lane; c < D; c += 32) acc = fmaf(q_s[h * D + c], p.c.k_min[bi + c], acc);
+        acc = warp_sum(acc);
+        if (lane == 0) qm_s[h] = acc;
+      }
+    }
+    if (r > 0) {
+      for (int e = tid; e < nt * (r / 2); e += kThreads) {
+        const int j = e / (r / 2), i = e - j * (r / 2);
+        zb_s[j * ZB + i] = p.c.z_codes[row0 * (r / 2) + e];
+      }
+      for (int j = tid; j < nt; j += kThreads) zs_s[j] = p.c.z_scale[row0 + j];
+    }
+    if (p.c.vmode == HEADQ_V_2BIT) {  // one thread per (token, 4 channels)
+      for (int e = tid; e < nt * (D / 4); e += kThreads) {
+        const int j = e / (D / 4), c4 = e - j * (D / 4), g = (4 * c4) / GS;
+        const size_t row = row0 + j;
+        const uint32_t cb = p.c.v_codes[row * (D / 4) + c4];
+        const float vsc = p.c.v_scale[row * NG + g], vmn = p.c.v_min[row * NG + g];
+        float4 v;
+        v.x = __fadd_rn(vmn, __fmul_rn(static_cast<float>(cb & 3u), vsc));
+        v.y = __fadd_rn(vmn, __fmul_rn(static_cast<float>((cb >> 2) & 3u), vsc));
+        v.z = __fadd_rn(vmn, __fmul_rn(static_cast<float>((cb >> 4) & 3u), vsc));
+        v.w = __fadd_rn(vmn, __fmul_rn(static_cast<float>(cb >> 6), vsc));
+        *reinterpret_cast<float4*>(v_s + j * D + 4 * c4) = v;
+      }
+    } else if (p.c.v_dtype == HEADQ_BF16) {  // one thread per (token, 8 channels)
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.c.v) + row0 * D);
+      for (int e = tid; e < nt * (D / 8); e += kThreads) {
+        const uint4 u = src[e];
+        float* dst = v_s + 8 * e;
+        *reinterpret_cast<float4*>(dst) =
+            make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                        __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+        *reinterpret_cast<float4*>(dst + 4) =
+            make_float4(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xffff0000u),
+                        __uint_as_float(u.w << 16), __uint_as_float(u.w & 0xffff0000u));
+      }
+    } else {  // fp32
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.c.v) + row0 * D);
+      for (int e = tid; e < nt * (D / 4); e += kThreads)
+        reinterpret_cast<float4*>(v_s)[e] = src[e];
+    }
     __syncthreads();
-    // phase 1: logits of (head, token) pairs
+    // ---- phase 1: logits of (head, token) pairs from the staged code words -----
     for (int idx = tid; idx < G * kTile; idx += kThreads) {
       const int h = idx / kTile, j = idx - h * kTile;
       float s = -INFINITY;
       if (j < nt) {
-        const size_t row = row0 + j;
-        const uint8_t* cr = p.c.k_codes + row * (D / 4);
-        const float* qh = q_s + h * D;
-        float acc = 0.0f;
-        if (p.c.kmode == HEADQ_K_CHANNEL) {  // per-channel minimum and scale of the block
-          for (int c = 0; c < D; ++c) {
-            const float kh =
-                __fadd_rn(kmn_s[c], __fmul_rn(static_cast<float>(code2(cr, c)), ksc_s[c]));
-            acc = fmaf(qh[c], kh, acc);
+        const uint32_t* kw = kc_s + j * CR::kStride;
+        float acc;
+        if (channel) {  // q.k^ = q.min + sum_c (q_c scale_c) code_c, per block
+          const float4* qh = reinterpret_cast<const float4*>(qs_s + h * D);
+          acc = qm_s[h];
+#pragma unroll
+          for (int w = 0; w < CR::kWords; ++w) {
+            const uint32_t word = kw[w];
+#pragma unroll
+            for (int k4 = 0; k4 < CR::kCodes / 4; ++k4) {
+              const float4 q4 = qh[w * 4 + k4];
+              acc = fmaf(q4.x, code_f(word, 4 * k4), acc);
+              acc = fmaf(q4.y, code_f(word, 4 * k4 + 1), acc);
+              acc = fmaf(q4.z, code_f(word, 4 * k4 + 2), acc);
+              acc = fmaf(q4.w, code_f(word, 4 * k4 + 3), acc);
+            }
           }
-        } else {
+        } else {  // sum_g ( min_g Q_g + scale_g sum_{c in g} q_c code_c )
+          const float4* qh = reinterpret_cast<const float4*>(q_s + h * D);
+          acc = 0.0f;
+#pragma unroll
           for (int g = 0; g < NG; ++g) {
             float pg = 0.0f;
-            for (int c = 0; c < GS; ++c)
-              pg = fmaf(qh[g * GS + c], static_cast<float>(code2(cr, g * GS + c)), pg);
-            acc = fmaf(p.c.k_min[row * NG + g], qg_s[h * NG + g], acc);
-            acc = fmaf(p.c.k_scale[row * NG + g], pg, acc);
+#pragma unroll
+            for (int c4 = 0; c4 < GS / 4; ++c4) {
+              const int cc = g * GS + 4 * c4;
+              const uint32_t word = kw[cc / CR::kCodes];
+              const int k = cc % CR::kCodes;
+              const float4 q4 = qh[cc / 4];
+              pg = fmaf(q4.x, code_f(word, k), pg);
+              pg = fmaf(q4.y, code_f(word, k + 1), pg);
+              pg = fmaf(q4.z, code_f(word, k + 2), pg);
+              pg = fmaf(q4.w, code_f(word, k + 3), pg);
+            }
+            acc = fmaf(km_s[j * KS + g], qg_s[h * NG + g], acc);
+            acc = fmaf(ks_s[j * KS + g], pg, acc);
           }
         }
         if (r > 0) {
-          const uint8_t* zr = p.c.z_codes + row * (r / 2);
+          const uint8_t* zr = zb_s + j * ZB;
           float cz = 0.0f;
           for (int i = 0; i < r; ++i)
             cz = fmaf(qt_s[h * r + i], static_cast<float>(nibble(zr, i)), cz);
-          acc = fmaf(p.c.z_scale[row], cz, acc);
+          acc = fmaf(zs_s[j], cz, acc);
         }
         s = acc * p.sm_scale;
       }
       s_s[idx] = s;
     }
     __syncthreads();
-    // phase 2: online softmax update, one warp per head
+    // ---- phase 2: online softmax update, one warp per head --------------------
     for (int h = warp; h < G; h += kThreads / 32) {
       const float s = s_s[h * kTile + lane];
       const float m_old = m_s[h];
@@ -171,7 +261,7 @@ decode_split_kernel(const DecodeParams p) {
       }
     }
     __syncthreads();
-    // phase 3: rescale and accumulate p_j v_j
+    // ---- phase 3: rescale and accumulate p_j v_j ------------------------------
 #pragma unroll
     for (int k = 0; k < kMaxOut; ++k) {
       const int idx = tid + k * kThreads;
@@ -264,15 +354,23 @@ decode_combine_kernel(const DecodeParams p) {
   if (threadIdx.x == 0 && p.lse) p.lse[bh] = L > 0.0f ? ML[0] + logf(L) : -INFINITY;
 }
 
+// shared memory of decode_split_kernel, in the order it is carved up
+template <int D>
+size_t decode_split_smem(int G, int r, bool channel) {
+  const int NG = num_groups(D), KS = NG + 1;
+  const int ZB = r > 0 ? ((r / 2 + 3) / 4 + 1) * 4 : 0;
+  size_t f = static_cast<size_t>(kTile) * D + G * D + (channel ? G * D : 0) + G * NG + G * r +
+             G * kTile + 4 * G + 2 * kTile * KS + kTile;
+  return f * sizeof(float) + sizeof(uint32_t) * kTile * CodeRow<D>::kStride + kTile * ZB;
+}
+
 template <int D>
 cudaError_t launch_d(const DecodeParams& p, bool mma, cudaStream_t s) {
   if (mma) {
     const cudaError_t e = launch_decode_mma(p, s);
     if (e != cudaSuccess) return e;
   } else {
-    const int G = p.G, r = p.c.r;
-    const size_t smem = sizeof(float) * (static_cast<size_t>(G) * D + G * num_groups(D) +
-                                         G * r + G * kTile + 3 * G + kTile * D + 2 * D);
+    const size_t smem = decode_split_smem<D>(p.G, p.c.r, p.c.kmode == HEADQ_K_CHANNEL);
     auto k = decode_split_kernel<D>;
     if (smem > 48 * 1024) {
       cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
