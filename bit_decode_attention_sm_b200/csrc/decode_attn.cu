@@ -26,6 +26,7 @@ namespace {
 constexpr int kTile = 32;      // tokens per inner step (one per lane in phase 2)
 constexpr int kThreads = 128;
 constexpr int kMaxOut = 16;    // (G * d) / kThreads outputs per thread at most
+static_assert(kThreads == 4 * kTile, "phase 1 maps the four warps to four channel quarters");
 constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -60,9 +61,11 @@ __device__ __forceinline__ float code_f(uint32_t w, int k) {
 // shared memory with vector loads; one thread per (head, token) forms the logit
 // from the staged code words; one warp per head updates the online softmax; one
 // thread per (channel, head set) accumulates p_j v_j.
-template <int D>
-__global__ void __launch_bounds__(kThreads, 4)
+template <int D, int GM>
+__global__ void __launch_bounds__(kThreads, D >= 256 ? 2 : 4)
 decode_split_kernel(const DecodeParams p) {
+  // (G * d) / kThreads outputs per thread (at most kMaxOut: G * d <= 2048)
+  constexpr int KO = GM * D / kThreads < 1 ? 1 : (GM * D / kThreads > kMaxOut ? kMaxOut : GM * D / kThreads);
   constexpr int NG = num_groups(D);
   constexpr int GS = group_size(D);
   using CR = CodeRow<D>;
@@ -76,8 +79,9 @@ decode_split_kernel(const DecodeParams p) {
   float* qs_s = q_s + G * D;         // [G][D]    per-channel code: q * scale of the block
   float* qg_s = qs_s + (channel ? G * D : 0);  // [G][NG] group sums of q
   float* qt_s = qg_s + G * NG;       // [G][r]    sigma * U_h^T q
-  float* s_s = qt_s + G * r;         // [G][kTile] logits, then weights
-  float* m_s = s_s + G * kTile;      // [G]
+  float* s_s = qt_s + G * r;         // [G][kTile] weights
+  float* ps_s = s_s + G * kTile;     // [4][G][kTile] partial logits of the channel quarters
+  float* m_s = ps_s + 4 * G * kTile; // [G]
   float* l_s = m_s + G;              // [G]
   float* a_s = l_s + G;              // [G]
   float* qm_s = a_s + G;             // [G]       per-channel code: q . minimum of the block
@@ -116,9 +120,9 @@ decode_split_kernel(const DecodeParams p) {
     qt_s[i] = p.corr_sign * acc;
   }
 
-  float o[kMaxOut];
+  float o[KO];
 #pragma unroll
-  for (int k = 0; k < kMaxOut; ++k) o[k] = 0.0f;
+  for (int k = 0; k < KO; ++k) o[k] = 0.0f;
 
   for (int t0 = t_begin; t0 < t_end; t0 += kTile) {
     const int nt = min(kTile, t_end - t0);
@@ -189,64 +193,106 @@ decode_split_kernel(const DecodeParams p) {
         reinterpret_cast<float4*>(v_s)[e] = src[e];
     }
     __syncthreads();
-    // ---- phase 1: logits of (head, token) pairs from the staged code words -----
-    for (int idx = tid; idx < G * kTile; idx += kThreads) {
-      const int h = idx / kTile, j = idx - h * kTile;
-      float s = -INFINITY;
-      if (j < nt) {
-        const uint32_t* kw = kc_s + j * CR::kStride;
-        float acc;
-        if (channel) {  // q.k^ = q.min + sum_c (q_c scale_c) code_c, per block
-          const float4* qh = reinterpret_cast<const float4*>(qs_s + h * D);
-          acc = qm_s[h];
+    // ---- phase 1: partial logits; warp = quarter of the channels, lane = token --
+    // Each code is decoded once for a batch of GM heads; a warp's lanes read the
+    // same query words (broadcasts) and code rows 9 words apart (distinct banks).
+    // The softmax warps add the four quarters in a fixed order.
+    {
+      constexpr int NP = kThreads / kTile;  // quarters (one per warp)
+      constexpr int PS = D / NP;            // channels per thread
+      constexpr int CS = PS >= 4 ? 4 : PS;  // channels per step
+      const int j = lane, part = warp;
+      const bool live = j < nt;
+      const int c0 = part * PS;
+      const uint32_t* kw = kc_s + j * CR::kStride;
+      for (int hb = 0; hb < G; hb += GM) {  // one pass unless G > 16
+        const int gn = min(GM, G - hb);
+        float acc[GM];
 #pragma unroll
-          for (int w = 0; w < CR::kWords; ++w) {
-            const uint32_t word = kw[w];
+        for (int h = 0; h < GM; ++h) acc[h] = 0.0f;
+        // sum_{c in [cb, cb + n)} q'_{h,c} code_c into sum[h], q' rows at qb
+        auto dot = [&](const float* qb, int cb, int n, float (&sum)[GM]) {
 #pragma unroll
-            for (int k4 = 0; k4 < CR::kCodes / 4; ++k4) {
-              const float4 q4 = qh[w * 4 + k4];
-              acc = fmaf(q4.x, code_f(word, 4 * k4), acc);
-              acc = fmaf(q4.y, code_f(word, 4 * k4 + 1), acc);
-              acc = fmaf(q4.z, code_f(word, 4 * k4 + 2), acc);
-              acc = fmaf(q4.w, code_f(word, 4 * k4 + 3), acc);
+          for (int i = 0; i < n; i += CS) {
+            const int c = cb + i;
+            const uint32_t word = kw[c / CR::kCodes] >> (2 * (c % CR::kCodes));
+            float e[CS];
+#pragma unroll
+            for (int k = 0; k < CS; ++k) e[k] = code_f(word, k);
+#pragma unroll
+            for (int h = 0; h < GM; ++h) {
+              if (h < gn) {
+                const float* qh = qb + h * D + c;
+                if constexpr (CS == 4) {
+                  const float4 q4 = *reinterpret_cast<const float4*>(qh);
+                  sum[h] = fmaf(q4.x, e[0], sum[h]);
+                  sum[h] = fmaf(q4.y, e[1], sum[h]);
+                  sum[h] = fmaf(q4.z, e[2], sum[h]);
+                  sum[h] = fmaf(q4.w, e[3], sum[h]);
+                } else {
+#pragma unroll
+                  for (int k = 0; k < CS; ++k) sum[h] = fmaf(qh[k], e[k], sum[h]);
+                }
+              }
             }
           }
-        } else {  // sum_g ( min_g Q_g + scale_g sum_{c in g} q_c code_c )
-          const float4* qh = reinterpret_cast<const float4*>(q_s + h * D);
-          acc = 0.0f;
+        };
+        if (live) {
+          if (channel) {  // q.k^ = q.min + sum_c (q_c scale_c) code_c, per block
+            if (part == 0) {
 #pragma unroll
-          for (int g = 0; g < NG; ++g) {
-            float pg = 0.0f;
-#pragma unroll
-            for (int c4 = 0; c4 < GS / 4; ++c4) {
-              const int cc = g * GS + 4 * c4;
-              const uint32_t word = kw[cc / CR::kCodes];
-              const int k = cc % CR::kCodes;
-              const float4 q4 = qh[cc / 4];
-              pg = fmaf(q4.x, code_f(word, k), pg);
-              pg = fmaf(q4.y, code_f(word, k + 1), pg);
-              pg = fmaf(q4.z, code_f(word, k + 2), pg);
-              pg = fmaf(q4.w, code_f(word, k + 3), pg);
+              for (int h = 0; h < GM; ++h)
+                if (h < gn) acc[h] = qm_s[hb + h];
             }
-            acc = fmaf(km_s[j * KS + g], qg_s[h * NG + g], acc);
-            acc = fmaf(ks_s[j * KS + g], pg, acc);
+            dot(qs_s + hb * D, c0, PS, acc);
+          } else {  // sum_g ( min_g Q_g + scale_g sum_{c in g} q_c code_c )
+            constexpr int SEG = PS < GS ? PS : GS;  // channels of one group in this thread
+#pragma unroll
+            for (int sg = 0; sg < PS / SEG; ++sg) {
+              const int cb = c0 + sg * SEG, g = cb / GS;
+              float pg[GM];
+#pragma unroll
+              for (int h = 0; h < GM; ++h) pg[h] = 0.0f;
+              dot(q_s + hb * D, cb, SEG, pg);
+              const float km = km_s[j * KS + g], ks = ks_s[j * KS + g];
+              const bool first = cb % GS == 0;  // this thread holds the group's start
+#pragma unroll
+              for (int h = 0; h < GM; ++h) {
+                if (h < gn) {
+                  if (first) acc[h] = fmaf(km, qg_s[(hb + h) * NG + g], acc[h]);
+                  acc[h] = fmaf(ks, pg[h], acc[h]);
+                }
+              }
+            }
+          }
+          if (r > 0) {  // side rows part, part + NP, ...
+            const uint8_t* zr = zb_s + j * ZB;
+            float cz[GM];
+#pragma unroll
+            for (int h = 0; h < GM; ++h) cz[h] = 0.0f;
+            for (int i = part; i < r; i += NP) {
+              const float w = static_cast<float>(nibble(zr, i));
+#pragma unroll
+              for (int h = 0; h < GM; ++h)
+                if (h < gn) cz[h] = fmaf(qt_s[(hb + h) * r + i], w, cz[h]);
+            }
+            const float zs = zs_s[j];
+#pragma unroll
+            for (int h = 0; h < GM; ++h) acc[h] = fmaf(zs, cz[h], acc[h]);
           }
         }
-        if (r > 0) {
-          const uint8_t* zr = zb_s + j * ZB;
-          float cz = 0.0f;
-          for (int i = 0; i < r; ++i)
-            cz = fmaf(qt_s[h * r + i], static_cast<float>(nibble(zr, i)), cz);
-          acc = fmaf(zs_s[j], cz, acc);
-        }
-        s = acc * p.sm_scale;
+#pragma unroll
+        for (int h = 0; h < GM; ++h)
+          if (h < gn) ps_s[(part * G + hb + h) * kTile + j] = acc[h];
       }
-      s_s[idx] = s;
     }
     __syncthreads();
     // ---- phase 2: online softmax update, one warp per head --------------------
     for (int h = warp; h < G; h += kThreads / 32) {
-      const float s = s_s[h * kTile + lane];
+      const float* ph = ps_s + h * kTile + lane;
+      const float s = lane < nt ? ((ph[0] + ph[G * kTile]) + (ph[2 * G * kTile] + ph[3 * G * kTile])) *
+                                      p.sm_scale
+                                : -INFINITY;
       const float m_old = m_s[h];
       const float m_new = fmaxf(m_old, warp_max(s));
       const float pj = lane < nt ? expf(s - m_new) : 0.0f;
@@ -263,7 +309,7 @@ decode_split_kernel(const DecodeParams p) {
     __syncthreads();
     // ---- phase 3: rescale and accumulate p_j v_j ------------------------------
 #pragma unroll
-    for (int k = 0; k < kMaxOut; ++k) {
+    for (int k = 0; k < KO; ++k) {
       const int idx = tid + k * kThreads;
       if (idx < G * D) {
         const int h = idx / D, c = idx - h * D;
@@ -279,7 +325,7 @@ decode_split_kernel(const DecodeParams p) {
   // epilogue: partial (o, m, l) or the final result
   const PartView pv = part_view(p.part, static_cast<size_t>(p.c.B) * p.Hq, p.splits, D);
 #pragma unroll
-  for (int k = 0; k < kMaxOut; ++k) {
+  for (int k = 0; k < KO; ++k) {
     const int idx = tid + k * kThreads;
     if (idx < G * D) {
       const int h = idx / D, c = idx - h * D;
@@ -360,8 +406,33 @@ size_t decode_split_smem(int G, int r, bool channel) {
   const int NG = num_groups(D), KS = NG + 1;
   const int ZB = r > 0 ? ((r / 2 + 3) / 4 + 1) * 4 : 0;
   size_t f = static_cast<size_t>(kTile) * D + G * D + (channel ? G * D : 0) + G * NG + G * r +
-             G * kTile + 4 * G + 2 * kTile * KS + kTile;
+             5 * G * kTile + 4 * G + 2 * kTile * KS + kTile;
   return f * sizeof(float) + sizeof(uint32_t) * kTile * CodeRow<D>::kStride + kTile * ZB;
+}
+
+// The split kernel for a batch of GM >= G heads (G > 16: several 16-head passes)
+template <int D, int GM>
+cudaError_t launch_split_gm(const DecodeParams& p, cudaStream_t s) {
+  const size_t smem = decode_split_smem<D>(p.G, p.c.r, p.c.kmode == HEADQ_K_CHANNEL);
+  auto k = decode_split_kernel<D, GM>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(p.splits, p.c.Hkv, p.c.B);
+  k<<<grid, kThreads, smem, s>>>(p);
+  return cudaSuccess;
+}
+
+template <int D>
+cudaError_t launch_split(const DecodeParams& p, cudaStream_t s) {
+  if (p.G <= 1) return launch_split_gm<D, 1>(p, s);
+  if (p.G <= 2) return launch_split_gm<D, 2>(p, s);
+  if (p.G <= 4) return launch_split_gm<D, 4>(p, s);
+  if (p.G <= 8) return launch_split_gm<D, 8>(p, s);
+  if constexpr (16 * D <= 2048) return launch_split_gm<D, 16>(p, s);  // G * d <= 2048
+  return cudaErrorInvalidValue;
 }
 
 template <int D>
@@ -370,15 +441,8 @@ cudaError_t launch_d(const DecodeParams& p, bool mma, cudaStream_t s) {
     const cudaError_t e = launch_decode_mma(p, s);
     if (e != cudaSuccess) return e;
   } else {
-    const size_t smem = decode_split_smem<D>(p.G, p.c.r, p.c.kmode == HEADQ_K_CHANNEL);
-    auto k = decode_split_kernel<D>;
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-    }
-    dim3 grid(p.splits, p.c.Hkv, p.c.B);
-    k<<<grid, kThreads, smem, s>>>(p);
+    const cudaError_t e = launch_split<D>(p, s);
+    if (e != cudaSuccess) return e;
   }
   if (p.splits > 1 && !(mma && p.fused)) {  // unless the split kernel merged its splits
     if (p.splits > kCombineMaxSplits) return cudaErrorInvalidConfiguration;
