@@ -325,17 +325,26 @@ struct KlStage {
   }
 };
 
-// copy `bytes_per_row` x rows (contiguous in global, rows of `rb` bytes) into
-// shared rows of stride `dst_stride`, zero-filling rows >= valid
-__device__ __forceinline__ void stage_rows(uint8_t* dst, int dst_stride, const uint8_t* src, int rb,
-                                           int valid, int tid) {
-  const int chunks = rb / 16;
-  for (int e = tid; e < kSTT * chunks; e += kSThreads) {
-    const int row = e / chunks, c = e - row * chunks;
+// copy kSTT rows of CH 16-byte chunks (contiguous in global) into shared rows of
+// stride `dst_stride`, zero-filling rows >= valid
+template <int CH>
+__device__ __forceinline__ void stage_rows_ch(uint8_t* dst, int dst_stride, const uint8_t* src,
+                                              int valid, int tid) {
+  for (int e = tid; e < kSTT * CH; e += kSThreads) {
+    const int row = e / CH, c = e - row * CH;
     const bool ok = row < valid;
-    cp_async16(dst + row * dst_stride + c * 16, ok ? src + static_cast<size_t>(row) * rb + c * 16 : src,
+    cp_async16(dst + row * dst_stride + c * 16, ok ? src + static_cast<size_t>(row) * CH * 16 + c * 16 : src,
                ok);
   }
+}
+// rows of rb = D * 2 or D * 4 bytes (the chunk count a compile-time constant)
+template <int D>
+__device__ __forceinline__ void stage_rows(uint8_t* dst, int dst_stride, const uint8_t* src, int rb,
+                                           int valid, int tid) {
+  if (rb == D * 2)
+    stage_rows_ch<D * 2 / 16>(dst, dst_stride, src, valid, tid);
+  else
+    stage_rows_ch<D * 4 / 16>(dst, dst_stride, src, valid, tid);
 }
 // a contiguous block (rows of rb bytes packed), valid rows only
 __device__ __forceinline__ void stage_block(uint8_t* dst, const uint8_t* src, int rb, int valid,
@@ -348,9 +357,22 @@ __device__ __forceinline__ void stage_block(uint8_t* dst, const uint8_t* src, in
   }
 }
 
-__device__ __forceinline__ float ld_smem_elem(const uint8_t* row, int c, bool bf16) {
-  return bf16 ? bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(row)[c])
-              : reinterpret_cast<const float*>(row)[c];
+// channels c .. c+7 of a staged row (bf16 or fp32), c a multiple of 8
+__device__ __forceinline__ void ld8(const uint8_t* row, int c, bool bf16, float (&x)[8]) {
+  if (bf16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(row + 2 * c);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      x[2 * k] = __uint_as_float(w[k] << 16);
+      x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(row + 4 * c);
+    const float4 b = *reinterpret_cast<const float4*>(row + 4 * c + 16);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
 }
 
 template <int D>
@@ -370,9 +392,9 @@ attn_kl_staged_kernel(const AttnKlParams p) {
   float* dv_s = dk_s + kSTT * DS;                              // [kSTT][DS]
   float* q_s = dv_s + kSTT * DS;                               // [G][D]
   float* qt_s = q_s + G * D;                                   // [G][r]
-  float* s_s = qt_s + G * (r > 0 ? r : 1);                     // [G][kSTT]
-  float* d_s = s_s + G * kSTT;                                 // [G][kSTT]
-  float* n2_s = d_s + G * kSTT;                                // [kSTT]
+  float* s_s = qt_s + G * (r > 0 ? r : 1);                     // [2][G][kSTT] s halves, then w
+  float* d_s = s_s + 2 * G * kSTT;                             // [2][G][kSTT] delta halves
+  float* n2_s = d_s + 2 * G * kSTT;                            // [kSTT]
   float* m_s = n2_s + kSTT;                                    // [G]
   float* md_s = m_s + G;                                       // [G]
   float* a_s = md_s + G;                                       // [G]
@@ -395,13 +417,13 @@ attn_kl_staged_kernel(const AttnKlParams p) {
     uint8_t* st = stg[i & 1];
     const size_t frow0 = bk * p.T + t0;
     const size_t crow0 = cache_row_read(p.c, b, kv, t0, tid == 0 ? p.err : nullptr);
-    stage_rows(st + L.kf, L.frow, static_cast<const uint8_t*>(p.k_full) + frow0 * D * esz,
+    stage_rows<D>(st + L.kf, L.frow, static_cast<const uint8_t*>(p.k_full) + frow0 * D * esz,
                D * esz, nv, tid);
-    stage_rows(st + L.vf, L.frow, static_cast<const uint8_t*>(p.v_full) + frow0 * D * esz,
+    stage_rows<D>(st + L.vf, L.frow, static_cast<const uint8_t*>(p.v_full) + frow0 * D * esz,
                D * esz, nv, tid);
     if (!v2) {
       const int cesz = cv_bf16 ? 2 : 4;
-      stage_rows(st + L.cv, L.cvrow, static_cast<const uint8_t*>(p.c.v) + crow0 * D * cesz,
+      stage_rows<D>(st + L.cv, L.cvrow, static_cast<const uint8_t*>(p.c.v) + crow0 * D * cesz,
                  D * cesz, nv, tid);
     } else {
       stage_block(st + L.vc, p.c.v_codes + crow0 * (D / 4), D / 4, nv, tid);
@@ -452,59 +474,66 @@ attn_kl_staged_kernel(const AttnKlParams p) {
     const uint8_t* st = stg[i & 1];
     const int t0 = t_begin + i * kSTT;
     const int nt = min(kSTT, t_end - t0);
-    // phase 0: key and value errors per (token, 4 channels); |dv|^2 per token
+    // phase 0: key and value errors per (token, 8 channels); |dv|^2 per token
     {
-      constexpr int CPT = D / 4;  // tasks per token
+      constexpr int CPT = D / 8;  // tasks per token
       for (int task = tid; task < kSTT * CPT; task += kSThreads) {
-        const int tt = task / CPT, c4 = task - tt * CPT, c = 4 * c4, g = c / 32;
+        const int tt = task / CPT, c8 = task - tt * CPT, c = 8 * c8, g = c / 32;
         float n2 = 0.0f;
         if (tt < nt) {
-          const uint8_t kb = st[L.kc + tt * (D / 4) + c4];
+          const uint32_t kb = *reinterpret_cast<const uint16_t*>(st + L.kc + tt * (D / 4) + 2 * c8);
           const float ksc = reinterpret_cast<const float*>(st + L.ks)[tt * NG + g];
           const float kmn = reinterpret_cast<const float*>(st + L.km)[tt * NG + g];
-          const uint8_t* kfr = st + L.kf + tt * L.frow;
-          const uint8_t* vfr = st + L.vf + tt * L.frow;
-          float4 dk, dv;
-          float* dkp = &dk.x;
-          float* dvp = &dv.x;
+          float kf[8], vf[8], vh[8];
+          ld8(st + L.kf + tt * L.frow, c, p.kv_bf16, kf);
+          ld8(st + L.vf + tt * L.frow, c, p.kv_bf16, vf);
+          if (v2) {
+            const uint32_t vb = *reinterpret_cast<const uint16_t*>(st + L.vc + tt * (D / 4) + 2 * c8);
+            const float vsc = reinterpret_cast<const float*>(st + L.vs)[tt * NG + g];
+            const float vmn = reinterpret_cast<const float*>(st + L.vm)[tt * NG + g];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float kh = __fadd_rn(kmn, __fmul_rn(static_cast<float>((kb >> (2 * k)) & 3), ksc));
-            dkp[k] = kh - ld_smem_elem(kfr, c + k, p.kv_bf16);
-            float vh;
-            if (v2) {
-              const uint8_t vb = st[L.vc + tt * (D / 4) + c4];
-              const float vsc = reinterpret_cast<const float*>(st + L.vs)[tt * NG + g];
-              const float vmn = reinterpret_cast<const float*>(st + L.vm)[tt * NG + g];
-              vh = __fadd_rn(vmn, __fmul_rn(static_cast<float>((vb >> (2 * k)) & 3), vsc));
-            } else {
-              vh = ld_smem_elem(st + L.cv + tt * L.cvrow, c + k, cv_bf16);
-            }
-            dvp[k] = vh - ld_smem_elem(vfr, c + k, p.kv_bf16);
-            n2 = fmaf(dvp[k], dvp[k], n2);
+            for (int k = 0; k < 8; ++k)
+              vh[k] = __fadd_rn(vmn, __fmul_rn(static_cast<float>((vb >> (2 * k)) & 3), vsc));
+          } else {
+            ld8(st + L.cv + tt * L.cvrow, c, cv_bf16, vh);
           }
-          *reinterpret_cast<float4*>(dk_s + tt * DS + c) = dk;
-          *reinterpret_cast<float4*>(dv_s + tt * DS + c) = dv;
+          float dk[8], dv[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float kh = __fadd_rn(kmn, __fmul_rn(static_cast<float>((kb >> (2 * k)) & 3), ksc));
+            dk[k] = kh - kf[k];
+            dv[k] = vh[k] - vf[k];
+            n2 = fmaf(dv[k], dv[k], n2);
+          }
+          float4* dkw = reinterpret_cast<float4*>(dk_s + tt * DS + c);
+          float4* dvw = reinterpret_cast<float4*>(dv_s + tt * DS + c);
+          dkw[0] = make_float4(dk[0], dk[1], dk[2], dk[3]);
+          dkw[1] = make_float4(dk[4], dk[5], dk[6], dk[7]);
+          dvw[0] = make_float4(dv[0], dv[1], dv[2], dv[3]);
+          dvw[1] = make_float4(dv[4], dv[5], dv[6], dv[7]);
         }
         // the CPT tasks of a token are CPT consecutive lanes of one warp
 #pragma unroll
-        for (int o = CPT >= 32 ? 16 : CPT / 2; o > 0; o >>= 1) n2 += __shfl_xor_sync(kFull, n2, o);
-        if (c4 == 0) n2_s[tt] = tt < nt ? n2 : 0.0f;
+        for (int o = CPT / 2; o > 0; o >>= 1) n2 += __shfl_xor_sync(kFull, n2, o);
+        if (c8 == 0) n2_s[tt] = tt < nt ? n2 : 0.0f;
       }
     }
     __syncthreads();
-    // phase 1: logits s and score perturbations delta per (head, token)
-    for (int task = tid; task < G * kSTT; task += kSThreads) {
-      const int h = task / kSTT, tt = task - h * kSTT;
-      float sv = -INFINITY, dl = 0.0f;
+    // phase 1: partial logits s and score perturbations delta per (half of the
+    // channels, head, token): the halves of a (head, token) are in different
+    // warps (one token per lane, distinct banks) and phase 2 adds them
+    for (int task = tid; task < 2 * G * kSTT; task += kSThreads) {
+      const int half = task / (G * kSTT), pair = task - half * (G * kSTT);
+      const int h = pair / kSTT, tt = pair - h * kSTT;
+      float sf = 0.0f, de = 0.0f;
       if (tt < nt) {
         const float* qh = q_s + h * D;
         const uint8_t* kfr = st + L.kf + tt * L.frow;
         const float* dkr = dk_s + tt * DS;
-        float sf = 0.0f, de = 0.0f;
+        const int c_lo = half * (D / 2);
         if (p.kv_bf16) {
 #pragma unroll 4
-          for (int c = 0; c < D; c += 8) {
+          for (int c = c_lo; c < c_lo + D / 2; c += 8) {
             const uint4 kw = *reinterpret_cast<const uint4*>(kfr + 2 * c);
             const uint32_t w4[4] = {kw.x, kw.y, kw.z, kw.w};
             const float4 d0 = *reinterpret_cast<const float4*>(dkr + c);
@@ -522,12 +551,12 @@ attn_kl_staged_kernel(const AttnKlParams p) {
             for (int k = 0; k < 8; ++k) de = fmaf(qv[k], dvv[k], de);
           }
         } else {
-          for (int c = 0; c < D; ++c) {
+          for (int c = c_lo; c < c_lo + D / 2; ++c) {
             sf = fmaf(qh[c], reinterpret_cast<const float*>(kfr)[c], sf);
             de = fmaf(qh[c], dkr[c], de);
           }
         }
-        if (r > 0) {
+        if (r > 0 && half == 1) {
           const uint8_t* zr = (kSTT * (r / 2)) % 16 == 0
                                   ? st + L.zc + tt * (r / 2)
                                   : p.c.z_codes + (cache_row_read(p.c, b, kv, t0, nullptr) + tt) * (r / 2);
@@ -536,18 +565,17 @@ attn_kl_staged_kernel(const AttnKlParams p) {
             cz = fmaf(qt_s[h * r + ii], static_cast<float>(nibble(zr, ii)), cz);
           de = fmaf(reinterpret_cast<const float*>(st + L.zs)[tt], cz, de);
         }
-        sv = sf * p.sm_scale;
-        dl = de * p.sm_scale;
       }
-      s_s[task] = sv;
-      d_s[task] = dl;
+      s_s[task] = sf;
+      d_s[task] = de;
     }
     __syncthreads();
     // phase 2: running fp64 accumulators, one warp per head
     for (int h = warp; h < G; h += kSThreads / 32) {
       const bool valid = lane < nt;
-      const float sv = s_s[h * kSTT + lane];
-      const float dl = d_s[h * kSTT + lane];
+      const int e0 = h * kSTT + lane, e1 = e0 + G * kSTT;
+      const float sv = valid ? (s_s[e0] + s_s[e1]) * p.sm_scale : -INFINITY;
+      const float dl = valid ? (d_s[e0] + d_s[e1]) * p.sm_scale : 0.0f;
       const float m_old = m_s[h], md_old = md_s[h];
       const float m_new = fmaxf(m_old, warp_maxf(sv));
       const float md_new = fmaxf(md_old, warp_maxf(valid ? dl : -INFINITY));
@@ -619,7 +647,7 @@ size_t staged_smem(const AttnKlParams& p) {
                      p.c.vmode == HEADQ_V_2BIT);
   const int G = p.G, r = p.c.r;
   return 2 * size_t(L.bytes) + sizeof(float) * (2 * kSTT * (D + 4) + G * D + G * (r > 0 ? r : 1) +
-                                                2 * G * kSTT + kSTT + 3 * G) +
+                                                4 * G * kSTT + kSTT + 3 * G) +
          8 + sizeof(double) * G * 5;
 }
 
