@@ -64,8 +64,12 @@ __device__ __forceinline__ float code_f(uint32_t w, int k) {
 template <int D, int GM>
 __global__ void __launch_bounds__(kThreads, D >= 256 ? 2 : 4)
 decode_split_kernel(const DecodeParams p) {
-  // (G * d) / kThreads outputs per thread (at most kMaxOut: G * d <= 2048)
-  constexpr int KO = GM * D / kThreads < 1 ? 1 : (GM * D / kThreads > kMaxOut ? kMaxOut : GM * D / kThreads);
+  // (G * d) / kThreads outputs per thread: at most GM * d / kThreads for G <= GM;
+  // the 16-head batch also serves G > 16 (several passes), up to kMaxOut (G * d <= 2048)
+  constexpr int KO = GM == 16 ? kMaxOut
+                              : (GM * D / kThreads < 1 ? 1
+                                                       : (GM * D / kThreads > kMaxOut ? kMaxOut
+                                                                                      : GM * D / kThreads));
   constexpr int NG = num_groups(D);
   constexpr int GS = group_size(D);
   using CR = CodeRow<D>;

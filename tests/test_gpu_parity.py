@@ -123,6 +123,8 @@ SMALL = [  # (d, r, Hq, Hkv, T, B) beyond the five workloads: every head dim, GQ
     (8, 4, 2, 1, 16, 2), (16, 2, 4, 2, 45, 1), (32, 8, 8, 1, 130, 2),
     (64, 16, 14, 2, 129, 1), (128, 32, 8, 8, 70, 1), (256, 16, 8, 2, 300, 1),
     (128, 0, 4, 4, 90, 1),
+    (64, 16, 24, 2, 100, 1),   # G = 12: the generic kernel's 16-head batch
+    (32, 8, 40, 2, 75, 1),     # G = 20: two head passes in the generic kernel
 ]
 
 
