@@ -26,10 +26,10 @@ constexpr int kThreads = 256;
 constexpr unsigned kFull = 0xffffffffu;
 
 // The residual tile in shared memory, one fp32 per channel.  Group g of a
-// token starts at 16-byte chunk g*GC (GC = 2 mod 8: two chunks of padding per
-// 32-channel group) and a token row spans RC chunks (RC odd): the (token, group)
-// writes of phase A and the per-token reads of phase B then fall in distinct
-// banks.
+// token starts at 16-byte chunk g*GC (two chunks of padding per group: GC = 10,
+// 2 mod 8, for 32-channel groups) and a token row spans RC chunks (RC odd): the
+// (token, group) writes of phase A and the per-token reads of phase B then fall
+// in distinct banks.
 template <int D>
 struct ResTile {
   static constexpr int GS = group_size(D);
@@ -107,8 +107,10 @@ __device__ __forceinline__ void unpack_raw(const RawGroup<GS, BF16>& g, float (&
 
 // The per-token base code of one group: the codes, scale, minimum and residuals
 // of codec::quantize_group, with fewer operations per channel.  With the scale
-// a normal number of at most 2^126, every quotient (x - min)/scale lies in
-// [0, 3 + 2^-21], and q = RN((x - min) * RN(1/scale)) rounds to the same integer
+// a normal number of at most 2^126, every product q = RN((x - min) * RN(1/scale))
+// lies in [0, 3(1 + 2^-21)]: RN(x - min) <= RN(max - min) = R, scale = RN(R/3),
+// and the three roundings (scale, 1/scale, the product) are each within a
+// relative 2^-24.  Then q rounds to the same integer
 // as RN((x - min)/scale) whenever q is more than 2^-16 away from a half-integer
 // (the error argument of codec::rint_quot), so no clamp is needed there; a
 // channel whose q lies that close to a half-integer (exact ties are common with
