@@ -9,6 +9,7 @@ back; no file uses fast-math, so division, square root and denormals keep
 IEEE semantics.
 """
 
+import concurrent.futures
 import os
 import shutil
 import subprocess
@@ -48,7 +49,7 @@ def build(force=False, verbose=False):
     os.makedirs(BUILD, exist_ok=True)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")]
     headers.append(os.path.join(INCLUDE, "headq.h"))
-    objs = []
+    objs, cmds = [], []
     for src in SOURCES:
         path = os.path.join(CSRC, src)
         obj = os.path.join(BUILD, src.replace(".cu", ".o"))
@@ -57,8 +58,12 @@ def build(force=False, verbose=False):
             cmd = [nvcc(), *ARCH, *COMMON, *PER_FILE_FLAGS.get(src, [])]
             if verbose:
                 cmd += ["-Xptxas", "-v"]
-            cmd += ["-c", path, "-o", obj]
-            subprocess.check_call(cmd)
+            cmds.append(cmd + ["-c", path, "-o", obj])
+    # the translation units are independent: compile them side by side
+    workers = max(1, min(len(cmds), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as ex:
+        for f in [ex.submit(subprocess.check_call, c) for c in cmds]:
+            f.result()
     if force or _stale(LIB, objs):
         tmp = LIB + ".tmp.%d" % os.getpid()
         subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs])
