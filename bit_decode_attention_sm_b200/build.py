@@ -3,10 +3,13 @@
     python -m bit_decode_attention_sm_b200.build [--verbose]
 
 Each translation unit is compiled to an object under ``_build/`` and linked
-into ``bit_decode_attention_sm_b200/libheadq.so``.  The codec file is compiled
-with ``-fmad=false`` so no multiply and add is fused behind the intrinsics'
-back; no file uses fast-math, so division, square root and denormals keep
-IEEE semantics.
+into ``bit_decode_attention_sm_b200/libheadq.so``.  The shared codec
+(``codec.cuh``) states every step with explicit round-to-nearest intrinsics
+(``__fmul_rn``, ``__fadd_rn``, ``mul.rn.f32x2``/``add.rn.f32x2``), which the
+compiler never contracts, so it is bit-exact in every file that includes it;
+``cache_write.cu`` is also compiled with ``-fmad=false`` for its own arithmetic
+around the codec.  No file uses fast-math, so division, square root and
+denormals keep IEEE semantics.
 """
 
 import concurrent.futures

@@ -13,8 +13,9 @@
 //      the exact codec near a rounding tie), codes/scale/min stored, the
 //      residual written to shared memory, values copied or coded
 //   B  one thread per (token, RB side rows), two threads per token for r = 16:
-//      y = U_h^T e in channel order, one fused multiply-add per term, two rows per
-//      packed fp32x2 FMA, U_h read as (nearly) warp-wide broadcasts; then max|y|
+//      y = U_h^T e in channel order, each term a rounded product then a rounded
+//      sum (packed fp32x2 multiply and add, two rows per instruction), U_h read
+//      as (nearly) warp-wide broadcasts; then max|y|
 //      shared by a warp shuffle and the 4-bit side code of each thread's rows
 #include "codec.cuh"
 
@@ -264,17 +265,18 @@ __device__ __forceinline__ void load_basis(const CacheWriteParams& p, int kv, fl
   }
 }
 
-// y (RB rows, as packed pairs) += U[c][rows] * e, for one channel c.
+// y (RB rows, as packed pairs) += U[c][rows] * e, for one channel c (each
+// product rounded, then each sum).
 template <int RB>
-__device__ __forceinline__ void fma_rows(uint64_t (&y)[RB / 2], const float* u, uint64_t e2) {
+__device__ __forceinline__ void muladd_rows(uint64_t (&y)[RB / 2], const float* u, uint64_t e2) {
   if constexpr (RB == 2) {
-    codec::fma2_pk(y[0], *reinterpret_cast<const uint64_t*>(u), e2);
+    codec::muladd2_pk(y[0], *reinterpret_cast<const uint64_t*>(u), e2);
   } else {
 #pragma unroll
     for (int k = 0; k < RB / 4; ++k) {
       const ulonglong2 uu = reinterpret_cast<const ulonglong2*>(u)[k];
-      codec::fma2_pk(y[2 * k], uu.x, e2);
-      codec::fma2_pk(y[2 * k + 1], uu.y, e2);
+      codec::muladd2_pk(y[2 * k], uu.x, e2);
+      codec::muladd2_pk(y[2 * k + 1], uu.y, e2);
     }
   }
 }
@@ -308,10 +310,10 @@ __device__ __forceinline__ void side_code_tile(const CacheWriteParams& p, const 
       for (int j = 0; j < L::GS / 4; ++j) {
         const int c = g * L::GS + 4 * j;
         const float4 ev = er[g * L::GC + j];  // e_c .. e_c+3
-        fma_rows<RB>(y, ub + c * RB, codec::dup2(ev.x));
-        fma_rows<RB>(y, ub + (c + 1) * RB, codec::dup2(ev.y));
-        fma_rows<RB>(y, ub + (c + 2) * RB, codec::dup2(ev.z));
-        fma_rows<RB>(y, ub + (c + 3) * RB, codec::dup2(ev.w));
+        muladd_rows<RB>(y, ub + c * RB, codec::dup2(ev.x));
+        muladd_rows<RB>(y, ub + (c + 1) * RB, codec::dup2(ev.y));
+        muladd_rows<RB>(y, ub + (c + 2) * RB, codec::dup2(ev.z));
+        muladd_rows<RB>(y, ub + (c + 3) * RB, codec::dup2(ev.w));
       }
     }
     const bool live = tile0 + tt < p.n;

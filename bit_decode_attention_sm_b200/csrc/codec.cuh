@@ -4,7 +4,7 @@
 // Shared by the cache-write kernel and the fused append of the decode kernel.
 //
 // Every arithmetic step is one IEEE fp32 operation through an explicit *_rn
-// intrinsic (or fma.rn), so no compiler contraction can change a result.
+// intrinsic, so no compiler contraction can change a result.
 #pragma once
 
 #include "headq_internal.cuh"
@@ -25,20 +25,14 @@ __device__ __forceinline__ float rint_quot(float a, float b, float rb) {
   return rintf(__fdiv_rn(a, b));
 }
 
-// Packed fp32 FMA (sm_100): y0 = fma(u0, e, y0), y1 = fma(u1, e, y1), each
-// correctly rounded exactly like two scalar fused multiply-adds.
-__device__ __forceinline__ void fma2(float& y0, float& y1, float u0, float u1, float e) {
-  asm("{\n .reg .b64 a, b, c;\n"
-      " mov.b64 a, {%2, %3};\n mov.b64 b, {%4, %4};\n mov.b64 c, {%0, %1};\n"
-      " fma.rn.f32x2 c, a, b, c;\n mov.b64 {%0, %1}, c;\n}\n"
-      : "+f"(y0), "+f"(y1)
-      : "f"(u0), "f"(u1), "f"(e));
-}
-
-// Packed fp32 FMA on 64-bit register pairs: y.lo = fma(u.lo, e.lo, y.lo),
-// y.hi = fma(u.hi, e.hi, y.hi), each correctly rounded like a scalar FMA.
-__device__ __forceinline__ void fma2_pk(uint64_t& y, uint64_t u, uint64_t e2) {
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(y) : "l"(u), "l"(e2));
+// Packed fp32 multiply, then add, on 64-bit register pairs (sm_100):
+// y.lo = RN(y.lo + RN(u.lo * e.lo)) and the same for .hi.  The product and the
+// sum are rounded separately (no fused multiply-add), the projection's
+// arithmetic in the cache write.
+__device__ __forceinline__ void muladd2_pk(uint64_t& y, uint64_t u, uint64_t e2) {
+  asm("{\n .reg .b64 t;\n mul.rn.f32x2 t, %1, %2;\n add.rn.f32x2 %0, %0, t;\n}"
+      : "+l"(y)
+      : "l"(u), "l"(e2));
 }
 __device__ __forceinline__ uint64_t dup2(float e) {
   const uint64_t b = __float_as_uint(e);

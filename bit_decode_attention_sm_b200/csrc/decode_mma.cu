@@ -259,7 +259,7 @@ __device__ __forceinline__ void encode_new_token(const DecodeParams& p, int b, i
   if (R > 0 && orow >= 0) {
     float y = 0.0f;
     if (lane < R)
-      for (int c = 0; c < D; ++c) y = __fmaf_rn(u_s[c * R + lane], enew_s[c], y);
+      for (int c = 0; c < D; ++c) y = __fadd_rn(y, __fmul_rn(u_s[c * R + lane], enew_s[c]));
     float a = lane < R ? fabsf(y) : 0.0f;
 #pragma unroll
     for (int o2 = 16; o2 > 0; o2 >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o2));

@@ -29,8 +29,9 @@
  *  - Q_q, the "low-bit side quantizer", is per-token 4-bit symmetric absmax:
  *    s = max|y| / 7, w = clamp(rint(y/s), -7, 7), all 0 when s == 0; w is stored
  *    as a 4-bit two's-complement nibble (even index in the low nibble), s as fp32.
- *  - The projection U_h^T e accumulates over channels c = 0..d-1 in order, one
- *    fused multiply-add (single rounding) per term.
+ *  - The projection U_h^T e accumulates over channels c = 0..d-1 in order; each
+ *    term U[c,i]*e_c is rounded to fp32 and then added with a second rounding
+ *    (a plain multiply, then an add: no fused multiply-add).
  *  - Packing: channel c of the 2-bit code lives in byte c/4 at bit 2*(c%4).
  *  - An empty sequence (length 0) reads as output 0 and lse = -inf; all
  *    diagnostics are 0 for it.
@@ -222,8 +223,10 @@ static void side_project(const float *e, const float *U, int d, int r, float *y)
 {
     for (int i = 0; i < r; ++i) y[i] = 0.0f;
     for (int c = 0; c < d; ++c)
-        for (int i = 0; i < r; ++i)
-            y[i] = fmaf(U[(size_t)c * r + i], e[c], y[i]);
+        for (int i = 0; i < r; ++i) {
+            const float term = U[(size_t)c * r + i] * e[c]; /* rounded product */
+            y[i] = y[i] + term;                              /* rounded sum */
+        }
 }
 
 static void side_quantize(const float *y, int r, uint8_t *zc, float *zs)

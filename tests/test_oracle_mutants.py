@@ -25,8 +25,10 @@ SRC_DIR = os.path.dirname(real_oracle.__file__)
 MUTANTS = [
     ("correction-sign", "s[j] = sm_scale * (base + sigma * corr);",
      "s[j] = sm_scale * (base - sigma * corr);"),
-    ("projection-U-transposed", "y[i] = fmaf(U[(size_t)c * r + i], e[c], y[i]);",
-     "y[i] = fmaf(U[(size_t)i * d + c], e[c], y[i]);"),
+    ("projection-U-transposed", "const float term = U[(size_t)c * r + i] * e[c];",
+     "const float term = U[(size_t)i * d + c] * e[c];"),
+    ("projection-fused", "y[i] = y[i] + term;",
+     "y[i] = fmaf(U[(size_t)c * r + i], e[c], y[i]);"),
     ("read-U-transposed",
      "acc += (double)U[(size_t)c * r + i] * zhat[(size_t)j * r + i];",
      "acc += (double)U[(size_t)i * d + c] * zhat[(size_t)j * r + i];"),
@@ -69,6 +71,11 @@ MUTANTS_PY = [
     ("a2-ties-to-higher-position", "order = sorted(range(Tb), key=lambda j: (-scores[b, kv, j], j))",
      "order = sorted(range(Tb), key=lambda j: (-scores[b, kv, j], -j))"),
     ("a2-kept-unsorted", "kept = sorted(order[:min(K, Tb)])", "kept = order[:min(K, Tb)]"),
+    ("calibrate-centre-dropped", "            X = X - X.mean(axis=0, keepdims=True)",
+     "            X = X"),
+    ("calibrate-centre-per-head",
+     "            X = X - X.mean(axis=0, keepdims=True)",
+     "            X = (X.reshape(N, G, d) - X.reshape(N, G, d).mean(axis=0, keepdims=True)).reshape(N * G, d)"),
     ("channel-block-of-32", "KBLOCK = 64  # tokens per block of the per-channel base code",
      "KBLOCK = 32  # tokens per block of the per-channel base code"),
 ]
@@ -78,7 +85,7 @@ PINS = [
     ("test_base_code_two_groups_hand_example", {}),
     ("test_side_code_hand_example", {}),
     ("test_base_code_is_nearest_level", {"d": 64}),
-    ("test_projection_exact_rational_sequential_fma", {}),
+    ("test_projection_exact_rational_sequential", {}),
     ("test_side_code_is_nearest_level", {"r": 16}),
     ("test_decode_brute_force_d8_T16", {}),
     ("test_sigma_zero_is_plain_base_code_attention", {}),
@@ -95,6 +102,8 @@ PINS = [
     ("test_a2_scores_uniform_attention_closed_form", {}),
     ("test_a2_selection_minimises_the_surrogate_brute_force", {}),
     ("test_a2_mixed_values_limits", {}),
+    ("test_calibration_centred_exact_rational", {}),
+    ("test_calibration_centred_translation_and_library", {"i": 2}),
 ]
 
 

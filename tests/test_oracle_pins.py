@@ -253,8 +253,9 @@ def test_null_space_intervention_hurts_only_the_non_equivariant_code():
         assert abs(fv["channel", "mean"] / fv["channel", "plain"] - 1) < 0.05
 
 
-def test_projection_exact_rational_sequential_fma():
-    """y_i = fl(... fl(fl(U_0i e_0) + U_1i e_1) ...) in channel order (d=8, r=4)."""
+def test_projection_exact_rational_sequential():
+    """y_i = fl(y_i + fl(U_ci e_c)) for c = 0..d-1 in order (d=8, r=4): every
+    product rounded to fp32, then every sum rounded (a multiply, then an add)."""
     rng = _rng(3)
     d, r, T = 8, 4, 16
     k = synth.round_bf16(rng.standard_normal((1, 1, T, d)).astype(np.float32) * 3)
@@ -270,8 +271,8 @@ def test_projection_exact_rational_sequential_fma():
         for i in range(r):
             y = np.float32(0.0)
             for j in range(d):
-                y = _round_f32(Fraction(float(U[0, j, i])) * Fraction(float(e[j]))
-                               + Fraction(float(y)))
+                term = _round_f32(Fraction(float(U[0, j, i])) * Fraction(float(e[j])))
+                y = _round_f32(Fraction(float(y)) + Fraction(float(term)))
             assert planes["y"][0, 0, t, i].view(np.uint32) == np.float32(y).view(np.uint32)
 
 
@@ -754,3 +755,66 @@ def test_calibration_basis(i):
         k = min(w.r, w.r_s)
         sv = np.linalg.svd(Qa.T @ Uk, compute_uv=False)
         assert sv[:k].min() > 0.99
+
+
+def _exact_centred_covariance(X):
+    """Covariance of the rows of an integer matrix about their mean, divided by
+    the row count, in exact rational arithmetic (the plain PCA matrix)."""
+    M, d = X.shape
+    mean = [Fraction(int(sum(int(X[m, c]) for m in range(M))), M) for c in range(d)]
+    C = np.zeros((d, d))
+    for a in range(d):
+        for b in range(d):
+            s = sum((int(X[m, a]) - mean[a]) * (int(X[m, b]) - mean[b]) for m in range(M))
+            C[a, b] = float(s / M)
+    return C
+
+
+def test_calibration_centred_exact_rational():
+    """center=True: the basis is the top eigenspace of the covariance about the
+    pooled mean of a KV head's G query heads (exact rationals on a small integer
+    case with head means far from 0 and from each other)."""
+    rng = _rng(41)
+    N, Hkv, G, d, r = 12, 2, 3, 8, 4
+    q = rng.integers(-4, 5, size=(N, Hkv * G, d)).astype(np.float32)
+    q += np.arange(Hkv * G, dtype=np.float32)[None, :, None] * 3 + 5  # shifted heads
+    U, eig = oracle.calibrate(q, Hkv, r, center=True)
+    for kv in range(Hkv):
+        X = q[:, kv * G:(kv + 1) * G].reshape(-1, d).astype(np.int64)
+        C = _exact_centred_covariance(X)
+        w = np.sort(np.linalg.eigvalsh(C))[::-1][:r]
+        np.testing.assert_allclose(eig[kv], w, rtol=1e-6, atol=1e-6 * w[0])
+        Uk = U[kv].astype(np.float64)
+        np.testing.assert_allclose(Uk.T @ Uk, np.eye(r), atol=1e-6)
+        np.testing.assert_allclose(C @ Uk, Uk * eig[kv].astype(np.float64), atol=1e-5 * w[0])
+        idx = np.argmax(np.abs(Uk), axis=0)
+        assert (Uk[idx, np.arange(r)] > 0).all()
+
+
+@pytest.mark.parametrize("i", [0, 2])
+def test_calibration_centred_translation_and_library(i):
+    """center=True equals numpy's biased covariance of the pooled queries, is
+    unchanged by a shared translation of every calibration query, and equals
+    the uncentred second moment minus the outer product of the mean."""
+    w = configs.workload(i)
+    L = synth.make_layer(w, T=16, B=1)
+    shift = (3.0 * _rng(42).standard_normal(w.d)).astype(np.float32)
+    U, eig = oracle.calibrate(L.q_cal, w.Hkv, w.r, center=True)
+    U2, eig2 = oracle.calibrate(L.q_cal + shift, w.Hkv, w.r, center=True)
+    G = w.G
+    for kv in range(w.Hkv):
+        X = L.q_cal[:, kv * G:(kv + 1) * G].reshape(-1, w.d).astype(np.float64)
+        C = np.cov(X, rowvar=False, bias=True)
+        m = X.mean(axis=0)
+        np.testing.assert_allclose(C, X.T @ X / X.shape[0] - np.outer(m, m),
+                                   atol=1e-9 * np.abs(C).max())
+        top = np.sort(np.linalg.eigvalsh(C))[::-1][:w.r]
+        np.testing.assert_allclose(eig[kv], top, rtol=1e-5)
+        Uk = U[kv].astype(np.float64)
+        np.testing.assert_allclose(C @ Uk, Uk * eig[kv].astype(np.float64),
+                                   atol=1e-5 * eig[kv].max())
+        # the translated queries give the same subspace and eigenvalues
+        np.testing.assert_allclose(eig2[kv], eig[kv], rtol=1e-4)
+        P = Uk @ Uk.T
+        P2 = U2[kv].astype(np.float64) @ U2[kv].astype(np.float64).T
+        assert np.linalg.norm(P - P2) < 1e-3
