@@ -131,6 +131,54 @@ def calibrate(q_cal, Hkv, r, center=False):
 
 
 # --------------------------------------------------------------------------
+# The same-budget counterexample (gist.science summary, section 4: a code with
+# lower key-storage error can still do worse on the attention; section 2: the
+# distortion that matters is the model-visible one, not the storage one).  The
+# side code's bit budget is fixed by r and the 4-bit levels whatever basis it
+# uses, so two bases give two codes of exactly the same size: HeadQ's
+# query-PCA basis, and the basis that is best for key storage -- the top-r
+# eigenvectors of the residuals' own second moment (1/M) E^T E, residuals
+# e = k - k^base of the base code, per KV head, with the sign rule of
+# calibrate().
+# --------------------------------------------------------------------------
+def residual_basis(k, r):
+    """[Hkv, d, r] fp32: per KV head, the top-r eigenvectors of the second moment
+    of the base-code residuals of keys k [B, Hkv, n, d] (all sequences pooled)."""
+    k = _f32(k)
+    B, Hkv, n, d = k.shape
+    codes, sc, mn = base_quantize(k)
+    e = k.astype(np.float64) - base_dequantize(codes, sc, mn).astype(np.float64)
+    U = np.zeros((Hkv, d, r), dtype=np.float32)
+    for kv in range(Hkv):
+        X = e[:, kv].reshape(B * n, d)
+        w, V = np.linalg.eigh((X.T @ X) / X.shape[0])
+        order = np.argsort(-w, kind="stable")[:r]
+        Vr = V[:, order]
+        for i in range(r):
+            j = int(np.argmax(np.abs(Vr[:, i])))
+            if Vr[j, i] < 0:
+                Vr[:, i] = -Vr[:, i]
+        U[kv] = Vr.astype(np.float32)
+    return U
+
+
+def key_mse(k, planes, U, kmode="token"):
+    """Key-storage error of a cache: the mean over tokens of the squared norm of
+    k - (k^base + U_h z^), the key the corrected logit q^T k^base + q^T U_h z^
+    reads.  fp64."""
+    k = np.asarray(k, np.float64)
+    if kmode == "token":
+        kb = base_dequantize(planes["kc"], planes["ks"], planes["km"])
+    else:
+        kb = base_dequantize_channel(planes["kc"], planes["ks"], planes["km"])
+    kh = kb.astype(np.float64)
+    if U.shape[-1] > 0:
+        z = side_dequantize(planes["zc"], planes["zs"]).astype(np.float64)
+        kh = kh + np.einsum("hdr,bhtr->bhtd", np.asarray(U, np.float64), z)
+    return float(np.mean(np.sum((k - kh) ** 2, axis=-1)))
+
+
+# --------------------------------------------------------------------------
 # Step 2: cache write.
 # --------------------------------------------------------------------------
 def base_quantize(x):

@@ -76,6 +76,10 @@ MUTANTS_PY = [
     ("calibrate-centre-per-head",
      "            X = X - X.mean(axis=0, keepdims=True)",
      "            X = (X.reshape(N, G, d) - X.reshape(N, G, d).mean(axis=0, keepdims=True)).reshape(N * G, d)"),
+    ("residual-basis-smallest", "        order = np.argsort(-w, kind=\"stable\")[:r]\n        Vr = V[:, order]\n        for i in range(r):\n            j = int(np.argmax(np.abs(Vr[:, i])))\n            if Vr[j, i] < 0:\n                Vr[:, i] = -Vr[:, i]\n        U[kv] = Vr.astype(np.float32)\n    return U\n",
+     "        order = np.argsort(w, kind=\"stable\")[:r]\n        Vr = V[:, order]\n        for i in range(r):\n            j = int(np.argmax(np.abs(Vr[:, i])))\n            if Vr[j, i] < 0:\n                Vr[:, i] = -Vr[:, i]\n        U[kv] = Vr.astype(np.float32)\n    return U\n"),
+    ("key-mse-without-side-term", "        kh = kh + np.einsum(\"hdr,bhtr->bhtd\", np.asarray(U, np.float64), z)",
+     "        kh = kh + 0.0 * np.einsum(\"hdr,bhtr->bhtd\", np.asarray(U, np.float64), z)"),
     ("channel-block-of-32", "KBLOCK = 64  # tokens per block of the per-channel base code",
      "KBLOCK = 32  # tokens per block of the per-channel base code"),
 ]
@@ -104,6 +108,8 @@ PINS = [
     ("test_a2_mixed_values_limits", {}),
     ("test_calibration_centred_exact_rational", {}),
     ("test_calibration_centred_translation_and_library", {"i": 2}),
+    ("test_residual_basis_is_the_residual_eigenbasis", {}),
+    ("test_key_mse_pythagoras_and_lossless_limit", {}),
 ]
 
 

@@ -818,3 +818,77 @@ def test_calibration_centred_translation_and_library(i):
         P = Uk @ Uk.T
         P2 = U2[kv].astype(np.float64) @ U2[kv].astype(np.float64).T
         assert np.linalg.norm(P - P2) < 1e-3
+
+
+# ---------------------------------------------------------------------------
+# The same-budget counterexample (summary, section 4): lower key-storage error,
+# higher attention KL.  residual_basis and key_mse are pinned first.
+# ---------------------------------------------------------------------------
+
+def test_residual_basis_is_the_residual_eigenbasis():
+    """residual_basis: orthonormal, the eigen-equation of the residuals' second
+    moment (residuals rebuilt here from the base code's definition, exact fp32
+    steps), the r largest eigenvalues, the sign rule."""
+    w = configs.workload(2)
+    L = synth.make_layer(w, T=128, B=2)
+    U = oracle.residual_basis(L.keys, w.r)
+    codes, sc, mn = oracle.base_quantize(L.keys)
+    c = _codes2(codes, w.d)
+    g = np.arange(w.d) // 32
+    khat = mn[..., g] + (c.astype(np.float32) * sc[..., g]).astype(np.float32)
+    e = (L.keys - khat).astype(np.float64)
+    for kv in range(w.Hkv):
+        X = e[:, kv].reshape(-1, w.d)
+        C = X.T @ X / X.shape[0]
+        Uk = U[kv].astype(np.float64)
+        np.testing.assert_allclose(Uk.T @ Uk, np.eye(w.r), atol=1e-6)
+        lam = np.diag(Uk.T @ C @ Uk)
+        np.testing.assert_allclose(C @ Uk, Uk * lam, atol=1e-5 * lam.max())
+        P = np.eye(w.d) - Uk @ Uk.T
+        assert np.linalg.eigvalsh(P @ C @ P).max() <= lam.min() * (1 + 1e-5)
+        assert (np.diff(lam) <= 1e-9 * lam.max()).all()
+        idx = np.argmax(np.abs(Uk), axis=0)
+        assert (Uk[idx, np.arange(w.r)] > 0).all()
+
+
+def test_key_mse_pythagoras_and_lossless_limit():
+    """key_mse: with orthonormal U the key error k - k^base - U z^ splits into
+    (I - U U^T) e and U (y - z^), so its squared norm is |e|^2 - |y|^2 + |y - z^|^2
+    (y = U^T e, the unquantised projection); and keys on the code grid give 0."""
+    rng = _rng(51)
+    w = configs.workload(1)
+    L = synth.make_layer(w, T=64, B=1)
+    U = synth.random_orthonormal(rng, w.d, w.r)[None].repeat(w.Hkv, 0)
+    pl = oracle.cache_write(L.keys, U)
+    codes, sc, mn = pl["kc"], pl["ks"], pl["km"]
+    c = _codes2(codes, w.d)
+    g = np.arange(w.d) // 32
+    khat = mn[..., g] + (c.astype(np.float32) * sc[..., g]).astype(np.float32)
+    e = (L.keys - khat).astype(np.float64)
+    y = pl["y"].astype(np.float64)
+    zh = _nibbles(pl["zc"], w.r) * pl["zs"][..., None].astype(np.float64)
+    want = np.mean(np.sum(e * e, -1) - np.sum(y * y, -1) + np.sum((y - zh) ** 2, -1))
+    assert abs(oracle.key_mse(L.keys, pl, U) - want) <= 1e-9 * max(1.0, want)
+    # on the grid: every group spans levels 0..3 exactly
+    kg = np.tile(np.array([0.0, 0.5, 1.0, 1.5], np.float32), (1, w.Hkv, 8, w.d // 4))
+    assert oracle.key_mse(kg, oracle.cache_write(kg, U), U) == 0.0
+
+
+@pytest.mark.parametrize("i", [0, 1, 2, 3, 4])
+def test_same_budget_counterexample(i):
+    """Summary, section 4: at the same bit budget, the side code fitted to the key
+    residuals (best for key storage) has the lower key-storage error but a far
+    higher attention KL than HeadQ's query-PCA side code."""
+    w = configs.workload(i)
+    L = synth.make_layer(w, T=256, B=min(w.B, 2))
+    Uq, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    Ue = oracle.residual_basis(L.keys, w.r)
+    res = {}
+    for tag, U in (("query", Uq), ("residual", Ue)):
+        pl = oracle.cache_write(L.keys, U)
+        kl, _, _, _ = oracle.attn_kl(L.queries, pl, U, L.keys, L.values, v=L.values)
+        res[tag] = (oracle.key_mse(L.keys, pl, U), float(np.mean(kl)),
+                    sum(pl[k].nbytes for k in ("kc", "ks", "km", "zc", "zs")))
+    assert res["residual"][2] == res["query"][2]          # the same bits
+    assert res["residual"][0] < 0.8 * res["query"][0]     # lower storage error
+    assert res["residual"][1] > 5.0 * res["query"][1]     # higher attention KL
