@@ -41,6 +41,8 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
@@ -61,6 +63,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["headq", "reference"], default="headq")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-rows", action="store_true", help="skip calibrate/write/kl rows")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the rows of the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
 
@@ -257,6 +261,72 @@ def oracle_decode_rate(w, L, U, budget_s=12.0, max_T=None):
                       "first %d of %d tokens of every sequence and KV head, all %d query "
                       "heads, %d call(s), %.1f s" % (T_s, T_full, L.queries.shape[1], reps,
                                                       total)}
+
+
+def _oracle_sample_timed(prepare, run, T_full, budget_s, T0=256):
+    """Grow a token-prefix sample T_s until one run() takes about a third of
+    budget_s, then repeat it until about two thirds of the budget is spent;
+    prepare(T_s) sets up a sample size outside the timing.  Returns (T_s,
+    calls, seconds)."""
+
+    def once():
+        t0 = time.perf_counter()
+        run()
+        return time.perf_counter() - t0
+
+    T_s = min(T0, T_full)
+    prepare(T_s)
+    dt = once()
+    while T_s < T_full and dt < budget_s / 3:
+        T_s = min(T_full, int(T_s * max(2.0, (budget_s / 3) / max(dt, 1e-3))))
+        prepare(T_s)
+        dt = once()
+    reps, total = 1, dt
+    while total < budget_s * 0.66:
+        total += once()
+        reps += 1
+    return T_s, reps, total
+
+
+def oracle_op_rates(w, L, U, budget_s=4.0):
+    """The oracle's cache write and KL diagnostic on the host cores, each on a
+    bounded token-prefix sample of every (sequence, KV head): cached tokens/s
+    (B * T_s per call, the decode metric's unit)."""
+    import oracle
+    cores = oracle.set_threads(host_cores())
+    T_full = L.keys.shape[2]
+    B = L.keys.shape[0]
+    st = {}
+
+    def prep_write(Ts):
+        st["k"] = np.ascontiguousarray(L.keys[:, :, :Ts])
+        st["v"] = np.ascontiguousarray(L.values[:, :, :Ts])
+
+    def write():
+        oracle.cache_write(st["k"], U, v=st["v"], vmode=w.vmode)
+
+    T_s, reps, total = _oracle_sample_timed(prep_write, write, T_full, budget_s)
+    out = {"cache_write": {
+        "value": B * T_s * reps / total, "unit": UNIT, "cores": cores, "kind": "oracle",
+        "sample": "oracle cache write (exact fp32 codec: base code, residual, projection, "
+                  "side code%s) of the first %d of %d tokens of every sequence and KV head, "
+                  "%d call(s), %.1f s" % (", 2-bit values" if w.vmode == "2bit" else "",
+                                          T_s, T_full, reps, total)}}
+
+    def prep_kl(Ts):
+        prep_write(Ts)
+        st["planes"] = oracle.cache_write(st["k"], U, v=st["v"], vmode=w.vmode)
+
+    def kl():
+        oracle.attn_kl(L.queries, st["planes"], U, st["k"], st["v"], v=st["v"], vmode=w.vmode)
+
+    T_s, reps, total = _oracle_sample_timed(prep_kl, kl, T_full, budget_s)
+    out["attn_kl"] = {
+        "value": B * T_s * reps / total, "unit": UNIT, "cores": cores, "kind": "oracle",
+        "sample": "oracle KL / Fisher / A^2 diagnostic (fp64) of the first %d of %d tokens of "
+                  "every sequence and KV head, all %d query heads, %d call(s), %.1f s"
+                  % (T_s, T_full, L.queries.shape[1], reps, total)}
+    return out
 
 
 def run_reference(args):
@@ -496,7 +566,11 @@ def run_headq(args):
     # rows beside the step: calibration, the full prefill write, the KL diagnostic
     rows = None
     if not args.no_rows and rank == 0:
-        rows = measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, caches[0], dt, stream, L)
+        with_cpu = world == 1 and not args.no_cpu_baseline
+        rows = measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, caches[0], dt, stream, L,
+                            with_cpu=with_cpu)
+        if not args.no_workloads:
+            rows["workloads"] = measure_workloads(torch, hq, stream, w.name, with_cpu)
 
     if world > 1:
         barrier(dev)
@@ -703,27 +777,32 @@ def channel_keys_row(torch, hq, w, q, U, k_all, v_all, dt, timed, gtimed, hbm_ro
     return row
 
 
-def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream, L):
-    """The other rows of the path, timed with CUDA events, each against its roofline:
-    the prefill cache write and the KL diagnostic against HBM bandwidth (bytes they
-    must move), calibration against the fp64 ALU peak (its Gram matrix FLOPs)."""
-    rows = {}
-    peak, peak_kind = measured_hbm_peak()
+class Timing:
+    """CUDA-event timing on one stream, and rows against the HBM roofline."""
 
-    def timed(fn, reps):
+    def __init__(self, torch, stream):
+        self.torch, self.stream = torch, stream
+        self.peak, self.peak_kind = measured_hbm_peak()
+        self.l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+        self._flush = None
+
+    def timed(self, fn, reps):
+        """Mean time of reps back-to-back calls (after one untimed call)."""
+        torch = self.torch
         fn()
         torch.cuda.synchronize()
         a, b = _events(torch)
-        a.record(stream)
+        a.record(self.stream)
         for _ in range(reps):
             fn()
-        b.record(stream)
+        b.record(self.stream)
         torch.cuda.synchronize()
         return a.elapsed_time(b) / reps
 
-    def gtimed(fn, reps=20, replays=10):
+    def gtimed(self, fn, reps=20, replays=10):
         """Per-call time of fn from a CUDA graph of `reps` back-to-back calls
         (no host launch cost between them); plain calls if capture fails."""
+        torch = self.torch
         try:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
@@ -732,23 +811,52 @@ def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream, L):
             g.replay()
             torch.cuda.synchronize()
             a, b = _events(torch)
-            a.record(stream)
+            a.record(self.stream)
             for _ in range(replays):
                 g.replay()
-            b.record(stream)
+            b.record(self.stream)
             torch.cuda.synchronize()
             del g
             return a.elapsed_time(b) / (replays * reps)
         except Exception:
-            return timed(fn, reps)
+            return self.timed(fn, reps)
 
-    def hbm_row(ms, nbytes, **extra):
+    def flushed(self, fn, reps=20):
+        """Mean time of single calls, each after the L2 is flushed (a buffer of
+        twice the L2 size written between the calls, outside the timing)."""
+        torch = self.torch
+        if self._flush is None:
+            self._flush = torch.empty(2 * self.l2, dtype=torch.uint8, device="cuda")
+        fn()
+        total = 0.0
+        for _ in range(reps):
+            self._flush.zero_()
+            a, b = _events(torch)
+            a.record(self.stream)
+            fn()
+            b.record(self.stream)
+            torch.cuda.synchronize()
+            total += a.elapsed_time(b)
+        return total / reps
+
+    def hbm_row(self, ms, nbytes, **extra):
         gbs = nbytes / (ms * 1e-3) / 1e9
         return dict(ms=ms, algorithmic_bytes=nbytes,
-                    roofline={"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
-                              "frac": gbs / peak, "peak_kind": peak_kind + " copy bandwidth"},
+                    roofline={"bound": "hbm", "achieved": gbs, "peak": self.peak,
+                              "unit": "GB/s", "frac": gbs / self.peak,
+                              "peak_kind": self.peak_kind + " copy bandwidth"},
                     **extra)
 
+
+def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream, L,
+                 with_cpu=False):
+    """The other rows of the path, timed with CUDA events, each against its roofline:
+    the prefill cache write and the KL diagnostic against HBM bandwidth (bytes they
+    must move), calibration against the fp64 ALU peak (its Gram matrix FLOPs); with
+    with_cpu, the oracle's cache write and diagnostic on the host cores beside them."""
+    rows = {}
+    tm = Timing(torch, stream)
+    timed, gtimed, hbm_row = tm.timed, tm.gtimed, tm.hbm_row
     B, Hkv, T, d = w.B, w.Hkv, w.T, w.d
     tok = B * Hkv * T
     kv_in = tok * d * 2 * k_all.element_size()          # the bf16 K and V read
@@ -759,6 +867,10 @@ def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream, L):
     ws = hq.attn_kl_workspace(cache, w.Hq, T)
     ms = timed(lambda: hq.headq_attn_kl(cache, q, U, k_all, v_all, ws=ws), 3)
     rows["attn_kl"] = hbm_row(ms, kv_in + planes, note="reads the packed cache and full K,V")
+    if with_cpu:
+        cpu = oracle_op_rates(w, L, U.cpu().numpy())
+        rows["cache_write_prefill"]["cpu_baseline"] = cpu["cache_write"]
+        rows["attn_kl"]["cpu_baseline"] = cpu["attn_kl"]
     rows["decode_paged"] = paged_decode_row(torch, hq, w, q, U, cache, gtimed, hbm_row)
     rows["context_parallel_rank"] = cp_rank_row(torch, hq, w, q, U, cache, gtimed, hbm_row)
     rows["channel_keys"] = channel_keys_row(torch, hq, w, q, U, k_all, v_all, dt, timed, gtimed,
@@ -777,6 +889,103 @@ def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream, L):
                                        "peak_kind": "fp64 from unit counts and max clock",
                                        "work": "Gram matrix, 2*Hkv*N*G*d^2 flops"})
     return rows
+
+
+def workload_rows(torch, hq, w, stream, with_cpu):
+    """Every row of the path on one more workload: the serving step and the
+    decode call (HBM roofline: the packed cache), the prefill cache write and
+    the KL diagnostic (HBM roofline: K and V read, every plane written or read),
+    the A^2 value policy on 2-bit-value workloads, and with with_cpu the
+    oracle's decode, cache write and diagnostic on the host cores.  A cache
+    larger than L2 is timed as two alternating copies from a CUDA graph;
+    smaller work is timed call by call with the L2 flushed before each call."""
+    tm = Timing(torch, stream)
+    L = synth.make_layer(w)
+    dt = torch.bfloat16 if w.kv_dtype == "bf16" else torch.float32
+    B, Hq, Hkv, d, T = w.B, w.Hq, w.Hkv, w.d, w.T
+    q_cal = torch.from_numpy(L.q_cal).cuda().to(dt)
+    U, _ = hq.headq_calibrate(q_cal, Hkv, w.r)
+    k_all = torch.from_numpy(L.keys).cuda().to(dt)
+    v_all = torch.from_numpy(L.values).cuda().to(dt)
+    q = torch.from_numpy(L.queries).cuda().to(dt)
+    k_new = k_all[:, :, T - 1].contiguous()
+    v_new = v_all[:, :, T - 1].contiguous()
+    c0 = hq.HeadQCache(B, Hkv, T, d, w.r, vmode=w.vmode, v_dtype=dt)
+    hq.headq_cache_write(c0, k_all, v_all, U)
+    tok = B * Hkv * T
+    planes = tok * c0.nbytes_per_token()
+    kv_in = tok * d * 2 * k_all.element_size()
+    big = planes > tm.l2
+    caches = [c0]
+    if big:
+        c1 = hq.HeadQCache(B, Hkv, T, d, w.r, vmode=w.vmode, v_dtype=dt)
+        hq.headq_cache_write(c1, k_all, v_all, U)
+        caches.append(c1)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device="cuda")
+    lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    ws = hq.decode_workspace(c0, Hq, T)
+    splits, chunk, n_dec, n_step = hq.decode_plan(c0, Hq, T)
+    ctr = [0]
+
+    def alternating(call):
+        def fn():
+            call(caches[ctr[0] % len(caches)])
+            ctr[0] += 1
+        return fn
+
+    dec = alternating(lambda c: hq.headq_decode_attn(c, q, U, T=T, out=out, lse=lse, ws=ws))
+    stp = alternating(lambda c: hq.headq_decode_append(c, k_new, v_new, q, U, T=T, out=out,
+                                                        lse=lse, ws=ws))
+    if big:
+        dec_ms, step_ms = tm.gtimed(dec), tm.gtimed(stp)
+        l2 = "two cache copies (each larger than L2) alternate, CUDA graph of 20 calls"
+    else:
+        dec_ms, step_ms = tm.flushed(dec), tm.flushed(stp)
+        l2 = "cache smaller than L2: L2 flushed before each timed call"
+    hq.headq_workspace_status(ws)
+    row = tm.hbm_row(dec_ms, planes, value=B * T / (step_ms * 1e-3), unit=UNIT,
+                     step_ms=step_ms, bytes_per_token_kv_head=c0.nbytes_per_token(),
+                     plan="%d splits of %d tokens, %d kernel(s) per decode call"
+                          % (splits, chunk, n_dec), l2=l2,
+                     note="ms / roofline: headq_decode_attn; value: cached tokens/s of the "
+                          "serving step (headq_decode_append)")
+    ops = {}
+    wr = lambda: hq.headq_cache_write(c0, k_all, v_all, U)
+    ms_w = tm.timed(wr, 5) if kv_in + planes > 2 * tm.l2 else tm.flushed(wr)
+    ops["cache_write_prefill"] = tm.hbm_row(ms_w, kv_in + planes, tokens_per_sequence=T,
+                                            note="prefill of every sequence: reads K,V and "
+                                                 "writes every plane")
+    kws = hq.attn_kl_workspace(c0, Hq, T)
+    kl = lambda: hq.headq_attn_kl(c0, q, U, k_all, v_all, ws=kws)
+    ms_k = tm.timed(kl, 3) if kv_in + planes > 2 * tm.l2 else tm.flushed(kl, 5)
+    ops["attn_kl"] = tm.hbm_row(ms_k, kv_in + planes,
+                                note="reads the packed cache and full K,V")
+    if w.vmode == "2bit":
+        ops["a2_policy"] = a2_policy_row(torch, hq, w, q, U, c0, k_all, v_all, dt, L, tm.timed,
+                                         tm.gtimed, tm.hbm_row)
+    if with_cpu:
+        U_np = U.cpu().numpy()
+        row["cpu_baseline"] = oracle_decode_rate(w, L, U_np, budget_s=4.0)
+        cpu = oracle_op_rates(w, L, U_np)
+        ops["cache_write_prefill"]["cpu_baseline"] = cpu["cache_write"]
+        ops["attn_kl"]["cpu_baseline"] = cpu["attn_kl"]
+    row.update(ops)
+    del caches, c0
+    return row
+
+
+def measure_workloads(torch, hq, stream, skip, with_cpu):
+    """workload_rows for every workload but `skip` (the headline's own)."""
+    res = {}
+    for w in configs.WORKLOADS:
+        if w.name == skip:
+            continue
+        try:
+            res[w.name] = workload_rows(torch, hq, w, stream, with_cpu)
+        except Exception as e:  # reported in the line, never silently dropped
+            res[w.name] = {"error": "%s: %s" % (type(e).__name__, e)}
+        torch.cuda.empty_cache()
+    return res
 
 
 def main(argv=None):

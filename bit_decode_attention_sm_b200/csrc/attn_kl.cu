@@ -654,6 +654,12 @@ size_t staged_smem(const AttnKlParams& p) {
 template <int D>
 cudaError_t launch_d(const AttnKlParams& p, cudaStream_t s) {
   const int G = p.G, r = p.c.r;
+  if (p.hm) {
+    const cudaError_t e = launch_attn_kl_hm(p, s);
+    if (e != cudaSuccess) return e;
+    attn_kl_combine_kernel<D><<<p.c.B * p.Hq, D < 32 ? 32 : (D > 128 ? 128 : D), 0, s>>>(p);
+    return cudaGetLastError();
+  }
   const size_t smem = sizeof(double) * G * 6 +
                       sizeof(float) * (static_cast<size_t>(G) * D + G * r + 2 * G * kTile +
                                        kTile + 3 * G);

@@ -25,14 +25,48 @@ __device__ __forceinline__ float rint_quot(float a, float b, float rb) {
   return rintf(__fdiv_rn(a, b));
 }
 
-// Packed fp32 multiply, then add, on 64-bit register pairs (sm_100):
-// y.lo = RN(y.lo + RN(u.lo * e.lo)) and the same for .hi.  The product and the
-// sum are rounded separately (no fused multiply-add), the projection's
-// arithmetic in the cache write.
-__device__ __forceinline__ void muladd2_pk(uint64_t& y, uint64_t u, uint64_t e2) {
-  asm("{\n .reg .b64 t;\n mul.rn.f32x2 t, %1, %2;\n add.rn.f32x2 %0, %0, t;\n}"
-      : "+l"(y)
-      : "l"(u), "l"(e2));
+// Packed fp32 pairs (sm_100).  A packed multiply followed by a packed add is
+// contracted into a fused multiply-add by the compiler even with explicit .rn
+// (measured: the results are those of fma.rn.f32x2), so a sum that must be
+// rounded on its own after a product is formed as fma.rn.f32x2(a, one, b) with
+// `one` a runtime 1.0 (from the kernel parameters, unknown to the compiler):
+// a * 1.0 is exact, so the lane is RN(a + b), and the product feeding it cannot
+// be fused into it.
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// y = RN(y + RN(u * e)) in each lane: the projection's multiply, then add
+__device__ __forceinline__ void muladd2_pk(uint64_t& y, uint64_t u, uint64_t e2, uint64_t one2) {
+  uint64_t t;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(u), "l"(e2));
+  y = fma2(t, one2, y);
+}
+// Packed fp32 pair helpers (sm_100), each lane one IEEE round-to-nearest op
+// (mind the contraction of mul2 followed by add2 / sub2: see fma2 above).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  return static_cast<uint64_t>(__float_as_uint(lo)) |
+         (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+__device__ __forceinline__ float pk_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float pk_hi(uint64_t v) {
+  return __uint_as_float(static_cast<uint32_t>(v >> 32));
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 __device__ __forceinline__ uint64_t dup2(float e) {
   const uint64_t b = __float_as_uint(e);

@@ -40,10 +40,12 @@
 #include <mutex>
 
 #include "codec.cuh"
+#include "decode_common.cuh"
 #include "headq_internal.cuh"
 
 namespace headq {
 namespace {
+using namespace dc;
 
 constexpr int kCW = 4;                   // consumer warps
 constexpr int kTile = 16 * kCW;          // tokens per stage
@@ -52,11 +54,11 @@ constexpr int kThreads = (kCW + 1) * 32; // + one producer warp
 // q fragments take the shared memory of the fourth) so that two CTAs fit per SM
 template <int NT>
 constexpr int kStagesFor = NT == 1 ? 4 : 3;
-constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at B200 clocks
-constexpr unsigned kFull = 0xffffffffu;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescale = 8.0f;         // log2 units the stale max may lag
+constexpr float kRescale = 8.0f;         // log2 units the stale max may lag (p <= 2^8)
+// 2-bit values: p * scale enters the fp16 operand relative to a power of two
+// 2^E per (warp, head slot, group) that is raised once a product reaches
+// 2^kRaiseLog2 of it (fp16 holds up to 2^16).
+constexpr int kRaiseLog2 = 12;
 
 // Shared-memory stage of kTile tokens.  Dense bf16 values (V2 = false): the
 // swizzled value boxes come first.  2-bit values (V2 = true): their code, scale
@@ -93,184 +95,13 @@ constexpr size_t smem_bytes() {
   // stages | per-warp value code tiles | q [GM][D] | group sums [GM][NG] |
   // sigma U^T q [GM][R] | U [D][R] | appended token's residual [D] and
   // projection [R] | barriers
-  // ... | the query as bulk-copied (raw bf16 or fp32) [GM][D] | barriers
+  // ... | max |q| per (head, group) [GM][NG] | the query as bulk-copied (raw bf16
+  // or fp32) [GM][D] | barriers
   return 1024 + size_t(kStagesFor<NT>) * L::kStage + size_t(kCW) * L::kCodeTile + bq_bytes +
          sizeof(float) * ((4 * NT) * (D + L::NG + (R > 0 ? R : 1)) + D * (R > 0 ? R : 1) + D +
-                          (R > 0 ? R : 1) + (4 * NT) * D) +
+                          (R > 0 ? R : 1) + (4 * NT) * L::NG + (4 * NT) * D) +
          32 * kStagesFor<NT> + 64;  // barriers (2 kStages + 2), stage tile starts,
                                     // two 16-byte alignments
-}
-
-// ---------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Wait for the phase of the given parity to complete; false after ~2 s.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long start = clock64();
-  for (;;) {
-    for (int k = 0; k < 32; ++k)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - start > kWaitCycles) return false;
-  }
-}
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
-                                         uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
-                                       uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4],
-                                        const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
-      " {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4],
-                                         const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
-      " {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-// ---------------------------------------------------------------- unpacking
-// y holds one 16-bit word of eight 2-bit codes c0..c7 (code k at bits 2k) in both
-// halves.  Returns fp16 pairs (c0,c1) (c2,c3) (c4,c5) (c6,c7), exactly.
-__device__ __forceinline__ void unpack_codes(uint32_t y, uint32_t (&v)[4]) {
-  const uint32_t z = y >> 8;
-  // (1024 + c, 1024 + 4c') * (1, 1/4) - (1024, 256)
-  v[0] = hfma2((y & 0x000C0003u) | 0x64006400u, 0x34003C00u, 0xDC00E400u);
-  // (1024 + 16c, 1024 + 64c') * (1/16, 1/64) - (64, 16)
-  v[1] = hfma2((y & 0x00C00030u) | 0x64006400u, 0x24002C00u, 0xCC00D400u);
-  v[2] = hfma2((z & 0x000C0003u) | 0x64006400u, 0x34003C00u, 0xDC00E400u);
-  v[3] = hfma2((z & 0x00C00030u) | 0x64006400u, 0x24002C00u, 0xCC00D400u);
-}
-// y holds one 16-bit word of four offset nibbles (w + 8, nibble k at bits 4k) in
-// both halves.  Returns fp16 pairs (w0,w1) (w2,w3), exactly.
-__device__ __forceinline__ void unpack_side(uint32_t y, uint32_t& n01, uint32_t& n23) {
-  const uint32_t z = y >> 8;
-  // (1024 + n, 1024 + 16n') * (1, 1/16) - (1032, 72)
-  n01 = hfma2((y & 0x00F0000Fu) | 0x64006400u, 0x2C003C00u, 0xD480E408u);
-  n23 = hfma2((z & 0x00F0000Fu) | 0x64006400u, 0x2C003C00u, 0xD480E408u);
-}
-__device__ __forceinline__ uint32_t half_part_pair(float a, float b, bool lo) {
-  __half ha = __float2half_rn(a), hb = __float2half_rn(b);
-  if (lo) {
-    ha = __float2half_rn(a - __half2float(ha));
-    hb = __float2half_rn(b - __half2float(hb));
-  }
-  return static_cast<uint32_t>(__half_as_ushort(ha)) |
-         (static_cast<uint32_t>(__half_as_ushort(hb)) << 16);
-}
-__device__ __forceinline__ uint32_t bf16_part_pair(float a, float b, bool lo) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  const float2 f = __bfloat1622float2(h);
-  const __nv_bfloat162 l = __floats2bfloat162_rn(a - f.x, b - f.y);
-  const __nv_bfloat162 r = lo ? l : h;
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
-// The new token of sequence b, KV head kv, encoded into cache position pos
-// exactly as the cache write does (bit-exact codec): lanes 0..NG-1 take the key
-// groups, NG..2NG-1 the value groups, lanes < R the side rows.  Warp-wide; U_h
-// is in shared memory, enew_s is [D] scratch.
-template <int D, int R, bool V2>
-__device__ __forceinline__ void encode_new_token(const DecodeParams& p, int b, int kv, int pos,
-                                                 const float* u_s, float* enew_s, int lane) {
-  constexpr int NG = D / 32;
-  const size_t bk = static_cast<size_t>(b) * p.c.Hkv + kv;
-  const long long orow = cache_row(p.c, b, kv, pos);
-  if (orow < 0 && lane == 0 && p.err) atomicOr(p.err, kDevErrBadPage);
-  const size_t row = orow < 0 ? 0 : static_cast<size_t>(orow);
-  const size_t in = bk * D;
-  if (orow < 0) {
-    // a block-table entry outside the pool: the token is not written
-  } else if (lane < NG) {
-    float x[32];
-    uint32_t packed[2];
-    float sc, mn;
-    codec::load_row<32>(p.k_new, in + lane * 32, p.new_bf16, x);
-    codec::quantize_group<32, true>(x, packed, sc, mn);
-    codec::store_codes<32>(p.c.k_codes + row * (D / 4) + lane * 8, packed);
-    p.c.k_scale[row * NG + lane] = sc;
-    p.c.k_min[row * NG + lane] = mn;
-#pragma unroll
-    for (int k = 0; k < 32; ++k) enew_s[lane * 32 + k] = x[k];
-  } else if (lane < 2 * NG && p.v_new != nullptr) {
-    const int gv = lane - NG;
-    float vv[32];
-    codec::load_row<32>(p.v_new, in + gv * 32, p.new_bf16, vv);
-    if constexpr (V2) {
-      uint32_t packed[2];
-      float sc, mn;
-      codec::quantize_group<32, false>(vv, packed, sc, mn);
-      codec::store_codes<32>(p.c.v_codes + row * (D / 4) + gv * 8, packed);
-      p.c.v_scale[row * NG + gv] = sc;
-      p.c.v_min[row * NG + gv] = mn;
-    } else {
-      codec::store_values<32>(p.c.v, row * D + gv * 32, true, vv);
-    }
-  }
-  __syncwarp();
-  if (R > 0 && orow >= 0) {
-    float y = 0.0f;
-    if (lane < R)
-      for (int c = 0; c < D; ++c) y = __fadd_rn(y, __fmul_rn(u_s[c * R + lane], enew_s[c]));
-    float a = lane < R ? fabsf(y) : 0.0f;
-#pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o2));
-    const float zs = codec::side_scale(a);
-    const int w = lane < R ? codec::side_level(y, zs, __frcp_rn(zs)) : 0;
-    const int w_next = __shfl_down_sync(kFull, w, 1);
-    if (lane < R && (lane & 1) == 0)
-      p.c.z_codes[row * (R / 2) + (lane >> 1)] =
-          static_cast<uint8_t>((w & 0xF) | ((w_next & 0xF) << 4));
-    if (lane == 0) p.c.z_scale[row] = zs;
-  }
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -299,10 +130,11 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   float* u_s = qt_s + GM * RR;                                                // [D][RR]
   float* enew_s = u_s + D * RR;                                               // [D]
   float* ynew_s = enew_s + D;                                                 // [RR]
+  float* qmax_s = ynew_s + RR;                                                // [GM][NG]
   // [GM][D] floats of room, 16-byte aligned (a bulk-copy destination): the query
   // as copied (bf16 or fp32)
   float* qraw_s = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(ynew_s + RR) + 15) & ~uintptr_t(15));
+      (reinterpret_cast<uintptr_t>(qmax_s + GM * NG) + 15) & ~uintptr_t(15));
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(qraw_s + GM * D) + 15) & ~uintptr_t(15));
   // bars[s] = stage full, bars[kStages + s] = stage empty, bars[2 kStages + 1] =
@@ -431,9 +263,14 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   for (int i = tid; i < GM * NG; i += kCT) {
     const int h = i / NG, g = i - h * NG;
-    float acc = 0.0f;
-    for (int c = 0; c < 32; ++c) acc += q_s[h * D + g * 32 + c];
+    float acc = 0.0f, amax = 0.0f;
+    for (int c = 0; c < 32; ++c) {
+      const float v = q_s[h * D + g * 32 + c];
+      acc += v;
+      amax = fmaxf(amax, fabsf(v));
+    }
     qsum_s[i] = acc;
+    qmax_s[i] = amax;
   }
   if constexpr (R > 0) {
     for (int i = tid; i < GM * R; i += kCT) {
@@ -452,6 +289,17 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   // B operands of q . code: column n = g is head (g >> 1), fp16 high (g even) or
   // low (g odd) part; k-step ks = 2*grp + e, k-slots (2t, 2t+1) <-> channels
   // 32*grp + 8t + 4e + {0, 1}, (2t+8, 2t+9) <-> 32*grp + 8t + 4e + {2, 3}.
+  // Every head's query enters the fp16 operands scaled by its own power of two
+  // (head_prescale): fb for the head of this thread's B column, fo / scale2 for
+  // the head of its output column.
+  float fb[NT], fo[NT], scale2[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float finv;
+    head_prescale<NG>(qmax_s, 4 * nt + (g >> 1), fb[nt], finv);
+    head_prescale<NG>(qmax_s, 4 * nt + t, fo[nt], finv);
+    scale2[nt] = p.sm_scale * kLog2e * finv;
+  }
   uint32_t bq[kBqInSmem<NT> ? 1 : KS][NT][2];
 #pragma unroll
   for (int ks = 0; ks < KS; ++ks) {
@@ -459,8 +307,9 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const float* qh = q_s + (4 * nt + (g >> 1)) * D + ch0;
-      const uint32_t b0 = half_part_pair(qh[0], qh[1], g & 1);
-      const uint32_t b1 = half_part_pair(qh[2], qh[3], g & 1);
+      const float f = fb[nt];
+      const uint32_t b0 = half_part_pair(qh[0] * f, qh[1] * f, g & 1);
+      const uint32_t b1 = half_part_pair(qh[2] * f, qh[3] * f, g & 1);
       if constexpr (kBqInSmem<NT>) {
         bq_s[(ks * NT + nt) * kCT + tid] = make_uint2(b0, b1);
       } else {
@@ -475,11 +324,13 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     bz[nt][0] = bz[nt][1] = 0;
     if constexpr (R == 16) {
       const float* z = qt_s + (4 * nt + (g >> 1)) * R + 4 * t;
-      bz[nt][0] = half_part_pair(z[0], z[1], g & 1);
-      bz[nt][1] = half_part_pair(z[2], z[3], g & 1);
+      const float f = fb[nt];
+      bz[nt][0] = half_part_pair(z[0] * f, z[1] * f, g & 1);
+      bz[nt][1] = half_part_pair(z[2] * f, z[3] * f, g & 1);
     } else if constexpr (R == 8) {
       const float* z = qt_s + (4 * nt + (g >> 1)) * R + 2 * t;
-      bz[nt][0] = half_part_pair(z[0], z[1], g & 1);
+      const float f = fb[nt];
+      bz[nt][0] = half_part_pair(z[0] * f, z[1] * f, g & 1);
     }
   }
   // group sums of this thread's output head (4*nt + t)
@@ -487,11 +338,10 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int gg = 0; gg < NG; ++gg) qsum[nt][gg] = qsum_s[(4 * nt + t) * NG + gg];
+    for (int gg = 0; gg < NG; ++gg) qsum[nt][gg] = qsum_s[(4 * nt + t) * NG + gg] * fo[nt];
 
   const uint32_t sel = (2 * t) | ((2 * t + 1) << 4) | ((2 * t) << 8) | ((2 * t + 1) << 12);
   const uint32_t sel8 = t | (4 << 4) | (t << 8) | (4 << 12);
-  const float scale2 = p.sm_scale * kLog2e;
   // ldmatrix row owned by this lane: matrix (lane >> 3), row (lane & 7)
   const int lm_tok = jw + 8 * (lane >> 4) + (lane & 7);
   const int lm_chunk_hi = (lane >> 3) & 1;
@@ -499,6 +349,14 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   float m2[NT], l[NT];
   float o[V2 ? 1 : MT][NT][4];      // dense values: columns (head, high/low part)
   float ov[V2 ? MT : 1][4];         // 2-bit values: columns = the 8 head slots (fp16 p.V)
+  int ve[V2 ? NG : 1];              // 2-bit values: ov of group g, head slot (lane >> 2),
+                                    // is in units of 2^ve[g]
+  float vf[V2 ? NG : 1];            // 2^-ve[g]
+#pragma unroll
+  for (int gg = 0; gg < (V2 ? NG : 1); ++gg) {
+    ve[gg] = -126;
+    vf[gg] = pow2_neg(-126);
+  }
   float vmin_acc[NT][V2 ? NG : 1];  // 2-bit values: sum_j p_j min_{j,g} per group
   uint8_t* ctile = ctiles + size_t(warp) * L::kCodeTile;
 #pragma unroll
@@ -639,8 +497,8 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
         s0 = fmaf(zs0, acc[NG][nt][0] + acc[NG][nt][1], s0);
         s1 = fmaf(zs1, acc[NG][nt][2] + acc[NG][nt][3], s1);
       }
-      const float x0 = val0 ? s0 * scale2 : -INFINITY;
-      const float x1 = val1 ? s1 * scale2 : -INFINITY;
+      const float x0 = val0 ? s0 * scale2[nt] : -INFINITY;
+      const float x1 = val1 ? s1 * scale2[nt] : -INFINITY;
       float mx = fmaxf(x0, x1);
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
@@ -691,8 +549,13 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     // 2-bit values: one fp16 B operand per 32-dim group over the 8 head slots.
     // Column g is head slot g; its p for tokens 2t, 2t+1 (2t+8, 2t+9) is p0 (p1)
     // of the lanes 4*(2t) + (g & 3) and 4*(2t+1) + (g & 3) in query tile g >> 2.
-    // p * scale_{j,g} lies in [0, a few]: one fp16 part (11-bit mantissa) is
-    // well inside the output tolerance; the codes are exact in fp16.
+    // p <= 2^8 (the lazy rescale) and p * scale_{j,g} enters as p * scale * 2^-E,
+    // E the running exponent of this warp's (head slot, group): raised (with
+    // that column of the group's accumulators rescaled by the exact power of
+    // two) as soon as a product reaches 2^kRaiseLog2 * 2^E, so the fp16 operand
+    // never overflows, and products within 2^-14 of their head's 2^E keep the
+    // full 11-bit mantissa.  One fp16 part is well inside the output tolerance;
+    // the codes are exact in fp16.
     uint32_t bpf[V2 ? NG : 1][2];
     if constexpr (V2) {
       const int src_a = 8 * t + (g & 3), src_b = src_a + 4;
@@ -715,7 +578,31 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
         const float qb = pb > 0.f ? pb * vs[(ta + 1) * NG + gg] : 0.f;
         const float qc = pc > 0.f ? pc * vs[(ta + 8) * NG + gg] : 0.f;
         const float qd = pd > 0.f ? pd * vs[(ta + 9) * NG + gg] : 0.f;
-        const __half2 h0 = __floats2half2_rn(qa, qb), h1 = __floats2half2_rn(qc, qd);
+        // the largest product of this lane's head slot g in this group (its four
+        // lanes; non-negative floats order like their bit patterns)
+        float hx = fmaxf(fmaxf(qa, qb), fmaxf(qc, qd));
+        hx = fmaxf(hx, __shfl_xor_sync(kFull, hx, 1));
+        hx = fmaxf(hx, __shfl_xor_sync(kFull, hx, 2));
+        const uint32_t mx = __float_as_uint(hx);
+        const bool raise = mx >= static_cast<uint32_t>(127 + ve[gg] + kRaiseLog2) << 23;
+        if (__any_sync(kFull, raise)) {
+          float r = 1.0f;
+          if (raise) {
+            const int en = max(-126, min(126, static_cast<int>(mx >> 23) - 127));
+            r = pow2_neg(-ve[gg]) * pow2_neg(en);  // 2^(E_old - E_new)
+            ve[gg] = en;
+            vf[gg] = pow2_neg(en);
+          }
+          // the output columns are head slots 2t, 2t+1: their factors live in
+          // lanes 8t and 8t + 4
+          const float r0 = __shfl_sync(kFull, r, 8 * t), r1 = __shfl_sync(kFull, r, 8 * t + 4);
+#pragma unroll
+          for (int mt = 2 * gg; mt < 2 * gg + 2 && mt < MT; ++mt) {
+            ov[mt][0] *= r0; ov[mt][1] *= r1; ov[mt][2] *= r0; ov[mt][3] *= r1;
+          }
+        }
+        const float f = vf[gg];
+        const __half2 h0 = __floats2half2_rn(qa * f, qb * f), h1 = __floats2half2_rn(qc * f, qd * f);
         bpf[gg][0] = *reinterpret_cast<const uint32_t*>(&h0);
         bpf[gg][1] = *reinterpret_cast<const uint32_t*>(&h1);
       }
@@ -812,6 +699,14 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     }
   }
   if constexpr (V2) {  // columns = head slots 2t, 2t+1; add the minima sum of the group
+    // back from units of 2^ve of each column's head slot (held by lanes 8t, 8t + 4)
+    float ue[2][V2 ? NG : 1];
+#pragma unroll
+    for (int gg = 0; gg < NG; ++gg) {
+      const float u = pow2_neg(-ve[gg]);
+      ue[0][gg] = __shfl_sync(kFull, u, 8 * t);
+      ue[1][gg] = __shfl_sync(kFull, u, 8 * t + 4);
+    }
     __syncwarp();
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -820,8 +715,9 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
           const float vmn = vms[(warp * GM + h) * NG + (mt >> 1)];
-          mo[(warp * GM + h) * D + 16 * mt + g] = ov[mt][e] + vmn;
-          mo[(warp * GM + h) * D + 16 * mt + g + 8] = ov[mt][2 + e] + vmn;
+          const float u = ue[e][mt >> 1];
+          mo[(warp * GM + h) * D + 16 * mt + g] = fmaf(ov[mt][e], u, vmn);
+          mo[(warp * GM + h) * D + 16 * mt + g + 8] = fmaf(ov[mt][2 + e], u, vmn);
         }
       }
     }

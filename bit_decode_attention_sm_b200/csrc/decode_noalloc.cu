@@ -74,3 +74,24 @@ HEADQ_API headq_status headq_decode_attn_noalloc(const headq_cache* cache, const
   return headq_decode_attn(cache, q, q_dtype, Hq, seq_lens, T, U, sm_scale, corr_sign, out,
                            lse, scratch, kNoAllocScratchBytes, stream);
 }
+
+// The device error word of the built-in scratch (its first 4 bytes, as in a
+// caller workspace).  A no-alloc call whose kernel gave up a bounded wait or met
+// a block-table entry outside the page pool raises it, exactly as it would in a
+// caller workspace; the caller never sees the array's address, so this call
+// reads and clears the word of the current device for it.
+HEADQ_API headq_status headq_decode_noalloc_status(headq_stream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return HEADQ_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return HEADQ_ERR_CUDA;
+  void* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_setup_mu);
+    ptr = g_scratch_addr[dev];
+  }
+  if (ptr == nullptr) return HEADQ_OK;  // no no-alloc call has run on this device
+  return headq_workspace_status(ptr, stream);
+}

@@ -103,8 +103,18 @@ static size_t decode_ws(const headq_cache* c, int Hq, int T) {
          round256(sizeof(float) * static_cast<size_t>(c->B) * Hq * dp.splits * (c->d + 2));
 }
 
+// the diagnostic's split plan: the tensor-core kernel's when it serves the shape
+static SplitPlan kl_plan(const headq_cache& c, int Hq, int T, bool kv_bf16, bool* hm) {
+  *hm = kl_hm_supported(c, Hq / c.Hkv, kv_bf16);
+  return *hm ? kl_hm_plan(c.B * c.Hkv, T) : plan_splits(c.B * c.Hkv, T, 256);
+}
+
+// sized for either kernel (the value dtype of the call is not known here)
 static size_t kl_ws(const headq_cache* c, int Hq, int T) {
-  const SplitPlan sp = plan_splits(c->B * c->Hkv, T, 256);
+  bool hm = false;
+  SplitPlan sp = plan_splits(c->B * c->Hkv, T, 256);
+  const SplitPlan sh = kl_plan(*c, Hq, T, true, &hm);
+  if (hm && sh.splits > sp.splits) sp = sh;
   return kWsHeaderBytes +
          round256(sizeof(double) * static_cast<size_t>(c->B) * Hq * sp.splits * (7 + c->d));
 }
@@ -324,8 +334,10 @@ HEADQ_API headq_status headq_attn_kl(const headq_cache* cache, const void* q,
   if (seq_lens && !aligned16(seq_lens)) return HEADQ_ERR_INVALID_ARG;
   if (!ws || !aligned16(ws) || ws_bytes < kl_ws(cache, Hq, T)) return HEADQ_ERR_WORKSPACE;
   if (cache->B == 0) return HEADQ_OK;
-  const SplitPlan sp = plan_splits(cache->B * cache->Hkv, T, 256);
+  bool hm = false;
+  const SplitPlan sp = kl_plan(*cache, Hq, T, kv_dtype == HEADQ_BF16, &hm);
   AttnKlParams p{};
+  p.hm = hm;
   p.c = *cache;
   p.q = q;
   p.q_bf16 = q_dtype == HEADQ_BF16;

@@ -104,6 +104,9 @@ struct CacheWriteParams {
   bool append;
   const int32_t* seq_lens;
   int T;
+  // 1.0f, set by the host: a value the compiler cannot see, so that the packed
+  // "multiply, then add" of the codec is not contracted (codec::fma2)
+  float one;
 };
 
 // Decode split partials: unnormalised outputs o [B*Hq][splits][d] (rows of d
@@ -155,6 +158,7 @@ struct AttnKlParams {
   float sm_scale;
   float corr_sign;
   int splits, chunk;
+  bool hm;         // the tensor-core kernel (attn_kl_hm.cu) with its own split plan
   double* part;    // [B, Hq, splits, 7 + d]
   unsigned* err;
   float *kl, *fvar, *a2v, *dout2;
@@ -179,6 +183,11 @@ headq_status check_read_args(const headq_cache* c, const void* q, headq_dtype qd
 
 cudaError_t launch_cache_write(const CacheWriteParams& p, cudaStream_t s);
 cudaError_t launch_attn_kl(const AttnKlParams& p, cudaStream_t s);
+// the tensor-core diagnostic kernel (attn_kl_hm.cu): its shapes, its split plan
+// and its launch (the split kernel only; the combine kernel follows it)
+struct SplitPlan;
+bool kl_hm_supported(const headq_cache& c, int G, bool kv_bf16);
+cudaError_t launch_attn_kl_hm(const AttnKlParams& p, cudaStream_t s);
 cudaError_t launch_calibrate(const CalibrateParams& p, cudaStream_t s);
 
 // split planning shared by the workspace-size query and the launch
@@ -186,6 +195,7 @@ struct SplitPlan {
   int splits, chunk;
 };
 SplitPlan plan_splits(int units, int T, int min_chunk, int ctas_per_sm = 2);
+SplitPlan kl_hm_plan(int units, int T);
 int sm_count();
 
 // The decode kernel and T-split plan chosen for these sizes on the current
@@ -202,5 +212,6 @@ constexpr int kMaxMmaSplits = 1024;  // the merging CTA keeps per-split weights 
 bool mma_decode_supported(const headq_cache& c, int G);
 int mma_decode_ctas_per_sm(const headq_cache& c, int G);
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s);
+
 
 }  // namespace headq

@@ -30,7 +30,8 @@ EXPORTS = ("headq_version", "headq_status_string", "headq_calibrate",
            "headq_calibrate_workspace_bytes", "headq_cache_write", "headq_decode_attn",
            "headq_decode_workspace_bytes", "headq_decode_plan", "headq_attn_kl",
            "headq_attn_kl_workspace_bytes", "headq_workspace_status",
-           "headq_decode_attn_noalloc", "headq_decode_append", "headq_shard_seq_lens",
+           "headq_decode_attn_noalloc", "headq_decode_noalloc_status",
+           "headq_decode_append", "headq_shard_seq_lens",
            "headq_merge_partials", "headq_a2_workspace_bytes", "headq_a2_scores",
            "headq_a2_select", "headq_a2_value_fixup")
 
@@ -86,6 +87,7 @@ def lib():
             "headq_attn_kl_workspace_bytes": ([CP, I, I], Z),
             "headq_workspace_status": ([P, P], I),
             "headq_decode_attn_noalloc": ([CP, P, I, I, P, I, P, F, I, P, P, P], I),
+            "headq_decode_noalloc_status": ([P], I),
             "headq_decode_append": ([CP, P, P, I, P, I, I, P, I, P, F, I, P, P, P, Z, P], I),
             "headq_shard_seq_lens": ([P, I, I, I, I, P, P], I),
             "headq_merge_partials": ([P, P, I, I, I, Z, P, P, P], I),

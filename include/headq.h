@@ -257,6 +257,21 @@ headq_status headq_decode_attn_noalloc(const headq_cache *cache, const void *q,
                                        float *lse, headq_stream_t stream);
 
 /*
+ * headq_decode_noalloc_status -- headq_workspace_status for the built-in scratch
+ * of headq_decode_attn_noalloc on the current device (the pages have no
+ * counterpart to this either).  A no-alloc call reports a device-side error the
+ * way headq_decode_attn does, through the error word at the start of its
+ * scratch: a bounded wait that gave up (no result written) or a block-table
+ * entry outside the page pool (result undefined).  Its caller does not hold the
+ * scratch's address, so this call waits for `stream`, reads the word, clears
+ * it and returns HEADQ_ERR_DEVICE if it was set, else HEADQ_OK (also when no
+ * no-alloc call has run on the device yet).  Because every no-alloc call on a
+ * device shares the one word, the status covers all of them since the last
+ * check.  Synchronous; allocates nothing; call it off the hot path.
+ */
+headq_status headq_decode_noalloc_status(headq_stream_t stream);
+
+/*
  * headq_attn_kl -- model-visible distortion of the cache against the
  * full-precision keys and values (summary section 2.1: score perturbation
  * delta_j = s^_j - s_j, attention KL and its local Fisher form; section 2.2:

@@ -237,6 +237,64 @@ def test_full_size_sampled_rows(i):
     torch.cuda.empty_cache()
 
 
+APPEND_FULL = [2, 3, 4]
+
+
+@pytest.mark.parametrize("i", APPEND_FULL, ids=["cfg%d-full-append" % i for i in APPEND_FULL])
+def test_full_size_decode_append(i):
+    """The benchmarked call at full size in the benchmark's launch plan:
+    headq_decode_append writes every sequence's token T-1 into a cache whose
+    position T-1 held other data, then attends over all T tokens.  The new
+    token's planes are bit-exact for every (b, kv); the outputs of every query
+    head are compared with the oracle on the long-context layer (one sequence,
+    8 KV heads, T = 131072), and on four sampled (b, kv) sequences of the
+    batched layers."""
+    import torch
+    hq = _headq()
+    w = configs.workload(i)
+    L = synth.make_layer(w)
+    B, Hkv, T, d = L.keys.shape
+    U, _ = oracle.calibrate(L.q_cal, w.Hkv, w.r)
+    stale = synth.LayerInputs(L.keys.copy(), L.values.copy(), L.queries, L.q_cal, {})
+    rng = np.random.default_rng(7)
+    stale.keys[:, :, T - 1] = synth.round_bf16(rng.standard_normal((B, Hkv, d)).astype(np.float32))
+    stale.values[:, :, T - 1] = synth.round_bf16(rng.standard_normal((B, Hkv, d)).astype(np.float32))
+    cache, Ut = gpu_cache(w, stale, U)
+    del stale
+    dt = torch_dtype(w)
+    k_new = torch.from_numpy(np.ascontiguousarray(L.keys[:, :, T - 1])).cuda().to(dt)
+    v_new = torch.from_numpy(np.ascontiguousarray(L.values[:, :, T - 1])).cuda().to(dt)
+    splits, chunk, _, _ = hq.decode_plan(cache, w.Hq, T)
+    assert splits >= 1
+    ws = hq.decode_workspace(cache, w.Hq, T)
+    out, lse = hq.headq_decode_append(cache, k_new, v_new, gpu_query(w, L), Ut, T=T, ws=ws)
+    hq.headq_workspace_status(ws)
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    # the appended token of every (b, kv), bit-exact
+    new_planes = oracle.cache_write(L.keys[:, :, T - 1:T], U, v=L.values[:, :, T - 1:T],
+                                    vmode=w.vmode)
+    got = planes_to_numpy(cache, T - 1, 1)
+    new_planes.pop("y", None)
+    assert_planes_equal(got, new_planes, w.r, w.vmode, w.kv_dtype,
+                        values=L.values[:, :, T - 1:T])
+    if B * Hkv <= 8:
+        pairs = [(b, kv) for b in range(B) for kv in range(Hkv)]
+    else:
+        r2 = np.random.default_rng(200 + i)
+        pairs = sorted({(int(r2.integers(B)), int(r2.integers(Hkv))) for _ in range(4)})
+    for b, kv in pairs:
+        sub = synth.LayerInputs(L.keys[b:b + 1, kv:kv + 1], L.values[b:b + 1, kv:kv + 1],
+                                L.queries[b:b + 1, kv * w.G:(kv + 1) * w.G], None, {})
+        w1 = w.with_(B=1, Hkv=1, Hq=w.G)
+        _, out_ref, lse_ref = oracle_side(w1, sub, U[kv:kv + 1])
+        o = out[b:b + 1, kv * w.G:(kv + 1) * w.G]
+        assert row_rel_err(o, out_ref) <= DECODE_RTOL, (b, kv)
+        np.testing.assert_allclose(lse[b:b + 1, kv * w.G:(kv + 1) * w.G], lse_ref,
+                                   rtol=1e-5, atol=1e-4)
+    del cache
+    torch.cuda.empty_cache()
+
+
 def test_one_workspace_reused_across_shapes():
     """A decode workspace sized for the largest call serves calls of different
     shapes in any order: partials of one call never disturb the next."""
