@@ -754,7 +754,7 @@ def a2_policy_row(torch, hq, w, q, U, cache, k_all, v_all, dt, L, timed, gtimed,
 
 def channel_keys_row(torch, hq, w, q, U, k_all, v_all, dt, timed, gtimed, hbm_row):
     """The alternative base code (per-channel keys over 64-token blocks) on this
-    workload: the prefill write and the decode (generic kernel), each against HBM."""
+    workload: the prefill write and the tensor-core decode, each against HBM."""
     B, Hkv, T, d = w.B, w.Hkv, w.T, w.d
     if T % 64:
         return None
@@ -769,7 +769,7 @@ def channel_keys_row(torch, hq, w, q, U, k_all, v_all, dt, timed, gtimed, hbm_ro
     tok = B * Hkv * T
     planes = tok * c.nbytes_per_token()
     row = hbm_row(ms_d, planes, write_ms=ms_w, bytes_per_token=c.nbytes_per_token(),
-                  note="ms: headq_decode_attn (generic kernel) on the per-channel code; "
+                  note="ms: headq_decode_attn (tensor-core kernel) on the per-channel code; "
                        "write_roofline: the prefill write")
     gbs = (tok * d * 2 * k_all.element_size() + planes) / (ms_w * 1e-3) / 1e9
     row["write_roofline"] = dict(row["roofline"], achieved=gbs, frac=gbs / row["roofline"]["peak"])
@@ -891,14 +891,18 @@ def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream, L,
     return rows
 
 
+COPIES_MAX = 16  # cache copies rotated to keep a small cache's reads out of L2
+
+
 def workload_rows(torch, hq, w, stream, with_cpu):
     """Every row of the path on one more workload: the serving step and the
     decode call (HBM roofline: the packed cache), the prefill cache write and
     the KL diagnostic (HBM roofline: K and V read, every plane written or read),
     the A^2 value policy on 2-bit-value workloads, and with with_cpu the
-    oracle's decode, cache write and diagnostic on the host cores.  A cache
-    larger than L2 is timed as two alternating copies from a CUDA graph;
-    smaller work is timed call by call with the L2 flushed before each call."""
+    oracle's decode, cache write and diagnostic on the host cores.  The decode
+    rotates cache copies whose total exceeds twice the L2 (at least two, at
+    most COPIES_MAX) in a CUDA graph; a cache too small for that is timed call
+    by call with the L2 flushed before each call."""
     tm = Timing(torch, stream)
     L = synth.make_layer(w)
     dt = torch.bfloat16 if w.kv_dtype == "bf16" else torch.float32
@@ -915,9 +919,10 @@ def workload_rows(torch, hq, w, stream, with_cpu):
     tok = B * Hkv * T
     planes = tok * c0.nbytes_per_token()
     kv_in = tok * d * 2 * k_all.element_size()
-    big = planes > tm.l2
+    ncopies = max(2, -(-2 * tm.l2 // planes))
+    big = ncopies <= COPIES_MAX
     caches = [c0]
-    if big:
+    for _ in range(ncopies - 1 if big else 0):
         c1 = hq.HeadQCache(B, Hkv, T, d, w.r, vmode=w.vmode, v_dtype=dt)
         hq.headq_cache_write(c1, k_all, v_all, U)
         caches.append(c1)
@@ -937,8 +942,9 @@ def workload_rows(torch, hq, w, stream, with_cpu):
     stp = alternating(lambda c: hq.headq_decode_append(c, k_new, v_new, q, U, T=T, out=out,
                                                         lse=lse, ws=ws))
     if big:
-        dec_ms, step_ms = tm.gtimed(dec), tm.gtimed(stp)
-        l2 = "two cache copies (each larger than L2) alternate, CUDA graph of 20 calls"
+        dec_ms, step_ms = tm.gtimed(dec, reps=max(20, 2 * ncopies)), tm.gtimed(stp, reps=max(20, 2 * ncopies))
+        l2 = ("%d cache copies (%.0f MB in all, more than twice the L2) rotate, CUDA graph of "
+              "%d calls" % (ncopies, ncopies * planes / 1e6, max(20, 2 * ncopies)))
     else:
         dec_ms, step_ms = tm.flushed(dec), tm.flushed(stp)
         l2 = "cache smaller than L2: L2 flushed before each timed call"

@@ -214,84 +214,6 @@ __device__ __forceinline__ void quantize_raw(const void* base, size_t off, RawGr
   }
 }
 
-// The base code of the 8 channels of one 16-byte chunk of a 32-channel group
-// whose other three chunks sit in the three neighbouring lanes (four aligned
-// lanes per group, all of them calling): the group's minimum and maximum go
-// round by two shuffles, then every channel takes exactly the operations of
-// quantize_group_fast (the short path, the exact quotient near a tie) or, for a
-// scale outside its range, those of codec::quantize_group.  Returns the eight
-// 2-bit codes (channel k at bits 2k); with RESIDUAL, x becomes the residual
-// x - (min + code * scale), the product rounded before the sum.
-template <bool RESIDUAL>
-__device__ __forceinline__ uint32_t quantize_chunk8(float (&x)[8], float& scale_out, float& min_out,
-                                                   float one) {
-  float lo = fmin3(x[0], x[1], x[2]), hi = fmax3(x[0], x[1], x[2]);
-  lo = fmin3(lo, x[3], x[4]);
-  hi = fmax3(hi, x[3], x[4]);
-  lo = fmin3(lo, x[5], x[6]);
-  hi = fmax3(hi, x[5], x[6]);
-  lo = fminf(lo, x[7]);
-  hi = fmaxf(hi, x[7]);
-  lo = fminf(lo, __shfl_xor_sync(kFull, lo, 1));
-  hi = fmaxf(hi, __shfl_xor_sync(kFull, hi, 1));
-  lo = fminf(lo, __shfl_xor_sync(kFull, lo, 2));
-  hi = fmaxf(hi, __shfl_xor_sync(kFull, hi, 2));
-  lo = __fadd_rn(lo, 0.0f);  // a -0 extreme is stored as +0
-  hi = __fadd_rn(hi, 0.0f);
-  const float scale = __fdiv_rn(__fsub_rn(hi, lo), 3.0f);
-  scale_out = scale;
-  min_out = lo;
-  if (scale == 0.0f) {  // all codes 0; the residual is x - (min + 0) = x - min
-    if constexpr (RESIDUAL) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) x[k] = __fsub_rn(x[k], lo);
-    }
-    return 0u;
-  }
-  const float rs = __frcp_rn(scale);
-  uint32_t bits = 0u;
-  if (scale >= 0x1p-126f && scale <= 0x1p126f) {
-    const uint64_t lo2 = codec::pk2(lo, lo), rs2 = codec::pk2(rs, rs), sc2 = codec::pk2(scale, scale);
-    const uint64_t one2 = codec::pk2(one, one), mone2 = codec::pk2(-one, -one);
-#pragma unroll
-    for (int k = 0; k < 8; k += 2) {
-      const uint64_t a2 = codec::sub2(codec::pk2(x[k], x[k + 1]), lo2);
-      const uint64_t q2 = codec::mul2(a2, rs2);
-      float c0 = rintf(codec::pk_lo(q2)), c1 = rintf(codec::pk_hi(q2));
-      const uint64_t d2 = codec::fma2(codec::pk2(c0, c1), mone2, q2);  // RN(q - c)
-      const bool ok0 = fabsf(codec::pk_lo(d2)) < 0.5f - 0x1p-16f;
-      const bool ok1 = fabsf(codec::pk_hi(d2)) < 0.5f - 0x1p-16f;
-      if (!(ok0 && ok1)) {  // near a half-integer (or NaN): the exact quotient
-        if (!ok0) {
-          const float t = rintf(__fdiv_rn(codec::pk_lo(a2), scale));
-          c0 = static_cast<float>(t < 0.0f ? 0 : (t > 3.0f ? 3 : static_cast<int>(t)));
-        }
-        if (!ok1) {
-          const float t = rintf(__fdiv_rn(codec::pk_hi(a2), scale));
-          c1 = static_cast<float>(t < 0.0f ? 0 : (t > 3.0f ? 3 : static_cast<int>(t)));
-        }
-      }
-      bits |= (static_cast<uint32_t>(c0) | (static_cast<uint32_t>(c1) << 2)) << (2 * k);
-      if constexpr (RESIDUAL) {
-        const uint64_t r2 = codec::sub2(codec::pk2(x[k], x[k + 1]),
-                                        codec::fma2(codec::mul2(codec::pk2(c0, c1), sc2), one2, lo2));
-        x[k] = codec::pk_lo(r2);
-        x[k + 1] = codec::pk_hi(r2);
-      }
-    }
-  } else {  // the exact codec, channel by channel
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float t = codec::rint_quot(__fsub_rn(x[k], lo), scale, rs);
-      const int code = t < 0.0f ? 0 : (t > 3.0f ? 3 : static_cast<int>(t));
-      bits |= static_cast<uint32_t>(code) << (2 * k);
-      if constexpr (RESIDUAL)
-        x[k] = __fsub_rn(x[k], __fadd_rn(lo, __fmul_rn(static_cast<float>(code), scale)));
-    }
-  }
-  return bits;
-}
-
 // Plane rows of a tile's tokens: when its first and last token share a slab, the
 // tile occupies consecutive rows from row0 (the common case: contiguous planes,
 // or a tile inside one page); otherwise each token is looked up.
@@ -553,89 +475,6 @@ cache_write_kernel(const CacheWriteParams p) {
     }
   };
   // ---- phase A: base code, residual, values ---------------------------------
-  // bf16 inputs in 32-channel groups: four lanes per (token, group), one 16-byte
-  // chunk (8 channels) each, so that consecutive lanes read consecutive chunks of
-  // the tile (coalesced) and the group's extremes go round by shuffles
-  constexpr bool kChunked = BF16 && GS == 32;
-  if constexpr (kChunked) {
-  if (v_copy || p.v == nullptr || p.c.vmode == HEADQ_V_2BIT) {
-    constexpr int CPT = D / 8;  // chunks per token row
-    static_assert(kTT * CPT % kThreads == 0, "every lane takes every round");
-    if (v_copy) v_load(0);
-    bool stored = false;
-#pragma unroll 1
-    for (int base = 0; base < kTT * CPT; base += kThreads) {
-      const int ci = base + tid;
-      const int tt = ci / CPT, c = ci - tt * CPT, g = c >> 2;
-      const bool live = tt < nt;
-      const size_t in_off = (bk * p.n + tile0 + tt) * D + 8 * c;
-      float x[8];
-      uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
-      const bool v2 = !v_copy && p.v != nullptr;  // 2-bit values
-      if (live) {
-        kw = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.k) + in_off);
-        if (v2) vw = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.v) + in_off);
-      }
-      if (v_copy && !stored) {  // the copy's first batch, while the keys load
-        v_store(0);
-        stored = true;
-      }
-      const long long row_s = live ? tile_row(p.c, tr, b, kv, t0 + tile0, tt) : -1;
-      {
-        const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          x[2 * j] = __uint_as_float(w[j] << 16);
-          x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-        }
-        float sc, mn;
-        const uint32_t bits = quantize_chunk8<true>(x, sc, mn, p.one);  // x: the residual e
-        if (row_s >= 0) {
-          const size_t row = static_cast<size_t>(row_s);
-          *reinterpret_cast<uint16_t*>(p.c.k_codes + row * (D / 4) + 2 * c) = static_cast<uint16_t>(bits);
-          if ((c & 3) == 0) {
-            p.c.k_scale[row * NG + g] = sc;
-            p.c.k_min[row * NG + g] = mn;
-          }
-        }
-        if (live) {
-          float4* er = reinterpret_cast<float4*>(e_s) + tt * L::RC + g * L::GC + 2 * (c & 3);
-          er[0] = make_float4(x[0], x[1], x[2], x[3]);
-          er[1] = make_float4(x[4], x[5], x[6], x[7]);
-        }
-      }
-      if (v2) {
-        const uint32_t w[4] = {vw.x, vw.y, vw.z, vw.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          x[2 * j] = __uint_as_float(w[j] << 16);
-          x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-        }
-        float sc, mn;
-        const uint32_t bits = quantize_chunk8<false>(x, sc, mn, p.one);
-        if (row_s >= 0) {
-          const size_t row = static_cast<size_t>(row_s);
-          *reinterpret_cast<uint16_t*>(p.c.v_codes + row * (D / 4) + 2 * c) = static_cast<uint16_t>(bits);
-          if ((c & 3) == 0) {
-            p.c.v_scale[row * NG + g] = sc;
-            p.c.v_min[row * NG + g] = mn;
-          }
-        }
-      }
-    }
-    if (v_copy) {
-      if (!stored) v_store(0);
-      for (int base = VC::kBatch * kThreads; base < v_chunks; base += VC::kBatch * kThreads) {
-        v_load(base);
-        v_store(base);
-      }
-    }
-    if (r == 0) return;  // no side code
-    __syncthreads();
-    side_code_tile<D, RB>(p, e_s, u_s, y_s, b, kv, tile0, t0, tr);
-    return;
-  }
-  }
   // one (token, group) task: the keys' code and residual from kraw
   auto key_group = [&](int tt, int g, size_t in_off, size_t row, RawGroup<GS, BF16>& kraw) {
     float x[GS];

@@ -462,9 +462,9 @@ DecodePlan decode_plan(const headq_cache& c, int Hq, int T) {
   const int G = c.Hkv > 0 ? Hq / c.Hkv : 0;
   const int units = c.B * c.Hkv;
   if (T <= 0 || units <= 0) return dp;
-  // the tensor-core kernel reads the per-token base code; the per-channel code
-  // goes to the generic kernel
-  const bool mma = c.kmode == HEADQ_K_TOKEN && mma_decode_supported(c, G);
+  // the tensor-core kernel reads either base code: per-channel keys fold each
+  // 64-token block's scale into the query fragments tile by tile
+  const bool mma = mma_decode_supported(c, G);
   const int occ = mma ? mma_decode_ctas_per_sm(c, G) : 0;
   if (occ > 0) {
     // one wave: every CTA resident, each streaming one contiguous chunk; the
@@ -474,8 +474,9 @@ DecodePlan decode_plan(const headq_cache& c, int Hq, int T) {
     s = s < 1 ? 1 : (s > max_s ? max_s : s);
     if (s > kMaxMmaSplits) s = kMaxMmaSplits;
     // a multiple of 16 tokens (so every bulk copy stays 16-byte aligned); of
-    // 64 for a paged cache, so that no 64-token tile straddles two pages
-    const int align = c.page_size > 0 ? 64 : 16;
+    // 64 for a paged cache, so that no 64-token tile straddles two pages, and
+    // for per-channel keys, so that every tile is one block
+    const int align = (c.page_size > 0 || c.kmode == HEADQ_K_CHANNEL) ? 64 : 16;
     int chunk = (T + s - 1) / s;
     chunk = (chunk + align - 1) / align * align;
     dp.chunk = chunk;

@@ -145,6 +145,14 @@ __device__ __forceinline__ void head_prescale(const float* qmax_s, int h, float&
   f = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
   finv = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
 }
+// 2^-e (f) and 2^e (finv), e the binary exponent of m >= 0 clamped to
+// [-126, 126] (0 for m == 0): m * f lies in [1, 2)
+__device__ __forceinline__ void pow2_prescale(float m, float& f, float& finv) {
+  int e = m > 0.f ? static_cast<int>((__float_as_uint(m) >> 23) & 0xffu) - 127 : 0;
+  e = max(-126, min(126, e));
+  f = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+  finv = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+}
 // 2^-E for a power-of-two exponent E in [-126, 126]
 __device__ __forceinline__ float pow2_neg(int E) {
   return __uint_as_float(static_cast<uint32_t>(127 - E) << 23);

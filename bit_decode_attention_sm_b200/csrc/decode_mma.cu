@@ -62,8 +62,10 @@ constexpr int kRaiseLog2 = 12;
 
 // Shared-memory stage of kTile tokens.  Dense bf16 values (V2 = false): the
 // swizzled value boxes come first.  2-bit values (V2 = true): their code, scale
-// and minimum planes are bulk-copied like the keys'.
-template <int D, int R, bool V2 = false>
+// and minimum planes are bulk-copied like the keys'.  Per-channel keys (KCH):
+// the tile is one 64-token block, whose scale and minimum rows (d floats each)
+// take the place of the per-token key scale and minimum planes.
+template <int D, int R, bool V2 = false, bool KCH = false>
 struct Layout {
   static constexpr int NG = D / 32;
   static constexpr int kVBoxes = V2 ? 0 : D / 64;    // 64-dim boxes per token row
@@ -79,8 +81,10 @@ struct Layout {
   static constexpr int kEnd = kVm + (V2 ? kTile * NG * 4 : 0);
   static constexpr int kStage = (kEnd + 1023) / 1024 * 1024;
   static constexpr int kRowBytes =
-      D / 4 + 8 * NG + (R > 0 ? R / 2 + 4 : 0) + (V2 ? D / 4 + 8 * NG : 0);
+      D / 4 + (KCH ? 0 : 8 * NG) + (R > 0 ? R / 2 + 4 : 0) + (V2 ? D / 4 + 8 * NG : 0);
+  static constexpr int kTileBytes = KCH ? 2 * D * 4 : 0;  // bytes per tile, besides the rows
   static constexpr int kCodeTile = V2 ? 16 * D * 2 : 0;  // per consumer warp, fp16 codes
+  static_assert(!KCH || D * 4 <= kTile * NG * 4, "a block row fits the per-token plane space");
 };
 
 // the two-N-tile variants keep each thread's q B-operand fragments in shared
@@ -88,9 +92,9 @@ struct Layout {
 template <int NT>
 constexpr bool kBqInSmem = NT == 2;
 
-template <int D, int R, int NT, bool V2>
+template <int D, int R, int NT, bool V2, bool KCH>
 constexpr size_t smem_bytes() {
-  using L = Layout<D, R, V2>;
+  using L = Layout<D, R, V2, KCH>;
   constexpr size_t bq_bytes = kBqInSmem<NT> ? size_t(kCW) * 32 * (D / 16) * NT * 8 : 0;
   // stages | per-warp value code tiles | q [GM][D] | group sums [GM][NG] |
   // sigma U^T q [GM][R] | U [D][R] | appended token's residual [D] and
@@ -105,10 +109,10 @@ constexpr size_t smem_bytes() {
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int D, int R, int NT, bool V2>
+template <int D, int R, int NT, bool V2, bool KCH>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap) {
-  using L = Layout<D, R, V2>;
+  using L = Layout<D, R, V2, KCH>;
   constexpr int NG = L::NG;
   constexpr int KS = D / 16;   // k-steps of 16 channels
   constexpr int MT = D / 16;   // 16-dim row blocks of the output
@@ -217,13 +221,19 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
           mbar_arrive(full);  // no more tiles: the consumers stop at this stage
         } else {
           const int n16 = (min(kTile, tile_end - t0) + 15) & ~15;
-          mbar_expect_tx(full, L::kVBoxes * L::kVBox + n16 * L::kRowBytes);
+          mbar_expect_tx(full, L::kVBoxes * L::kVBox + n16 * L::kRowBytes + L::kTileBytes);
           uint8_t* st = stages + size_t(s) * L::kStage;
           const CacheSlab sl = cache_slab_read(p.c, b, kv, t0, p.err);
           const size_t row0 = static_cast<size_t>(sl.slab) * slab_rows(p.c) + sl.off;
           bulk_g2s(smem_addr(st + L::kKc), p.c.k_codes + row0 * (D / 4), n16 * (D / 4), full);
-          bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + row0 * NG, n16 * NG * 4, full);
-          bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + row0 * NG, n16 * NG * 4, full);
+          if constexpr (KCH) {  // the tile is one block: its scale and minimum rows
+            const size_t brow = row0 / kTile;
+            bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + brow * D, D * 4, full);
+            bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + brow * D, D * 4, full);
+          } else {
+            bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + row0 * NG, n16 * NG * 4, full);
+            bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + row0 * NG, n16 * NG * 4, full);
+          }
           if constexpr (R > 0) {
             bulk_g2s(smem_addr(st + L::kZc), p.c.z_codes + row0 * (R / 2), n16 * (R / 2), full);
             bulk_g2s(smem_addr(st + L::kZs), p.c.z_scale + row0, n16 * 4, full);
@@ -292,17 +302,18 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   // Every head's query enters the fp16 operands scaled by its own power of two
   // (head_prescale): fb for the head of this thread's B column, fo / scale2 for
   // the head of its output column.
-  float fb[NT], fo[NT], scale2[NT];
+  float fb[NT], fo[NT], scale2[NT], foinv[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     float finv;
     head_prescale<NG>(qmax_s, 4 * nt + (g >> 1), fb[nt], finv);
     head_prescale<NG>(qmax_s, 4 * nt + t, fo[nt], finv);
     scale2[nt] = p.sm_scale * kLog2e * finv;
+    foinv[nt] = finv;
   }
   uint32_t bq[kBqInSmem<NT> ? 1 : KS][NT][2];
 #pragma unroll
-  for (int ks = 0; ks < KS; ++ks) {
+  for (int ks = 0; ks < (KCH ? 0 : KS); ++ks) {  // per-channel keys: rebuilt per tile
     const int ch0 = 32 * (ks >> 1) + 8 * t + 4 * (ks & 1);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -414,6 +425,64 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       __syncwarp();
     }
 
+    // ---- per-channel keys: the B operands of q . code are the query times the
+    // block's scale, (q * scale)_c, rebuilt for each tile (one 64-token block),
+    // prescaled by a power of two per (head, block) from their largest
+    // magnitude; the minimum enters as one term q . min per (head, block)
+    float kfinv[KCH ? NT : 1], kqmin[KCH ? NT : 1];
+    if constexpr (KCH) {
+      const float* ksc = reinterpret_cast<const float*>(st + L::kKs);  // [D] block scale
+      const float* kmn = reinterpret_cast<const float*>(st + L::kKm);  // [D] block minimum
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float* qh = q_s + (4 * nt + (g >> 1)) * D;
+        float qv[KS][4];
+        float mx = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const int ch0 = 32 * (ks >> 1) + 8 * t + 4 * (ks & 1);
+          const float4 a = *reinterpret_cast<const float4*>(qh + ch0);
+          const float4 c = *reinterpret_cast<const float4*>(ksc + ch0);
+          qv[ks][0] = a.x * c.x; qv[ks][1] = a.y * c.y; qv[ks][2] = a.z * c.z; qv[ks][3] = a.w * c.w;
+          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(qv[ks][0]), fabsf(qv[ks][1])),
+                               fmaxf(fabsf(qv[ks][2]), fabsf(qv[ks][3]))));
+        }
+        // the head of this B column: its eight lanes (lane >> 3)
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+        float fk, fkinv;
+        pow2_prescale(mx, fk, fkinv);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const uint32_t b0 = half_part_pair(qv[ks][0] * fk, qv[ks][1] * fk, g & 1);
+          const uint32_t b1 = half_part_pair(qv[ks][2] * fk, qv[ks][3] * fk, g & 1);
+          if constexpr (kBqInSmem<NT>) {
+            bq_s[(ks * NT + nt) * kCT + tid] = make_uint2(b0, b1);
+          } else {
+            bq[ks][nt][0] = b0;
+            bq[ks][nt][1] = b1;
+          }
+        }
+        // the output head 4 nt + t: its factor from lane 8t; q . min over the
+        // eight lanes of the same t, 16 channels each
+        kfinv[nt] = __shfl_sync(kFull, fkinv, 8 * t);
+        const int cb = (D / 8) * g;  // this lane's d/8 channels
+        const float* qo = q_s + (4 * nt + t) * D + cb;
+        float qm = 0.f;
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+          const float4 a = *reinterpret_cast<const float4*>(qo + 4 * c4);
+          const float4 m = *reinterpret_cast<const float4*>(kmn + cb + 4 * c4);
+          qm = fmaf(a.x, m.x, fmaf(a.y, m.y, fmaf(a.z, m.z, fmaf(a.w, m.w, qm))));
+        }
+        qm += __shfl_xor_sync(kFull, qm, 4);
+        qm += __shfl_xor_sync(kFull, qm, 8);
+        qm += __shfl_xor_sync(kFull, qm, 16);
+        kqmin[nt] = qm;
+      }
+    }
+
     // ---- q . code and the side-code correction on tensor cores
     float acc[NG + (R > 0 ? 1 : 0)][NT][4];
 #pragma unroll
@@ -472,7 +541,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     }
     float ks0[NG], km0[NG], ks1[NG], km1[NG];
 #pragma unroll
-    for (int gg = 0; gg < NG; ++gg) {
+    for (int gg = 0; gg < (KCH ? 0 : NG); ++gg) {
       ks0[gg] = reinterpret_cast<const float*>(st + L::kKs)[j0 * NG + gg];
       km0[gg] = reinterpret_cast<const float*>(st + L::kKm)[j0 * NG + gg];
       ks1[gg] = reinterpret_cast<const float*>(st + L::kKs)[j1 * NG + gg];
@@ -486,19 +555,37 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       float s0 = 0.f, s1 = 0.f;
+      float x0, x1;
+      if constexpr (KCH) {  // q . k^ = q . min + sum_c (q scale)_c code_c, in true units
+        float c0 = 0.f, c1 = 0.f;
 #pragma unroll
-      for (int gg = 0; gg < NG; ++gg) {
-        s0 = fmaf(ks0[gg], acc[gg][nt][0] + acc[gg][nt][1], s0);
-        s0 = fmaf(km0[gg], qsum[nt][gg], s0);
-        s1 = fmaf(ks1[gg], acc[gg][nt][2] + acc[gg][nt][3], s1);
-        s1 = fmaf(km1[gg], qsum[nt][gg], s1);
+        for (int gg = 0; gg < NG; ++gg) {
+          c0 += acc[gg][nt][0] + acc[gg][nt][1];
+          c1 += acc[gg][nt][2] + acc[gg][nt][3];
+        }
+        s0 = fmaf(c0, kfinv[nt], kqmin[nt]);
+        s1 = fmaf(c1, kfinv[nt], kqmin[nt]);
+        if constexpr (R > 0) {  // the side term is in units of the head's prescale
+          s0 = fmaf(zs0 * foinv[nt], acc[NG][nt][0] + acc[NG][nt][1], s0);
+          s1 = fmaf(zs1 * foinv[nt], acc[NG][nt][2] + acc[NG][nt][3], s1);
+        }
+        x0 = val0 ? s0 * (p.sm_scale * kLog2e) : -INFINITY;
+        x1 = val1 ? s1 * (p.sm_scale * kLog2e) : -INFINITY;
+      } else {
+#pragma unroll
+        for (int gg = 0; gg < NG; ++gg) {
+          s0 = fmaf(ks0[gg], acc[gg][nt][0] + acc[gg][nt][1], s0);
+          s0 = fmaf(km0[gg], qsum[nt][gg], s0);
+          s1 = fmaf(ks1[gg], acc[gg][nt][2] + acc[gg][nt][3], s1);
+          s1 = fmaf(km1[gg], qsum[nt][gg], s1);
+        }
+        if constexpr (R > 0) {
+          s0 = fmaf(zs0, acc[NG][nt][0] + acc[NG][nt][1], s0);
+          s1 = fmaf(zs1, acc[NG][nt][2] + acc[NG][nt][3], s1);
+        }
+        x0 = val0 ? s0 * scale2[nt] : -INFINITY;
+        x1 = val1 ? s1 * scale2[nt] : -INFINITY;
       }
-      if constexpr (R > 0) {
-        s0 = fmaf(zs0, acc[NG][nt][0] + acc[NG][nt][1], s0);
-        s1 = fmaf(zs1, acc[NG][nt][2] + acc[NG][nt][3], s1);
-      }
-      const float x0 = val0 ? s0 * scale2[nt] : -INFINITY;
-      const float x1 = val1 ? s1 * scale2[nt] : -INFINITY;
       float mx = fmaxf(x0, x1);
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
@@ -874,7 +961,7 @@ EncodeTiled encode_fn() {
 
 constexpr int kMaxDev = 64;
 
-template <int D, int R, int NT, bool V2>
+template <int D, int R, int NT, bool V2, bool KCH>
 struct Variant {
   static int occupancy[kMaxDev];  // CTAs per SM, 0 = not yet known
   static std::mutex mu;
@@ -889,8 +976,8 @@ struct Variant {
     }
     std::lock_guard<std::mutex> lock(mu);
     if (occupancy[dev] == 0) {
-      auto k = decode_mma_kernel<D, R, NT, V2>;
-      const int smem = static_cast<int>(smem_bytes<D, R, NT, V2>());
+      auto k = decode_mma_kernel<D, R, NT, V2, KCH>;
+      const int smem = static_cast<int>(smem_bytes<D, R, NT, V2, KCH>());
       int n = 0;
       if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
               cudaSuccess ||
@@ -909,7 +996,7 @@ struct Variant {
     dim3 grid(p.splits, p.c.Hkv, p.c.B);
     if (V2) {  // no value tensor map: the 2-bit value planes are bulk-copied
       memset(&vmap, 0, sizeof(vmap));
-      decode_mma_kernel<D, R, NT, V2><<<grid, kThreads, smem_bytes<D, R, NT, V2>(), s>>>(p, vmap);
+      decode_mma_kernel<D, R, NT, V2, KCH><<<grid, kThreads, smem_bytes<D, R, NT, V2, KCH>(), s>>>(p, vmap);
       return cudaGetLastError();
     }
     EncodeTiled enc = encode_fn();
@@ -927,32 +1014,38 @@ struct Variant {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
-    decode_mma_kernel<D, R, NT, V2><<<grid, kThreads, smem_bytes<D, R, NT, V2>(), s>>>(p, vmap);
+    decode_mma_kernel<D, R, NT, V2, KCH><<<grid, kThreads, smem_bytes<D, R, NT, V2, KCH>(), s>>>(p, vmap);
     return cudaGetLastError();
   }
 };
-template <int D, int R, int NT, bool V2>
-int Variant<D, R, NT, V2>::occupancy[kMaxDev];
-template <int D, int R, int NT, bool V2>
-std::mutex Variant<D, R, NT, V2>::mu;
+template <int D, int R, int NT, bool V2, bool KCH>
+int Variant<D, R, NT, V2, KCH>::occupancy[kMaxDev];
+template <int D, int R, int NT, bool V2, bool KCH>
+std::mutex Variant<D, R, NT, V2, KCH>::mu;
 
 template <typename F>
-auto dispatch(int d, int r, int G, bool v2, F&& f) -> decltype(f(Variant<128, 16, 1, false>{})) {
+auto dispatch(int d, int r, int G, bool v2, bool kch, F&& f)
+    -> decltype(f(Variant<128, 16, 1, false, false>{})) {
   const int nt = G <= 4 ? 1 : 2;
-#define HEADQ_MMA_CASE(DD, RR, NN, VV) \
-  if (d == DD && r == RR && nt == NN && v2 == VV) return f(Variant<DD, RR, NN, VV>{});
-  HEADQ_MMA_CASE(128, 16, 1, false) HEADQ_MMA_CASE(128, 16, 2, false)
-  HEADQ_MMA_CASE(128, 8, 1, false) HEADQ_MMA_CASE(128, 8, 2, false)
-  HEADQ_MMA_CASE(128, 0, 1, false) HEADQ_MMA_CASE(128, 0, 2, false)
-  HEADQ_MMA_CASE(64, 16, 1, false) HEADQ_MMA_CASE(64, 16, 2, false)
-  HEADQ_MMA_CASE(64, 8, 1, false) HEADQ_MMA_CASE(64, 8, 2, false)
-  HEADQ_MMA_CASE(64, 0, 1, false) HEADQ_MMA_CASE(64, 0, 2, false)
-  HEADQ_MMA_CASE(128, 16, 1, true) HEADQ_MMA_CASE(128, 16, 2, true)
-  HEADQ_MMA_CASE(128, 8, 1, true) HEADQ_MMA_CASE(128, 8, 2, true)
-  HEADQ_MMA_CASE(64, 16, 1, true) HEADQ_MMA_CASE(64, 16, 2, true)
-  HEADQ_MMA_CASE(64, 8, 1, true) HEADQ_MMA_CASE(64, 8, 2, true)
+#define HEADQ_MMA_CASE(DD, RR, NN, VV, KK) \
+  if (d == DD && r == RR && nt == NN && v2 == VV && kch == KK) \
+    return f(Variant<DD, RR, NN, VV, KK>{});
+#define HEADQ_MMA_CASES(KK)                                                         \
+  HEADQ_MMA_CASE(128, 16, 1, false, KK) HEADQ_MMA_CASE(128, 16, 2, false, KK)       \
+  HEADQ_MMA_CASE(128, 8, 1, false, KK) HEADQ_MMA_CASE(128, 8, 2, false, KK)         \
+  HEADQ_MMA_CASE(128, 0, 1, false, KK) HEADQ_MMA_CASE(128, 0, 2, false, KK)         \
+  HEADQ_MMA_CASE(64, 16, 1, false, KK) HEADQ_MMA_CASE(64, 16, 2, false, KK)         \
+  HEADQ_MMA_CASE(64, 8, 1, false, KK) HEADQ_MMA_CASE(64, 8, 2, false, KK)           \
+  HEADQ_MMA_CASE(64, 0, 1, false, KK) HEADQ_MMA_CASE(64, 0, 2, false, KK)           \
+  HEADQ_MMA_CASE(128, 16, 1, true, KK) HEADQ_MMA_CASE(128, 16, 2, true, KK)         \
+  HEADQ_MMA_CASE(128, 8, 1, true, KK) HEADQ_MMA_CASE(128, 8, 2, true, KK)           \
+  HEADQ_MMA_CASE(64, 16, 1, true, KK) HEADQ_MMA_CASE(64, 16, 2, true, KK)           \
+  HEADQ_MMA_CASE(64, 8, 1, true, KK) HEADQ_MMA_CASE(64, 8, 2, true, KK)
+  HEADQ_MMA_CASES(false)
+  HEADQ_MMA_CASES(true)
+#undef HEADQ_MMA_CASES
 #undef HEADQ_MMA_CASE
-  return decltype(f(Variant<128, 16, 1, false>{}))();
+  return decltype(f(Variant<128, 16, 1, false, false>{}))();
 }
 
 bool is_v2(const headq_cache& c) { return c.vmode == HEADQ_V_2BIT; }
@@ -961,6 +1054,7 @@ bool is_v2(const headq_cache& c) { return c.vmode == HEADQ_V_2BIT; }
 
 bool mma_decode_supported(const headq_cache& c, int G) {
   if (c.d != 64 && c.d != 128) return false;
+  if (c.kmode != HEADQ_K_TOKEN && c.kmode != HEADQ_K_CHANNEL) return false;
   if (G < 1 || G > 8) return false;
   if (c.vmode == HEADQ_V_2BIT) return c.r == 8 || c.r == 16;
   return c.vmode == HEADQ_V_DENSE && c.v_dtype == HEADQ_BF16 &&
@@ -968,12 +1062,13 @@ bool mma_decode_supported(const headq_cache& c, int G) {
 }
 
 int mma_decode_ctas_per_sm(const headq_cache& c, int G) {
-  return dispatch(c.d, c.r, G, is_v2(c), [](auto v) { return decltype(v)::ctas_per_sm(); });
+  return dispatch(c.d, c.r, G, is_v2(c), c.kmode == HEADQ_K_CHANNEL,
+                  [](auto v) { return decltype(v)::ctas_per_sm(); });
 }
 
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s) {
   // 0 means no variant matched; otherwise the launch status + 1
-  const int e = dispatch(p.c.d, p.c.r, p.G, is_v2(p.c), [&](auto v) {
+  const int e = dispatch(p.c.d, p.c.r, p.G, is_v2(p.c), p.c.kmode == HEADQ_K_CHANNEL, [&](auto v) {
     return static_cast<int>(decltype(v)::launch(p, s)) + 1;
   });
   return e == 0 ? cudaErrorInvalidValue : static_cast<cudaError_t>(e - 1);

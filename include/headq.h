@@ -108,8 +108,7 @@ typedef enum {
  *   k_scale, k_min  fp32 [B, Hkv, T_cap/64, d]  (paged: [num_pages, Hkv, page_size/64, d])
  * T_cap is a multiple of 64, writes start on a block boundary (t0 % 64 == 0)
  * and a block's codes are fixed once written (headq_decode_append and the A^2
- * fixup are unsupported in this mode); the tensor-core decode serves only the
- * per-token code, the channel code is decoded by the generic kernel.
+ * fixup are unsupported in this mode).
  */
 typedef struct {
     int B, Hkv, T_cap, d, r;

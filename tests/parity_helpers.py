@@ -29,20 +29,20 @@ def layer(i, **kw):
     return w, synth.make_layer(w, **kw)
 
 
-def oracle_side(w, L, U, seq_lens=None, sigma=1.0):
-    planes = oracle.cache_write(L.keys, U, v=L.values, vmode=w.vmode)
+def oracle_side(w, L, U, seq_lens=None, sigma=1.0, kmode="token"):
+    planes = oracle.cache_write(L.keys, U, v=L.values, vmode=w.vmode, kmode=kmode)
     out, lse = oracle.decode(L.queries, planes, U, v=L.values, vmode=w.vmode,
-                             sigma=sigma, seq_lens=seq_lens)
+                             sigma=sigma, seq_lens=seq_lens, kmode=kmode)
     return planes, out, lse
 
 
-def gpu_cache(w, L, U, T_cap=None, t0=0):
+def gpu_cache(w, L, U, T_cap=None, t0=0, kmode="token"):
     import torch
     from bit_decode_attention_sm_b200 import headq
     dt = torch_dtype(w)
     B, Hkv, T, d = L.keys.shape
-    T_cap = roundup(t0 + T, 16) if T_cap is None else T_cap
-    cache = headq.HeadQCache(B, Hkv, T_cap, d, w.r, vmode=w.vmode, v_dtype=dt)
+    T_cap = roundup(t0 + T, 64 if kmode == "channel" else 16) if T_cap is None else T_cap
+    cache = headq.HeadQCache(B, Hkv, T_cap, d, w.r, vmode=w.vmode, v_dtype=dt, kmode=kmode)
     k = torch.from_numpy(L.keys).to("cuda").to(dt)
     v = torch.from_numpy(L.values).to("cuda").to(dt)
     Ut = torch.from_numpy(np.ascontiguousarray(U)).to("cuda")
