@@ -539,8 +539,7 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
   float* lse_s = qt_s + G * r;        // [G]
   float* p_s = lse_s + G;             // [kFixTok][G]
   int* idx_s = reinterpret_cast<int*>(p_s + kFixTok * G);            // [kFixTok]
-  size_t* row_s = reinterpret_cast<size_t*>(                          // [kFixTok], 8-aligned
-      (reinterpret_cast<uintptr_t>(idx_s + kFixTok) + 7) & ~uintptr_t(7));
+  size_t* row_s = reinterpret_cast<size_t*>(smem_align(idx_s + kFixTok, 8));  // [kFixTok]
   uint32_t* kc_s = reinterpret_cast<uint32_t*>(row_s + kFixTok);     // [kFixTok][D/16]
   float* ks_s = reinterpret_cast<float*>(kc_s + kFixTok * FS::kKcWords);  // [kFixTok][NG]
   float* km_s = ks_s + kFixTok * NG;                                  // [kFixTok][NG]

@@ -398,8 +398,7 @@ attn_kl_staged_kernel(const AttnKlParams p) {
   float* m_s = n2_s + kSTT;                                    // [G]
   float* md_s = m_s + G;                                       // [G]
   float* a_s = md_s + G;                                       // [G]
-  double* acc_s = reinterpret_cast<double*>(
-      (reinterpret_cast<uintptr_t>(a_s + G) + 7) & ~uintptr_t(7));  // [G][5]
+  double* acc_s = reinterpret_cast<double*>(smem_align(a_s + G, 8));  // [G][5]
 
   const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

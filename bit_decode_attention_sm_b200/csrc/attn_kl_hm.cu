@@ -135,8 +135,7 @@ attn_kl_hm_kernel(const AttnKlParams p, const __grid_constant__ CUtensorMap kmap
   constexpr int MT = D / 16;  // 16-dim row blocks of the readout-error product
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align(smem_raw, 1024);
   uint8_t* stages = smem;
   float* q_s = reinterpret_cast<float*>(stages + size_t(kStages) * L::kStage);  // [kGM][D]
   float* qsum_s = q_s + kGM * D;     // [kGM][NG]

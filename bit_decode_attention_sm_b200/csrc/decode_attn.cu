@@ -18,6 +18,8 @@
 // their log-sum-exp.  When there is a single split the CTA writes the result.
 #include <math.h>
 
+#include <algorithm>
+
 #include "headq_internal.cuh"
 
 namespace headq {
@@ -467,18 +469,36 @@ DecodePlan decode_plan(const headq_cache& c, int Hq, int T) {
   const bool mma = mma_decode_supported(c, G);
   const int occ = mma ? mma_decode_ctas_per_sm(c, G) : 0;
   if (occ > 0) {
-    // one wave: every CTA resident, each streaming one contiguous chunk; the
-    // last CTA of each (b, kv) merges the splits, so one kernel per call
-    int s = (occ * sm_count()) / units;
+    // Each CTA streams one contiguous chunk; the last CTA of each (b, kv)
+    // merges the splits, so one kernel per call.  The split count minimises
+    // waves x (tiles per CTA + kTileOverhead): with `slots` resident CTAs a
+    // call takes ceil(units * splits / slots) waves of CTAs whose time is their
+    // tile count plus a fixed cost (query preparation, merge) worth about
+    // kTileOverhead tiles.  Ties go to fewer splits.
+    constexpr long long kTileOverhead = 2;
+    const long long slots = static_cast<long long>(occ) * sm_count();
     const int max_s = (T + 63) / 64;
-    s = s < 1 ? 1 : (s > max_s ? max_s : s);
-    if (s > kMaxMmaSplits) s = kMaxMmaSplits;
     // a multiple of 16 tokens (so every bulk copy stays 16-byte aligned); of
     // 64 for a paged cache, so that no 64-token tile straddles two pages, and
     // for per-channel keys, so that every tile is one block
     const int align = (c.page_size > 0 || c.kmode == HEADQ_K_CHANNEL) ? 64 : 16;
-    int chunk = (T + s - 1) / s;
-    chunk = (chunk + align - 1) / align * align;
+    const long long per_unit = (slots + units - 1) / units;
+    const int s_hi = static_cast<int>(
+        std::min<long long>({static_cast<long long>(max_s), kMaxMmaSplits, 4 * per_unit + 4}));
+    long long best = -1;
+    int chunk = T;
+    for (int s = 1; s <= s_hi; ++s) {
+      int ch = (T + s - 1) / s;
+      ch = (ch + align - 1) / align * align;
+      const int sp = (T + ch - 1) / ch;
+      if (sp != s) continue;  // the same chunk as a smaller count
+      const long long waves = (static_cast<long long>(units) * sp + slots - 1) / slots;
+      const long long cost = waves * ((ch + 63) / 64 + kTileOverhead);
+      if (best < 0 || cost < best) {
+        best = cost;
+        chunk = ch;
+      }
+    }
     dp.chunk = chunk;
     dp.splits = (T + chunk - 1) / chunk;
     dp.mma = true;

@@ -83,7 +83,15 @@ struct Layout {
   static constexpr int kRowBytes =
       D / 4 + (KCH ? 0 : 8 * NG) + (R > 0 ? R / 2 + 4 : 0) + (V2 ? D / 4 + 8 * NG : 0);
   static constexpr int kTileBytes = KCH ? 2 * D * 4 : 0;  // bytes per tile, besides the rows
-  static constexpr int kCodeTile = V2 ? 16 * D * 2 : 0;  // per consumer warp, fp16 codes
+  // 2-bit values: per consumer warp, the fp16 codes of its D/4 channels for the
+  // kTile tokens of a stage (the warp's readout slice)
+  static constexpr int kCodeTile = V2 ? kTile * (D / kCW) * 2 : 0;
+  // 2-bit values: the probabilities p [2 buffers][kCW warps][8 head slots][24]
+  // (16 tokens, rows padded for conflict-free stores and loads) and each warp's
+  // running max [2][8 head slots][kCW], passed from the logit warps to the
+  // readout warps
+  static constexpr int kPexFloats = 2 * kCW * 8 * 24;
+  static constexpr int kExBytes = V2 ? (kPexFloats + 2 * 8 * kCW) * 4 : 0;
   static_assert(!KCH || D * 4 <= kTile * NG * 4, "a block row fits the per-token plane space");
 };
 
@@ -96,21 +104,29 @@ template <int D, int R, int NT, bool V2, bool KCH>
 constexpr size_t smem_bytes() {
   using L = Layout<D, R, V2, KCH>;
   constexpr size_t bq_bytes = kBqInSmem<NT> ? size_t(kCW) * 32 * (D / 16) * NT * 8 : 0;
-  // stages | per-warp value code tiles | q [GM][D] | group sums [GM][NG] |
-  // sigma U^T q [GM][R] | U [D][R] | appended token's residual [D] and
-  // projection [R] | barriers
-  // ... | max |q| per (head, group) [GM][NG] | the query as bulk-copied (raw bf16
-  // or fp32) [GM][D] | barriers
-  return 1024 + size_t(kStagesFor<NT>) * L::kStage + size_t(kCW) * L::kCodeTile + bq_bytes +
-         sizeof(float) * ((4 * NT) * (D + L::NG + (R > 0 ? R : 1)) + D * (R > 0 ? R : 1) + D +
-                          (R > 0 ? R : 1) + (4 * NT) * L::NG + (4 * NT) * D) +
-         32 * kStagesFor<NT> + 64;  // barriers (2 kStages + 2), stage tile starts,
+  // stages | per-warp value code tiles | p exchange | q fragments | q [GM][D] |
+  // group sums [GM][NG] | sigma U^T q [GM][R] | U [D][R] | appended token's
+  // residual [D] and projection [R] | max |q| per (head, group) [GM][NG] | the
+  // query as bulk-copied (raw bf16 or fp32) [GM][D] | barriers.  2-bit values
+  // (three CTAs per SM) read U_h from global memory and land the raw query in
+  // the code tiles, which are free until the main loop.
+  return 1024 + size_t(kStagesFor<NT>) * L::kStage + size_t(kCW) * L::kCodeTile + L::kExBytes +
+         bq_bytes +
+         sizeof(float) * ((4 * NT) * (D + L::NG + (R > 0 ? R : 1)) +
+                          (V2 ? 0 : D * (R > 0 ? R : 1)) + D + (R > 0 ? R : 1) +
+                          (4 * NT) * L::NG + (V2 ? 0 : (4 * NT) * D)) +
+         32 * kStagesFor<NT> + 80;  // barriers (2 kStages + 4), stage tile starts,
                                     // two 16-byte alignments
 }
 
 // ---------------------------------------------------------------- the kernel
+// CTAs per SM the registers are budgeted for: 2-bit values keep a small
+// readout accumulator (their channel slice), so three fit
+template <bool V2>
+constexpr int kMinCtas = V2 ? 3 : 2;
+
 template <int D, int R, int NT, bool V2, bool KCH>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kMinCtas<V2>)
 decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap) {
   using L = Layout<D, R, V2, KCH>;
   constexpr int NG = L::NG;
@@ -122,28 +138,31 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   constexpr int kStages = kStagesFor<NT>;
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align(smem_raw, 1024);
   uint8_t* stages = smem;
   uint8_t* ctiles = smem + size_t(kStagesFor<NT>) * L::kStage;  // [kCW][16][D] fp16 value codes
-  uint2* bq_s = reinterpret_cast<uint2*>(ctiles + size_t(kCW) * L::kCodeTile);  // [KS][NT][128]
+  float* pex_s = reinterpret_cast<float*>(ctiles + size_t(kCW) * L::kCodeTile);  // 2-bit values
+  float* mex_s = pex_s + L::kPexFloats;
+  uint2* bq_s = reinterpret_cast<uint2*>(ctiles + size_t(kCW) * L::kCodeTile +
+                                         L::kExBytes);  // [KS][NT][128]
   float* q_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bq_s) +
                                         (kBqInSmem<NT> ? size_t(kCW) * 32 * KS * NT * 8 : 0));
   float* qsum_s = q_s + GM * D;                                               // [GM][NG]
   float* qt_s = qsum_s + GM * NG;                                             // [GM][RR]
-  float* u_s = qt_s + GM * RR;                                                // [D][RR]
-  float* enew_s = u_s + D * RR;                                               // [D]
+  // U_h [D][RR]: in shared memory, or (2-bit values) read from global memory
+  const float* u_s = V2 ? p.U + static_cast<size_t>(blockIdx.y) * D * R : qt_s + GM * RR;
+  float* enew_s = qt_s + GM * RR + (V2 ? 0 : D * RR);                         // [D]
   float* ynew_s = enew_s + D;                                                 // [RR]
   float* qmax_s = ynew_s + RR;                                                // [GM][NG]
   // [GM][D] floats of room, 16-byte aligned (a bulk-copy destination): the query
   // as copied (bf16 or fp32)
-  float* qraw_s = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(qmax_s + GM * NG) + 15) & ~uintptr_t(15));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(qraw_s + GM * D) + 15) & ~uintptr_t(15));
+  float* qraw_s = V2 ? reinterpret_cast<float*>(ctiles) : smem_align(qmax_s + GM * NG, 16);
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(smem_align(V2 ? qmax_s + GM * NG : qraw_s + GM * D, 16));
   // bars[s] = stage full, bars[kStages + s] = stage empty, bars[2 kStages + 1] =
-  // the query and U_h are in shared memory (bars[2 kStages] unused)
-  int* stile_s = reinterpret_cast<int*>(bars + 2 * kStages + 2);  // [kStages] tile start, -1: end
+  // the query and U_h are in shared memory (bars[2 kStages] unused),
+  // bars[2 kStages + 2 + b] = exchange buffer b holds every warp's p (2-bit values)
+  int* stile_s = reinterpret_cast<int*>(bars + 2 * kStages + 4);  // [kStages] tile start, -1: end
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
@@ -166,6 +185,8 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     }
     mbar_init(smem_addr(&bars[2 * kStages]), 1);
     mbar_init(smem_addr(&bars[2 * kStages + 1]), 1);
+    mbar_init(smem_addr(&bars[2 * kStages + 2]), kCW);
+    mbar_init(smem_addr(&bars[2 * kStages + 3]), kCW);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -178,12 +199,12 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       // preparation does not wait behind the cache stream
       const uint32_t qbar = smem_addr(&bars[2 * kStages + 1]);
       const uint32_t qbytes = static_cast<uint32_t>(G * D * (p.q_bf16 ? 2 : 4));
-      mbar_expect_tx(qbar, qbytes + (R > 0 ? D * R * 4 : 0));
+      mbar_expect_tx(qbar, qbytes + (R > 0 && !V2 ? D * R * 4 : 0));
       bulk_g2s(smem_addr(qraw_s),
                static_cast<const uint8_t*>(p.q) +
                    (static_cast<size_t>(b) * p.Hq + h0) * D * (p.q_bf16 ? 2 : 4),
                qbytes, qbar);
-      if constexpr (R > 0)
+      if constexpr (R > 0 && !V2)
         bulk_g2s(smem_addr(u_s), p.U + static_cast<size_t>(kv) * D * R, D * R * 4, qbar);
     }
     // The tiles of this CTA's chunk in order, one per stage, then an end marker.
@@ -359,16 +380,19 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
 
   float m2[NT], l[NT];
   float o[V2 ? 1 : MT][NT][4];      // dense values: columns (head, high/low part)
-  float ov[V2 ? MT : 1][4];         // 2-bit values: columns = the 8 head slots (fp16 p.V)
-  int ve[V2 ? NG : 1];              // 2-bit values: ov of group g, head slot (lane >> 2),
-                                    // is in units of 2^ve[g]
-  float vf[V2 ? NG : 1];            // 2^-ve[g]
-#pragma unroll
-  for (int gg = 0; gg < (V2 ? NG : 1); ++gg) {
-    ve[gg] = -126;
-    vf[gg] = pow2_neg(-126);
-  }
-  float vmin_acc[NT][V2 ? NG : 1];  // 2-bit values: sum_j p_j min_{j,g} per group
+  // 2-bit values.  Logits and softmax are per warp (its 16 tokens of each tile,
+  // as for dense values); the readout is split by channel: this warp reads out
+  // channels [cw0, cw0 + CW) of all kTile tokens of each tile (p of the other
+  // warps' tokens through shared memory), into ov with columns = the 8 head
+  // slots (C columns 2t, 2t+1).  ov is relative to Mref, the running maximum of
+  // the warps' maxima for head slot g (this thread's B column), and in units of
+  // 2^ve, the exponent of head slot g in this channel slice.
+  constexpr int CW = D / kCW, MTW = CW / 16, CPR = CW / 8;
+  const int cw0 = warp * CW, gw = cw0 / 32;
+  float ov[V2 ? MTW : 1][4];
+  int ve = -126;
+  float Mref = -INFINITY;
+  float vmin_acc[NT][V2 ? NG : 1];  // 2-bit values: sum_j p_j min_{j,g} per group (this warp's tokens)
   uint8_t* ctile = ctiles + size_t(warp) * L::kCodeTile;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -380,7 +404,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     for (int mt = 0; mt < (V2 ? 1 : MT); ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
   }
 #pragma unroll
-  for (int mt = 0; mt < (V2 ? MT : 1); ++mt) ov[mt][0] = ov[mt][1] = ov[mt][2] = ov[mt][3] = 0.f;
+  for (int mt = 0; mt < (V2 ? MTW : 1); ++mt) ov[mt][0] = ov[mt][1] = ov[mt][2] = ov[mt][3] = 0.f;
 
   bool ok = true;
   for (int i = 0;; ++i) {
@@ -397,20 +421,23 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     const bool val0 = j0 < nvalid, val1 = j1 < nvalid;
 
     if constexpr (V2) {
-      // this warp's 16 tokens of value codes -> fp16 code tile (chunk c of row t
-      // stored at c ^ (t & 7): conflict-free ldmatrix)
-      for (int task = lane; task < 16 * (D / 16); task += 32) {
-        const int tt = task / (D / 16), blk = task - tt * (D / 16);
-        const uint32_t wv = *reinterpret_cast<const uint32_t*>(st + L::kVc + (jw + tt) * (D / 4) +
-                                                               4 * blk);
-        uint32_t lo4[4], hi4[4];
-        unpack_codes(__byte_perm(wv, 0u, 0x1010u), lo4);
-        unpack_codes(__byte_perm(wv, 0u, 0x3232u), hi4);
-        const int c0 = 2 * blk, c1 = 2 * blk + 1;
-        *reinterpret_cast<uint4*>(ctile + tt * (D * 2) + ((c0 ^ (tt & 7)) << 4)) =
-            make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
-        *reinterpret_cast<uint4*>(ctile + tt * (D * 2) + ((c1 ^ (tt & 7)) << 4)) =
-            make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+      // the fp16 codes of this warp's channel slice for all kTile tokens: row r =
+      // token r (CW * 2 bytes), its 16-byte chunk c stored at c ^ sz(r),
+      // sz(r) = (r / (8 / CPR)) % CPR, so that the 16-byte stores of 8 lanes and
+      // the 8 rows read by an ldmatrix each cover all 8 bank groups
+      constexpr int WPT = CW / 16;  // 32-bit code words of the slice per token
+      for (int task = lane; task < kTile * WPT; task += 32) {
+        const int r = task / WPT, wd = task - r * WPT;
+        const uint32_t wv = *reinterpret_cast<const uint32_t*>(st + L::kVc + r * (D / 4) +
+                                                               cw0 / 4 + 4 * wd);
+        uint32_t v1[4], v2[4];
+        unpack_codes(__byte_perm(wv, 0u, 0x1010u), v1);  // channels 16 wd + 0..7 of the slice
+        unpack_codes(__byte_perm(wv, 0u, 0x3232u), v2);  // 16 wd + 8..15
+        const int sz = (r / (8 / CPR)) % CPR;
+        uint8_t* row = ctile + r * (CW * 2);
+        *reinterpret_cast<uint4*>(row + (((2 * wd) ^ sz) << 4)) = make_uint4(v1[0], v1[1], v1[2], v1[3]);
+        *reinterpret_cast<uint4*>(row + (((2 * wd + 1) ^ sz) << 4)) =
+            make_uint4(v2[0], v2[1], v2[2], v2[3]);
       }
       __syncwarp();
     } else if (nvalid < jw + 16) {  // tail of the split: clear value rows past the end
@@ -550,8 +577,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
 
     // ---- logits, online softmax, p in the B-operand layout
     uint32_t bp[NT][2];
-    float pv0[NT], pv1[NT], al[NT];  // 2-bit values: p of tokens j0, j1 and the rescale
-    bool any_resc = false;
+    const int pb = i & 1;  // 2-bit values: the exchange buffer of this tile
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       float s0 = 0.f, s1 = 0.f;
@@ -592,16 +618,13 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
       const float mnew = fmaxf(m2[nt], mx);
       const bool resc = mnew > m2[nt] + kRescale;
-      al[nt] = 1.0f;
       if (__any_sync(kFull, resc)) {
         const float alpha = resc ? exp2f(m2[nt] - mnew) : 1.0f;
         if (resc) m2[nt] = mnew;
         l[nt] *= alpha;
-        if constexpr (V2) {
+        if constexpr (V2) {  // the readout rescales to the warps' common maximum itself
 #pragma unroll
           for (int gg = 0; gg < NG; ++gg) vmin_acc[nt][gg] *= alpha;
-          al[nt] = alpha;
-          any_resc = true;
         } else {
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
@@ -614,8 +637,11 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       const float p1 = x1 == -INFINITY ? 0.f : exp2f(x1 - m2[nt]);
       l[nt] += p0 + p1;
       if constexpr (V2) {
-        pv0[nt] = p0;
-        pv1[nt] = p1;
+        // p and this warp's maximum to the readout warps
+        float* pw = pex_s + ((pb * kCW + warp) * 8 + 4 * nt + t) * 24;
+        pw[g] = p0;
+        pw[g + 8] = p1;
+        if (g == 0) mex_s[(pb * 8 + 4 * nt + t) * kCW + warp] = m2[nt];
         // the running sum of p_j * min_{j,g} (masked tokens add nothing)
         const float* vm = reinterpret_cast<const float*>(st + L::kVm);
 #pragma unroll
@@ -633,98 +659,105 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       }
     }
 
-    // 2-bit values: one fp16 B operand per 32-dim group over the 8 head slots.
-    // Column g is head slot g; its p for tokens 2t, 2t+1 (2t+8, 2t+9) is p0 (p1)
-    // of the lanes 4*(2t) + (g & 3) and 4*(2t+1) + (g & 3) in query tile g >> 2.
-    // p <= 2^8 (the lazy rescale) and p * scale_{j,g} enters as p * scale * 2^-E,
-    // E the running exponent of this warp's (head slot, group): raised (with
-    // that column of the group's accumulators rescaled by the exact power of
-    // two) as soon as a product reaches 2^kRaiseLog2 * 2^E, so the fp16 operand
-    // never overflows, and products within 2^-14 of their head's 2^E keep the
-    // full 11-bit mantissa.  One fp16 part is well inside the output tolerance;
-    // the codes are exact in fp16.
-    uint32_t bpf[V2 ? NG : 1][2];
+    // ---- 2-bit values: the readout of this warp's channel slice over the
+    // kTile tokens.  Column g of the B operand is head slot g; its entries for
+    // the tokens 16 kb + {2t, 2t+1 | 2t+8, 2t+9} are p_j * scale_{j,gw} of logit
+    // warp kb, brought to the common reference Mref (factor 2^(m_kb - Mref), m_kb
+    // that warp's running maximum) and to 2^-E, E the running exponent of
+    // (head slot, slice): raised, with that column of ov rescaled by the exact
+    // power of two, as soon as an entry reaches 2^kRaiseLog2 * 2^E, so the fp16
+    // operand never overflows and entries within 2^-14 of 2^E keep the full
+    // 11-bit mantissa.  p <= 2^8 (the lazy rescale); the codes are exact in fp16.
     if constexpr (V2) {
-      const int src_a = 8 * t + (g & 3), src_b = src_a + 4;
-      float pa = 0.f, pb = 0.f, pc = 0.f, pd = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const float a_ = __shfl_sync(kFull, pv0[nt], src_a);
-        const float b_ = __shfl_sync(kFull, pv0[nt], src_b);
-        const float c_ = __shfl_sync(kFull, pv1[nt], src_a);
-        const float d_ = __shfl_sync(kFull, pv1[nt], src_b);
-        if ((g >> 2) == nt) {
-          pa = a_; pb = b_; pc = c_; pd = d_;
-        }
+      __syncwarp();
+      const uint32_t xbar = smem_addr(&bars[2 * kStages + 2 + pb]);
+      if (lane == 0) mbar_arrive(xbar);
+      if (!mbar_wait(xbar, (i >> 1) & 1)) {
+        ok = false;
+        break;
       }
+      const bool hv = g < GM;  // head slot g exists
+      float mw[kCW];
+      {
+        const float4 m4 = *reinterpret_cast<const float4*>(mex_s + (pb * 8 + g) * kCW);
+        mw[0] = hv ? m4.x : -INFINITY;
+        mw[1] = hv ? m4.y : -INFINITY;
+        mw[2] = hv ? m4.z : -INFINITY;
+        mw[3] = hv ? m4.w : -INFINITY;
+      }
+      float Mn = Mref;
+#pragma unroll
+      for (int kb = 0; kb < kCW; ++kb) Mn = fmaxf(Mn, mw[kb]);
+      float rfac = 1.0f;  // factor of the ov column of head slot g
+      if (Mn > Mref) {
+        rfac = exp2f(Mref - Mn);
+        Mref = Mn;
+      }
+      float fk[kCW];
+#pragma unroll
+      for (int kb = 0; kb < kCW; ++kb) fk[kb] = mw[kb] == -INFINITY ? 0.f : exp2f(mw[kb] - Mref);
       const float* vs = reinterpret_cast<const float*>(st + L::kVs);
-      const int ta = jw + 2 * t;
+      float wq[kCW][4];
+      float hx = 0.f;
 #pragma unroll
-      for (int gg = 0; gg < NG; ++gg) {
-        const float qa = pa > 0.f ? pa * vs[ta * NG + gg] : 0.f;
-        const float qb = pb > 0.f ? pb * vs[(ta + 1) * NG + gg] : 0.f;
-        const float qc = pc > 0.f ? pc * vs[(ta + 8) * NG + gg] : 0.f;
-        const float qd = pd > 0.f ? pd * vs[(ta + 9) * NG + gg] : 0.f;
-        // the largest product of this lane's head slot g in this group (its four
-        // lanes; non-negative floats order like their bit patterns)
-        float hx = fmaxf(fmaxf(qa, qb), fmaxf(qc, qd));
-        hx = fmaxf(hx, __shfl_xor_sync(kFull, hx, 1));
-        hx = fmaxf(hx, __shfl_xor_sync(kFull, hx, 2));
-        const uint32_t mx = __float_as_uint(hx);
-        const bool raise = mx >= static_cast<uint32_t>(127 + ve[gg] + kRaiseLog2) << 23;
-        if (__any_sync(kFull, raise)) {
-          float r = 1.0f;
-          if (raise) {
-            const int en = max(-126, min(126, static_cast<int>(mx >> 23) - 127));
-            r = pow2_neg(-ve[gg]) * pow2_neg(en);  // 2^(E_old - E_new)
-            ve[gg] = en;
-            vf[gg] = pow2_neg(en);
-          }
-          // the output columns are head slots 2t, 2t+1: their factors live in
-          // lanes 8t and 8t + 4
-          const float r0 = __shfl_sync(kFull, r, 8 * t), r1 = __shfl_sync(kFull, r, 8 * t + 4);
-#pragma unroll
-          for (int mt = 2 * gg; mt < 2 * gg + 2 && mt < MT; ++mt) {
-            ov[mt][0] *= r0; ov[mt][1] *= r1; ov[mt][2] *= r0; ov[mt][3] *= r1;
-          }
-        }
-        const float f = vf[gg];
-        const __half2 h0 = __floats2half2_rn(qa * f, qb * f), h1 = __floats2half2_rn(qc * f, qd * f);
-        bpf[gg][0] = *reinterpret_cast<const uint32_t*>(&h0);
-        bpf[gg][1] = *reinterpret_cast<const uint32_t*>(&h1);
+      for (int kb = 0; kb < kCW; ++kb) {
+        const float* pr = pex_s + ((pb * kCW + kb) * 8 + g) * 24 + 2 * t;
+        const float2 pa = hv ? *reinterpret_cast<const float2*>(pr) : make_float2(0.f, 0.f);
+        const float2 pc = hv ? *reinterpret_cast<const float2*>(pr + 8) : make_float2(0.f, 0.f);
+        const int ja = 16 * kb + 2 * t;
+        // masked tokens have p = 0 and may have no scale in the stage
+        wq[kb][0] = pa.x > 0.f ? pa.x * vs[ja * NG + gw] : 0.f;
+        wq[kb][1] = pa.y > 0.f ? pa.y * vs[(ja + 1) * NG + gw] : 0.f;
+        wq[kb][2] = pc.x > 0.f ? pc.x * vs[(ja + 8) * NG + gw] : 0.f;
+        wq[kb][3] = pc.y > 0.f ? pc.y * vs[(ja + 9) * NG + gw] : 0.f;
+        hx = fmaxf(hx, fk[kb] * fmaxf(fmaxf(wq[kb][0], wq[kb][1]), fmaxf(wq[kb][2], wq[kb][3])));
       }
-      if (__any_sync(kFull, any_resc)) {
-        // rescale the output columns (head slots 2t, 2t+1) by their heads' factors
-        float f0 = 1.0f, f1 = 1.0f;
+      // the largest entry of head slot g (its four lanes; non-negative floats
+      // order like their bit patterns)
+      hx = fmaxf(hx, __shfl_xor_sync(kFull, hx, 1));
+      hx = fmaxf(hx, __shfl_xor_sync(kFull, hx, 2));
+      const uint32_t mxb = __float_as_uint(hx);
+      if (mxb >= static_cast<uint32_t>(127 + ve + kRaiseLog2) << 23) {
+        const int en = max(-126, min(126, static_cast<int>(mxb >> 23) - 127));
+        rfac *= pow2_neg(-ve) * pow2_neg(en);  // 2^(E_old - E_new)
+        ve = en;
+      }
+      if (__any_sync(kFull, rfac != 1.0f)) {
+        // the output columns are head slots 2t, 2t+1: their factors live in
+        // lanes 8t and 8t + 4
+        const float r0 = __shfl_sync(kFull, rfac, 8 * t), r1 = __shfl_sync(kFull, rfac, 8 * t + 4);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const float x0 = __shfl_sync(kFull, al[nt], (2 * t) & 3);
-          const float x1 = __shfl_sync(kFull, al[nt], (2 * t + 1) & 3);
-          if (((2 * t) >> 2) == nt) {
-            f0 = x0;
-            f1 = x1;
-          }
-        }
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          ov[mt][0] *= f0; ov[mt][1] *= f1;
-          ov[mt][2] *= f0; ov[mt][3] *= f1;
+        for (int mt = 0; mt < MTW; ++mt) {
+          ov[mt][0] *= r0; ov[mt][1] *= r1; ov[mt][2] *= r0; ov[mt][3] *= r1;
         }
       }
-    }
-
-    // ---- p . V on tensor cores (A = V^T from the swizzled tile)
-    if constexpr (V2) {
+      const float fE = pow2_neg(ve);
+      uint32_t bpf[kCW][2];
+#pragma unroll
+      for (int kb = 0; kb < kCW; ++kb) {
+        const float c = fk[kb] * fE;
+        const __half2 h0 = __floats2half2_rn(wq[kb][0] * c, wq[kb][1] * c);
+        const __half2 h1 = __floats2half2_rn(wq[kb][2] * c, wq[kb][3] * c);
+        bpf[kb][0] = *reinterpret_cast<const uint32_t*>(&h0);
+        bpf[kb][1] = *reinterpret_cast<const uint32_t*>(&h1);
+      }
+      // p . V on tensor cores: A = V^T of the slice from the code tile
       const uint32_t cbase = smem_addr(ctile);
-      const int lt = lm_tok - jw;  // row within this warp's code tile
+      const int lr = 8 * (lane >> 4) + (lane & 7);  // ldmatrix row of this lane in a k-step
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        const int chunk = 2 * mt + lm_chunk_hi;
-        uint32_t a[4];
-        ldsm_x4_trans(cbase + lt * (D * 2) + ((chunk ^ (lt & 7)) << 4), a);
-        mma_f16(ov[mt], a, bpf[mt >> 1]);
+      for (int kb = 0; kb < kCW; ++kb) {
+        const int r = 16 * kb + lr;
+        const int sz = (r / (8 / CPR)) % CPR;
+#pragma unroll
+        for (int mt = 0; mt < MTW; ++mt) {
+          const int chunk = 2 * mt + lm_chunk_hi;
+          uint32_t a[4];
+          ldsm_x4_trans(cbase + r * (CW * 2) + ((chunk ^ sz) << 4), a);
+          mma_f16(ov[mt], a, bpf[kb]);
+        }
       }
     } else {
+      // ---- p . V on tensor cores (A = V^T from the swizzled tile)
       const uint32_t vbase = smem_addr(st);
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
@@ -758,7 +791,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
-  float* mo = reinterpret_cast<float*>(stages);  // [kCW][GM][D]
+  float* mo = reinterpret_cast<float*>(stages);  // [kCW][GM][D] ([GM][D] for 2-bit values)
   float* mm = mo + kCW * GM * D;                 // [kCW][GM]
   float* ml = mm + kCW * GM;                     // [kCW][GM]
   float* vms = ml + kCW * GM;                    // [kCW][GM][NG] (2-bit values) sum p min
@@ -785,26 +818,20 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       }
     }
   }
-  if constexpr (V2) {  // columns = head slots 2t, 2t+1; add the minima sum of the group
-    // back from units of 2^ve of each column's head slot (held by lanes 8t, 8t + 4)
-    float ue[2][V2 ? NG : 1];
-#pragma unroll
-    for (int gg = 0; gg < NG; ++gg) {
-      const float u = pow2_neg(-ve[gg]);
-      ue[0][gg] = __shfl_sync(kFull, u, 8 * t);
-      ue[1][gg] = __shfl_sync(kFull, u, 8 * t + 4);
-    }
-    __syncwarp();
+  if constexpr (V2) {
+    // this warp's channel slice, columns = head slots 2t, 2t+1: back from units
+    // of 2^ve of each column's head slot (held by lanes 8t, 8t + 4); relative to
+    // Mref, the largest of the warps' final maxima
+    const float u = pow2_neg(-ve);
+    const float ue[2] = {__shfl_sync(kFull, u, 8 * t), __shfl_sync(kFull, u, 8 * t + 4)};
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int h = 2 * t + e;
       if (h < GM) {
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const float vmn = vms[(warp * GM + h) * NG + (mt >> 1)];
-          const float u = ue[e][mt >> 1];
-          mo[(warp * GM + h) * D + 16 * mt + g] = fmaf(ov[mt][e], u, vmn);
-          mo[(warp * GM + h) * D + 16 * mt + g + 8] = fmaf(ov[mt][2 + e], u, vmn);
+        for (int mt = 0; mt < MTW; ++mt) {
+          mo[h * D + cw0 + 16 * mt + g] = ov[mt][e] * ue[e];
+          mo[h * D + cw0 + 16 * mt + g + 8] = ov[mt][2 + e] * ue[e];
         }
       }
     }
@@ -824,9 +851,13 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
 #pragma unroll
       for (int w = 0; w < kCW; ++w) {
         const float f = exp2f(mm[w * GM + h] - M);
-        O = fmaf(f, mo[(w * GM + h) * D + c], O);
+        if constexpr (V2)  // sum_j p_j min_{j,g}
+          O = fmaf(f, vms[(w * GM + h) * NG + c / 32], O);
+        else
+          O = fmaf(f, mo[(w * GM + h) * D + c], O);
         Ls = fmaf(f, ml[w * GM + h], Ls);
       }
+      if constexpr (V2) O += mo[h * D + c];  // sum_j p_j scale_{j,g} code_{j,c}, relative to M
     }
     const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
     if (single) {

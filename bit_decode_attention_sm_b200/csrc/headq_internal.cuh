@@ -28,6 +28,17 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
 
+// p (a pointer into shared memory) advanced to the next multiple of `align` (a
+// power of two) bytes of the shared window, by pointer arithmetic on p itself so
+// that the compiler keeps its address space (shared loads and stores, not
+// generic ones)
+template <typename T>
+__device__ __forceinline__ T* smem_align(T* p, uint32_t align) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(p) +
+                              (((a + align - 1) & ~(align - 1)) - a));
+}
+
 // element i of a tensor that is either fp32 or bf16
 __device__ __forceinline__ float load_elem(const void* p, size_t i, bool bf16) {
   return bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(p)[i])
