@@ -861,12 +861,15 @@ def measure_rows(torch, hq, w, q_cal, k_all, v_all, q, U, cache, dt, stream, L,
     tok = B * Hkv * T
     kv_in = tok * d * 2 * k_all.element_size()          # the bf16 K and V read
     planes = tok * cache.nbytes_per_token()              # the packed cache
-    ms = timed(lambda: hq.headq_cache_write(cache, k_all, v_all, U), 5)
+    # inputs larger than L2; CUDA graphs of back-to-back calls, as for the decode
+    ms = gtimed(lambda: hq.headq_cache_write(cache, k_all, v_all, U), reps=5, replays=3)
     rows["cache_write_prefill"] = hbm_row(ms, kv_in + planes, tokens=B * T,
-                                          note="reads K,V and writes every plane")
+                                          note="reads K,V and writes every plane (CUDA graph "
+                                               "of 5 calls)")
     ws = hq.attn_kl_workspace(cache, w.Hq, T)
-    ms = timed(lambda: hq.headq_attn_kl(cache, q, U, k_all, v_all, ws=ws), 3)
-    rows["attn_kl"] = hbm_row(ms, kv_in + planes, note="reads the packed cache and full K,V")
+    ms = gtimed(lambda: hq.headq_attn_kl(cache, q, U, k_all, v_all, ws=ws), reps=5, replays=3)
+    rows["attn_kl"] = hbm_row(ms, kv_in + planes, note="reads the packed cache and full K,V "
+                                                       "(CUDA graph of 5 calls)")
     if with_cpu:
         cpu = oracle_op_rates(w, L, U.cpu().numpy())
         rows["cache_write_prefill"]["cpu_baseline"] = cpu["cache_write"]
@@ -957,13 +960,13 @@ def workload_rows(torch, hq, w, stream, with_cpu):
                           "serving step (headq_decode_append)")
     ops = {}
     wr = lambda: hq.headq_cache_write(c0, k_all, v_all, U)
-    ms_w = tm.timed(wr, 5) if kv_in + planes > 2 * tm.l2 else tm.flushed(wr)
+    ms_w = tm.gtimed(wr, reps=5, replays=3) if kv_in + planes > 2 * tm.l2 else tm.flushed(wr)
     ops["cache_write_prefill"] = tm.hbm_row(ms_w, kv_in + planes, tokens_per_sequence=T,
                                             note="prefill of every sequence: reads K,V and "
                                                  "writes every plane")
     kws = hq.attn_kl_workspace(c0, Hq, T)
     kl = lambda: hq.headq_attn_kl(c0, q, U, k_all, v_all, ws=kws)
-    ms_k = tm.timed(kl, 3) if kv_in + planes > 2 * tm.l2 else tm.flushed(kl, 5)
+    ms_k = tm.gtimed(kl, reps=5, replays=3) if kv_in + planes > 2 * tm.l2 else tm.flushed(kl, 5)
     ops["attn_kl"] = tm.hbm_row(ms_k, kv_in + planes,
                                 note="reads the packed cache and full K,V")
     if w.vmode == "2bit":

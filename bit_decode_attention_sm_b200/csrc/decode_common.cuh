@@ -212,8 +212,12 @@ __device__ __forceinline__ void encode_new_token(const DecodeParams& p, int b, i
   __syncwarp();
   if (R > 0 && orow >= 0) {
     float y = 0.0f;
-    if (lane < R)
+    // channels in order (the codec's rounding sequence); unrolled so that the
+    // loads of U_h (shared or global memory) are issued ahead of the adds
+    if (lane < R) {
+#pragma unroll 16
       for (int c = 0; c < D; ++c) y = __fadd_rn(y, __fmul_rn(u_s[c * R + lane], enew_s[c]));
+    }
     float a = lane < R ? fabsf(y) : 0.0f;
 #pragma unroll
     for (int o2 = 16; o2 > 0; o2 >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o2));

@@ -108,8 +108,9 @@ constexpr size_t smem_bytes() {
   // group sums [GM][NG] | sigma U^T q [GM][R] | U [D][R] | appended token's
   // residual [D] and projection [R] | max |q| per (head, group) [GM][NG] | the
   // query as bulk-copied (raw bf16 or fp32) [GM][D] | barriers.  2-bit values
-  // (three CTAs per SM) read U_h from global memory and land the raw query in
-  // the code tiles, which are free until the main loop.
+  // (three CTAs per SM) land the raw query and U_h in the code tiles, which are
+  // free until the main loop (the fused append then reads U_h from global
+  // memory).
   return 1024 + size_t(kStagesFor<NT>) * L::kStage + size_t(kCW) * L::kCodeTile + L::kExBytes +
          bq_bytes +
          sizeof(float) * ((4 * NT) * (D + L::NG + (R > 0 ? R : 1)) +
@@ -149,8 +150,10 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
                                         (kBqInSmem<NT> ? size_t(kCW) * 32 * KS * NT * 8 : 0));
   float* qsum_s = q_s + GM * D;                                               // [GM][NG]
   float* qt_s = qsum_s + GM * NG;                                             // [GM][RR]
-  // U_h [D][RR]: in shared memory, or (2-bit values) read from global memory
-  const float* u_s = V2 ? p.U + static_cast<size_t>(blockIdx.y) * D * R : qt_s + GM * RR;
+  // U_h [D][RR] in shared memory (2-bit values: in the code tiles, after the query)
+  float* u_s = V2 ? reinterpret_cast<float*>(ctiles + GM * D * 4) : qt_s + GM * RR;
+  static_assert(!V2 || (4 * NT) * D * 4 + D * (R > 0 ? R : 1) * 4 <= kCW * L::kCodeTile,
+                "the query and U_h fit in the code tiles");
   float* enew_s = qt_s + GM * RR + (V2 ? 0 : D * RR);                         // [D]
   float* ynew_s = enew_s + D;                                                 // [RR]
   float* qmax_s = ynew_s + RR;                                                // [GM][NG]
@@ -199,12 +202,12 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       // preparation does not wait behind the cache stream
       const uint32_t qbar = smem_addr(&bars[2 * kStages + 1]);
       const uint32_t qbytes = static_cast<uint32_t>(G * D * (p.q_bf16 ? 2 : 4));
-      mbar_expect_tx(qbar, qbytes + (R > 0 && !V2 ? D * R * 4 : 0));
+      mbar_expect_tx(qbar, qbytes + (R > 0 ? D * R * 4 : 0));
       bulk_g2s(smem_addr(qraw_s),
                static_cast<const uint8_t*>(p.q) +
                    (static_cast<size_t>(b) * p.Hq + h0) * D * (p.q_bf16 ? 2 : 4),
                qbytes, qbar);
-      if constexpr (R > 0 && !V2)
+      if constexpr (R > 0)
         bulk_g2s(smem_addr(u_s), p.U + static_cast<size_t>(kv) * D * R, D * R * 4, qbar);
     }
     // The tiles of this CTA's chunk in order, one per stage, then an end marker.
@@ -228,7 +231,9 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
         // memory), then publish it to the bulk copies (async proxy)
         if (!mbar_wait(smem_addr(&bars[2 * kStages + 1]), 0) && lane == 0 && p.err)
           atomicOr(p.err, kDevErrWaitTimeout);
-        encode_new_token<D, R, V2>(p, b, kv, pos, u_s, enew_s, lane);
+        encode_new_token<D, R, V2>(p, b, kv, pos,
+                                   V2 ? p.U + static_cast<size_t>(kv) * D * R : u_s, enew_s,
+                                   lane);
         __threadfence();
         asm volatile("fence.proxy.async.global;" ::: "memory");
         __syncwarp();
