@@ -578,7 +578,8 @@ def run_headq(args):
     alg_bytes = B * Hkv * T * bytes_tok
     peak, peak_kind = measured_hbm_peak()
     achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
-    traffic = (recorded_traffic(["decode_mma.cu", "codec.cuh"], "decode_mma_longctx.md")
+    traffic = (recorded_traffic(["decode_mma.cu", "decode_common.cuh", "codec.cuh"],
+                                "decode_mma_longctx.md")
                if w.name == DEFAULT_WORKLOAD else None)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
