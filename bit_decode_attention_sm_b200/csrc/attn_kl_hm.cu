@@ -606,39 +606,11 @@ attn_kl_hm_kernel(const AttnKlParams p, const __grid_constant__ CUtensorMap kmap
 }
 
 // ---------------------------------------------------------------- host side
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encode_fn() {
-  static EncodeTiled fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(f);
-    cudaGetLastError();
-  });
-  return fn;
-}
-
 // bf16 rows of D channels in slabs: [slab][row][channel], 64-channel x kTile-row
 // boxes with the 128-byte swizzle
 template <int D>
 bool encode_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t slabs) {
-  EncodeTiled enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), rows, slabs};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, rows * D * 2};
-  const cuuint32_t box[3] = {64, kTile, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return encode_bf16_rows(map, base, D, rows, slabs, kTile);
 }
 
 template <int D, int R, bool V2>
@@ -677,7 +649,7 @@ bool kl_hm_supported(const headq_cache& c, int G, bool kv_bf16) {
   if (c.r != 0 && c.r != 8 && c.r != 16) return false;
   if (c.page_size > 0 && c.page_size % kTile != 0) return false;  // whole tiles per page
   if (c.vmode == HEADQ_V_2BIT) return true;
-  return c.v_dtype == HEADQ_BF16 && encode_fn() != nullptr;
+  return c.v_dtype == HEADQ_BF16 && tensor_maps_available();
 }
 
 // Splits for one CTA per SM: chunks a multiple of the tile (112 tokens), the

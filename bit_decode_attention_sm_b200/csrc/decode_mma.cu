@@ -975,26 +975,6 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
 }
 
 // ---------------------------------------------------------------- host side
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encode_fn() {
-  static EncodeTiled fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(f);
-    cudaGetLastError();
-  });
-  return fn;
-}
-
 constexpr int kMaxDev = 64;
 
 template <int D, int R, int NT, bool V2, bool KCH>
@@ -1035,21 +1015,12 @@ struct Variant {
       decode_mma_kernel<D, R, NT, V2, KCH><<<grid, kThreads, smem_bytes<D, R, NT, V2, KCH>(), s>>>(p, vmap);
       return cudaGetLastError();
     }
-    EncodeTiled enc = encode_fn();
-    if (!enc) return cudaErrorNotSupported;
+    if (!tensor_maps_available()) return cudaErrorNotSupported;
     // [slab][row in slab][channel]: one slab per (b, kv), or per (page, kv)
     const bool paged = p.c.page_size > 0;
-    const cuuint64_t rows = static_cast<cuuint64_t>(paged ? p.c.page_size : p.c.T_cap);
-    const cuuint64_t slabs = static_cast<cuuint64_t>(paged ? p.c.num_pages : p.c.B) * p.c.Hkv;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), rows, slabs};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, rows * D * 2};
-    const cuuint32_t box[3] = {64, kTile, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    if (enc(&vmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.c.v, dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
-        CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
+    const uint64_t rows = static_cast<uint64_t>(paged ? p.c.page_size : p.c.T_cap);
+    const uint64_t slabs = static_cast<uint64_t>(paged ? p.c.num_pages : p.c.B) * p.c.Hkv;
+    if (!encode_bf16_rows(&vmap, p.c.v, D, rows, slabs, kTile)) return cudaErrorInvalidValue;
     decode_mma_kernel<D, R, NT, V2, KCH><<<grid, kThreads, smem_bytes<D, R, NT, V2, KCH>(), s>>>(p, vmap);
     return cudaGetLastError();
   }
@@ -1094,7 +1065,7 @@ bool mma_decode_supported(const headq_cache& c, int G) {
   if (G < 1 || G > 8) return false;
   if (c.vmode == HEADQ_V_2BIT) return c.r == 8 || c.r == 16;
   return c.vmode == HEADQ_V_DENSE && c.v_dtype == HEADQ_BF16 &&
-         (c.r == 0 || c.r == 8 || c.r == 16) && encode_fn() != nullptr;
+         (c.r == 0 || c.r == 8 || c.r == 16) && tensor_maps_available();
 }
 
 int mma_decode_ctas_per_sm(const headq_cache& c, int G) {

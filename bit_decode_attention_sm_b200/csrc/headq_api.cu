@@ -3,6 +3,8 @@
 // allocates device memory; a failed check returns before any launch.
 #include <string.h>
 
+#include <mutex>
+
 #include "headq_internal.cuh"
 
 #define HEADQ_API extern "C" __attribute__((visibility("default")))
@@ -15,6 +17,45 @@ bool aligned16(const void* p) {
 
 static bool supported_d(int d) {
   return d == 8 || d == 16 || d == 32 || d == 64 || d == 128 || d == 256;
+}
+
+namespace {
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library); null when the driver does not offer it
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(f);
+    cudaGetLastError();
+  });
+  return fn;
+}
+}  // namespace
+
+bool tensor_maps_available() { return encode_fn() != nullptr; }
+
+bool encode_bf16_rows(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                      uint64_t slabs, uint32_t box_rows) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {inner, rows, slabs};
+  const cuuint64_t strides[2] = {inner * 2, rows * inner * 2};
+  const cuuint32_t box[3] = {64, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int sm_count() {

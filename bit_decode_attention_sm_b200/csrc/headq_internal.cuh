@@ -3,6 +3,7 @@
 // one launcher taking a plain parameter struct.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -185,6 +186,14 @@ struct CalibrateParams {
   float* U;
   float* eig;
 };
+
+// Tensor map of bf16 rows of `inner` channels in slabs ([slab][row][channel],
+// row stride inner * 2 bytes), boxes of 64 channels x box_rows rows with the
+// 128-byte swizzle (headq_api.cu).  False when the driver offers no encoder or
+// the encoding fails (a base or stride not 16-byte aligned).
+bool tensor_maps_available();
+bool encode_bf16_rows(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                      uint64_t slabs, uint32_t box_rows);
 
 // host-side argument checks shared by the entry points (headq_api.cu)
 bool aligned16(const void* p);
