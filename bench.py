@@ -711,8 +711,8 @@ A2_OBS = 16        # observation queries per sequence
 A2_KEEP = 0.05     # fraction of each sequence's tokens whose values stay exact
 def a2_policy_row(torch, hq, w, q, U, cache, k_all, v_all, dt, L, timed, gtimed, hbm_row):
     """The A^2 value policy on this workload: scores from A2_OBS observation
-    queries per sequence (two logit passes on CUDA cores, against the fp32 ALU
-    peak), the top-K selection with the copy of the kept values, and the decode
+    queries per sequence (two logit passes, on tensor cores for bf16, plus the
+    per-token value error; CUDA graph of 5 calls, against HBM), the top-K selection with the copy of the kept values, and the decode
     followed by the value fixup (against HBM, the cache plus the kept values)."""
     B, Hq, Hkv, d, T = w.B, w.Hq, w.Hkv, w.d, w.T
     qo = torch.from_numpy(synth.make_observation_queries(w, L, A2_OBS)).to(q.device).to(dt)
@@ -721,7 +721,8 @@ def a2_policy_row(torch, hq, w, q, U, cache, k_all, v_all, dt, L, timed, gtimed,
     scores = torch.empty((B, Hkv, T), dtype=torch.float32, device=q.device)
     keep_idx = torch.empty((B, Hkv, K), dtype=torch.int32, device=q.device)
     keep_v = torch.empty((B, Hkv, K, d), dtype=dt, device=q.device)
-    ms_sc = timed(lambda: hq.headq_a2_scores(cache, qo, k_all, v_all, ws=ws, out=scores), 3)
+    ms_sc = gtimed(lambda: hq.headq_a2_scores(cache, qo, k_all, v_all, ws=ws, out=scores),
+                   reps=5, replays=3)
     ms_sel = timed(lambda: hq.headq_a2_select(scores, K, v_all, keep_idx=keep_idx, keep_v=keep_v), 5)
     hq.headq_workspace_status(ws)
     out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)

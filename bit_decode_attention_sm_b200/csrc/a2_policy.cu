@@ -27,6 +27,8 @@
 //                        (same softmax weights; exact algebra).
 #include <math.h>
 
+#include <mutex>
+
 #include "headq_internal.cuh"
 
 #define HEADQ_API extern "C" __attribute__((visibility("default")))
@@ -217,14 +219,24 @@ __global__ void __launch_bounds__(kAThreads) a2_pass_kernel(const A2Params p) {
 }
 
 // ---- the same two passes on tensor cores, for bf16 keys and queries ---------
-// A 64-token tile, 4 warps of 16 tokens; observation queries in chunks of 64.
-// Logits = K_tile (A, row-major, tokens x channels) times Q^T (B: each query's
-// channels are a column), mma.sync m16n8k16 bf16 -> fp32: products of bf16
-// values are exact, so this differs from the CUDA-core pass only in the order
-// of the fp32 sums.  Both operands come from padded shared-memory rows with
-// 32-bit loads (row stride D + 8: lanes of a fragment hit distinct banks).
-constexpr int kMT = 128;   // threads: 4 warps x 16 tokens
-constexpr int kMQ = 64;    // queries per chunk: 8 n8 tiles
+// Observation queries on the MMA M side: warp w holds queries [16 w, 16 w + 16)
+// of a chunk of kQW * 16 as A fragments (all k-steps, in registers for the
+// CTA's whole walk), and a CTA walks kTPC 64-token tiles of one (b, kv), each
+// tile's keys (the B operand: tokens on N, from padded rows with 32-bit loads,
+// lanes on distinct banks) streamed through two cp.async buffers so the next
+// tile loads during the current tile's MMAs.  Logits = Q K^T on mma.sync
+// m16n8k16 bf16 -> fp32: products of bf16 values are exact, so this differs from
+// the CUDA-core pass only in the order of the fp32 sums.
+//   pass 0: a running max and sum per query row in each lane (its two columns
+//           of every n8 tile), merged over the row's four lanes at the end: one
+//           (max, sum) partial per (CTA, query)
+//   pass 1: p^2 per (query, token) summed over the chunk's queries per token:
+//           the row pair in each lane, the rows by warp shuffles, the warps in
+//           shared memory
+// |v^_j - v_j|^2 comes from a2_dv2_kernel, already in `scores`.
+constexpr int kQW = 8;           // query warps: 16 queries each
+constexpr int kMT = 32 * kQW;    // threads
+constexpr int kTPC = 8;          // tiles per CTA
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
                                                uint32_t b1) {
@@ -234,74 +246,79 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// 16 bytes global -> shared, asynchronously; zero-filled when `valid` is false
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// four 8x8 b16 matrices; lane l gives the row address of matrix l / 8, row l % 8
+__device__ __forceinline__ void ldsm_x4(const void* row, uint32_t (&r)[4]) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(row));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+
+template <int D>
+constexpr size_t a2_mma_smem() {
+  return sizeof(uint16_t) * (2 * kAT + 16 * kQW) * (D + 8) +
+         sizeof(float) * (kQW * kAT + kTPC * kAT);
+}
 
 template <int D, bool SCORE>
 __global__ void __launch_bounds__(kMT) a2_pass_mma_kernel(const A2Params p) {
   constexpr int RS = D + 8;  // bf16 elements per shared row
   constexpr int KSTEPS = D / 16;
+  constexpr int CPR = D / 8; // 16-byte chunks per row
+  constexpr int QC = 16 * kQW;
+  constexpr float kL2e = 1.4426950408889634f;
+  constexpr float kLn2f = 0.6931471805599453f;
   extern __shared__ __align__(16) unsigned char a2m_smem[];
-  uint16_t* k_s = reinterpret_cast<uint16_t*>(a2m_smem);          // [kAT][RS]
-  uint16_t* q_s = k_s + kAT * RS;                                   // [kMQ][RS]
-  float* dv2_s = reinterpret_cast<float*>(q_s + kMQ * RS);         // [kAT]
+  uint16_t* k_s = reinterpret_cast<uint16_t*>(a2m_smem);          // [2][kAT][RS]
+  uint16_t* q_s = k_s + 2 * kAT * RS;                               // [QC][RS]
+  float* red_s = reinterpret_cast<float*>(q_s + QC * RS);          // [kQW][kAT] per-warp sums
+  float* acc_s = red_s + kQW * kAT;                                 // [kTPC][kAT] sum p^2
 
-  const int tile = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
+  const int kv = blockIdx.y, b = blockIdx.z;
+  const int tile_first = blockIdx.x * kTPC;
+  const int ntl = min(kTPC, p.ntiles - tile_first);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int Tb = seq_len(p.seq_lens, b, p.T);
-  const int t0 = tile * kAT;
   const int G = p.G, NQ = p.n_obs * G;
   const size_t bk = static_cast<size_t>(b) * p.c.Hkv + kv;
   const uint16_t* kf = static_cast<const uint16_t*>(p.k_full);
   const uint16_t* qo = static_cast<const uint16_t*>(p.q_obs);
+  const float s2 = p.sm_scale * kL2e;  // logits in log2 units
 
-  for (int e = tid; e < kAT * (D / 8); e += kMT) {
-    const int row = e / (D / 8), c8 = e - row * (D / 8);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (t0 + row < Tb) v = *reinterpret_cast<const uint4*>(kf + (bk * p.T + t0 + row) * D + c8 * 8);
-    *reinterpret_cast<uint4*>(k_s + row * RS + c8 * 8) = v;
-  }
-  if constexpr (SCORE) {  // |v^_j - v_j|^2: two threads per token, half the channels each
-    const int j = tid >> 1, half = tid & 1;
-    float a = 0.0f;
-    if (t0 + j < Tb) {
-      const size_t row = cache_row_read(p.c, b, kv, t0 + j, half == 0 ? p.err : nullptr);
-      for (int c0 = half * (D / 2); c0 < (half + 1) * (D / 2); c0 += 8) {
-        float v[8], vh[8];
-        load8(p.v_full, (bk * p.T + t0 + j) * D + c0, true, v);
-        value_hat8(p.c, row, c0, D, vh);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float dv = vh[k] - v[k];
-          a = fmaf(dv, dv, a);
-        }
-      }
+  // the key rows of local tile k into buffer buf (rows past T_b read as zero)
+  auto load_tile = [&](int k, int buf) {
+    const int t0 = (tile_first + k) * kAT;
+    uint16_t* dst = k_s + buf * kAT * RS;
+    for (int e = tid; e < kAT * CPR; e += kMT) {
+      const int row = e / CPR, c8 = e - row * CPR;
+      const bool valid = t0 + row < Tb;
+      const uint16_t* src = kf + (bk * p.T + (valid ? t0 + row : 0)) * D + c8 * 8;
+      cp_async16(dst + row * RS + c8 * 8, src, valid);
     }
-    a += __shfl_xor_sync(0xffffffffu, a, 1);
-    if (half == 0) dv2_s[j] = a;
-  }
-  __syncthreads();
+    cp_async_commit();
+  };
+  if constexpr (SCORE)
+    for (int e = tid; e < kTPC * kAT; e += kMT) acc_s[e] = 0.0f;
 
-  // this warp's 16 tokens as A fragments, all k-steps
-  uint32_t af[KSTEPS][4];
-  {
-    const uint16_t* r0 = k_s + (16 * warp + g) * RS + 2 * t;
-    const uint16_t* r1 = r0 + 8 * RS;
-#pragma unroll
-    for (int ks = 0; ks < KSTEPS; ++ks) {
-      af[ks][0] = *reinterpret_cast<const uint32_t*>(r0 + 16 * ks);
-      af[ks][1] = *reinterpret_cast<const uint32_t*>(r1 + 16 * ks);
-      af[ks][2] = *reinterpret_cast<const uint32_t*>(r0 + 16 * ks + 8);
-      af[ks][3] = *reinterpret_cast<const uint32_t*>(r1 + 16 * ks + 8);
-    }
-  }
-  const int tok0 = t0 + 16 * warp + g, tok1 = tok0 + 8;
-  const bool v0 = tok0 < Tb, v1 = tok1 < Tb;
-  float acc0 = 0.0f, acc1 = 0.0f;  // SCORE: sum of p^2 for tokens tok0, tok1
-
-  for (int q0 = 0; q0 < NQ; q0 += kMQ) {
-    const int nq = min(kMQ, NQ - q0);
-    __syncthreads();  // every warp is done with the previous chunk
-    for (int e = tid; e < kMQ * (D / 8); e += kMT) {
-      const int qq = e / (D / 8), c8 = e - qq * (D / 8);
+  for (int q0 = 0; q0 < NQ; q0 += QC) {
+    const int nq = min(QC, NQ - q0);
+    __syncthreads();  // every warp is done with the previous query chunk
+    for (int e = tid; e < QC * CPR; e += kMT) {
+      const int qq = e / CPR, c8 = e - qq * CPR;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (qq < nq) {
         const int qi = q0 + qq, o = qi / G, gq = qi - o * G;
@@ -310,69 +327,164 @@ __global__ void __launch_bounds__(kMT) a2_pass_mma_kernel(const A2Params p) {
       }
       *reinterpret_cast<uint4*>(q_s + qq * RS + c8 * 8) = v;
     }
-    __syncthreads();
-    float c[kMQ / 8][4];
+    load_tile(0, 0);
+    __syncthreads();  // the query chunk in shared memory
+    // this warp's 16 queries as A fragments (rows g and g + 8)
+    const bool wlive = 16 * warp < nq;
+    const int qr0 = q0 + 16 * warp + g, qr1 = qr0 + 8;  // query indices of the two rows
+    const bool r0 = qr0 < q0 + nq, r1 = qr1 < q0 + nq;
+    uint32_t qa[KSTEPS][4];
+    {
+      const uint16_t* a0 = q_s + (16 * warp + g) * RS + 2 * t;
+      const uint16_t* a1 = a0 + 8 * RS;
 #pragma unroll
-    for (int nt = 0; nt < kMQ / 8; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.0f;
-#pragma unroll
-    for (int ks = 0; ks < KSTEPS; ++ks) {
-#pragma unroll
-      for (int nt = 0; nt < kMQ / 8; ++nt) {
-        if (8 * nt >= nq) break;  // uniform across the CTA
-        const uint16_t* qr = q_s + (8 * nt + g) * RS + 16 * ks + 2 * t;
-        mma_bf16_16816(c[nt], af[ks], *reinterpret_cast<const uint32_t*>(qr),
-                       *reinterpret_cast<const uint32_t*>(qr + 8));
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        qa[ks][0] = *reinterpret_cast<const uint32_t*>(a0 + 16 * ks);
+        qa[ks][1] = *reinterpret_cast<const uint32_t*>(a1 + 16 * ks);
+        qa[ks][2] = *reinterpret_cast<const uint32_t*>(a0 + 16 * ks + 8);
+        qa[ks][3] = *reinterpret_cast<const uint32_t*>(a1 + 16 * ks + 8);
       }
     }
-#pragma unroll
-    for (int nt = 0; nt < kMQ / 8; ++nt) {
-      if (8 * nt >= nq) break;
-      const int n0 = 8 * nt + 2 * t;  // this lane's two query columns n0, n0 + 1
-      const float s00 = v0 ? c[nt][0] * p.sm_scale : -INFINITY;
-      const float s01 = v0 ? c[nt][1] * p.sm_scale : -INFINITY;
-      const float s10 = v1 ? c[nt][2] * p.sm_scale : -INFINITY;
-      const float s11 = v1 ? c[nt][3] * p.sm_scale : -INFINITY;
-      if constexpr (!SCORE) {
-        float m0 = fmaxf(s00, s10), m1 = fmaxf(s01, s11);
-#pragma unroll
-        for (int o2 = 4; o2 < 32; o2 <<= 1) {
-          m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o2));
-          m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o2));
-        }
-        float l0 = (v0 ? expf(s00 - m0) : 0.0f) + (v1 ? expf(s10 - m0) : 0.0f);
-        float l1 = (v0 ? expf(s01 - m1) : 0.0f) + (v1 ? expf(s11 - m1) : 0.0f);
-#pragma unroll
-        for (int o2 = 4; o2 < 32; o2 <<= 1) {
-          l0 += __shfl_xor_sync(0xffffffffu, l0, o2);
-          l1 += __shfl_xor_sync(0xffffffffu, l1, o2);
-        }
-        if (g == 0) {
-          float2* dst = p.part + ((bk * p.ntiles + tile) * p.ppt + warp) * NQ + q0;
-          if (n0 < nq) dst[n0] = make_float2(m0, l0);
-          if (n0 + 1 < nq) dst[n0 + 1] = make_float2(m1, l1);
-        }
+    // pass 0: running max (log2 units) and sum of the two rows over this lane's
+    // columns; pass 1: the rows' lse in log2 units
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
+    float lse2[2] = {0.0f, 0.0f};
+    if constexpr (SCORE) {
+      if (r0) lse2[0] = p.lse[bk * NQ + qr0] * kL2e;
+      if (r1) lse2[1] = p.lse[bk * NQ + qr1] * kL2e;
+    }
+
+    for (int k = 0; k < ntl; ++k) {
+      const int tile = tile_first + k;
+      if (k + 1 < ntl) {
+        load_tile(k + 1, (k + 1) & 1);
+        cp_async_wait<1>();
       } else {
-        const float* lse = p.lse + bk * NQ + q0;
-        const float l0 = n0 < nq ? lse[n0] : 0.0f, l1 = n0 + 1 < nq ? lse[n0 + 1] : 0.0f;
-        const float p00 = (v0 && n0 < nq) ? expf(s00 - l0) : 0.0f;
-        const float p01 = (v0 && n0 + 1 < nq) ? expf(s01 - l1) : 0.0f;
-        const float p10 = (v1 && n0 < nq) ? expf(s10 - l0) : 0.0f;
-        const float p11 = (v1 && n0 + 1 < nq) ? expf(s11 - l1) : 0.0f;
-        acc0 = fmaf(p00, p00, fmaf(p01, p01, acc0));
-        acc1 = fmaf(p10, p10, fmaf(p11, p11, acc1));
+        cp_async_wait<0>();
+      }
+      __syncthreads();  // tile k in shared memory
+      const uint16_t* kb = k_s + (k & 1) * kAT * RS;
+      if (wlive) {
+#pragma unroll
+        for (int nt = 0; nt < kAT / 8; ++nt) {
+          float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          // B fragments of two k-steps per ldmatrix: matrices = channels
+          // [32 kk, +8), [+8, +16), [+16, +24), [+24, +32) of tokens 8 nt .. 8 nt + 7
+          const uint16_t* br = kb + (8 * nt + (lane & 7)) * RS + 8 * (lane >> 3);
+#pragma unroll
+          for (int kk = 0; kk < KSTEPS / 2; ++kk) {
+            uint32_t bf[4];
+            ldsm_x4(br + 32 * kk, bf);
+            mma_bf16_16816(c, qa[2 * kk], bf[0], bf[1]);
+            mma_bf16_16816(c, qa[2 * kk + 1], bf[2], bf[3]);
+          }
+          // c: (row g | g + 8) x (tokens j, j + 1) of this lane
+          const int j = tile * kAT + 8 * nt + 2 * t;
+          const bool c0 = j < Tb, c1 = j + 1 < Tb;
+          if constexpr (!SCORE) {
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+              const float xa = c0 ? c[2 * rr] * s2 : -INFINITY;
+              const float xb = c1 ? c[2 * rr + 1] * s2 : -INFINITY;
+              const float mx = fmaxf(xa, xb);
+              if (mx > m[rr]) {  // a new maximum: rescale the sum (exp2(-inf) = 0)
+                l[rr] *= exp2f(m[rr] - mx);
+                m[rr] = mx;
+              }
+              if (m[rr] != -INFINITY) l[rr] += exp2f(xa - m[rr]) + exp2f(xb - m[rr]);
+            }
+          } else {
+            const float p00 = (c0 && r0) ? exp2f(c[0] * s2 - lse2[0]) : 0.0f;
+            const float p01 = (c1 && r0) ? exp2f(c[1] * s2 - lse2[0]) : 0.0f;
+            const float p10 = (c0 && r1) ? exp2f(c[2] * s2 - lse2[1]) : 0.0f;
+            const float p11 = (c1 && r1) ? exp2f(c[3] * s2 - lse2[1]) : 0.0f;
+            // column sums over the warp's 16 rows
+            float sa = fmaf(p00, p00, p10 * p10), sb = fmaf(p01, p01, p11 * p11);
+#pragma unroll
+            for (int o2 = 4; o2 < 32; o2 <<= 1) {
+              sa += __shfl_xor_sync(0xffffffffu, sa, o2);
+              sb += __shfl_xor_sync(0xffffffffu, sb, o2);
+            }
+            if (g == 0) {
+              red_s[warp * kAT + 8 * nt + 2 * t] = sa;
+              red_s[warp * kAT + 8 * nt + 2 * t + 1] = sb;
+            }
+          }
+        }
+      }
+      if constexpr (SCORE) {
+        __syncthreads();  // every warp's token sums in red_s
+        if (tid < kAT) {
+          float a = 0.0f;
+          for (int w = 0; w < kQW; ++w)
+            if (16 * w < nq) a += red_s[w * kAT + tid];
+          acc_s[k * kAT + tid] += a;
+        }
+      }
+      __syncthreads();  // every warp is done with buffer k & 1 (and red_s) before reuse
+    }
+    if constexpr (!SCORE) {
+      // merge the rows' (max, sum) over their four lanes; one partial per query
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+#pragma unroll
+        for (int o2 = 1; o2 < 4; o2 <<= 1) {
+          const float mo = __shfl_xor_sync(0xffffffffu, m[rr], o2);
+          const float lo = __shfl_xor_sync(0xffffffffu, l[rr], o2);
+          const float mx = fmaxf(m[rr], mo);
+          if (mx != -INFINITY) {
+            l[rr] = (m[rr] == -INFINITY ? 0.0f : l[rr] * exp2f(m[rr] - mx)) +
+                    (mo == -INFINITY ? 0.0f : lo * exp2f(mo - mx));
+            m[rr] = mx;
+          }
+        }
+      }
+      if (wlive && t == 0) {
+        float2* dst = p.part + (bk * gridDim.x + blockIdx.x) * NQ;  // gridDim.x partials per (b, kv)
+        // natural-log max; the sum is the same in either base
+        if (r0) dst[qr0] = make_float2(m[0] == -INFINITY ? -INFINITY : m[0] * kLn2f, l[0]);
+        if (r1) dst[qr1] = make_float2(m[1] == -INFINITY ? -INFINITY : m[1] * kLn2f, l[1]);
       }
     }
   }
   if constexpr (SCORE) {
-    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
-    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
-    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
-    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
-    if (t == 0) {
-      if (tok0 < p.T) p.scores[bk * p.T + tok0] = v0 ? acc0 * dv2_s[16 * warp + g] : 0.0f;
-      if (tok1 < p.T) p.scores[bk * p.T + tok1] = v1 ? acc1 * dv2_s[16 * warp + g + 8] : 0.0f;
+    // scores holds |v^_j - v_j|^2 (a2_dv2_kernel); times sum_{o,h} p^2
+    for (int e = tid; e < ntl * kAT; e += kMT) {
+      const int tok = tile_first * kAT + e;
+      if (tok >= p.T) continue;
+      float* sc = p.scores + bk * p.T + tok;
+      *sc = tok < Tb ? acc_s[e] * *sc : 0.0f;
     }
   }
+}
+
+// |v^_j - v_j|^2 of every token j < T into scores (0 for j >= T_b): D/8 lanes
+// per token, 8 channels each, summed by shuffles within the token's lanes; CTA
+// (token block, kv, b)
+template <int D>
+__global__ void __launch_bounds__(256) a2_dv2_kernel(const A2Params p) {
+  constexpr int LPT = D / 8;           // lanes per token (a power of two, <= 32)
+  constexpr int TPB = 256 / LPT;       // tokens per CTA
+  const int kv = blockIdx.y, b = blockIdx.z;
+  const int tt = blockIdx.x * TPB + threadIdx.x / LPT;
+  const int c0 = (threadIdx.x % LPT) * 8;
+  const size_t bk = static_cast<size_t>(b) * p.c.Hkv + kv;
+  const bool live = tt < seq_len(p.seq_lens, b, p.T);
+  float a = 0.0f;
+  if (live) {
+    const size_t row = cache_row_read(p.c, b, kv, tt, c0 == 0 ? p.err : nullptr);
+    float v[8], vh[8];
+    load8(p.v_full, (bk * p.T + tt) * D + c0, true, v);
+    value_hat8(p.c, row, c0, D, vh);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float dv = vh[k] - v[k];
+      a = fmaf(dv, dv, a);
+    }
+  }
+#pragma unroll
+  for (int o2 = 1; o2 < LPT; o2 <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o2);
+  if (tt < p.T && c0 == 0) p.scores[bk * p.T + tt] = live ? a : 0.0f;
 }
 
 // lse of every observation query from the tile partials; one CTA per (b, kv)
@@ -704,10 +816,27 @@ cudaError_t launch_scores(A2Params p, cudaStream_t s) {
   if constexpr (D == 64 || D == 128) {
     if (p.kv_bf16 && p.q_bf16) {  // tensor cores
       p.ppt = 4;
-      const size_t smem = sizeof(uint16_t) * (kAT + kMQ) * (D + 8) + sizeof(float) * kAT;
-      a2_pass_mma_kernel<D, false><<<grid, kMT, smem, s>>>(p);
-      a2_lse_kernel<<<p.c.B * p.c.Hkv, NQ < 1024 ? (NQ + 31) / 32 * 32 : 1024, 0, s>>>(p);
-      a2_pass_mma_kernel<D, true><<<grid, kMT, smem, s>>>(p);
+      constexpr size_t smem = a2_mma_smem<D>();
+      static std::once_flag once;
+      static cudaError_t attr = cudaSuccess;
+      std::call_once(once, [] {
+        attr = cudaFuncSetAttribute(a2_pass_mma_kernel<D, false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (attr == cudaSuccess)
+          attr = cudaFuncSetAttribute(a2_pass_mma_kernel<D, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      });
+      if (attr != cudaSuccess) return attr;
+      const int parts = (p.ntiles + kTPC - 1) / kTPC;  // CTAs per (b, kv)
+      const dim3 mgrid(parts, p.c.Hkv, p.c.B);
+      a2_pass_mma_kernel<D, false><<<mgrid, kMT, smem, s>>>(p);
+      A2Params pl = p;  // the normaliser merges one partial per CTA
+      pl.ntiles = parts;
+      pl.ppt = 1;
+      a2_lse_kernel<<<p.c.B * p.c.Hkv, NQ < 1024 ? (NQ + 31) / 32 * 32 : 1024, 0, s>>>(pl);
+      constexpr int kDv2Tok = 256 / (D / 8);
+      a2_dv2_kernel<D><<<dim3((p.T + kDv2Tok - 1) / kDv2Tok, p.c.Hkv, p.c.B), 256, 0, s>>>(p);
+      a2_pass_mma_kernel<D, true><<<mgrid, kMT, smem, s>>>(p);
       return cudaGetLastError();
     }
   }
