@@ -712,8 +712,9 @@ A2_KEEP = 0.05     # fraction of each sequence's tokens whose values stay exact
 def a2_policy_row(torch, hq, w, q, U, cache, k_all, v_all, dt, L, timed, gtimed, hbm_row):
     """The A^2 value policy on this workload: scores from A2_OBS observation
     queries per sequence (two logit passes, on tensor cores for bf16, plus the
-    per-token value error; CUDA graph of 5 calls, against HBM), the top-K selection with the copy of the kept values, and the decode
-    followed by the value fixup (against HBM, the cache plus the kept values)."""
+    per-token value error; CUDA graph of 5 calls, against HBM), the top-K
+    selection with the copy of the kept values, and the decode followed by the
+    value fixup (against HBM, the cache plus the kept values)."""
     B, Hq, Hkv, d, T = w.B, w.Hq, w.Hkv, w.d, w.T
     qo = torch.from_numpy(synth.make_observation_queries(w, L, A2_OBS)).to(q.device).to(dt)
     K = max(1, int(A2_KEEP * T))
