@@ -655,24 +655,26 @@ bool kl_hm_supported(const headq_cache& c, int G, bool kv_bf16) {
 // Splits for one CTA per SM: chunks a multiple of the tile (112 tokens), the
 // count chosen so the grid fills whole waves best (ties: fewer splits).
 SplitPlan kl_hm_plan(int units, int T) {
+  // One CTA per SM.  The split count minimises waves x (tiles per CTA +
+  // kTileOverhead), the 2 standing for a CTA's fixed cost (query and U_h
+  // preparation, the fp64 merge and partial store); ties go to fewer splits.
+  constexpr long long kTileOverhead = 2;
   SplitPlan best{1, (T + kTile - 1) / kTile * kTile};
   if (units <= 0 || T <= 0) return best;
   const long long slots = sm_count();
-  double best_eff = -1.0;
+  long long best_cost = -1;
   const int max_s = (T + kTile - 1) / kTile;
   for (int s = 1; s <= max_s && s <= 256; ++s) {
     int chunk = (T + s - 1) / s;
     chunk = (chunk + kTile - 1) / kTile * kTile;
     const int sp = (T + chunk - 1) / chunk;
     if (sp != s) continue;
-    const long long ctas = static_cast<long long>(units) * sp;
-    const long long waves = (ctas + slots - 1) / slots;
-    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
+    const long long waves = (static_cast<long long>(units) * sp + slots - 1) / slots;
+    const long long cost = waves * (chunk / kTile + kTileOverhead);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
       best = SplitPlan{sp, chunk};
     }
-    if (ctas >= 16 * slots) break;  // deep enough: the tail is small
   }
   return best;
 }
