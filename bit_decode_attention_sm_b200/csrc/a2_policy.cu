@@ -745,35 +745,78 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
       dst[1] = make_float4(dv[4], dv[5], dv[6], dv[7]);
     }
     __syncthreads();
-    // weights exp(s^_j - lse) of the kept tokens, per head, from shared memory
-    for (int pr = tid; pr < kFixTok * G; pr += kFixThreads) {
-      const int tt = pr / G, h = pr - tt * G;
-      float w = 0.0f;
-      if (idx_s[tt] >= 0) {
-        const uint32_t* cw = kc_s + tt * FS::kKcWords;
-        const float* qh = q_s + h * D;
-        float s = 0.0f;
+    // weights exp(s^_j - lse) of the kept tokens, per head.  D >= 16: kFP lanes
+    // per token (aligned in a warp), each with one 16-channel slice (inside one
+    // group) for every head and every kFP-th side row; the slices are summed by
+    // shuffles.  d = 8: one lane per (token, head).
+    if constexpr (D >= 16) {
+      constexpr int kFP = D / 16;                  // lanes per token, a power of two <= 16
+      constexpr int kTPP = kFixThreads / kFP;      // tokens per pass
+      const int part = tid % kFP, c0 = 16 * part, g = c0 / GS;
+      const bool first_of_group = (c0 % GS) == 0;
+      for (int tt = tid / kFP; tt < kFixTok; tt += kTPP) {
+        const bool live = idx_s[tt] >= 0;
+        const uint32_t cw = kc_s[tt * FS::kKcWords + part];
+        float code[16];
 #pragma unroll
-        for (int g = 0; g < NG; ++g) {
+        for (int k = 0; k < 16; ++k) code[k] = static_cast<float>((cw >> (2 * k)) & 3u);
+        const float ksc = ks_s[tt * NG + g], kmn = km_s[tt * NG + g];
+        const float zs = r > 0 ? zs_s[tt] : 0.0f;  // (not staged without a side code)
+        const uint8_t* zr = zc_s + tt * FS::kZcBytes;
+        for (int h = 0; h < G; ++h) {
+          const float4* qh = reinterpret_cast<const float4*>(q_s + h * D + c0);
           float pg = 0.0f;
 #pragma unroll
-          for (int c = 0; c < GS; ++c) {
-            const int ch = g * GS + c;
-            const uint32_t code = (cw[ch >> 4] >> (2 * (ch & 15))) & 3u;
-            pg = fmaf(qh[ch], static_cast<float>(code), pg);
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const float4 qv = qh[k4];
+            pg = fmaf(qv.x, code[4 * k4], pg);
+            pg = fmaf(qv.y, code[4 * k4 + 1], pg);
+            pg = fmaf(qv.z, code[4 * k4 + 2], pg);
+            pg = fmaf(qv.w, code[4 * k4 + 3], pg);
           }
-          s = fmaf(km_s[tt * NG + g], qg_s[h * NG + g], s);
-          s = fmaf(ks_s[tt * NG + g], pg, s);
+          float sp = ksc * pg;
+          if (first_of_group) sp = fmaf(kmn, qg_s[h * NG + g], sp);
+          if (r > 0) {
+            float cz = 0.0f;
+            for (int i = part; i < r; i += kFP)
+              cz = fmaf(qt_s[h * r + i], static_cast<float>(nibble(zr, i)), cz);
+            sp = fmaf(zs, cz, sp);
+          }
+#pragma unroll
+          for (int o2 = 1; o2 < kFP; o2 <<= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o2);
+          if (part == 0) p_s[tt * G + h] = live ? expf(sp * p.sm_scale - lse_s[h]) : 0.0f;
         }
-        if (r > 0) {
-          const uint8_t* zr = zc_s + tt * FS::kZcBytes;
-          float cz = 0.0f;
-          for (int i = 0; i < r; ++i) cz = fmaf(qt_s[h * r + i], static_cast<float>(nibble(zr, i)), cz);
-          s = fmaf(zs_s[tt], cz, s);
-        }
-        w = expf(s * p.sm_scale - lse_s[h]);
       }
-      p_s[tt * G + h] = w;
+    } else {
+      for (int pr = tid; pr < kFixTok * G; pr += kFixThreads) {
+        const int tt = pr / G, h = pr - tt * G;
+        float w = 0.0f;
+        if (idx_s[tt] >= 0) {
+          const uint32_t* cw = kc_s + tt * FS::kKcWords;
+          const float* qh = q_s + h * D;
+          float s = 0.0f;
+#pragma unroll
+          for (int g = 0; g < NG; ++g) {
+            float pg = 0.0f;
+#pragma unroll
+            for (int c = 0; c < GS; ++c) {
+              const int ch = g * GS + c;
+              const uint32_t code = (cw[ch >> 4] >> (2 * (ch & 15))) & 3u;
+              pg = fmaf(qh[ch], static_cast<float>(code), pg);
+            }
+            s = fmaf(km_s[tt * NG + g], qg_s[h * NG + g], s);
+            s = fmaf(ks_s[tt * NG + g], pg, s);
+          }
+          if (r > 0) {
+            const uint8_t* zr = zc_s + tt * FS::kZcBytes;
+            float cz = 0.0f;
+            for (int i = 0; i < r; ++i) cz = fmaf(qt_s[h * r + i], static_cast<float>(nibble(zr, i)), cz);
+            s = fmaf(zs_s[tt], cz, s);
+          }
+          w = expf(s * p.sm_scale - lse_s[h]);
+        }
+        p_s[tt * G + h] = w;
+      }
     }
     __syncthreads();
 #pragma unroll

@@ -216,8 +216,29 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     // already in flight.
     bool ok = true;
     int issued = 0;
+    // Appending: this warp encodes the new token once the first stages are in
+    // flight (or before the tile holding it, if that comes sooner), so the
+    // codec's latency overlaps the consumers' first tiles; the tile holding the
+    // token is copied only after the encoded planes are published.
+    const int enc_i = (pos >= t_begin && pos < tile_end) ? min((pos - t_begin) / kTile, kStages)
+                                                         : -1;
     for (int i = 0;; ++i) {
       const int s = i % kStages, use = i / kStages;
+      if (i == enc_i) {
+        // dense values read U_h from shared memory (bulk-copied with the
+        // query); 2-bit values, which keep no copy there, from global memory
+        if (!V2 && !mbar_wait(smem_addr(&bars[2 * kStages + 1]), 0) && lane == 0 && p.err)
+          atomicOr(p.err, kDevErrWaitTimeout);
+        encode_new_token<D, R, V2>(p, b, kv, pos,
+                                   V2 ? p.U + static_cast<size_t>(kv) * D * R : u_s, enew_s,
+                                   lane);
+        // publish the token's planes to the bulk copies (async proxy): every
+        // lane's writes, then the issuing lane
+        __threadfence();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
       int t0 = -1;
       if (lane == 0) {
         if (use > 0 && !mbar_wait(smem_addr(&bars[kStages + s]), (use - 1) & 1)) ok = false;
@@ -226,20 +247,6 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
       ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
       t0 = __shfl_sync(kFull, t0, 0);
       if (!ok) break;
-      if (t0 >= 0 && pos >= t0 && pos < t0 + kTile) {
-        // this tile holds the new token: encode it (U_h must be in shared
-        // memory), then publish it to the bulk copies (async proxy)
-        if (!mbar_wait(smem_addr(&bars[2 * kStages + 1]), 0) && lane == 0 && p.err)
-          atomicOr(p.err, kDevErrWaitTimeout);
-        encode_new_token<D, R, V2>(p, b, kv, pos,
-                                   V2 ? p.U + static_cast<size_t>(kv) * D * R : u_s, enew_s,
-                                   lane);
-        __threadfence();
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        __syncwarp();
-        // the issuing lane orders every lane's writes before its bulk copies
-        if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");
-      }
       if (lane == 0) {
         stile_s[s] = t0;
         const uint32_t full = smem_addr(&bars[s]);
