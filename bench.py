@@ -584,7 +584,7 @@ def run_headq(args):
     alg_bytes = B * Hkv * T * bytes_tok
     peak, peak_kind = measured_hbm_peak()
     achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
-    traffic = (recorded_traffic(["decode_mma.cu", "decode_common.cuh", "codec.cuh"],
+    traffic = (recorded_traffic(["decode_mma.cu", "decode_pipe.cuh", "decode_common.cuh", "codec.cuh"],
                                 "decode_mma_longctx.md")
                if w.name == DEFAULT_WORKLOAD else None)
     cpu = None

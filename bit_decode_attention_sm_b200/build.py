@@ -26,7 +26,7 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libheadq.so")
 
 SOURCES = ["headq_api.cu", "cache_write.cu", "decode_attn.cu", "attn_kl.cu",
-           "calibrate.cu", "decode_noalloc.cu", "decode_mma.cu", "attn_kl_hm.cu", "merge.cu",
+           "calibrate.cu", "decode_noalloc.cu", "decode_mma.cu", "decode_hm.cu", "attn_kl_hm.cu", "merge.cu",
            "a2_policy.cu"]
 PER_FILE_FLAGS = {"cache_write.cu": ["-fmad=false"]}
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -40,7 +40,7 @@
 #include <mutex>
 
 #include "codec.cuh"
-#include "decode_common.cuh"
+#include "decode_pipe.cuh"
 #include "headq_internal.cuh"
 
 namespace headq {
@@ -48,7 +48,7 @@ namespace {
 using namespace dc;
 
 constexpr int kCW = 4;                   // consumer warps
-constexpr int kTile = 16 * kCW;          // tokens per stage
+constexpr int kTile = kPipeTile;         // tokens per stage (16 per consumer warp)
 constexpr int kThreads = (kCW + 1) * 32; // + one producer warp
 // pipeline depth: 4 stages of 64 tokens, 3 for the two-N-tile variants (their
 // q fragments take the shared memory of the fourth) so that two CTAs fit per SM
@@ -60,29 +60,10 @@ constexpr float kRescale = 8.0f;         // log2 units the stale max may lag (p 
 // 2^kRaiseLog2 of it (fp16 holds up to 2^16).
 constexpr int kRaiseLog2 = 12;
 
-// Shared-memory stage of kTile tokens.  Dense bf16 values (V2 = false): the
-// swizzled value boxes come first.  2-bit values (V2 = true): their code, scale
-// and minimum planes are bulk-copied like the keys'.  Per-channel keys (KCH):
-// the tile is one 64-token block, whose scale and minimum rows (d floats each)
-// take the place of the per-token key scale and minimum planes.
+// Shared-memory stage of kTile tokens (StageLayout), plus this kernel's
+// per-warp scratch for 2-bit values.
 template <int D, int R, bool V2 = false, bool KCH = false>
-struct Layout {
-  static constexpr int NG = D / 32;
-  static constexpr int kVBoxes = V2 ? 0 : D / 64;    // 64-dim boxes per token row
-  static constexpr int kVBox = kTile * 128;          // 64 tokens x 128 bytes
-  static constexpr int kKc = kVBoxes * kVBox;
-  static constexpr int kKs = kKc + kTile * (D / 4);
-  static constexpr int kKm = kKs + kTile * NG * 4;
-  static constexpr int kZc = kKm + kTile * NG * 4;
-  static constexpr int kZs = kZc + kTile * (R / 2);
-  static constexpr int kVc = kZs + (R > 0 ? kTile * 4 : 0);
-  static constexpr int kVs = kVc + (V2 ? kTile * (D / 4) : 0);
-  static constexpr int kVm = kVs + (V2 ? kTile * NG * 4 : 0);
-  static constexpr int kEnd = kVm + (V2 ? kTile * NG * 4 : 0);
-  static constexpr int kStage = (kEnd + 1023) / 1024 * 1024;
-  static constexpr int kRowBytes =
-      D / 4 + (KCH ? 0 : 8 * NG) + (R > 0 ? R / 2 + 4 : 0) + (V2 ? D / 4 + 8 * NG : 0);
-  static constexpr int kTileBytes = KCH ? 2 * D * 4 : 0;  // bytes per tile, besides the rows
+struct Layout : StageLayout<D, R, V2, KCH> {
   // 2-bit values: per consumer warp, the fp16 codes of its D/4 channels for the
   // kTile tokens of a stage (the warp's readout slice)
   static constexpr int kCodeTile = V2 ? kTile * (D / kCW) * 2 : 0;
@@ -92,7 +73,6 @@ struct Layout {
   // readout warps
   static constexpr int kPexFloats = 2 * kCW * 8 * 24;
   static constexpr int kExBytes = V2 ? (kPexFloats + 2 * 8 * kCW) * 4 : 0;
-  static_assert(!KCH || D * 4 <= kTile * NG * 4, "a block row fits the per-token plane space");
 };
 
 // the two-N-tile variants keep each thread's q B-operand fragments in shared
@@ -197,103 +177,12 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   // ------------------------------------------------------------ producer warp
   // starts streaming at once; the consumers prepare the query meanwhile
   if (warp == kCW) {
-    if (lane == 0) {
-      // the query and U_h first: they head the copy queue, so the consumers'
-      // preparation does not wait behind the cache stream
-      const uint32_t qbar = smem_addr(&bars[2 * kStages + 1]);
-      const uint32_t qbytes = static_cast<uint32_t>(G * D * (p.q_bf16 ? 2 : 4));
-      mbar_expect_tx(qbar, qbytes + (R > 0 ? D * R * 4 : 0));
-      bulk_g2s(smem_addr(qraw_s),
-               static_cast<const uint8_t*>(p.q) +
-                   (static_cast<size_t>(b) * p.Hq + h0) * D * (p.q_bf16 ? 2 : 4),
-               qbytes, qbar);
-      if constexpr (R > 0)
-        bulk_g2s(smem_addr(u_s), p.U + static_cast<size_t>(kv) * D * R, D * R * 4, qbar);
-    }
-    // The tiles of this CTA's chunk in order, one per stage, then an end marker.
-    // Appending: before issuing the tile that holds the new token (the chunk's
-    // last) this warp encodes the token, while the consumers drain the stages
-    // already in flight.
-    bool ok = true;
-    int issued = 0;
-    // Appending: this warp encodes the new token once the first stages are in
-    // flight (or before the tile holding it, if that comes sooner), so the
-    // codec's latency overlaps the consumers' first tiles; the tile holding the
-    // token is copied only after the encoded planes are published.
-    const int enc_i = (pos >= t_begin && pos < tile_end) ? min((pos - t_begin) / kTile, kStages)
-                                                         : -1;
-    for (int i = 0;; ++i) {
-      const int s = i % kStages, use = i / kStages;
-      if (i == enc_i) {
-        // dense values read U_h from shared memory (bulk-copied with the
-        // query); 2-bit values, which keep no copy there, from global memory
-        if (!V2 && !mbar_wait(smem_addr(&bars[2 * kStages + 1]), 0) && lane == 0 && p.err)
-          atomicOr(p.err, kDevErrWaitTimeout);
-        encode_new_token<D, R, V2>(p, b, kv, pos,
-                                   V2 ? p.U + static_cast<size_t>(kv) * D * R : u_s, enew_s,
-                                   lane);
-        // publish the token's planes to the bulk copies (async proxy): every
-        // lane's writes, then the issuing lane
-        __threadfence();
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");
-      }
-      int t0 = -1;
-      if (lane == 0) {
-        if (use > 0 && !mbar_wait(smem_addr(&bars[kStages + s]), (use - 1) & 1)) ok = false;
-        if (ok && i < ntiles) t0 = t_begin + i * kTile;
-      }
-      ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
-      t0 = __shfl_sync(kFull, t0, 0);
-      if (!ok) break;
-      if (lane == 0) {
-        stile_s[s] = t0;
-        const uint32_t full = smem_addr(&bars[s]);
-        if (t0 < 0) {
-          mbar_arrive(full);  // no more tiles: the consumers stop at this stage
-        } else {
-          const int n16 = (min(kTile, tile_end - t0) + 15) & ~15;
-          mbar_expect_tx(full, L::kVBoxes * L::kVBox + n16 * L::kRowBytes + L::kTileBytes);
-          uint8_t* st = stages + size_t(s) * L::kStage;
-          const CacheSlab sl = cache_slab_read(p.c, b, kv, t0, p.err);
-          const size_t row0 = static_cast<size_t>(sl.slab) * slab_rows(p.c) + sl.off;
-          bulk_g2s(smem_addr(st + L::kKc), p.c.k_codes + row0 * (D / 4), n16 * (D / 4), full);
-          if constexpr (KCH) {  // the tile is one block: its scale and minimum rows
-            const size_t brow = row0 / kTile;
-            bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + brow * D, D * 4, full);
-            bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + brow * D, D * 4, full);
-          } else {
-            bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + row0 * NG, n16 * NG * 4, full);
-            bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + row0 * NG, n16 * NG * 4, full);
-          }
-          if constexpr (R > 0) {
-            bulk_g2s(smem_addr(st + L::kZc), p.c.z_codes + row0 * (R / 2), n16 * (R / 2), full);
-            bulk_g2s(smem_addr(st + L::kZs), p.c.z_scale + row0, n16 * 4, full);
-          }
-          if constexpr (V2) {
-            bulk_g2s(smem_addr(st + L::kVc), p.c.v_codes + row0 * (D / 4), n16 * (D / 4), full);
-            bulk_g2s(smem_addr(st + L::kVs), p.c.v_scale + row0 * NG, n16 * NG * 4, full);
-            bulk_g2s(smem_addr(st + L::kVm), p.c.v_min + row0 * NG, n16 * NG * 4, full);
-          } else {
-#pragma unroll
-            for (int bx = 0; bx < L::kVBoxes; ++bx)
-              tma_3d(smem_addr(st + bx * L::kVBox), &vmap, bx * 64, sl.off, static_cast<int>(sl.slab),
-                     full);
-          }
-        }
-        ++issued;
-      }
-      if (t0 < 0) break;
-    }
-    if (lane == 0) {
-      if (!ok && p.err) atomicOr(p.err, kDevErrWaitTimeout);
-      // never leave with copies in flight: wait (bounded) for the last use of each stage
-      for (int s = 0; s < kStages && s < issued; ++s) {
-        const int last_use = (issued - 1 - s) / kStages;
-        mbar_wait(smem_addr(&bars[s]), last_use & 1);
-      }
-    }
+    // 2-bit values reuse u_s (in the code tiles) once the main loop starts: the
+    // fused append's encoder reads U_h from global memory
+    produce_tiles<D, R, V2, KCH, kStages, !V2>(p, &vmap, stages, bars, bars + kStages,
+                                               bars + 2 * kStages + 1, stile_s, qraw_s, u_s,
+                                               enew_s, b, kv, h0, t_begin, tile_end, ntiles,
+                                               pos, lane);
     return;
   }
 
@@ -896,87 +785,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   if (!flags[1]) return;
   __threadfence();
-  const int S = p.splits;
-  float* w_s = reinterpret_cast<float*>(flags + 4);  // [G][S] split weights, past the flags
-  // One warp per head, no CTA barrier, few round trips to L2: the first issues
-  // the (m, l) of the splits (lane-strided) together with the partial outputs
-  // of the first kMR splits (lane = 4 output dims); while those are in flight
-  // the warp reduces the maximum and writes the split weights w_s to shared
-  // memory; further rounds load the remaining splits' outputs.
-  constexpr int kSPL = 4;   // splits per lane held in registers (S <= 128)
-  constexpr int kMR = 16;   // splits per round of output loads
-  for (int h = warp; h < G; h += kCW) {
-    const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
-    const bool has_c4 = lane < D / 4;
-    const float4* po = reinterpret_cast<const float4*>(pv.o + bh * S * D) + lane;
-    float4 v[kMR];
-#pragma unroll
-    for (int u = 0; u < kMR; ++u)
-      v[u] = (has_c4 && u < S) ? __ldcg(po + u * (D / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    float mv[kSPL], lv[kSPL];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < kSPL; ++k) {
-      const int sI = lane + 32 * k;
-      mv[k] = -INFINITY;
-      lv[k] = 0.f;
-      if (sI < S) {
-        mv[k] = __ldcg(pv.m + bh * S + sI);
-        lv[k] = __ldcg(pv.l + bh * S + sI);
-      }
-      mx = fmaxf(mx, mv[k]);
-    }
-    for (int sI = lane + 32 * kSPL; sI < S; sI += 32) mx = fmaxf(mx, __ldcg(pv.m + bh * S + sI));
-#pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o2));
-    float ls = 0.f;
-    float* w = w_s + h * S;
-#pragma unroll
-    for (int k = 0; k < kSPL; ++k) {
-      const int sI = lane + 32 * k;
-      if (sI < S) {
-        const float wk = mv[k] > -INFINITY ? expf(mv[k] - mx) : 0.f;
-        w[sI] = wk;
-        ls = fmaf(wk, lv[k], ls);
-      }
-    }
-    for (int sI = lane + 32 * kSPL; sI < S; sI += 32) {
-      const float m = __ldcg(pv.m + bh * S + sI);
-      const float wk = m > -INFINITY ? expf(m - mx) : 0.f;
-      w[sI] = wk;
-      ls = fmaf(wk, __ldcg(pv.l + bh * S + sI), ls);
-    }
-    for (int o2 = 16; o2 > 0; o2 >>= 1) ls += __shfl_xor_sync(kFull, ls, o2);
-    __syncwarp();
-    float4 acc[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0;;) {
-#pragma unroll
-      for (int u = 0; u < kMR; ++u) {
-        const float wu = s0 + u < S ? w[s0 + u] : 0.f;
-        float4& a4 = acc[u & 3];
-        a4.x = fmaf(wu, v[u].x, a4.x); a4.y = fmaf(wu, v[u].y, a4.y);
-        a4.z = fmaf(wu, v[u].z, a4.z); a4.w = fmaf(wu, v[u].w, a4.w);
-      }
-      s0 += kMR;
-      if (s0 >= S) break;
-#pragma unroll
-      for (int u = 0; u < kMR; ++u)
-        v[u] = (has_c4 && s0 + u < S) ? __ldcg(po + (s0 + u) * (D / 4))
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    const float inv = ls > 0.f ? 1.0f / ls : 0.f;
-    if (has_c4) {
-      float4 r;
-      r.x = ((acc[0].x + acc[1].x) + (acc[2].x + acc[3].x)) * inv;
-      r.y = ((acc[0].y + acc[1].y) + (acc[2].y + acc[3].y)) * inv;
-      r.z = ((acc[0].z + acc[1].z) + (acc[2].z + acc[3].z)) * inv;
-      r.w = ((acc[0].w + acc[1].w) + (acc[2].w + acc[3].w)) * inv;
-      reinterpret_cast<float4*>(p.out + bh * D)[lane] = r;
-    }
-    if (lane == 0 && p.lse) p.lse[bh] = ls > 0.f ? mx + logf(ls) : -INFINITY;
-  }
+  merge_splits_last<D>(p, b, h0, reinterpret_cast<float*>(flags + 4), warp, kCW, lane);
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   if (tid == 0) p.counters[bk] = 0;  // ready for the next call
 }
@@ -1044,20 +853,17 @@ auto dispatch(int d, int r, int G, bool v2, bool kch, F&& f)
 #define HEADQ_MMA_CASE(DD, RR, NN, VV, KK) \
   if (d == DD && r == RR && nt == NN && v2 == VV && kch == KK) \
     return f(Variant<DD, RR, NN, VV, KK>{});
-#define HEADQ_MMA_CASES(KK)                                                         \
-  HEADQ_MMA_CASE(128, 16, 1, false, KK) HEADQ_MMA_CASE(128, 16, 2, false, KK)       \
-  HEADQ_MMA_CASE(128, 8, 1, false, KK) HEADQ_MMA_CASE(128, 8, 2, false, KK)         \
-  HEADQ_MMA_CASE(128, 0, 1, false, KK) HEADQ_MMA_CASE(128, 0, 2, false, KK)         \
-  HEADQ_MMA_CASE(64, 16, 1, false, KK) HEADQ_MMA_CASE(64, 16, 2, false, KK)         \
-  HEADQ_MMA_CASE(64, 8, 1, false, KK) HEADQ_MMA_CASE(64, 8, 2, false, KK)           \
-  HEADQ_MMA_CASE(64, 0, 1, false, KK) HEADQ_MMA_CASE(64, 0, 2, false, KK)           \
-  HEADQ_MMA_CASE(128, 16, 1, true, KK) HEADQ_MMA_CASE(128, 16, 2, true, KK)         \
-  HEADQ_MMA_CASE(128, 8, 1, true, KK) HEADQ_MMA_CASE(128, 8, 2, true, KK)           \
-  HEADQ_MMA_CASE(64, 16, 1, true, KK) HEADQ_MMA_CASE(64, 16, 2, true, KK)           \
-  HEADQ_MMA_CASE(64, 8, 1, true, KK) HEADQ_MMA_CASE(64, 8, 2, true, KK)
-  HEADQ_MMA_CASES(false)
-  HEADQ_MMA_CASES(true)
-#undef HEADQ_MMA_CASES
+// per-token keys with G > 4 run in decode_hm.cu: only one N-tile here
+#define HEADQ_MMA_CASES_NT(NN, KK)                                               \
+  HEADQ_MMA_CASE(128, 16, NN, false, KK) HEADQ_MMA_CASE(128, 8, NN, false, KK)   \
+  HEADQ_MMA_CASE(128, 0, NN, false, KK) HEADQ_MMA_CASE(64, 16, NN, false, KK)    \
+  HEADQ_MMA_CASE(64, 8, NN, false, KK) HEADQ_MMA_CASE(64, 0, NN, false, KK)      \
+  HEADQ_MMA_CASE(128, 16, NN, true, KK) HEADQ_MMA_CASE(128, 8, NN, true, KK)     \
+  HEADQ_MMA_CASE(64, 16, NN, true, KK) HEADQ_MMA_CASE(64, 8, NN, true, KK)
+  HEADQ_MMA_CASES_NT(1, false)
+  HEADQ_MMA_CASES_NT(1, true)
+  HEADQ_MMA_CASES_NT(2, true)
+#undef HEADQ_MMA_CASES_NT
 #undef HEADQ_MMA_CASE
   return decltype(f(Variant<128, 16, 1, false, false>{}))();
 }
@@ -1076,11 +882,13 @@ bool mma_decode_supported(const headq_cache& c, int G) {
 }
 
 int mma_decode_ctas_per_sm(const headq_cache& c, int G) {
+  if (hm_decode_supported(c, G)) return hm_decode_ctas_per_sm(c);
   return dispatch(c.d, c.r, G, is_v2(c), c.kmode == HEADQ_K_CHANNEL,
                   [](auto v) { return decltype(v)::ctas_per_sm(); });
 }
 
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s) {
+  if (hm_decode_supported(p.c, p.G)) return launch_decode_hm(p, s);
   // 0 means no variant matched; otherwise the launch status + 1
   const int e = dispatch(p.c.d, p.c.r, p.G, is_v2(p.c), p.c.kmode == HEADQ_K_CHANNEL, [&](auto v) {
     return static_cast<int>(decltype(v)::launch(p, s)) + 1;

@@ -232,6 +232,11 @@ constexpr int kMaxMmaSplits = 1024;  // the merging CTA keeps per-split weights 
 bool mma_decode_supported(const headq_cache& c, int G);
 int mma_decode_ctas_per_sm(const headq_cache& c, int G);
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t s);
+// the tensor-core kernel for 5..8 query heads per KV head with per-token keys
+// (decode_hm.cu); launch_decode_mma and mma_decode_ctas_per_sm route to it
+bool hm_decode_supported(const headq_cache& c, int G);
+int hm_decode_ctas_per_sm(const headq_cache& c);
+cudaError_t launch_decode_hm(const DecodeParams& p, cudaStream_t s);
 
 
 }  // namespace headq
