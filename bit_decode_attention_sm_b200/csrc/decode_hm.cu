@@ -142,7 +142,6 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
   if (p.seq_lens) Tb = max(0, min(p.seq_lens[b], p.T));
   const int t_begin = split * p.chunk;
   const int tile_end = min(Tb, t_begin + p.chunk);
-  const int ntiles = tile_end > t_begin ? (tile_end - t_begin + kTile - 1) / kTile : 0;
   const size_t bk = static_cast<size_t>(b) * Hkv + kv;
   const int h0 = kv * G;
   const int pos = (p.k_new != nullptr && Tb > 0) ? Tb - 1 : -1;
@@ -160,8 +159,7 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
   if (warp == kCW) {
     produce_tiles<D, R, V2, false, kStages, true>(p, &vmap, stages, bars, bars + kStages,
                                                   bars + 2 * kStages, stile_s, qraw_s, u_s,
-                                                  enew_s, b, kv, h0, t_begin, tile_end,
-                                                  ntiles, pos, lane);
+                                                  enew_s, b, kv, t_begin, tile_end, pos, lane);
     return;
   }
 
@@ -187,10 +185,12 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
   if constexpr (R > 0) {
     for (int i = tid; i < kGM * R; i += kCT) {
       const int h = i / R, ii = i - h * R;
-      float acc = 0.0f;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll 8
-      for (int c = 0; c < D; ++c) acc = fmaf(u_s[c * R + ii], q_s[h * D + c], acc);
-      qt_s[i] = p.corr_sign * acc;
+      for (int c = 0; c < D; c += 4)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[k] = fmaf(u_s[(c + k) * R + ii], q_s[h * D + c + k], acc[k]);
+      qt_s[i] = p.corr_sign * ((acc[0] + acc[1]) + (acc[2] + acc[3]));
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
@@ -398,8 +398,25 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
       float vs[4][NG];
 #pragma unroll
       for (int k = 0; k < 4; ++k) load_groups<NG>(st + L::kVs + jr[k] * NG * 4, vs[k]);
+      // A operands of p . V: this thread's code byte (channels 32 gg + 4 g .. + 3)
+      // of its four tokens, paired by token and split into two row blocks
+      uint32_t aa[NG][4], ab[NG][4];
+#pragma unroll
+      for (int gg = 0; gg < NG; ++gg) {
+        const uint8_t* vc = st + L::kVc + 8 * gg + 4 * (g >> 2);
+        const uint32_t c0 = *reinterpret_cast<const uint32_t*>(vc + jr[0] * (D / 4));
+        const uint32_t c1 = *reinterpret_cast<const uint32_t*>(vc + jr[1] * (D / 4));
+        const uint32_t c2 = *reinterpret_cast<const uint32_t*>(vc + jr[2] * (D / 4));
+        const uint32_t c3 = *reinterpret_cast<const uint32_t*>(vc + jr[3] * (D / 4));
+        const uint32_t z01 = __byte_perm(c0, c1, vsel), z23 = __byte_perm(c2, c3, vsel);
+        aa[gg][0] = z01 & 0x00030003u; aa[gg][1] = z01 & 0x000C000Cu;
+        aa[gg][2] = z23 & 0x00030003u; aa[gg][3] = z23 & 0x000C000Cu;
+        ab[gg][0] = z01 & 0x00300030u; ab[gg][1] = z01 & 0x00C000C0u;
+        ab[gg][2] = z23 & 0x00300030u; ab[gg][3] = z23 & 0x00C000C0u;
+      }
       // B entries p_j scale_{j,g} of head g; their largest in the 16 tokens
       // (the quad's lanes) decides whether 2^E of (head g, group g) is raised
+      // (branch-free: a raise is rare, but keeps the block one basic block)
       float w[NG][4];
       float rf[NG];
       bool raise = false;
@@ -410,24 +427,25 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
         float hx = fmaxf(fmaxf(w[gg][0], w[gg][1]), fmaxf(w[gg][2], w[gg][3]));
         hx = fmaxf(hx, __shfl_xor_sync(kFull, hx, 1));
         hx = fmaxf(hx, __shfl_xor_sync(kFull, hx, 2));
-        rf[gg] = alpha;
         const uint32_t hb = __float_as_uint(hx);
-        if (hb >= static_cast<uint32_t>(127 + ve[gg] + kRaiseLog2) << 23) {
-          const int en = max(-126, min(126, static_cast<int>(hb >> 23) - 127));
-          rf[gg] *= pow2_neg(-ve[gg]) * pow2_neg(en);  // 2^(E_old - E_new)
-          ve[gg] = en;
-          raise = true;
-        }
+        const bool up = hb >= static_cast<uint32_t>(127 + ve[gg] + kRaiseLog2) << 23;
+        const int en = max(-126, min(126, static_cast<int>(hb >> 23) - 127));
+        // 2^(E_old - E_new) on a raise
+        rf[gg] = up ? alpha * (pow2_neg(-ve[gg]) * pow2_neg(en)) : alpha;
+        ve[gg] = up ? en : ve[gg];
+        raise |= up;
       }
+      {
+        float vm[4][NG];
 #pragma unroll
-      for (int gg = 0; gg < NG; ++gg) {
-        float a = vmin[gg] * alpha;
+        for (int k = 0; k < 4; ++k) load_groups<NG>(st + L::kVm + jr[k] * NG * 4, vm[k]);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float vmk = reinterpret_cast<const float*>(st + L::kVm)[jr[k] * NG + gg];
-          a = fmaf(pr[k], vmk, a);
+        for (int gg = 0; gg < NG; ++gg) {
+          float a = vmin[gg] * alpha;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) a = fmaf(pr[k], vm[k][gg], a);
+          vmin[gg] = a;
         }
-        vmin[gg] = a;
       }
       if (__any_sync(kFull, resc || raise)) {
         // output columns = head slots 2t, 2t+1: their factors live in lanes 8t, 8t+4
@@ -444,18 +462,8 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
         const float fe = pow2_neg(ve[gg]);
         const uint32_t bv[2] = {f16x2(w[gg][0] * fe, w[gg][1] * fe),
                                 f16x2(w[gg][2] * fe, w[gg][3] * fe)};
-        const uint8_t* vc = st + L::kVc + 8 * gg + 4 * (g >> 2);
-        const uint32_t c0 = *reinterpret_cast<const uint32_t*>(vc + jr[0] * (D / 4));
-        const uint32_t c1 = *reinterpret_cast<const uint32_t*>(vc + jr[1] * (D / 4));
-        const uint32_t c2 = *reinterpret_cast<const uint32_t*>(vc + jr[2] * (D / 4));
-        const uint32_t c3 = *reinterpret_cast<const uint32_t*>(vc + jr[3] * (D / 4));
-        const uint32_t z01 = __byte_perm(c0, c1, vsel), z23 = __byte_perm(c2, c3, vsel);
-        const uint32_t aa[4] = {z01 & 0x00030003u, z01 & 0x000C000Cu, z23 & 0x00030003u,
-                                z23 & 0x000C000Cu};
-        const uint32_t ab[4] = {z01 & 0x00300030u, z01 & 0x00C000C0u, z23 & 0x00300030u,
-                                z23 & 0x00C000C0u};
-        mma_f16(oa[gg], aa, bv);
-        mma_f16(ob[gg], ab, bv);
+        mma_f16(oa[gg], aa[gg], bv);
+        mma_f16(ob[gg], ab[gg], bv);
       }
     } else {
       if (__any_sync(kFull, resc)) {
@@ -588,7 +596,7 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
   if (!flags[1]) return;
   __threadfence();
   // the split weights overwrite the (consumed) warp partials
-  merge_splits_last<D>(p, b, h0, reinterpret_cast<float*>(stages), warp, kCW, lane);
+  merge_splits_last<D>(p, b, h0, p.splits, reinterpret_cast<float*>(stages), warp, kCW, lane);
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   if (tid == 0) p.counters[bk] = 0;  // ready for the next call
 }
