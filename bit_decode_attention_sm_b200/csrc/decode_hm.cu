@@ -142,6 +142,7 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
   if (p.seq_lens) Tb = max(0, min(p.seq_lens[b], p.T));
   const int t_begin = split * p.chunk;
   const int tile_end = min(Tb, t_begin + p.chunk);
+  const int ntiles = tile_end > t_begin ? (tile_end - t_begin + kTile - 1) / kTile : 0;
   const size_t bk = static_cast<size_t>(b) * Hkv + kv;
   const int h0 = kv * G;
   const int pos = (p.k_new != nullptr && Tb > 0) ? Tb - 1 : -1;
@@ -159,7 +160,8 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
   if (warp == kCW) {
     produce_tiles<D, R, V2, false, kStages, true>(p, &vmap, stages, bars, bars + kStages,
                                                   bars + 2 * kStages, stile_s, qraw_s, u_s,
-                                                  enew_s, b, kv, t_begin, tile_end, pos, lane);
+                                                  enew_s, b, kv, h0, t_begin, tile_end,
+                                                  ntiles, pos, lane);
     return;
   }
 
@@ -596,7 +598,7 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
   if (!flags[1]) return;
   __threadfence();
   // the split weights overwrite the (consumed) warp partials
-  merge_splits_last<D>(p, b, h0, p.splits, reinterpret_cast<float*>(stages), warp, kCW, lane);
+  merge_splits_last<D>(p, b, h0, reinterpret_cast<float*>(stages), warp, kCW, lane);
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   if (tid == 0) p.counters[bk] = 0;  // ready for the next call
 }

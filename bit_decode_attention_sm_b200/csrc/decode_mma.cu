@@ -154,6 +154,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   if (p.seq_lens) Tb = max(0, min(p.seq_lens[b], p.T));
   const int t_begin = split * p.chunk;
   const int t_end = min(Tb, t_begin + p.chunk);
+  const int ntiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
   const size_t bk = static_cast<size_t>(b) * Hkv + kv;
   const int h0 = kv * G;
   // position of this step's new token (fused append), -1 when none
@@ -180,7 +181,8 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
     // fused append's encoder reads U_h from global memory
     produce_tiles<D, R, V2, KCH, kStages, !V2>(p, &vmap, stages, bars, bars + kStages,
                                                bars + 2 * kStages + 1, stile_s, qraw_s, u_s,
-                                               enew_s, b, kv, t_begin, tile_end, pos, lane);
+                                               enew_s, b, kv, h0, t_begin, tile_end, ntiles,
+                                               pos, lane);
     return;
   }
 
@@ -783,7 +785,7 @@ decode_mma_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   if (!flags[1]) return;
   __threadfence();
-  merge_splits_last<D>(p, b, h0, p.splits, reinterpret_cast<float*>(flags + 4), warp, kCW, lane);
+  merge_splits_last<D>(p, b, h0, reinterpret_cast<float*>(flags + 4), warp, kCW, lane);
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
   if (tid == 0) p.counters[bk] = 0;  // ready for the next call
 }

@@ -43,27 +43,26 @@ struct StageLayout {
   static_assert(!KCH || D * 4 <= kTile * NG * 4, "a block row fits the per-token plane space");
 };
 
-// One (b, kv) segment of a decode CTA's producer warp: bulk-copies the query
-// of the G heads of KV head kv (into qraw_s) and U_h (into u_s, when R > 0)
-// behind barrier qbar, then the tiles of [t_begin, tile_end) in order, one per
-// stage, each behind its stage's full barrier, continuing the CTA's stage
-// sequence at issue index `it`; a stage is reused once its empty barrier
-// completes (the consumers' arrivals).  stile_s[stage] receives each tile's
-// first token when stile_s is given.  When the call appends (pos inside the
-// segment), the warp encodes the new token once the first stages are in
-// flight, or before the tile holding it if that comes sooner, and publishes it
-// to the copies (async proxy) before that tile is issued; the encoder reads U_h
-// from u_s (after qbar) when kEncSmemU, else from global memory (a kernel that
-// reuses u_s once its main loop starts).  `it` counts the tiles issued so far
-// (also when a wait expired); false when a wait expired (the error word is
-// flagged).
+// The producer warp of a decode CTA.  Bulk-copies the query of the CTA's G
+// heads (into qraw_s) and U_h (into u_s, when R > 0) behind barrier qbar,
+// then the tiles of [t_begin, tile_end) in order, one per stage, each behind
+// its stage's full barrier; then an end marker (stile_s[s] = -1).  A stage is
+// reused once its empty barrier completes (the consumers' arrivals).  When the
+// call appends (pos inside the chunk), the warp encodes the new token once the
+// first stages are in flight, or before the tile holding it if that comes
+// sooner, and publishes it to the copies (async proxy) before that tile is
+// issued; the encoder reads U_h from u_s (after qbar) when kEncSmemU, else from
+// global memory (a kernel that reuses u_s once its main loop starts).  Every
+// wait is bounded; on expiry the error word is flagged and the warp stops
+// issuing, and it never leaves with copies in flight.
 template <int D, int R, bool V2, bool KCH, int kStages, bool kEncSmemU>
-__device__ __forceinline__ bool produce_segment(const DecodeParams& p, const CUtensorMap* vmap,
-                                                uint8_t* stages, uint64_t* full_bars,
-                                                uint64_t* empty_bars, uint64_t* qbar_p,
-                                                int* stile_s, float* qraw_s, float* u_s,
-                                                float* enew_s, int b, int kv, int t_begin,
-                                                int tile_end, int pos, int lane, int& it) {
+__device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUtensorMap* vmap,
+                                              uint8_t* stages, uint64_t* full_bars,
+                                              uint64_t* empty_bars, uint64_t* qbar_p,
+                                              int* stile_s, float* qraw_s, float* u_s,
+                                              float* enew_s, int b, int kv, int h0,
+                                              int t_begin, int tile_end, int ntiles, int pos,
+                                              int lane) {
   using L = StageLayout<D, R, V2, KCH>;
   constexpr int NG = L::NG;
   constexpr int kTile = L::kTile;
@@ -76,16 +75,17 @@ __device__ __forceinline__ bool produce_segment(const DecodeParams& p, const CUt
     mbar_expect_tx(qbar, qbytes + (R > 0 ? D * R * 4 : 0));
     bulk_g2s(smem_addr(qraw_s),
              static_cast<const uint8_t*>(p.q) +
-                 (static_cast<size_t>(b) * p.Hq + static_cast<size_t>(kv) * G) * D *
-                     (p.q_bf16 ? 2 : 4),
+                 (static_cast<size_t>(b) * p.Hq + h0) * D * (p.q_bf16 ? 2 : 4),
              qbytes, qbar);
     if (R > 0)
       bulk_g2s(smem_addr(u_s), p.U + static_cast<size_t>(kv) * D * R, D * R * 4, qbar);
   }
-  const int ntiles = tile_end > t_begin ? (tile_end - t_begin + kTile - 1) / kTile : 0;
+  bool ok = true;
+  int issued = 0;
   const int enc_i =
       (pos >= t_begin && pos < tile_end) ? min((pos - t_begin) / kTile, kStages) : -1;
-  for (int i = 0; i < ntiles; ++i, ++it) {
+  for (int i = 0;; ++i) {
+    const int s = i % kStages, use = i / kStages;
     if (i == enc_i) {
       if (kEncSmemU && !mbar_wait(qbar, 0) && lane == 0 && p.err)
         atomicOr(p.err, kDevErrWaitTimeout);
@@ -99,114 +99,81 @@ __device__ __forceinline__ bool produce_segment(const DecodeParams& p, const CUt
       __syncwarp();
       if (lane == 0) asm volatile("fence.proxy.async.global;" ::: "memory");
     }
-    const int s = it % kStages, use = it / kStages;
-    bool ok = true;
-    if (lane == 0 && use > 0) ok = mbar_wait(smem_addr(&empty_bars[s]), (use - 1) & 1);
-    if (__shfl_sync(kFull, ok ? 1 : 0, 0) == 0) {
-      if (lane == 0 && p.err) atomicOr(p.err, kDevErrWaitTimeout);
-      return false;
-    }
+    int t0 = -1;
     if (lane == 0) {
-      const int t0 = t_begin + i * kTile;
-      if (stile_s != nullptr) stile_s[s] = t0;
+      if (use > 0 && !mbar_wait(smem_addr(&empty_bars[s]), (use - 1) & 1)) ok = false;
+      if (ok && i < ntiles) t0 = t_begin + i * kTile;
+    }
+    ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+    t0 = __shfl_sync(kFull, t0, 0);
+    if (!ok) break;
+    if (lane == 0) {
+      stile_s[s] = t0;
       const uint32_t full = smem_addr(&full_bars[s]);
-      const int n16 = (min(kTile, tile_end - t0) + 15) & ~15;
-      mbar_expect_tx(full, L::kVBoxes * L::kVBox + n16 * L::kRowBytes + L::kTileBytes);
-      uint8_t* st = stages + size_t(s) * L::kStage;
-      const CacheSlab sl = cache_slab_read(p.c, b, kv, t0, p.err);
-      const size_t row0 = static_cast<size_t>(sl.slab) * slab_rows(p.c) + sl.off;
-      bulk_g2s(smem_addr(st + L::kKc), p.c.k_codes + row0 * (D / 4), n16 * (D / 4), full);
-      if constexpr (KCH) {  // the tile is one block: its scale and minimum rows
-        const size_t brow = row0 / kTile;
-        bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + brow * D, D * 4, full);
-        bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + brow * D, D * 4, full);
+      if (t0 < 0) {
+        mbar_arrive(full);  // no more tiles: the consumers stop at this stage
       } else {
-        bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + row0 * NG, n16 * NG * 4, full);
-        bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + row0 * NG, n16 * NG * 4, full);
-      }
-      if constexpr (R > 0) {
-        bulk_g2s(smem_addr(st + L::kZc), p.c.z_codes + row0 * (R / 2), n16 * (R / 2), full);
-        bulk_g2s(smem_addr(st + L::kZs), p.c.z_scale + row0, n16 * 4, full);
-      }
-      if constexpr (V2) {
-        bulk_g2s(smem_addr(st + L::kVc), p.c.v_codes + row0 * (D / 4), n16 * (D / 4), full);
-        bulk_g2s(smem_addr(st + L::kVs), p.c.v_scale + row0 * NG, n16 * NG * 4, full);
-        bulk_g2s(smem_addr(st + L::kVm), p.c.v_min + row0 * NG, n16 * NG * 4, full);
-      } else {
+        const int n16 = (min(kTile, tile_end - t0) + 15) & ~15;
+        mbar_expect_tx(full, L::kVBoxes * L::kVBox + n16 * L::kRowBytes + L::kTileBytes);
+        uint8_t* st = stages + size_t(s) * L::kStage;
+        const CacheSlab sl = cache_slab_read(p.c, b, kv, t0, p.err);
+        const size_t row0 = static_cast<size_t>(sl.slab) * slab_rows(p.c) + sl.off;
+        bulk_g2s(smem_addr(st + L::kKc), p.c.k_codes + row0 * (D / 4), n16 * (D / 4), full);
+        if constexpr (KCH) {  // the tile is one block: its scale and minimum rows
+          const size_t brow = row0 / kTile;
+          bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + brow * D, D * 4, full);
+          bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + brow * D, D * 4, full);
+        } else {
+          bulk_g2s(smem_addr(st + L::kKs), p.c.k_scale + row0 * NG, n16 * NG * 4, full);
+          bulk_g2s(smem_addr(st + L::kKm), p.c.k_min + row0 * NG, n16 * NG * 4, full);
+        }
+        if constexpr (R > 0) {
+          bulk_g2s(smem_addr(st + L::kZc), p.c.z_codes + row0 * (R / 2), n16 * (R / 2), full);
+          bulk_g2s(smem_addr(st + L::kZs), p.c.z_scale + row0, n16 * 4, full);
+        }
+        if constexpr (V2) {
+          bulk_g2s(smem_addr(st + L::kVc), p.c.v_codes + row0 * (D / 4), n16 * (D / 4), full);
+          bulk_g2s(smem_addr(st + L::kVs), p.c.v_scale + row0 * NG, n16 * NG * 4, full);
+          bulk_g2s(smem_addr(st + L::kVm), p.c.v_min + row0 * NG, n16 * NG * 4, full);
+        } else {
 #pragma unroll
-        for (int bx = 0; bx < L::kVBoxes; ++bx)
-          tma_3d(smem_addr(st + bx * L::kVBox), vmap, bx * 64, sl.off, static_cast<int>(sl.slab),
-                 full);
+          for (int bx = 0; bx < L::kVBoxes; ++bx)
+            tma_3d(smem_addr(st + bx * L::kVBox), vmap, bx * 64, sl.off,
+                   static_cast<int>(sl.slab), full);
+        }
       }
+      ++issued;
     }
+    if (t0 < 0) break;
   }
-  return true;
-}
-
-// The producer's last act: wait (bounded) for the last use of each of the first
-// min(issued, kStages) stages, so that the warp never leaves with copies in flight.
-template <int kStages>
-__device__ __forceinline__ void drain_stages(uint64_t* full_bars, int issued, int lane) {
-  if (lane != 0) return;
-  for (int s = 0; s < kStages && s < issued; ++s) {
-    const int last_use = (issued - 1 - s) / kStages;
-    mbar_wait(smem_addr(&full_bars[s]), last_use & 1);
-  }
-}
-
-// The producer warp of a single-chunk decode CTA: its one segment, then an end
-// marker (stile_s[stage] = -1, arrived on the stage's full barrier) that stops
-// the consumers, then the drain.  Every wait is bounded; on expiry the error
-// word is flagged and the warp stops issuing.
-template <int D, int R, bool V2, bool KCH, int kStages, bool kEncSmemU>
-__device__ __forceinline__ void produce_tiles(const DecodeParams& p, const CUtensorMap* vmap,
-                                              uint8_t* stages, uint64_t* full_bars,
-                                              uint64_t* empty_bars, uint64_t* qbar_p,
-                                              int* stile_s, float* qraw_s, float* u_s,
-                                              float* enew_s, int b, int kv, int t_begin,
-                                              int tile_end, int pos, int lane) {
-  int it = 0;
-  if (!produce_segment<D, R, V2, KCH, kStages, kEncSmemU>(p, vmap, stages, full_bars, empty_bars,
-                                                          qbar_p, stile_s, qraw_s, u_s, enew_s,
-                                                          b, kv, t_begin, tile_end, pos, lane,
-                                                          it)) {
-    drain_stages<kStages>(full_bars, it, lane);  // the consumers time out on their own
-    return;
-  }
-  const int s = it % kStages, use = it / kStages;
-  bool ok = true;
   if (lane == 0) {
-    if (use > 0) ok = mbar_wait(smem_addr(&empty_bars[s]), (use - 1) & 1);
-    if (ok) {
-      stile_s[s] = -1;
-      mbar_arrive(smem_addr(&full_bars[s]));  // no more tiles: the consumers stop here
-    } else if (p.err) {
-      atomicOr(p.err, kDevErrWaitTimeout);
+    if (!ok && p.err) atomicOr(p.err, kDevErrWaitTimeout);
+    // never leave with copies in flight: wait (bounded) for the last use of each stage
+    for (int s = 0; s < kStages && s < issued; ++s) {
+      const int last_use = (issued - 1 - s) / kStages;
+      mbar_wait(smem_addr(&full_bars[s]), last_use & 1);
     }
   }
-  ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
-  drain_stages<kStages>(full_bars, ok ? it + 1 : it, lane);
 }
 
-// The last CTA of a (b, kv) merges the S partials of its G heads (slots
-// 0..S-1 of p.splits per head) into the output (log-sum-exp combine), one warp
-// per head (warps 0..nwarps-1), no
+// The last CTA of a (b, kv) merges all p.splits partials of its G heads into
+// the output (log-sum-exp combine), one warp per head (warps 0..nwarps-1), no
 // CTA barrier, few round trips to L2: the first round issues the (m, l) of the
 // splits (lane-strided) together with the partial outputs of the first kMR
 // splits (lane = 4 output dims); while those are in flight the warp reduces
 // the maximum and writes the split weights to w_s ([G][splits] floats of
 // shared memory); further rounds load the remaining splits' outputs.
 template <int D>
-__device__ __forceinline__ void merge_splits_last(const DecodeParams& p, int b, int h0, int S,
+__device__ __forceinline__ void merge_splits_last(const DecodeParams& p, int b, int h0,
                                                   float* w_s, int warp, int nwarps, int lane) {
-  const int SP = p.splits, G = p.G;  // SP: the partial slots per head
-  const PartView pv = part_view(p.part, static_cast<size_t>(p.c.B) * p.Hq, SP, D);
+  const int S = p.splits, G = p.G;
+  const PartView pv = part_view(p.part, static_cast<size_t>(p.c.B) * p.Hq, S, D);
   constexpr int kSPL = 4;   // splits per lane held in registers (S <= 128)
   constexpr int kMR = 16;   // splits per round of output loads
   for (int h = warp; h < G; h += nwarps) {
     const size_t bh = static_cast<size_t>(b) * p.Hq + h0 + h;
     const bool has_c4 = lane < D / 4;
-    const float4* po = reinterpret_cast<const float4*>(pv.o + bh * SP * D) + lane;
+    const float4* po = reinterpret_cast<const float4*>(pv.o + bh * S * D) + lane;
     float4 v[kMR];
 #pragma unroll
     for (int u = 0; u < kMR; ++u)
@@ -219,12 +186,12 @@ __device__ __forceinline__ void merge_splits_last(const DecodeParams& p, int b, 
       mv[k] = -INFINITY;
       lv[k] = 0.f;
       if (sI < S) {
-        mv[k] = __ldcg(pv.m + bh * SP + sI);
-        lv[k] = __ldcg(pv.l + bh * SP + sI);
+        mv[k] = __ldcg(pv.m + bh * S + sI);
+        lv[k] = __ldcg(pv.l + bh * S + sI);
       }
       mx = fmaxf(mx, mv[k]);
     }
-    for (int sI = lane + 32 * kSPL; sI < S; sI += 32) mx = fmaxf(mx, __ldcg(pv.m + bh * SP + sI));
+    for (int sI = lane + 32 * kSPL; sI < S; sI += 32) mx = fmaxf(mx, __ldcg(pv.m + bh * S + sI));
 #pragma unroll
     for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o2));
     float ls = 0.f;
@@ -239,10 +206,10 @@ __device__ __forceinline__ void merge_splits_last(const DecodeParams& p, int b, 
       }
     }
     for (int sI = lane + 32 * kSPL; sI < S; sI += 32) {
-      const float m = __ldcg(pv.m + bh * SP + sI);
+      const float m = __ldcg(pv.m + bh * S + sI);
       const float wk = m > -INFINITY ? expf(m - mx) : 0.f;
       w[sI] = wk;
-      ls = fmaf(wk, __ldcg(pv.l + bh * SP + sI), ls);
+      ls = fmaf(wk, __ldcg(pv.l + bh * S + sI), ls);
     }
     for (int o2 = 16; o2 > 0; o2 >>= 1) ls += __shfl_xor_sync(kFull, ls, o2);
     __syncwarp();
