@@ -27,8 +27,10 @@
 //                        (same softmax weights; exact algebra).
 #include <math.h>
 
+#include <algorithm>
 #include <mutex>
 
+#include "codec.cuh"
 #include "headq_internal.cuh"
 
 #define HEADQ_API extern "C" __attribute__((visibility("default")))
@@ -43,6 +45,7 @@ constexpr int kSelThreads = 1024;
 constexpr int kFixThreads = 512;
 constexpr int kFixTok = 64;      // kept tokens per fixup step
 constexpr int kFixMaxOut = 2048 / kFixThreads;
+constexpr int kFixHeads = 8;     // heads per KV head accumulated per thread (G <= 8)
 
 struct A2Params {
   headq_cache c;
@@ -458,33 +461,73 @@ __global__ void __launch_bounds__(kMT) a2_pass_mma_kernel(const A2Params p) {
   }
 }
 
-// |v^_j - v_j|^2 of every token j < T into scores (0 for j >= T_b): D/8 lanes
-// per token, 8 channels each, summed by shuffles within the token's lanes; CTA
-// (token block, kv, b)
+// |v^_j - v_j|^2 of every token j < T into scores (0 for j >= T_b): one lane per
+// (token, 32-channel group), summed over the token's D/32 lanes by shuffles;
+// CTA (token block, kv, b).  2-bit values: the group's 32 exact bf16 values (four
+// 16-byte loads), its 8 code bytes, scale and minimum; v^ = min + code * scale
+// rounded as the codec rounds it (a rounded product, then a rounded sum), in
+// packed fp32 pairs (each lane one IEEE round-to-nearest operation; separate
+// PTX statements, so nothing is contracted); each code becomes an exact float
+// as (2^23 | code) - 2^23.  Dense values: the cached values.
 template <int D>
 __global__ void __launch_bounds__(256) a2_dv2_kernel(const A2Params p) {
-  constexpr int LPT = D / 8;           // lanes per token (a power of two, <= 32)
+  constexpr int LPT = D / 32;          // lanes per token (one per group)
   constexpr int TPB = 256 / LPT;       // tokens per CTA
   const int kv = blockIdx.y, b = blockIdx.z;
   const int tt = blockIdx.x * TPB + threadIdx.x / LPT;
-  const int c0 = (threadIdx.x % LPT) * 8;
+  const int g = threadIdx.x % LPT;
   const size_t bk = static_cast<size_t>(b) * p.c.Hkv + kv;
   const bool live = tt < seq_len(p.seq_lens, b, p.T);
   float a = 0.0f;
   if (live) {
-    const size_t row = cache_row_read(p.c, b, kv, tt, c0 == 0 ? p.err : nullptr);
-    float v[8], vh[8];
-    load8(p.v_full, (bk * p.T + tt) * D + c0, true, v);
-    value_hat8(p.c, row, c0, D, vh);
+    const size_t row = cache_row_read(p.c, b, kv, tt, g == 0 ? p.err : nullptr);
+    const uint4* vp = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.v_full) +
+                                                     (bk * p.T + tt) * D + 32 * g);
+    uint32_t vw[16];  // the 32 exact values, bf16 pairs
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float dv = vh[k] - v[k];
-      a = fmaf(dv, dv, a);
+    for (int k = 0; k < 4; ++k) {
+      const uint4 u = vp[k];
+      vw[4 * k] = u.x; vw[4 * k + 1] = u.y; vw[4 * k + 2] = u.z; vw[4 * k + 3] = u.w;
     }
+    uint64_t acc = 0;  // (+0, +0)
+    if (p.c.vmode == HEADQ_V_2BIT) {
+      const uint2 cw = *reinterpret_cast<const uint2*>(p.c.v_codes + row * (D / 4) + 8 * g);
+      const uint64_t sc = codec::dup2(p.c.v_scale[row * (D / 32) + g]);
+      const uint64_t mn = codec::dup2(p.c.v_min[row * (D / 32) + g]);
+      const uint64_t magic = codec::dup2(8388608.0f);  // 2^23
+#pragma unroll
+      for (int w = 0; w < 16; ++w) {  // channels 2w, 2w + 1 of the group
+        const uint32_t word = w < 8 ? cw.x : cw.y;
+        const uint32_t sh = 4 * (w & 7);
+        const uint64_t code =
+            codec::sub2(codec::pk2(__uint_as_float(((word >> sh) & 3u) | 0x4B000000u),
+                                   __uint_as_float(((word >> (sh + 2)) & 3u) | 0x4B000000u)),
+                        magic);
+        const uint64_t vh = codec::add2(mn, codec::mul2(code, sc));
+        const uint64_t v = codec::pk2(__uint_as_float(vw[w] << 16), __uint_as_float(vw[w] & 0xffff0000u));
+        const uint64_t dv = codec::sub2(vh, v);
+        acc = codec::fma2(dv, dv, acc);
+      }
+    } else {
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float vh[8];
+        value_hat8(p.c, row, 32 * g + 8 * c8, D, vh);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t u = vw[4 * c8 + k];
+          const uint64_t dv = codec::sub2(codec::pk2(vh[2 * k], vh[2 * k + 1]),
+                                          codec::pk2(__uint_as_float(u << 16),
+                                                     __uint_as_float(u & 0xffff0000u)));
+          acc = codec::fma2(dv, dv, acc);
+        }
+      }
+    }
+    a = codec::pk_lo(acc) + codec::pk_hi(acc);
   }
 #pragma unroll
   for (int o2 = 1; o2 < LPT; o2 <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o2);
-  if (tt < p.T && c0 == 0) p.scores[bk * p.T + tt] = live ? a : 0.0f;
+  if (tt < p.T && g == 0) p.scores[bk * p.T + tt] = live ? a : 0.0f;
 }
 
 // lse of every observation query from the tile partials; one CTA per (b, kv)
@@ -649,8 +692,12 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
   float* qg_s = q_s + G * D;          // [G][NG]
   float* qt_s = qg_s + G * NG;        // [G][r]
   float* lse_s = qt_s + G * r;        // [G]
-  float* p_s = lse_s + G;             // [kFixTok][G]
-  int* idx_s = reinterpret_cast<int*>(p_s + kFixTok * G);            // [kFixTok]
+  // weights exp(s^_j - lse) [kFixTok][PS]: PS = kFixHeads (16-byte rows, heads
+  // G.. zero) when the accumulation is blocked by channel, else G
+  const bool blocked = D >= 64 && G <= kFixHeads;
+  const int PS = blocked ? kFixHeads : G;
+  float* p_s = smem_align(lse_s + G, 16);
+  int* idx_s = reinterpret_cast<int*>(p_s + kFixTok * PS);           // [kFixTok]
   size_t* row_s = reinterpret_cast<size_t*>(smem_align(idx_s + kFixTok, 8));  // [kFixTok]
   uint32_t* kc_s = reinterpret_cast<uint32_t*>(row_s + kFixTok);     // [kFixTok][D/16]
   float* ks_s = reinterpret_cast<float*>(kc_s + kFixTok * FS::kKcWords);  // [kFixTok][NG]
@@ -667,6 +714,7 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
   for (int i = tid; i < G * D; i += kFixThreads)
     q_s[i] = load_elem(p.q, (static_cast<size_t>(b) * p.Hq + h0) * D + i, p.q_bf16);
   for (int h = tid; h < G; h += kFixThreads) lse_s[h] = p.lse[static_cast<size_t>(b) * p.Hq + h0 + h];
+  for (int e = tid; e < kFixTok * PS; e += kFixThreads) p_s[e] = 0.0f;  // padded heads stay 0
   __syncthreads();
   for (int i = tid; i < G * NG; i += kFixThreads) {
     const int h = i / NG, g = i - h * NG;
@@ -685,9 +733,15 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
     qt_s[i] = p.corr_sign * acc;
   }
 
-  float acc[kFixMaxOut];
+  // blocked (G <= kFixHeads, D >= 64, so that the [TQ][kFixHeads][D] class sums
+  // fit in the value-difference tile): acc[h] = head h, channel cf, the tokens of
+  // class tq; else acc[k] = output tid + k * kFixThreads over all tokens
+  static_assert(D < 64 || kFixThreads * kFixHeads <= kFixTok * D, "class sums fit");
+  constexpr int kAcc = kFixMaxOut > kFixHeads ? kFixMaxOut : kFixHeads;
+  const int cf = tid % D, tq = tid / D;
+  float acc[kAcc];
 #pragma unroll
-  for (int k = 0; k < kFixMaxOut; ++k) acc[k] = 0.0f;
+  for (int k = 0; k < kAcc; ++k) acc[k] = 0.0f;
 
   for (int k0 = 0; k0 < p.K; k0 += kFixTok) {
     __syncthreads();
@@ -784,7 +838,7 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
           }
 #pragma unroll
           for (int o2 = 1; o2 < kFP; o2 <<= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o2);
-          if (part == 0) p_s[tt * G + h] = live ? expf(sp * p.sm_scale - lse_s[h]) : 0.0f;
+          if (part == 0) p_s[tt * PS + h] = live ? expf(sp * p.sm_scale - lse_s[h]) : 0.0f;
         }
       }
     } else {
@@ -815,28 +869,60 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
           }
           w = expf(s * p.sm_scale - lse_s[h]);
         }
-        p_s[tt * G + h] = w;
+        p_s[tt * PS + h] = w;
       }
     }
     __syncthreads();
+    if (blocked) {
+      // thread (c, tq): channel c for every head over the tokens tt = tq mod TQ
+      // of the step (one value load, the heads' weights as broadcasts)
+#pragma unroll 4
+      for (int tt = tq; tt < kFixTok; tt += kFixThreads / D) {
+        const float dv = dv_s[tt * D + cf];
+        const float4 pa = reinterpret_cast<const float4*>(p_s + tt * kFixHeads)[0];
+        const float4 pb = reinterpret_cast<const float4*>(p_s + tt * kFixHeads)[1];
+        acc[0] = fmaf(pa.x, dv, acc[0]); acc[1] = fmaf(pa.y, dv, acc[1]);
+        acc[2] = fmaf(pa.z, dv, acc[2]); acc[3] = fmaf(pa.w, dv, acc[3]);
+        acc[4] = fmaf(pb.x, dv, acc[4]); acc[5] = fmaf(pb.y, dv, acc[5]);
+        acc[6] = fmaf(pb.z, dv, acc[6]); acc[7] = fmaf(pb.w, dv, acc[7]);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < kFixMaxOut; ++k) {
+        const int idx = tid + k * kFixThreads;
+        if (idx < G * D) {
+          const int h = idx / D, c = idx - h * D;
+          float a = acc[k];
+#pragma unroll
+          for (int tt = 0; tt < kFixTok; ++tt) a = fmaf(p_s[tt * PS + h], dv_s[tt * D + c], a);
+          acc[k] = a;
+        }
+      }
+    }
+  }
+  if (blocked) {
+    // the token classes' sums, in a fixed order, through shared memory
+    constexpr int TQ = kFixThreads / D;
+    __syncthreads();
+    float* red = dv_s;  // [TQ][kFixHeads][D], inside the (consumed) value-difference tile
+#pragma unroll
+    for (int h = 0; h < kFixHeads; ++h)
+      if (h < G) red[(tq * kFixHeads + h) * D + cf] = acc[h];
+    __syncthreads();
+    for (int idx = tid; idx < G * D; idx += kFixThreads) {
+      const int h = idx / D, c = idx - h * D;
+      float a = 0.0f;
+      for (int q = 0; q < TQ; ++q) a += red[(q * kFixHeads + h) * D + c];
+      p.out[(static_cast<size_t>(b) * p.Hq + h0 + h) * D + c] += a;
+    }
+  } else {
 #pragma unroll
     for (int k = 0; k < kFixMaxOut; ++k) {
       const int idx = tid + k * kFixThreads;
       if (idx < G * D) {
         const int h = idx / D, c = idx - h * D;
-        float a = acc[k];
-#pragma unroll
-        for (int tt = 0; tt < kFixTok; ++tt) a = fmaf(p_s[tt * G + h], dv_s[tt * D + c], a);
-        acc[k] = a;
+        p.out[(static_cast<size_t>(b) * p.Hq + h0 + h) * D + c] += acc[k];
       }
-    }
-  }
-#pragma unroll
-  for (int k = 0; k < kFixMaxOut; ++k) {
-    const int idx = tid + k * kFixThreads;
-    if (idx < G * D) {
-      const int h = idx / D, c = idx - h * D;
-      p.out[(static_cast<size_t>(b) * p.Hq + h0 + h) * D + c] += acc[k];
     }
   }
 }
@@ -877,7 +963,7 @@ cudaError_t launch_scores(A2Params p, cudaStream_t s) {
       pl.ntiles = parts;
       pl.ppt = 1;
       a2_lse_kernel<<<p.c.B * p.c.Hkv, NQ < 1024 ? (NQ + 31) / 32 * 32 : 1024, 0, s>>>(pl);
-      constexpr int kDv2Tok = 256 / (D / 8);
+      constexpr int kDv2Tok = 256 / (D / 32);
       a2_dv2_kernel<D><<<dim3((p.T + kDv2Tok - 1) / kDv2Tok, p.c.Hkv, p.c.B), 256, 0, s>>>(p);
       a2_pass_mma_kernel<D, true><<<mgrid, kMT, smem, s>>>(p);
       return cudaGetLastError();
@@ -905,7 +991,8 @@ template <int D>
 cudaError_t launch_fixup(const FixParams& p, cudaStream_t s) {
   const int G = p.G;
   const size_t smem = sizeof(float) * (static_cast<size_t>(G) * D + G * num_groups(D) +
-                                       G * p.c.r + G + kFixTok * G + kFixTok * D) +
+                                       G * p.c.r + G + kFixTok * std::max(G, kFixHeads) +
+                                       kFixTok * D) + 16 +
                       sizeof(int) * 2 * kFixTok + sizeof(size_t) * kFixTok + FixStage<D>::bytes();
   auto k = a2_fixup_kernel<D>;
   if (smem > 48 * 1024) {
