@@ -249,6 +249,12 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// 2^x, results below 2^-126 flushed to zero (2^-inf = 0)
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 // 16 bytes global -> shared, asynchronously; zero-filled when `valid` is false
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
@@ -278,7 +284,7 @@ constexpr size_t a2_mma_smem() {
 }
 
 template <int D, bool SCORE>
-__global__ void __launch_bounds__(kMT) a2_pass_mma_kernel(const A2Params p) {
+__global__ void __launch_bounds__(kMT, 3) a2_pass_mma_kernel(const A2Params p) {
   constexpr int RS = D + 8;  // bf16 elements per shared row
   constexpr int KSTEPS = D / 16;
   constexpr int CPR = D / 8; // 16-byte chunks per row
@@ -368,9 +374,11 @@ __global__ void __launch_bounds__(kMT) a2_pass_mma_kernel(const A2Params p) {
       __syncthreads();  // tile k in shared memory
       const uint16_t* kb = k_s + (k & 1) * kAT * RS;
       if (wlive) {
+        // the tile's logits of this lane: rows g | g + 8 x tokens 8 nt + 2t, + 1
+        float cv[kAT / 8][4];
 #pragma unroll
         for (int nt = 0; nt < kAT / 8; ++nt) {
-          float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          cv[nt][0] = cv[nt][1] = cv[nt][2] = cv[nt][3] = 0.0f;
           // B fragments of two k-steps per ldmatrix: matrices = channels
           // [32 kk, +8), [+8, +16), [+16, +24), [+24, +32) of tokens 8 nt .. 8 nt + 7
           const uint16_t* br = kb + (8 * nt + (lane & 7)) * RS + 8 * (lane >> 3);
@@ -378,41 +386,66 @@ __global__ void __launch_bounds__(kMT) a2_pass_mma_kernel(const A2Params p) {
           for (int kk = 0; kk < KSTEPS / 2; ++kk) {
             uint32_t bf[4];
             ldsm_x4(br + 32 * kk, bf);
-            mma_bf16_16816(c, qa[2 * kk], bf[0], bf[1]);
-            mma_bf16_16816(c, qa[2 * kk + 1], bf[2], bf[3]);
+            mma_bf16_16816(cv[nt], qa[2 * kk], bf[0], bf[1]);
+            mma_bf16_16816(cv[nt], qa[2 * kk + 1], bf[2], bf[3]);
           }
-          // c: (row g | g + 8) x (tokens j, j + 1) of this lane
-          const int j = tile * kAT + 8 * nt + 2 * t;
-          const bool c0 = j < Tb, c1 = j + 1 < Tb;
-          if constexpr (!SCORE) {
+        }
+        // tokens past T_b (the last tile of a sequence) take logit -inf
+        if ((tile + 1) * kAT > Tb) {
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-              const float xa = c0 ? c[2 * rr] * s2 : -INFINITY;
-              const float xb = c1 ? c[2 * rr + 1] * s2 : -INFINITY;
-              const float mx = fmaxf(xa, xb);
-              if (mx > m[rr]) {  // a new maximum: rescale the sum (exp2(-inf) = 0)
-                l[rr] *= exp2f(m[rr] - mx);
-                m[rr] = mx;
-              }
-              if (m[rr] != -INFINITY) l[rr] += exp2f(xa - m[rr]) + exp2f(xb - m[rr]);
-            }
-          } else {
-            const float p00 = (c0 && r0) ? exp2f(c[0] * s2 - lse2[0]) : 0.0f;
-            const float p01 = (c1 && r0) ? exp2f(c[1] * s2 - lse2[0]) : 0.0f;
-            const float p10 = (c0 && r1) ? exp2f(c[2] * s2 - lse2[1]) : 0.0f;
-            const float p11 = (c1 && r1) ? exp2f(c[3] * s2 - lse2[1]) : 0.0f;
-            // column sums over the warp's 16 rows
-            float sa = fmaf(p00, p00, p10 * p10), sb = fmaf(p01, p01, p11 * p11);
+          for (int nt = 0; nt < kAT / 8; ++nt) {
+            const int j = tile * kAT + 8 * nt + 2 * t;
+            if (j >= Tb) cv[nt][0] = cv[nt][2] = -INFINITY;
+            if (j + 1 >= Tb) cv[nt][1] = cv[nt][3] = -INFINITY;
+          }
+        }
+        if constexpr (!SCORE) {
+          // per row: the tile's maximum, then one rescale of the running sum
 #pragma unroll
-            for (int o2 = 4; o2 < 32; o2 <<= 1) {
-              sa += __shfl_xor_sync(0xffffffffu, sa, o2);
-              sb += __shfl_xor_sync(0xffffffffu, sb, o2);
-            }
-            if (g == 0) {
-              red_s[warp * kAT + 8 * nt + 2 * t] = sa;
-              red_s[warp * kAT + 8 * nt + 2 * t + 1] = sb;
+          for (int rr = 0; rr < 2; ++rr) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < kAT / 8; ++nt)
+              mx = fmaxf(mx, fmaxf(cv[nt][2 * rr], cv[nt][2 * rr + 1]));
+            const float mnew = fmaxf(m[rr], mx * s2);  // log2 units (s2 > 0)
+            if (mnew != -INFINITY) {
+              float acc = 0.0f;
+#pragma unroll
+              for (int nt = 0; nt < kAT / 8; ++nt)
+                acc += ex2_ftz(fmaf(cv[nt][2 * rr], s2, -mnew)) +
+                       ex2_ftz(fmaf(cv[nt][2 * rr + 1], s2, -mnew));
+              l[rr] = fmaf(l[rr], ex2_ftz(m[rr] - mnew), acc);  // 2^-inf = 0
+              m[rr] = mnew;
             }
           }
+        } else {
+          // p^2 summed over the warp's 16 rows for each of the lane's 16 columns
+          // (v[2 nt + e] = token 8 nt + 2t + e), then a butterfly over the lanes
+          // of the same t (xor 16, 8, 4): each step keeps half of the columns,
+          // so that lane (g, t) ends with the sums of tokens 8g + 2t + {0, 1}
+          float v[kAT / 4];
+#pragma unroll
+          for (int nt = 0; nt < kAT / 8; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float pa = r0 ? ex2_ftz(fmaf(cv[nt][e], s2, -lse2[0])) : 0.0f;
+              const float pb = r1 ? ex2_ftz(fmaf(cv[nt][2 + e], s2, -lse2[1])) : 0.0f;
+              v[2 * nt + e] = fmaf(pa, pa, pb * pb);
+            }
+          }
+#pragma unroll
+          for (int step = 0; step < 3; ++step) {
+            const int bit = 16 >> step, n = 8 >> step;  // lanes apart, values kept
+            const bool up = (lane & bit) != 0;
+#pragma unroll
+            for (int i = 0; i < n; ++i) {
+              const float keep = up ? v[n + i] : v[i];
+              const float give = up ? v[i] : v[n + i];
+              v[i] = keep + __shfl_xor_sync(0xffffffffu, give, bit);
+            }
+          }
+          red_s[warp * kAT + 8 * g + 2 * t] = v[0];
+          red_s[warp * kAT + 8 * g + 2 * t + 1] = v[1];
         }
       }
       if constexpr (SCORE) {
