@@ -628,24 +628,42 @@ a2_select_kernel(const float* scores, int Hkv, const int32_t* seq_lens, int T, i
     s_rem = Keff;
   }
   unsigned mask = 0u;
+  const int lane = tid & 31;
   for (int shift = 24; shift >= 0 && Keff > 0; shift -= 8) {
     for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0u;
     __syncthreads();
     const unsigned pre = s_pre;
-    for (int t = tid; t < Tb; t += kSelThreads) {
-      const unsigned u = key[t];
-      if ((u & mask) == pre) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    for (int t0 = 0; t0 < Tb; t0 += kSelThreads) {
+      const int t = t0 + tid;
+      const unsigned u = t < Tb ? key[t] : 0u;
+      const bool in = t < Tb && (u & mask) == pre;
+      // the lanes of this warp with the same bin (lanes outside share 256): one
+      // atomic per distinct bin, by its lowest lane
+      const unsigned bin = in ? (u >> shift) & 255u : 256u;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<unsigned>(__popc(peers)));
     }
     __syncthreads();
-    if (tid == 0) {
-      int rem = s_rem, bin = 255;
-      for (; bin > 0; --bin) {
-        const int h = static_cast<int>(hist[bin]);
-        if (h >= rem) break;
-        rem -= h;
+    // the bin holding the s_rem-th largest: counts summed from the top bin down
+    // (thread i <-> bin 255 - i), an inclusive scan over the 256 threads
+    if (tid < 256) {
+      const int rem = s_rem;
+      const unsigned h = hist[255 - tid];
+      unsigned c = h;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, c, o);
+        if (lane >= o) c += y;
       }
-      s_rem = rem;
-      s_pre = pre | (static_cast<unsigned>(bin) << shift);
+      if (lane == 31) wsum[tid >> 5] = static_cast<int>(c);
+      asm volatile("bar.sync 2, 256;" ::: "memory");
+      unsigned before = 0u;
+      for (int w = 0; w < (tid >> 5); ++w) before += static_cast<unsigned>(wsum[w]);
+      c += before;
+      if (c >= static_cast<unsigned>(rem) && c - h < static_cast<unsigned>(rem)) {
+        s_rem = rem - static_cast<int>(c - h);
+        s_pre = pre | (static_cast<unsigned>(255 - tid) << shift);
+      }
     }
     mask |= 255u << shift;
     __syncthreads();
