@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kAThreads) a2_pass_kernel(const A2Params p) {
 // |v^_j - v_j|^2 comes from a2_dv2_kernel, already in `scores`.
 constexpr int kQW = 8;           // query warps: 16 queries each
 constexpr int kMT = 32 * kQW;    // threads
-constexpr int kTPC = 8;          // tiles per CTA
+constexpr int kTPC = 16;         // tiles per CTA
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
                                                uint32_t b1) {
