@@ -61,9 +61,8 @@ constexpr float kMaxInit = -1e30f;        // running max before the first logit 
 // pipeline depth (the stages also hold the merging CTA's [G][splits] weights)
 // and CTAs per SM: two, with registers for the operand fragments, the output
 // and the per-(head, group) exponents without spilling
-template <int D, bool V2>
-constexpr int kStagesHM = V2 ? 8 : 4;
 template <bool V2>
+constexpr int kStagesHM = V2 ? 8 : 4;
 constexpr int kMinCtasHM = 2;
 
 // stages | q [8][D] | group sums and maxima [8][NG] each | sigma U^T q [8][R] |
@@ -73,9 +72,9 @@ template <int D, int R, bool V2>
 constexpr size_t hm_smem_bytes() {
   using L = StageLayout<D, R, V2>;
   constexpr int RR = R > 0 ? R : 1;
-  return 1024 + size_t(kStagesHM<D, V2>) * L::kStage +
+  return 1024 + size_t(kStagesHM<V2>) * L::kStage +
          sizeof(float) * (kGM * D + 2 * kGM * L::NG + kGM * RR + D * RR + kGM * D + D) + 16 +
-         8 * (2 * kStagesHM<D, V2> + 1) + 4 * kStagesHM<D, V2> + 16;
+         8 * (2 * kStagesHM<V2> + 1) + 4 * kStagesHM<V2> + 16;
 }
 
 // 2^x, flushing results below 2^-126 to zero (2^-inf = 0)
@@ -112,14 +111,14 @@ __device__ __forceinline__ void load_groups(const uint8_t* row, float (&v)[N]) {
 }
 
 template <int D, int R, bool V2>
-__global__ void __launch_bounds__(kThreads, kMinCtasHM<V2>)
+__global__ void __launch_bounds__(kThreads, kMinCtasHM)
 decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap) {
   using L = StageLayout<D, R, V2>;
   constexpr int NG = L::NG;
   constexpr int KS = D / 16;   // k-steps of 16 channels
   constexpr int MT = D / 16;   // 16-channel row blocks of the output
   constexpr int RR = R > 0 ? R : 1;
-  constexpr int kStages = kStagesHM<D, V2>;
+  constexpr int kStages = kStagesHM<V2>;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = smem_align(smem_raw, 1024);
@@ -615,10 +614,10 @@ struct HmVariant {
   // the warps' partials (outputs, maxima, sums, group minima), and later the
   // merging CTA's [G][splits] split weights, lie inside the stages
   static_assert(sizeof(float) * kCW * kGM * (D + 2 + D / 32) <=
-                    size_t(kStagesHM<D, V2>) * StageLayout<D, R, V2>::kStage,
+                    size_t(kStagesHM<V2>) * StageLayout<D, R, V2>::kStage,
                 "warp partials fit in the stages");
   static_assert(sizeof(float) * kGM * kMaxMmaSplits <=
-                    size_t(kStagesHM<D, V2>) * StageLayout<D, R, V2>::kStage,
+                    size_t(kStagesHM<V2>) * StageLayout<D, R, V2>::kStage,
                 "split weights fit in the stages");
 
   static int ctas_per_sm() {
