@@ -42,6 +42,7 @@ constexpr int kAT = 64;          // tokens per score tile
 constexpr int kAThreads = 256;   // 64 tokens x 4 query lanes
 constexpr int kAQC = 16;         // observation queries staged per chunk
 constexpr int kSelThreads = 1024;
+constexpr int kSelReg = 4;       // scores per select thread kept in registers
 constexpr int kFixThreads = 512;
 constexpr int kFixTok = 64;      // kept tokens per fixup step
 constexpr int kFixMaxOut = 2048 / kFixThreads;
@@ -627,21 +628,33 @@ a2_select_kernel(const float* scores, int Hkv, const int32_t* seq_lens, int T, i
     s_pre = 0u;
     s_rem = Keff;
   }
+  // the first kSelReg * kSelThreads scores stay in registers for all passes
+  unsigned kr[kSelReg];
+#pragma unroll
+  for (int c = 0; c < kSelReg; ++c) {
+    const int t = c * kSelThreads + tid;
+    kr[c] = t < Tb ? key[t] : 0u;
+  }
   unsigned mask = 0u;
   const int lane = tid & 31;
   for (int shift = 24; shift >= 0 && Keff > 0; shift -= 8) {
     for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0u;
     __syncthreads();
     const unsigned pre = s_pre;
-    for (int t0 = 0; t0 < Tb; t0 += kSelThreads) {
-      const int t = t0 + tid;
-      const unsigned u = t < Tb ? key[t] : 0u;
-      const bool in = t < Tb && (u & mask) == pre;
-      // the lanes of this warp with the same bin (lanes outside share 256): one
-      // atomic per distinct bin, by its lowest lane
+    // the lanes of a warp with the same bin (lanes outside share 256): one atomic
+    // per distinct bin, by its lowest lane
+    auto count = [&](unsigned u, bool valid) {
+      const bool in = valid && (u & mask) == pre;
       const unsigned bin = in ? (u >> shift) & 255u : 256u;
       const unsigned peers = __match_any_sync(0xffffffffu, bin);
       if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<unsigned>(__popc(peers)));
+    };
+#pragma unroll
+    for (int c = 0; c < kSelReg; ++c)
+      if (c * kSelThreads < Tb) count(kr[c], c * kSelThreads + tid < Tb);
+    for (int t0 = kSelReg * kSelThreads; t0 < Tb; t0 += kSelThreads) {
+      const int t = t0 + tid;
+      count(t < Tb ? key[t] : 0u, t < Tb);
     }
     __syncthreads();
     // the bin holding the s_rem-th largest: counts summed from the top bin down
@@ -673,9 +686,7 @@ a2_select_kernel(const float* scores, int Hkv, const int32_t* seq_lens, int T, i
 
   // ordered compaction: every token above tau, and the first need_eq equal to it
   int base = 0, eq_base = 0;
-  for (int t0 = 0; t0 < Tb && Keff > 0; t0 += kSelThreads) {
-    const int t = t0 + tid;
-    const unsigned u = t < Tb ? key[t] : 0u;
+  auto compact = [&](unsigned u, int t) {
     const bool eq = t < Tb && u == tau;
     int eq_total = 0;
     const int eq_rank = block_excl_count(eq, wsum, &eq_total);
@@ -685,6 +696,15 @@ a2_select_kernel(const float* scores, int Hkv, const int32_t* seq_lens, int T, i
     if (take && base + pos < Keff) out_idx[base + pos] = t;
     base += take_total;
     eq_base += eq_total;
+  };
+  if (Keff > 0) {
+#pragma unroll
+    for (int c = 0; c < kSelReg; ++c)
+      if (c * kSelThreads < Tb) compact(kr[c], c * kSelThreads + tid);
+    for (int t0 = kSelReg * kSelThreads; t0 < Tb; t0 += kSelThreads) {
+      const int t = t0 + tid;
+      compact(t < Tb ? key[t] : 0u, t);
+    }
   }
   for (int k = Keff + tid; k < K; k += kSelThreads) out_idx[k] = -1;
   __syncthreads();
