@@ -45,6 +45,7 @@ constexpr int kSelThreads = 1024;
 constexpr int kSelReg = 4;       // scores per select thread kept in registers
 constexpr int kFixThreads = 512;
 constexpr int kFixTok = 64;      // kept tokens per fixup step
+constexpr int kFixIdx = 512;     // kept-token indices loaded at once (a multiple of kFixTok)
 constexpr int kFixMaxOut = 2048 / kFixThreads;
 constexpr int kFixHeads = 8;     // heads per KV head accumulated per thread (G <= 8)
 
@@ -250,6 +251,7 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+constexpr float kLog2eF = 1.4426950408889634f;
 // 2^x, results below 2^-126 flushed to zero (2^-inf = 0)
 __device__ __forceinline__ float ex2_ftz(float x) {
   float y;
@@ -768,9 +770,10 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
   const bool blocked = D >= 64 && G <= kFixHeads;
   const int PS = blocked ? kFixHeads : G;
   float* p_s = smem_align(lse_s + G, 16);
-  int* idx_s = reinterpret_cast<int*>(p_s + kFixTok * PS);           // [kFixTok]
-  size_t* row_s = reinterpret_cast<size_t*>(smem_align(idx_s + kFixTok, 8));  // [kFixTok]
-  uint32_t* kc_s = reinterpret_cast<uint32_t*>(row_s + kFixTok);     // [kFixTok][D/16]
+  // kept-token indices and cache rows of a chunk of kFixIdx (every step of it)
+  int* idx_all = reinterpret_cast<int*>(p_s + kFixTok * PS);         // [kFixIdx]
+  size_t* row_all = reinterpret_cast<size_t*>(smem_align(idx_all + kFixIdx, 8));  // [kFixIdx]
+  uint32_t* kc_s = reinterpret_cast<uint32_t*>(row_all + kFixIdx);   // [kFixTok][D/16]
   float* ks_s = reinterpret_cast<float*>(kc_s + kFixTok * FS::kKcWords);  // [kFixTok][NG]
   float* km_s = ks_s + kFixTok * NG;                                  // [kFixTok][NG]
   float* zs_s = km_s + kFixTok * NG;                                  // [kFixTok]
@@ -816,13 +819,17 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
 
   for (int k0 = 0; k0 < p.K; k0 += kFixTok) {
     __syncthreads();
-    if (tid < kFixTok) {
-      const int t = k0 + tid < p.K ? p.keep_idx[bk * p.K + k0 + tid] : -1;
-      const bool ok = t >= 0 && t < Tb;
-      idx_s[tid] = ok ? t : -1;
-      row_s[tid] = ok ? cache_row_read(p.c, b, kv, t, nullptr) : 0;
+    if (k0 % kFixIdx == 0) {  // a new chunk: every step's indices and rows at once
+      for (int k = tid; k < kFixIdx; k += kFixThreads) {
+        const int t = k0 + k < p.K ? p.keep_idx[bk * p.K + k0 + k] : -1;
+        const bool ok = t >= 0 && t < Tb;
+        idx_all[k] = ok ? t : -1;
+        row_all[k] = ok ? cache_row_read(p.c, b, kv, t, nullptr) : 0;
+      }
+      __syncthreads();
     }
-    __syncthreads();
+    const int* idx_s = idx_all + k0 % kFixIdx;     // this step's kFixTok entries
+    const size_t* row_s = row_all + k0 % kFixIdx;
     // stage the kept tokens' key planes (word-wide, all threads)
     if constexpr (D >= 16) {
       for (int e = tid; e < kFixTok * FS::kKcWords; e += kFixThreads) {
@@ -909,7 +916,7 @@ __global__ void __launch_bounds__(kFixThreads) a2_fixup_kernel(const FixParams p
           }
 #pragma unroll
           for (int o2 = 1; o2 < kFP; o2 <<= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o2);
-          if (part == 0) p_s[tt * PS + h] = live ? expf(sp * p.sm_scale - lse_s[h]) : 0.0f;
+          if (part == 0) p_s[tt * PS + h] = live ? ex2_ftz((sp * p.sm_scale - lse_s[h]) * kLog2eF) : 0.0f;
         }
       }
     } else {
@@ -1064,7 +1071,7 @@ cudaError_t launch_fixup(const FixParams& p, cudaStream_t s) {
   const size_t smem = sizeof(float) * (static_cast<size_t>(G) * D + G * num_groups(D) +
                                        G * p.c.r + G + kFixTok * std::max(G, kFixHeads) +
                                        kFixTok * D) + 16 +
-                      sizeof(int) * 2 * kFixTok + sizeof(size_t) * kFixTok + FixStage<D>::bytes();
+                      sizeof(int) * (kFixIdx + 2) + sizeof(size_t) * kFixIdx + FixStage<D>::bytes();
   auto k = a2_fixup_kernel<D>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
