@@ -31,9 +31,11 @@
 //    group g, in fp16 relative to a power of two 2^E per (warp, head, group)
 //    that is raised once an entry reaches 2^12 of it; the minimum enters as
 //    sum_j p_j min_{j,g} in fp32.
-//  * each consumer warp takes 16 tokens of every 64-token stage with its own
-//    online softmax (log2 domain, lazily rescaled max); the four warps merge
-//    through shared memory at the end and the splits by the last CTA.
+//  * five consumer warps take the four 16-token slices of the 64-token stages in
+//    turn, each with its own online softmax (log2 domain, lazily rescaled max);
+//    a stage is released after its four slices.  Five, because two CTAs of six
+//    warps at this register count still fit an SM.  The warps merge through
+//    shared memory at the end and the splits by the last CTA.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -49,7 +51,8 @@ namespace headq {
 namespace {
 using namespace dc;
 
-constexpr int kCW = 4;                    // consumer warps
+constexpr int kCW = 5;                    // consumer warps
+constexpr int kSlices = 4;                // 16-token slices per 64-token stage
 constexpr int kTile = kPipeTile;          // tokens per stage
 constexpr int kThreads = (kCW + 1) * 32;  // + one producer warp
 constexpr int kGM = 8;                    // head slots
@@ -149,7 +152,7 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_addr(&bars[s]), 1);
-      mbar_init(smem_addr(&bars[kStages + s]), kCW);
+      mbar_init(smem_addr(&bars[kStages + s]), kSlices);
     }
     mbar_init(smem_addr(&bars[2 * kStages]), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -197,7 +200,6 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
   asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory");
 
   const int g = lane >> 2, t = lane & 3;
-  const int jw = 16 * warp;  // this warp's tokens in a stage
 
   // Operand fields of this thread: its code bits sit at 4t (and 4t + 16) of each
   // 32-bit key-code word; after the shift sh they sit at p0 = 4 (t & 1), so the
@@ -280,18 +282,21 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
   // and byte 2 (token 2t+1 or 2t+9)
   const uint32_t vsel = static_cast<uint32_t>((g & 3) | ((4 + (g & 3)) << 8));
   // ldmatrix row owned by this lane (dense values): matrix (lane >> 3), row (lane & 7)
-  const int lm_tok = jw + 8 * (lane >> 4) + (lane & 7);
+  const int lm_row = 8 * (lane >> 4) + (lane & 7);  // + the slice's first token
   const int lm_chunk_hi = (lane >> 3) & 1;
 
   bool ok = true;
-  for (int i = 0;; ++i) {
+  // The kCW warps take the kSlices 16-token slices of the stages in turn (slice
+  // j = tile j / kSlices, tokens 16 (j % kSlices) ..), each with its own online
+  // softmax; a stage is released after its kSlices slices.
+  for (int j = warp; j < ntiles * kSlices; j += kCW) {
+    const int i = j / kSlices, jw = 16 * (j - i * kSlices);
     const int s = i % kStages;
     if (!mbar_wait(smem_addr(&bars[s]), (i / kStages) & 1)) {
       ok = false;
       break;
     }
-    const int t0 = stile_s[s];  // the producer's tile for this stage, -1: no more
-    if (t0 < 0) break;
+    const int t0 = t_begin + i * kTile;
     uint8_t* st = stages + size_t(s) * L::kStage;
     const int nvalid = min(kTile, tile_end - t0);
 
@@ -485,8 +490,8 @@ decode_hm_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap)
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
         const int chunk = 2 * mt + lm_chunk_hi;
-        const uint32_t addr = vbase + (chunk >> 3) * L::kVBox + lm_tok * 128 +
-                              (((chunk & 7) ^ (lm_tok & 7)) << 4);
+        const uint32_t addr = vbase + (chunk >> 3) * L::kVBox + (jw + lm_row) * 128 +
+                              (((chunk & 7) ^ ((jw + lm_row) & 7)) << 4);
         uint32_t a[4];
         ldsm_x4_trans(addr, a);
         mma_bf16(o[mt], a, bh);
