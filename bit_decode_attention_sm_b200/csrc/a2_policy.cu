@@ -232,12 +232,14 @@ __global__ void __launch_bounds__(kAThreads) a2_pass_kernel(const A2Params p) {
 // tile loads during the current tile's MMAs.  Logits = Q K^T on mma.sync
 // m16n8k16 bf16 -> fp32: products of bf16 values are exact, so this differs from
 // the CUDA-core pass only in the order of the fp32 sums.
-//   pass 0: a running max and sum per query row in each lane (its two columns
-//           of every n8 tile), merged over the row's four lanes at the end: one
-//           (max, sum) partial per (CTA, query)
+//   pass 0: a running max and sum per query row in each lane (its sixteen
+//           columns of a tile: the tile's maximum first, then one exponential
+//           per logit and one rescale of the sum), merged over the row's four
+//           lanes at the end: one (max, sum) partial per (CTA, query)
 //   pass 1: p^2 per (query, token) summed over the chunk's queries per token:
-//           the row pair in each lane, the rows by warp shuffles, the warps in
-//           shared memory
+//           the row pair in each lane, the warp's rows by a butterfly over the
+//           lanes of a column (each step keeps half of the columns), the warps
+//           in shared memory
 // |v^_j - v_j|^2 comes from a2_dv2_kernel, already in `scores`.
 constexpr int kQW = 8;           // query warps: 16 queries each
 constexpr int kMT = 32 * kQW;    // threads
